@@ -1,0 +1,348 @@
+"""Pins of the fp64 oracle against facts other than itself (CPU only).
+
+Each check is chosen so that a plausible slip in the oracle (a dropped term, a wrong sign, a
+transposed state, the gate applied after instead of before the delta correction, an off-by-one
+in a window or a page index) fails at least one of them:
+
+* hand-worked two-token examples (tests/golden/delta_hand_examples.json);
+* closed forms: beta=0 & g=1 is the identity; beta=0 is pure decay; the delta-rule write
+  M_t^T k_t = (1-beta) M'^T k_t + beta v_t for unit k; orthonormal keys store and retrieve
+  values; one token from a zero state gives o = beta (k.q) v;
+* KDA with a uniform per-channel gate equals GDN (two differently oriented formulas);
+* the chunked UT-transform form equals the token-by-token recurrence (any chunk size, ragged T);
+* FA equals torch's scaled_dot_product_attention and a numpy softmax(QK^T/sqrt(d))V in fp64;
+  SWA with w >= L equals FA; w = 1 and L = 1 return the new token's value;
+* paged indexing: bijectivity of the FA map, injectivity of the SWA ring over every window,
+  and a new token's ring slot never holding a position inside the window.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_mixer_decoding_b200 import inputs as I
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _hand():
+    with open(os.path.join(GOLD, "delta_hand_examples.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_hand_worked_example(oracle_mod, kind):
+    O = oracle_mod
+    ex = _hand()
+    key = "gdn" if kind == I.GDN else "kda"
+    inp = ex["inputs"]
+    k = np.array(inp["k"])[None, :, None, :]
+    v = np.array(inp["v"])[None, :, None, :]
+    q = np.array(inp["q"])[None, :, None, :]
+    beta = np.array(inp["beta"])[None, :, None]
+    gate = np.array(ex[key]["gate"], dtype=np.float64)
+    log_gate = np.log(gate)[None, :, None] if kind == I.GDN else np.log(gate)[None, :, None, :]
+    s0 = np.zeros((1, 1, 2, 2))
+    for fn in (lambda: O.delta_recurrent(kind, q, k, v, beta, log_gate, s0),
+               lambda: O.delta_chunked(kind, q, k, v, beta, log_gate, s0, chunk=2),
+               lambda: O.delta_chunked(kind, q, k, v, beta, log_gate, s0, chunk=1)):
+        o, st = fn()
+        np.testing.assert_allclose(o[0, :, 0, :], np.array(ex[key]["o"]), atol=1e-12)
+        np.testing.assert_allclose(st[0, 0], np.array(ex[key]["final_state_M"]), atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_identity_when_beta0_g1(oracle_mod, kind):
+    """beta = 0 and g = 1 leave the state unchanged, and o = M0^T q."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 2, 7, 3, 8, 5, dtype="f32", seed=1, state0="randn")
+    lg = np.zeros_like(d.log_gate)
+    o, st = O.delta_recurrent(kind, d.q, d.k, d.v, np.zeros_like(d.beta), lg, d.state0)
+    np.testing.assert_array_equal(st, d.state0.astype(np.float64))
+    expect = np.einsum("bthi,bhij->bthj", d.q.astype(np.float64), d.state0.astype(np.float64))
+    np.testing.assert_allclose(o, expect, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_pure_decay_when_beta0(oracle_mod, kind):
+    """beta = 0: M_T = Diag(prod_t a_t) M0 (scalar product for GDN)."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 1, 9, 2, 6, 4, dtype="f32", seed=2, state0="randn")
+    _, st = O.delta_recurrent(kind, d.q, d.k, d.v, np.zeros_like(d.beta), d.log_gate, d.state0)
+    tot = np.exp(d.log_gate.astype(np.float64).sum(axis=1))  # [B,H] or [B,H,dk]
+    if kind == I.GDN:
+        expect = tot[:, :, None, None] * d.state0
+    else:
+        expect = tot[:, :, :, None] * d.state0
+    np.testing.assert_allclose(st, expect, rtol=1e-12)
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_delta_rule_write(oracle_mod, kind):
+    """After each token, M_t^T k_t = (1-beta) (Diag(a_t) M_{t-1})^T k_t + beta v_t (unit k)."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 1, 6, 2, 8, 5, dtype="f32", seed=3, state0="randn")
+    k = d.k.astype(np.float64)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)  # exactly unit in fp64
+    st = d.state0.astype(np.float64)
+    for t in range(d.T):
+        sl = slice(t, t + 1)
+        lg = d.log_gate[:, sl]
+        _, st_new = O.delta_recurrent(kind, d.q[:, sl], k[:, sl], d.v[:, sl], d.beta[:, sl], lg,
+                                      st)
+        a = np.exp(lg[0, 0].astype(np.float64))  # [H] or [H,dk]
+        for h in range(d.H):
+            ah = a[h] if kind == I.GDN else a[h][:, None]
+            Mp = ah * st[0, h]
+            b = float(d.beta[0, t, h])
+            lhs = st_new[0, h].T @ k[0, t, h]
+            rhs = (1 - b) * (Mp.T @ k[0, t, h]) + b * d.v[0, t, h].astype(np.float64)
+            np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+        st = st_new
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_orthonormal_keys_store_and_retrieve(oracle_mod, kind):
+    """k_t = e_t, beta = 1, g = 1, M0 = 0: M_T = sum_t e_t v_t^T, so q = e_t returns v_t."""
+    O = oracle_mod
+    dk, dv, T = 6, 4, 6
+    rs = np.random.default_rng(4)
+    k = np.eye(dk)[None, :, None, :]
+    v = rs.standard_normal((1, T, 1, dv))
+    q = np.eye(dk)[None, :, None, :]  # token t queries e_t after writing it
+    beta = np.ones((1, T, 1))
+    lg = np.zeros((1, T, 1)) if kind == I.GDN else np.zeros((1, T, 1, dk))
+    o, st = O.delta_recurrent(kind, q, k, v, beta, lg, np.zeros((1, 1, dk, dv)))
+    np.testing.assert_allclose(st[0, 0], v[0, :, 0, :], atol=1e-14)
+    np.testing.assert_allclose(o[0, :, 0, :], v[0, :, 0, :], atol=1e-14)
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_single_token_from_zero(oracle_mod, kind):
+    """One token from a zero state: o = scale * beta (k.q) v, state = beta k v^T."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 2, 1, 3, 8, 5, dtype="f32", seed=5)
+    o, st = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0, scale=0.25)
+    q, k, v, b = (x.astype(np.float64) for x in (d.q, d.k, d.v, d.beta))
+    kq = np.einsum("bthi,bthi->bth", k, q)
+    np.testing.assert_allclose(o, 0.25 * (b * kq)[..., None] * v, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(st, np.einsum("bth,bthi,bthj->bhij", b, k, v), rtol=1e-13)
+
+
+def test_kda_uniform_gate_equals_gdn(oracle_mod):
+    O = oracle_mod
+    d = I.delta_inputs(I.GDN, 2, 20, 3, 8, 6, dtype="f32", seed=6, state0="randn")
+    o_g, s_g = O.delta_recurrent(I.GDN, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    lg_k = np.repeat(d.log_gate[..., None], d.dk, axis=-1)
+    o_k, s_k = O.delta_recurrent(I.KDA, d.q, d.k, d.v, d.beta, lg_k, d.state0)
+    assert O.rel_err(o_k, o_g) < 1e-12 and O.rel_err(s_k, s_g) < 1e-12
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+@pytest.mark.parametrize("T,C", [(37, 1), (37, 2), (37, 16), (200, 64), (64, 64), (37, 37),
+                                 (130, 64)])
+def test_chunked_equals_recurrent(oracle_mod, kind, T, C):
+    O = oracle_mod
+    d = I.delta_inputs(kind, 1, T, 2, 16, 8, dtype="f32", seed=7 + T + C, state0="randn")
+    o_r, s_r = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    o_c, s_c = O.delta_chunked(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0, chunk=C)
+    assert O.rel_err(o_c, o_r) < 1e-12
+    assert O.rel_err(s_c, s_r) < 1e-12
+
+
+def test_oracle_thread_count_invariance(oracle_mod):
+    O = oracle_mod
+    d = I.delta_inputs(I.KDA, 2, 30, 4, 8, 8, dtype="f32", seed=8, state0="randn")
+    a = O.delta_recurrent(I.KDA, d.q, d.k, d.v, d.beta, d.log_gate, d.state0, n_threads=1)
+    b = O.delta_recurrent(I.KDA, d.q, d.k, d.v, d.beta, d.log_gate, d.state0, n_threads=4)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_oracle_rejects_bad_kind(oracle_mod):
+    O = oracle_mod
+    d = I.delta_inputs(I.GDN, 1, 2, 1, 4, 4, dtype="f32", seed=9)
+    with pytest.raises(ValueError):
+        O.delta_recurrent(I.FA, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+
+
+# --------------------------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------------------------
+
+def _logical_kv(a: I.AttnInputs, O):
+    """Logical K/V [B][L][Hkv][d] for an identity page table (reshape, no oracle indexing)."""
+    B, PT = a.B, a.page_tokens
+    P = a.k_pool.shape[0]
+    pps = P // B
+    K = O.bf16_bits_to_f64(a.k_pool).reshape(B, pps, a.Hkv, PT, a.d).transpose(0, 1, 3, 2, 4)
+    V = O.bf16_bits_to_f64(a.v_pool).reshape(B, pps, a.Hkv, PT, a.d).transpose(0, 1, 3, 2, 4)
+    return K.reshape(B, pps * PT, a.Hkv, a.d), V.reshape(B, pps * PT, a.Hkv, a.d)
+
+
+def _brute(a: I.AttnInputs, O, lo_fn):
+    K, V = _logical_kv(a, O)
+    q = O.bf16_bits_to_f64(a.q)
+    nk, nv = O.bf16_bits_to_f64(a.new_k), O.bf16_bits_to_f64(a.new_v)
+    out = np.zeros((a.B, a.Hq, a.d))
+    grp = a.Hq // a.Hkv
+    for b in range(a.B):
+        L = int(a.seq_lens[b])
+        Kb, Vb = K[b, :L].copy(), V[b, :L].copy()
+        Kb[L - 1], Vb[L - 1] = nk[b], nv[b]
+        lo = lo_fn(L)
+        for h in range(a.Hq):
+            s = Kb[lo:L, h // grp] @ q[b, h] / math.sqrt(a.d)
+            p = np.exp(s - s.max())
+            out[b, h] = (p / p.sum()) @ Vb[lo:L, h // grp]
+    return out
+
+
+def test_fa_matches_brute_force_and_torch_sdpa(oracle_mod):
+    O = oracle_mod
+    a = I.attn_inputs(I.FA, 3, 8, 2, 16, 150, page_tokens=16, seed=10, permute=False,
+                      seq_lens=np.array([150, 1, 77]))
+    o = O.attn_decode(I.FA, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                      a.seq_lens)
+    ref = _brute(a, O, lambda L: 0)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+    # torch's fp64 CPU attention on the same logical sequences
+    K, V = _logical_kv(a, O)
+    q = O.bf16_bits_to_f64(a.q)
+    for b in range(a.B):
+        L = int(a.seq_lens[b])
+        Kb, Vb = K[b, :L].copy(), V[b, :L].copy()
+        Kb[L - 1], Vb[L - 1] = O.bf16_bits_to_f64(a.new_k)[b], O.bf16_bits_to_f64(a.new_v)[b]
+        Kt = torch.from_numpy(np.repeat(Kb.transpose(1, 0, 2), a.Hq // a.Hkv, axis=0))
+        Vt = torch.from_numpy(np.repeat(Vb.transpose(1, 0, 2), a.Hq // a.Hkv, axis=0))
+        qt = torch.from_numpy(q[b][:, None, :])
+        st = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt)
+        np.testing.assert_allclose(o[b], st[:, 0, :].numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_fa_page_permutation_invariance(oracle_mod):
+    """Same logical data under a permuted page table gives the same result."""
+    O = oracle_mod
+    a = I.attn_inputs(I.FA, 2, 4, 2, 8, 100, page_tokens=16, seed=11, permute=False)
+    o1 = O.attn_decode(I.FA, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                       a.seq_lens)
+    perm = np.random.default_rng(0).permutation(a.k_pool.shape[0])
+    inv = np.argsort(perm)
+    kp, vp = a.k_pool[perm], a.v_pool[perm]  # physical page x holds old page perm[x]
+    table = inv[a.page_table].astype(np.int32)
+    o2 = O.attn_decode(I.FA, 0, a.q, a.new_k, a.new_v, kp, vp, table, a.seq_lens)
+    np.testing.assert_array_equal(o1, o2)
+
+
+def test_swa_wide_window_equals_fa(oracle_mod):
+    O = oracle_mod
+    a = I.attn_inputs(I.FA, 2, 4, 1, 8, 90, page_tokens=16, seed=12)
+    o_fa = O.attn_decode(I.FA, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                         a.seq_lens)
+    for w in (90, 91, 500):
+        # a ring of R >= ceil(L/PT) pages never wraps, so the FA table is a valid ring table
+        R = -(-w // 16)
+        table = np.full((a.B, R), -1, np.int32)
+        table[:, :a.page_table.shape[1]] = a.page_table
+        o_swa = O.attn_decode(I.SWA, w, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, table,
+                              a.seq_lens)
+        np.testing.assert_array_equal(o_swa, o_fa)
+
+
+def test_swa_matches_brute_force_window(oracle_mod):
+    O = oracle_mod
+    w = 40
+    # contiguous layout long enough to hold every position, so the brute force can index it
+    a = I.attn_inputs(I.FA, 2, 4, 2, 8, 130, page_tokens=16, seed=13, permute=False)
+    ref = _brute(a, O, lambda L: max(0, L - w))
+    # build the SWA ring (R = 3 pages of 16) holding positions of the last window
+    R, PT = 3, 16
+    P = a.B * R
+    kp = np.zeros((P, a.Hkv, PT, a.d), np.uint16)
+    vp = np.zeros_like(kp)
+    table = np.arange(P, dtype=np.int32).reshape(a.B, R)[:, ::-1].copy()
+    for b in range(a.B):
+        L = int(a.seq_lens[b])
+        for j in range(max(0, L - R * PT), L - 1):
+            src_pg, src_off = b * (a.k_pool.shape[0] // a.B) + j // PT, j % PT
+            r = j % (R * PT)
+            kp[table[b, r // PT], :, r % PT] = a.k_pool[src_pg, :, src_off]
+            vp[table[b, r // PT], :, r % PT] = a.v_pool[src_pg, :, src_off]
+    o = O.attn_decode(I.SWA, w, a.q, a.new_k, a.new_v, kp, vp, table, a.seq_lens)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_degenerate_attention(oracle_mod):
+    O = oracle_mod
+    # L = 1 (FA) and w = 1 (SWA): output is the new token's value
+    a = I.attn_inputs(I.FA, 2, 4, 2, 8, 50, page_tokens=16, seed=14,
+                      seq_lens=np.array([1, 50]))
+    o = O.attn_decode(I.FA, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                      a.seq_lens)
+    nv = O.bf16_bits_to_f64(a.new_v)
+    np.testing.assert_allclose(o[0], np.repeat(nv[0], 2, axis=0), rtol=1e-15)
+    s = I.attn_inputs(I.SWA, 2, 4, 2, 8, 50, window=1, page_tokens=16, seed=15)
+    o1 = O.attn_decode(I.SWA, 1, s.q, s.new_k, s.new_v, s.k_pool, s.v_pool, s.page_table,
+                       s.seq_lens)
+    np.testing.assert_allclose(o1, np.repeat(O.bf16_bits_to_f64(s.new_v), 2, axis=1),
+                               rtol=1e-15)
+    # all keys equal: output is the mean of the values
+    e = I.attn_inputs(I.FA, 1, 2, 1, 8, 20, page_tokens=16, seed=16, permute=False)
+    e.k_pool[:] = e.k_pool[0, 0, 0]
+    e.new_k[:] = e.k_pool[0, 0, 0]
+    o2 = O.attn_decode(I.FA, 0, e.q, e.new_k, e.new_v, e.k_pool, e.v_pool, e.page_table,
+                       e.seq_lens)
+    vals = np.concatenate([O.bf16_bits_to_f64(e.v_pool)[0, 0, :16],
+                           O.bf16_bits_to_f64(e.v_pool)[1, 0, :3],
+                           O.bf16_bits_to_f64(e.new_v)[0]], axis=0)
+    np.testing.assert_allclose(o2[0, 0], vals.mean(axis=0), rtol=1e-13, atol=1e-15)
+
+
+def test_attention_hand_example(oracle_mod):
+    """q = (1,1), keys (0,0) and (1,1), values (1,0) and (0,2), d = 2:
+    scores (0, sqrt 2), so o = ((1, 0) + e^sqrt2 (0, 2)) / (1 + e^sqrt2)."""
+    O = oracle_mod
+    one, two = I.bf16_bits(np.array([1.0], np.float32))[0], I.bf16_bits(np.array([2.0], np.float32))[0]
+    kp = np.zeros((1, 1, 4, 2), np.uint16)
+    vp = np.zeros((1, 1, 4, 2), np.uint16)
+    vp[0, 0, 0, 0] = one
+    q = np.array([[[one, one]]], np.uint16)
+    nk = np.array([[[one, one]]], np.uint16)
+    nv = np.array([[[0, two]]], np.uint16)
+    o = O.attn_decode(I.FA, 0, q, nk, nv, kp, vp, np.array([[0]], np.int32),
+                      np.array([2], np.int32))
+    e = math.exp(math.sqrt(2.0))
+    np.testing.assert_allclose(o[0, 0], [1 / (1 + e), 2 * e / (1 + e)], rtol=1e-15)
+
+
+def test_fa_index_map_is_a_bijection(oracle_mod):
+    O = oracle_mod
+    PT, n = 16, 7
+    row = np.random.default_rng(1).permutation(40)[:n].astype(np.int32)
+    seen = set()
+    for pos in range(n * PT):
+        pg, off = O.kv_slot(I.FA, 0, PT, row, pos)
+        assert pg in set(row.tolist()) and 0 <= off < PT
+        seen.add((pg, off))
+    assert len(seen) == n * PT  # every (page, offset) of the sequence used exactly once
+
+
+@pytest.mark.parametrize("w", [1, 15, 16, 17, 40, 48])
+def test_swa_ring_injective_over_every_window(oracle_mod, w):
+    O = oracle_mod
+    PT = 16
+    R = -(-w // PT)
+    row = np.random.default_rng(w).permutation(50)[:R].astype(np.int32)
+    slots = [O.kv_slot(I.SWA, w, PT, row, p) for p in range(300)]
+    for L in range(1, 300):
+        lo = max(0, L - w)
+        win = slots[lo:L]
+        assert len(set(win)) == len(win)  # the window's positions never share a slot
+        if L >= 2:
+            # the new token (position L-1) overwrites a slot whose previous occupant, if any,
+            # is older than the window
+            prev = [p for p in range(L - 1) if slots[p] == slots[L - 1]]
+            assert all(p < lo for p in prev)
