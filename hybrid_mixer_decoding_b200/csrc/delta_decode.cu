@@ -1,0 +1,204 @@
+// Delta-rule decode step (GDN and KDA), one token per sequence.
+//
+// The pages name GDN (scalar gate) and KDA (channel-wise gate) as the two O(n) recurrent mixers
+// of every supernet layer ("Super Apriel: One Checkpoint, Many Speeds", abstract; gist.science
+// technical summary, section 2a). With the state stored as M[d_k][d_v] (M = S^T for GDN, M = S
+// for KDA), one token of either standard definition is
+//     M' = Diag(a) M,   u = beta (v - M'^T k),   M = M' + k u^T,   o = scale * M^T q,
+// a = exp(log_gate) (a scalar broadcast over d_k for GDN). Since M^T q = M'^T q + u (k.q), one
+// read of M gives both column reductions M'^T k and M'^T q, and one write stores the update:
+// the state crosses HBM exactly twice (read + write), which is the algorithmic minimum.
+//
+// Work split: one CTA of 128 threads per (sequence, head, 32-column slice of d_v). A thread
+// owns 4 adjacent columns (one 16-byte vector) of d_k/16 rows; the 8 threads of a row group
+// cover 128 contiguous bytes, so every warp-wide load or store is four full 128-byte lines.
+// Column sums are reduced over rows with warp shuffles (xor 8, 16), then across the 4 warps
+// through shared memory. No tensor cores: the step is ~1 flop per byte, far below any ridge.
+#include "kernels.h"
+#include "ptx.cuh"
+#include "../../include/hmd.h"
+
+namespace hmd {
+namespace {
+
+__device__ unsigned int g_err;
+
+constexpr int kThreads = 128;
+constexpr int kColThreads = 8;                     // float4 columns across a slice
+constexpr int kSliceCols = 4 * kColThreads;        // 32 columns of d_v per CTA
+constexpr int kRowThreads = kThreads / kColThreads;  // 16 row groups
+constexpr int kWarps = kThreads / 32;
+
+template <bool BF16>
+__device__ __forceinline__ float act(const void *p, size_t i) {
+    if constexpr (BF16) {
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    } else {
+        return reinterpret_cast<const float *>(p)[i];
+    }
+}
+
+template <int DK, bool BF16>
+__global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecodeArgs a,
+                                                                int n_slices) {
+    constexpr int RPT = DK / kRowThreads;  // rows per thread
+    const int slice = blockIdx.x % n_slices;
+    const int bh = blockIdx.x / n_slices;
+    const int b = bh / a.H;
+    const int h = bh - b * a.H;
+    const int tid = threadIdx.x;
+    const int ct = tid % kColThreads;
+    const int rt = tid / kColThreads;
+    const int col = slice * kSliceCols + ct * 4;
+    const bool active = col < a.dv;
+
+    const int slot = a.slots ? a.slots[b] : b;
+    if (slot < 0 || slot >= a.n_slots) {
+        if (tid == 0) atomicOr(&g_err, HMD_DEVERR_SLOT);
+        return;
+    }
+    float *M = a.state + ((size_t)slot * a.H + h) * (size_t)DK * a.dv;
+
+    // Issue every state load first: RPT independent 16-byte loads per thread in flight.
+    float4 m[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        if (active) {
+            m[r] = *reinterpret_cast<const float4 *>(M + (size_t)(rt + r * kRowThreads) * a.dv + col);
+        } else {
+            m[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    __shared__ float sk[DK], sq[DK], sa[DK];
+    __shared__ float red[kWarps][kColThreads][9];
+    const size_t tok = (size_t)b * a.H + h;
+    if (a.kind == HMD_GDN) {
+        const float g = expf(a.log_gate[tok]);
+        for (int i = tid; i < DK; i += kThreads) sa[i] = g;
+    } else {
+        for (int i = tid; i < DK; i += kThreads) sa[i] = expf(a.log_gate[tok * DK + i]);
+    }
+    for (int i = tid; i < DK; i += kThreads) {
+        sk[i] = act<BF16>(a.k, tok * DK + i);
+        sq[i] = act<BF16>(a.q, tok * DK + i);
+    }
+    __syncthreads();
+
+    // M' = Diag(a) M in registers, and the partial column sums of M'^T k, M'^T q, k.q.
+    float w[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f}, kq = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rt + r * kRowThreads;
+        const float ai = sa[i], ki = sk[i], qi = sq[i];
+        m[r].x *= ai; m[r].y *= ai; m[r].z *= ai; m[r].w *= ai;
+        w[0] += ki * m[r].x; w[1] += ki * m[r].y; w[2] += ki * m[r].z; w[3] += ki * m[r].w;
+        pq[0] += qi * m[r].x; pq[1] += qi * m[r].y; pq[2] += qi * m[r].z; pq[3] += qi * m[r].w;
+        kq += ki * qi;
+    }
+    // Reduce over the 4 row groups of this warp (lanes differing in bits 3 and 4).
+#pragma unroll
+    for (int off = 8; off < 32; off <<= 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            w[c] += __shfl_xor_sync(0xffffffffu, w[c], off);
+            pq[c] += __shfl_xor_sync(0xffffffffu, pq[c], off);
+        }
+        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    }
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < kColThreads) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            red[warp][lane][c] = w[c];
+            red[warp][lane][4 + c] = pq[c];
+        }
+        red[warp][lane][8] = kq;
+    }
+    __syncthreads();
+    float W[4] = {0.f, 0.f, 0.f, 0.f}, PQ[4] = {0.f, 0.f, 0.f, 0.f}, KQ = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < kWarps; ++wi) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            W[c] += red[wi][ct][c];
+            PQ[c] += red[wi][ct][4 + c];
+        }
+        KQ += red[wi][ct][8];
+    }
+    if (!active) return;
+
+    const float beta = a.beta[tok];
+    float u[4], o[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float vc = act<BF16>(a.v, tok * a.dv + col + c);
+        u[c] = beta * (vc - W[c]);
+        o[c] = a.scale * (PQ[c] + u[c] * KQ);
+    }
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int i = rt + r * kRowThreads;
+        const float ki = sk[i];
+        float4 nm;
+        nm.x = m[r].x + ki * u[0];
+        nm.y = m[r].y + ki * u[1];
+        nm.z = m[r].z + ki * u[2];
+        nm.w = m[r].w + ki * u[3];
+        *reinterpret_cast<float4 *>(M + (size_t)i * a.dv + col) = nm;
+    }
+    if (rt == 0) {
+        if constexpr (BF16) {
+            uint2 pk;
+            pk.x = pack_bf16x2(o[0], o[1]);
+            pk.y = pack_bf16x2(o[2], o[3]);
+            *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(a.o) + tok * a.dv + col) = pk;
+        } else {
+            *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.o) + tok * a.dv + col) =
+                make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+template <int DK>
+cudaError_t launch_dk(const DeltaDecodeArgs &a, cudaStream_t s) {
+    const int n_slices = (a.dv + kSliceCols - 1) / kSliceCols;
+    const long long grid = (long long)a.B * a.H * n_slices;
+    if (grid <= 0) return cudaSuccess;
+    if (a.bf16) {
+        delta_decode_kernel<DK, true><<<(unsigned)grid, kThreads, 0, s>>>(a, n_slices);
+    } else {
+        delta_decode_kernel<DK, false><<<(unsigned)grid, kThreads, 0, s>>>(a, n_slices);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool delta_decode_supported(int dk, int dv) {
+    const bool dk_ok = dk == 16 || dk == 32 || dk == 64 || dk == 128 || dk == 256;
+    return dk_ok && dv >= 4 && dv <= 1024 && dv % 4 == 0;
+}
+
+cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s) {
+    switch (a.dk) {
+        case 16: return launch_dk<16>(a, s);
+        case 32: return launch_dk<32>(a, s);
+        case 64: return launch_dk<64>(a, s);
+        case 128: return launch_dk<128>(a, s);
+        case 256: return launch_dk<256>(a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+uint32_t delta_decode_read_errors(bool clear) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err, sizeof v) != cudaSuccess) return 0;
+    if (clear && v) {
+        const unsigned int z = 0;
+        cudaMemcpyToSymbol(g_err, &z, sizeof z);
+    }
+    return v;
+}
+
+}  // namespace hmd

@@ -1,0 +1,337 @@
+// C ABI of libhmd.so: argument validation, the recurrent-state and paged-KV caches, and the
+// per-layer placement dispatcher. Every check here runs on the host before anything is
+// launched, so a rejected call leaves device memory untouched.
+//
+// A placement picks one of four mixers per layer and can change between requests without
+// reloading weights ("Super Apriel: One Checkpoint, Many Speeds", abstract; gist.science
+// technical summary, section 2d). Here every layer's caches stay registered in the handles for
+// their whole life, so a switch is a different placement array: nothing is copied.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "kernels.h"
+#include "../../include/hmd.h"
+
+struct hmd_state_cache {
+    int n_layers, slots, H, dk, dv;
+    float *base;
+    size_t layer_elems;
+};
+
+struct hmd_kv_cache {
+    int n_layers, n_pools, n_pages, Hkv, d, page_tokens;
+    std::vector<int32_t> layer_pool;
+    std::vector<void *> k_pools, v_pools;
+};
+
+namespace {
+
+thread_local hmd_status_t t_last = HMD_OK;
+
+hmd_status_t fail(hmd_status_t s) {
+    t_last = s;
+    return s;
+}
+
+hmd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? HMD_OK : fail(HMD_ERR_CUDA); }
+
+cudaStream_t as_stream(hmd_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hmd_status_t check_delta_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
+                                const void *q, const void *k, const void *v, const float *beta,
+                                const float *log_gate, const float *state, int n_slots,
+                                const void *o) {
+    if (kind != HMD_GDN && kind != HMD_KDA) return HMD_ERR_ARG;
+    if (dtype != HMD_F32 && dtype != HMD_BF16) return HMD_ERR_DTYPE;
+    if (B < 0 || H < 1 || dk < 1 || dv < 1 || n_slots < 0) return HMD_ERR_SHAPE;
+    if (B == 0) return HMD_OK;
+    if (!q || !k || !v || !beta || !log_gate || !state || !o) return HMD_ERR_ARG;
+    if (!hmd::delta_decode_supported(dk, dv)) return HMD_ERR_UNSUPPORTED;
+    if (!aligned16(state) || !aligned16(o) || !aligned16(v)) return HMD_ERR_ARG;
+    return HMD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hmd_version(void) { return "hmd 0.1 (sm_100a)"; }
+
+const char *hmd_status_string(hmd_status_t s) {
+    switch (s) {
+        case HMD_OK: return "ok";
+        case HMD_ERR_ARG: return "invalid argument";
+        case HMD_ERR_SHAPE: return "inconsistent shape";
+        case HMD_ERR_DTYPE: return "unsupported dtype";
+        case HMD_ERR_OOM: return "out of device memory";
+        case HMD_ERR_CUDA: return "CUDA error";
+        case HMD_ERR_UNSUPPORTED: return "unsupported configuration";
+        case HMD_ERR_DEVICE_CHECK: return "device-side check fired";
+    }
+    return "unknown status";
+}
+
+hmd_status_t hmd_last_error(void) {
+    const hmd_status_t s = t_last;
+    t_last = HMD_OK;
+    return s;
+}
+
+hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
+    if (!bits) return fail(HMD_ERR_ARG);
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
+    *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
+            hmd::delta_prefill_read_errors(clear != 0);
+    return HMD_OK;
+}
+
+// ---- delta-rule mixers -------------------------------------------------------------------
+
+hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
+                               const void *q, const void *k, const void *v, const float *beta,
+                               const float *log_gate, float *state, int n_slots,
+                               const int32_t *slots, void *o, float scale, hmd_stream_t stream) {
+    const hmd_status_t st = check_delta_decode(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate,
+                                               state, n_slots, o);
+    if (st != HMD_OK) return fail(st);
+    if (B == 0) return HMD_OK;
+    if (!slots && n_slots < B) return fail(HMD_ERR_SHAPE);
+    hmd::DeltaDecodeArgs a{};
+    a.kind = kind; a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
+    a.n_slots = n_slots; a.slots = slots; a.o = o; a.scale = scale;
+    return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
+}
+
+hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                        hmd_dtype_t dtype, const void *q, const void *k,
+                                        const void *v, const float *beta, const float *log_gate,
+                                        float *state, int n_slots, const int32_t *slots, void *o,
+                                        int chunk, float scale, hmd_stream_t stream) {
+    if (kind != HMD_GDN && kind != HMD_KDA) return fail(HMD_ERR_ARG);
+    if (dtype != HMD_F32 && dtype != HMD_BF16) return fail(HMD_ERR_DTYPE);
+    if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || n_slots < 0 || chunk < 1)
+        return fail(HMD_ERR_SHAPE);
+    if (B == 0 || T == 0) return HMD_OK;
+    if (!q || !k || !v || !beta || !log_gate || !state || !o) return fail(HMD_ERR_ARG);
+    if (!slots && n_slots < B) return fail(HMD_ERR_SHAPE);
+    if (!hmd::delta_prefill_supported(dk, dv, dtype == HMD_BF16, chunk))
+        return fail(HMD_ERR_UNSUPPORTED);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return fail(HMD_ERR_ARG);
+    hmd::DeltaPrefillArgs a{};
+    a.kind = kind; a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
+    a.n_slots = n_slots; a.slots = slots; a.o = o; a.chunk = chunk; a.scale = scale;
+    return from_cuda(hmd::launch_delta_prefill(a, as_stream(stream)));
+}
+
+// ---- attention mixers --------------------------------------------------------------------
+
+size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                                  int page_tokens, int max_seq_len) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || max_seq_len < 1) return 16;
+    const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, B, Hq, Hkv, d,
+                                                   page_tokens, max_seq_len);
+    return pl.ws_bytes < 16 ? 16 : pl.ws_bytes;
+}
+
+hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                         int page_tokens, const void *q, const void *new_k, const void *new_v,
+                         void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
+                         int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
+                         void *workspace, size_t ws_bytes, hmd_stream_t stream) {
+    if (kind != HMD_FA && kind != HMD_SWA) return fail(HMD_ERR_ARG);
+    if (kind == HMD_SWA && window < 1) return fail(HMD_ERR_ARG);
+    if (B < 0 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
+        max_pages < 1 || max_seq_len < 1)
+        return fail(HMD_ERR_SHAPE);
+    if (Hq % Hkv) return fail(HMD_ERR_SHAPE);
+    if (B == 0) return HMD_OK;
+    if (!q || !new_k || !new_v || !k_pool || !v_pool || !page_table || !seq_lens || !o ||
+        !workspace)
+        return fail(HMD_ERR_ARG);
+    if (!hmd::attn_decode_supported(d, page_tokens, Hq / Hkv)) return fail(HMD_ERR_UNSUPPORTED);
+    // the table must be wide enough for the longest sequence (FA) or for the ring (SWA)
+    const long long need = kind == HMD_SWA
+        ? (window + page_tokens - 1) / page_tokens < (max_seq_len + page_tokens - 1) / page_tokens
+              ? (window + page_tokens - 1) / page_tokens
+              : (max_seq_len + page_tokens - 1) / page_tokens
+        : (max_seq_len + page_tokens - 1) / page_tokens;
+    if (max_pages < need) return fail(HMD_ERR_SHAPE);
+    if ((long long)n_pages * Hkv * page_tokens >= (1LL << 31)) return fail(HMD_ERR_UNSUPPORTED);
+    if (!aligned16(q) || !aligned16(new_k) || !aligned16(new_v) || !aligned16(k_pool) ||
+        !aligned16(v_pool) || !aligned16(workspace))
+        return fail(HMD_ERR_ARG);
+    const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, B, Hq, Hkv, d,
+                                                   page_tokens, max_seq_len);
+    if (ws_bytes < pl.ws_bytes) return fail(HMD_ERR_SHAPE);
+    hmd::AttnDecodeArgs a{};
+    a.swa = kind == HMD_SWA; a.window = window; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.page_tokens = page_tokens; a.q = q; a.new_k = new_k; a.new_v = new_v;
+    a.k_pool = k_pool; a.v_pool = v_pool; a.n_pages = n_pages; a.page_table = page_table;
+    a.max_pages = max_pages; a.seq_lens = seq_lens; a.max_seq_len = max_seq_len; a.o = o;
+    a.workspace = workspace; a.ws_bytes = ws_bytes;
+    return from_cuda(hmd::launch_attn_decode(a, as_stream(stream)));
+}
+
+// ---- caches ------------------------------------------------------------------------------
+
+hmd_status_t state_cache_alloc(int n_layers, int slots, int H, int dk, int dv,
+                               hmd_stream_t stream, hmd_state_cache_t **out) {
+    if (!out) return fail(HMD_ERR_ARG);
+    *out = nullptr;
+    if (n_layers < 1 || slots < 1 || H < 1 || dk < 1 || dv < 1) return fail(HMD_ERR_SHAPE);
+    auto *c = new (std::nothrow) hmd_state_cache{n_layers, slots, H, dk, dv, nullptr, 0};
+    if (!c) return fail(HMD_ERR_OOM);
+    c->layer_elems = (size_t)slots * H * dk * dv;
+    const size_t bytes = c->layer_elems * n_layers * sizeof(float);
+    cudaStream_t s = as_stream(stream);
+    if (cudaMallocAsync(reinterpret_cast<void **>(&c->base), bytes, s) != cudaSuccess) {
+        cudaGetLastError();
+        delete c;
+        return fail(HMD_ERR_OOM);
+    }
+    if (cudaMemsetAsync(c->base, 0, bytes, s) != cudaSuccess) {
+        cudaFreeAsync(c->base, s);
+        delete c;
+        return fail(HMD_ERR_CUDA);
+    }
+    *out = c;
+    return HMD_OK;
+}
+
+hmd_status_t state_cache_free(hmd_state_cache_t *c, hmd_stream_t stream) {
+    if (!c) return fail(HMD_ERR_ARG);
+    const cudaError_t e = cudaFreeAsync(c->base, as_stream(stream));
+    delete c;
+    return from_cuda(e);
+}
+
+hmd_status_t state_cache_layer(hmd_state_cache_t *c, int layer, float **out) {
+    if (!c || !out) return fail(HMD_ERR_ARG);
+    if (layer < 0 || layer >= c->n_layers) return fail(HMD_ERR_ARG);
+    *out = c->base + c->layer_elems * layer;
+    return HMD_OK;
+}
+
+hmd_status_t state_cache_reset(hmd_state_cache_t *c, int layer, const int32_t *slot_ids, int n,
+                               const float *init, hmd_stream_t stream) {
+    if (!c || (n > 0 && !slot_ids)) return fail(HMD_ERR_ARG);
+    if (layer < 0 || layer >= c->n_layers || n < 0) return fail(HMD_ERR_ARG);
+    for (int i = 0; i < n; ++i)
+        if (slot_ids[i] < 0 || slot_ids[i] >= c->slots) return fail(HMD_ERR_ARG);
+    const size_t per = (size_t)c->H * c->dk * c->dv;
+    float *blk = c->base + c->layer_elems * layer;
+    cudaStream_t s = as_stream(stream);
+    for (int i = 0; i < n; ++i) {
+        float *dst = blk + per * slot_ids[i];
+        const cudaError_t e = init ? cudaMemcpyAsync(dst, init + per * i, per * sizeof(float),
+                                                     cudaMemcpyDeviceToDevice, s)
+                                   : cudaMemsetAsync(dst, 0, per * sizeof(float), s);
+        if (e != cudaSuccess) return fail(HMD_ERR_CUDA);
+    }
+    return HMD_OK;
+}
+
+hmd_status_t kv_cache_alloc(int n_layers, const int32_t *layer_pool, int n_pools, int n_pages,
+                            int Hkv, int d, int page_tokens, hmd_stream_t stream,
+                            hmd_kv_cache_t **out) {
+    if (!out || !layer_pool) return fail(HMD_ERR_ARG);
+    *out = nullptr;
+    if (n_layers < 1 || n_pools < 0 || n_pages < 1 || Hkv < 1 || d < 1 || page_tokens < 1)
+        return fail(HMD_ERR_SHAPE);
+    for (int l = 0; l < n_layers; ++l)
+        if (layer_pool[l] < -1 || layer_pool[l] >= n_pools) return fail(HMD_ERR_ARG);
+    auto *c = new (std::nothrow) hmd_kv_cache;
+    if (!c) return fail(HMD_ERR_OOM);
+    c->n_layers = n_layers; c->n_pools = n_pools; c->n_pages = n_pages; c->Hkv = Hkv; c->d = d;
+    c->page_tokens = page_tokens;
+    c->layer_pool.assign(layer_pool, layer_pool + n_layers);
+    const size_t bytes = (size_t)n_pages * Hkv * page_tokens * d * 2;
+    cudaStream_t s = as_stream(stream);
+    for (int i = 0; i < n_pools; ++i) {
+        void *kp = nullptr, *vp = nullptr;
+        if (cudaMallocAsync(&kp, bytes, s) != cudaSuccess ||
+            cudaMallocAsync(&vp, bytes, s) != cudaSuccess) {
+            cudaGetLastError();
+            if (kp) cudaFreeAsync(kp, s);
+            for (size_t j = 0; j < c->k_pools.size(); ++j) {
+                cudaFreeAsync(c->k_pools[j], s);
+                cudaFreeAsync(c->v_pools[j], s);
+            }
+            delete c;
+            return fail(HMD_ERR_OOM);
+        }
+        cudaMemsetAsync(kp, 0, bytes, s);
+        cudaMemsetAsync(vp, 0, bytes, s);
+        c->k_pools.push_back(kp);
+        c->v_pools.push_back(vp);
+    }
+    *out = c;
+    return HMD_OK;
+}
+
+hmd_status_t kv_cache_free(hmd_kv_cache_t *c, hmd_stream_t stream) {
+    if (!c) return fail(HMD_ERR_ARG);
+    cudaError_t e = cudaSuccess;
+    for (size_t j = 0; j < c->k_pools.size(); ++j) {
+        if (cudaFreeAsync(c->k_pools[j], as_stream(stream)) != cudaSuccess) e = cudaErrorUnknown;
+        if (cudaFreeAsync(c->v_pools[j], as_stream(stream)) != cudaSuccess) e = cudaErrorUnknown;
+    }
+    delete c;
+    return from_cuda(e);
+}
+
+hmd_status_t kv_cache_layer(hmd_kv_cache_t *c, int layer, void **k_pool, void **v_pool) {
+    if (!c || !k_pool || !v_pool) return fail(HMD_ERR_ARG);
+    if (layer < 0 || layer >= c->n_layers) return fail(HMD_ERR_ARG);
+    const int p = c->layer_pool[layer];
+    if (p < 0) return fail(HMD_ERR_ARG);
+    *k_pool = c->k_pools[p];
+    *v_pool = c->v_pools[p];
+    return HMD_OK;
+}
+
+// ---- the placement dispatcher -------------------------------------------------------------
+
+hmd_status_t mixer_decode_step(const int8_t *placement, int n_layers, int layer,
+                               const hmd_decode_io_t *io, hmd_state_cache_t *sc,
+                               hmd_kv_cache_t *kc, void *workspace, size_t ws_bytes,
+                               hmd_stream_t stream) {
+    if (!placement || !io || n_layers < 1 || layer < 0 || layer >= n_layers)
+        return fail(HMD_ERR_ARG);
+    const int kind = placement[layer];
+    switch (kind) {
+        case HMD_GDN:
+        case HMD_KDA: {
+            if (!sc || layer >= sc->n_layers) return fail(HMD_ERR_ARG);
+            if (io->H != sc->H || io->d != sc->dk || io->d != sc->dv) return fail(HMD_ERR_SHAPE);
+            if (!io->slots && io->B > sc->slots) return fail(HMD_ERR_SHAPE);
+            float *state = sc->base + sc->layer_elems * layer;
+            const float *lg = kind == HMD_GDN ? io->log_gate_scalar : io->log_gate_channel;
+            return delta_rule_decode(static_cast<hmd_kind_t>(kind), io->B, io->H, io->d, io->d,
+                                     io->dtype, io->q, io->k, io->v, io->beta, lg, state,
+                                     sc->slots, io->slots, io->o, io->scale, stream);
+        }
+        case HMD_FA:
+        case HMD_SWA: {
+            if (!kc || layer >= kc->n_layers || kc->layer_pool[layer] < 0) return fail(HMD_ERR_ARG);
+            if (io->dtype != HMD_BF16) return fail(HMD_ERR_DTYPE);
+            if (io->Hkv != kc->Hkv || io->d != kc->d) return fail(HMD_ERR_SHAPE);
+            const int p = kc->layer_pool[layer];
+            return attn_decode(static_cast<hmd_kind_t>(kind), io->window, io->B, io->H, io->Hkv,
+                               io->d, kc->page_tokens, io->q, io->k, io->v, kc->k_pools[p],
+                               kc->v_pools[p], kc->n_pages, io->page_table, io->max_pages,
+                               io->seq_lens, io->max_seq_len, io->o, workspace, ws_bytes, stream);
+        }
+        default:
+            return fail(HMD_ERR_ARG);
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Internal launchers shared between the C-ABI layer (hmd_api.cu) and the kernel files.
+// Every launcher validates nothing (the API layer already did) and returns the launch status.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hmd {
+
+struct DeltaDecodeArgs {
+    int kind;  // 2 = KDA (per-channel gate), 3 = GDN (scalar gate)
+    int B, H, dk, dv;
+    bool bf16;  // activations bf16 (else fp32)
+    const void *q, *k, *v;
+    const float *beta, *log_gate;
+    float *state;
+    int n_slots;
+    const int32_t *slots;
+    void *o;
+    float scale;
+};
+cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s);
+bool delta_decode_supported(int dk, int dv);
+uint32_t delta_decode_read_errors(bool clear);
+
+struct AttnDecodeArgs {
+    bool swa;
+    int window;
+    int B, Hq, Hkv, d, page_tokens;
+    const void *q, *new_k, *new_v;
+    void *k_pool, *v_pool;
+    int n_pages;
+    const int32_t *page_table;
+    int max_pages;
+    const int32_t *seq_lens;
+    int max_seq_len;
+    void *o;
+    void *workspace;
+    size_t ws_bytes;
+};
+struct AttnPlan {
+    int n_splits;
+    int pages_per_split;
+    size_t ws_bytes;
+};
+AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, int page_tokens,
+                          int max_seq_len);
+cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);
+bool attn_decode_supported(int d, int page_tokens, int group);
+uint32_t attn_decode_read_errors(bool clear);
+
+struct DeltaPrefillArgs {
+    int kind;
+    int B, T, H, dk, dv;
+    bool bf16;
+    const void *q, *k, *v;
+    const float *beta, *log_gate;
+    float *state;
+    int n_slots;
+    const int32_t *slots;
+    void *o;
+    int chunk;
+    float scale;
+};
+cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s);
+bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk);
+uint32_t delta_prefill_read_errors(bool clear);
+
+}  // namespace hmd

@@ -1,0 +1,211 @@
+/*
+ * hmd.h — C ABI of the hybrid-mixer decoding library (libhmd.so, sm_100a).
+ *
+ * The library runs the per-layer token-mixer step of a hybrid "supernet" decoder in which every
+ * layer offers four mixers — full attention (FA), sliding-window attention (SWA), Kimi Delta
+ * Attention (KDA) and Gated DeltaNet (GDN) — and a placement vector picks one mixer per layer
+ * ("Super Apriel: One Checkpoint, Many Speeds", abstract; gist.science technical summary of the
+ * same paper, section 2a "Supernet architecture").
+ *
+ * Conventions for every entry point:
+ *  - Tensors are DEVICE pointers owned by the caller (the library owns only the caches it
+ *    allocates through *_alloc and frees through *_free). They are dense and contiguous in the
+ *    row-major layouts stated, and 16-byte aligned.
+ *  - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Every call is asynchronous on that stream, never synchronises, allocates nothing on the
+ *    decode/prefill paths, and can be captured into a CUDA graph (cache alloc/free excepted).
+ *  - Errors: no exception crosses the ABI. Argument, shape and dtype errors return a status
+ *    before anything is launched and leave every output untouched. A failed launch returns
+ *    HMD_ERR_CUDA. Faults detected inside a kernel (an out-of-range page id or state slot, a
+ *    wait that timed out) skip the offending access and set a bit in a per-device error word,
+ *    read (and cleared) by hmd_device_errors().
+ *  - Precision: activations (q, k, v, o) are bf16 or fp32; gates, beta and recurrent states are
+ *    fp32; attention KV caches are bf16. Outputs take the activation dtype (bf16 stores round to
+ *    nearest even).
+ */
+#ifndef HMD_H
+#define HMD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HMD_API __attribute__((visibility("default")))
+#else
+#define HMD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { HMD_FA = 0, HMD_SWA = 1, HMD_KDA = 2, HMD_GDN = 3 } hmd_kind_t;
+typedef enum { HMD_F32 = 0, HMD_BF16 = 1 } hmd_dtype_t;
+typedef enum {
+    HMD_OK = 0,
+    HMD_ERR_ARG = 1,          /* null pointer, bad enum, negative size, bad layer/window */
+    HMD_ERR_SHAPE = 2,        /* sizes inconsistent with each other or with a cache */
+    HMD_ERR_DTYPE = 3,        /* dtype not accepted by this entry point */
+    HMD_ERR_OOM = 4,          /* cache allocation failed */
+    HMD_ERR_CUDA = 5,         /* a CUDA call or a kernel launch failed */
+    HMD_ERR_UNSUPPORTED = 6,  /* valid but not implemented (e.g. a head size with no kernel) */
+    HMD_ERR_DEVICE_CHECK = 7  /* a kernel-side check fired (see hmd_device_errors) */
+} hmd_status_t;
+
+/* Bits of the per-device error word. */
+#define HMD_DEVERR_TIMEOUT   0x1u  /* a bounded wait on a copy barrier gave up */
+#define HMD_DEVERR_PAGE      0x2u  /* a page-table entry was outside [0, n_pages) */
+#define HMD_DEVERR_SLOT      0x4u  /* a state-slot index was outside [0, n_slots) */
+#define HMD_DEVERR_SEQLEN    0x8u  /* a sequence length was < 1 or above the stated maximum */
+
+typedef void *hmd_stream_t;
+
+/* ------------------------------------------------------------------------------------------ */
+/* Delta-rule mixers (GDN, KDA).                                                              */
+/* The pages name GDN as a recurrence with a scalar gate and KDA as one with channel-wise     */
+/* gating, both O(n) with a constant-size state (gist.science summary, section 2a). The       */
+/* library implements the standard definitions, with the state stored as M[d_k][d_v]:         */
+/*   GDN: S_t = g_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T, o_t = S_t q_t, M = S^T       */
+/*   KDA: S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T, o_t = S_t^T q_t, M = S */
+/* i.e. for both: M' = Diag(a) M, u = b (v - M'^T k), M <- M' + k u^T, o = scale * M^T q,      */
+/* with a = exp(log_gate) broadcast over d_k for GDN.                                          */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One decode token per sequence for one layer.
+ *   q, k      [B][H][dk]   (dtype)        v, o  [B][H][dv] (dtype)
+ *   beta      [B][H]       fp32
+ *   log_gate  [B][H] fp32 (GDN) or [B][H][dk] fp32 (KDA); values <= 0
+ *   state     [n_slots][H][dk][dv] fp32, updated in place; sequence b uses slot slots[b]
+ *             (slots == NULL: slot b). Two sequences must not share a slot.
+ *   scale     multiplies o (1.0 reproduces the definitions).
+ * Supported: dk in {16, 32, 64, 128, 256}; dv a multiple of 4, 4 <= dv <= 1024.
+ * Returns HMD_ERR_ARG for a bad kind / null pointer, HMD_ERR_UNSUPPORTED for other dk/dv.     */
+HMD_API hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
+                               const void *q, const void *k, const void *v, const float *beta,
+                               const float *log_gate, float *state, int n_slots,
+                               const int32_t *slots, void *o, float scale, hmd_stream_t stream);
+
+/* Chunked (WY / UT-transform) prefill over T tokens per sequence for one layer: the same
+ * recurrence as delta_rule_decode applied to tokens 0..T-1 in order, computed chunk by chunk.
+ *   q, k [B][T][H][dk]; v, o [B][T][H][dv] (dtype); beta [B][T][H] fp32;
+ *   log_gate [B][T][H] (GDN) or [B][T][H][dk] (KDA) fp32;
+ *   state [n_slots][H][dk][dv] fp32: read as the initial state and overwritten with the final
+ *   one (slot slots[b], or b when slots == NULL).
+ *   chunk: tokens per chunk; 64 is the supported value. T need not be a multiple of it.
+ * Supported: bf16 with dk = dv = 128 on the tensor-core path; fp32 or other sizes (dk, dv in
+ * {16..128}, multiples of 16) on the CUDA-core path.                                          */
+HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                        hmd_dtype_t dtype, const void *q, const void *k,
+                                        const void *v, const float *beta, const float *log_gate,
+                                        float *state, int n_slots, const int32_t *slots, void *o,
+                                        int chunk, float scale, hmd_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Attention mixers (FA, SWA) over a paged bf16 KV cache.                                     */
+/* FA is standard causal attention, O(n^2) over a KV cache that grows with the context; SWA   */
+/* attends to a local window, O(n*w) (gist.science summary, sections 1 and 2a).               */
+/* One decode step: append the new token's k, v at logical position L-1 (L = seq_lens[b],     */
+/* counting the new token), then o = softmax(q K^T / sqrt(d)) V over keys j in [lo, L-1],     */
+/* lo = 0 (FA) or max(0, L - window) (SWA). Query head h uses kv-head h / (Hq / Hkv).         */
+/* Paged layout: k_pool, v_pool [n_pages][Hkv][page_tokens][d] bf16. FA: position p is at      */
+/* (page_table[b][p / page_tokens], p % page_tokens). SWA keeps a ring of                      */
+/* R = ceil(window / page_tokens) pages: position p is at ring index r = p mod (R*page_tokens),*/
+/* i.e. (page_table[b][r / page_tokens], r % page_tokens).                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Workspace bytes attn_decode needs for these sizes (split-K partials; 0 is never returned).  */
+HMD_API size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                                  int page_tokens, int max_seq_len);
+
+/*   q [B][Hq][d] bf16; new_k, new_v [B][Hkv][d] bf16; o [B][Hq][d] bf16.
+ *   page_table [B][max_pages] int32 (device); seq_lens [B] int32 (device), each in
+ *   [1, max_seq_len]; max_seq_len is a host-side upper bound that sizes the launch.
+ *   workspace: device scratch of at least attn_decode_workspace_size(...) bytes.
+ * Supported: d in {64, 128}; page_tokens == 64; Hq / Hkv <= 16. The pools must hold finite
+ * values (freshly allocated pools from kv_cache_alloc are zero-filled).                       */
+HMD_API hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                         int page_tokens, const void *q, const void *new_k, const void *new_v,
+                         void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
+                         int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
+                         void *workspace, size_t ws_bytes, hmd_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Caches and the placement dispatcher.                                                       */
+/* A placement selects one mixer per layer and can change between requests without reloading */
+/* weights (abstract; gist.science summary, section 2d "Inference and serving"). The library  */
+/* keeps every layer's caches registered for the life of the handles, so switching placements */
+/* is passing a different placement array: nothing is copied or reallocated.                 */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct hmd_state_cache hmd_state_cache_t;
+typedef struct hmd_kv_cache hmd_kv_cache_t;
+
+/* Recurrent-state cache: n_layers blocks of [slots][H][dk][dv] fp32, zero-filled.
+ * Memory comes from cudaMallocAsync on `stream`; the handle is freed by state_cache_free.      */
+HMD_API hmd_status_t state_cache_alloc(int n_layers, int slots, int H, int dk, int dv,
+                               hmd_stream_t stream, hmd_state_cache_t **out);
+HMD_API hmd_status_t state_cache_free(hmd_state_cache_t *cache, hmd_stream_t stream);
+/* Device pointer of layer `layer`'s [slots][H][dk][dv] block.                                 */
+HMD_API hmd_status_t state_cache_layer(hmd_state_cache_t *cache, int layer, float **out);
+/* Reset n slots (host array `slot_ids`) of one layer to zero, or to init [n][H][dk][dv] fp32
+ * (device) when init is not NULL.                                                            */
+HMD_API hmd_status_t state_cache_reset(hmd_state_cache_t *cache, int layer, const int32_t *slot_ids,
+                               int n, const float *init, hmd_stream_t stream);
+
+/* Paged KV cache: n_pools pairs of K and V pools [n_pages][Hkv][page_tokens][d] bf16,
+ * zero-filled. layer_pool (host, n_layers entries) maps each layer to a pool, or -1 for none;
+ * several layers may share a pool (aliasing, for placements whose KV exceeds memory).         */
+HMD_API hmd_status_t kv_cache_alloc(int n_layers, const int32_t *layer_pool, int n_pools, int n_pages,
+                            int Hkv, int d, int page_tokens, hmd_stream_t stream,
+                            hmd_kv_cache_t **out);
+HMD_API hmd_status_t kv_cache_free(hmd_kv_cache_t *cache, hmd_stream_t stream);
+HMD_API hmd_status_t kv_cache_layer(hmd_kv_cache_t *cache, int layer, void **k_pool, void **v_pool);
+
+/* Per-layer decode inputs. Delta layers read q, k, v with H heads and dk = dv = d, beta and
+ * log_gate_scalar (GDN, [B][H]) or log_gate_channel (KDA, [B][H][d]), and the state slots.
+ * Attention layers read q with H heads, k, v (the new token) with Hkv heads, page_table,
+ * seq_lens, max_seq_len and window (SWA). o has H heads. A layer's io may fill only the fields
+ * of the mixer kinds it can be switched to.                                                    */
+typedef struct {
+    int B, H, Hkv, d;
+    hmd_dtype_t dtype;         /* activations; attention layers require HMD_BF16 */
+    const void *q, *k, *v;
+    const float *beta;
+    const float *log_gate_scalar;
+    const float *log_gate_channel;
+    const int32_t *slots;      /* state slot per sequence (NULL: b) */
+    const int32_t *page_table; /* [B][max_pages] */
+    int max_pages;
+    const int32_t *seq_lens;   /* [B], counting the new token */
+    int max_seq_len;
+    int window;                /* SWA window (keys, including the current token) */
+    float scale;               /* delta layers: output scale (1.0 = the definition) */
+    void *o;
+} hmd_decode_io_t;
+
+/* One decode token for layer `layer`: runs the mixer placement[layer] (host int8 array of
+ * n_layers kinds) on that layer's registered caches. Attention layers need a workspace of
+ * attn_decode_workspace_size(...) bytes. Returns HMD_ERR_ARG if the chosen mixer's cache is not
+ * registered for the layer (no pool for FA/SWA, no state block for GDN/KDA).                 */
+HMD_API hmd_status_t mixer_decode_step(const int8_t *placement, int n_layers, int layer,
+                               const hmd_decode_io_t *io, hmd_state_cache_t *state_cache,
+                               hmd_kv_cache_t *kv_cache, void *workspace, size_t ws_bytes,
+                               hmd_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Diagnostics.                                                                               */
+/* ------------------------------------------------------------------------------------------ */
+HMD_API const char *hmd_status_string(hmd_status_t status);
+/* The status of the most recent failing call on this host thread (HMD_OK if none), cleared on
+ * read.                                                                                       */
+HMD_API hmd_status_t hmd_last_error(void);
+/* Synchronise `stream`, then read the current device's error word (HMD_DEVERR_* bits) into
+ * *bits and clear it when clear != 0.                                                         */
+HMD_API hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear);
+/* Library version string. */
+HMD_API const char *hmd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HMD_H */

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: libhmd.so loads, exports every entry point include/hmd.h declares,
+and rejects bad arguments on the host (a status, no launch). These calls never reach a kernel:
+validation returns before any CUDA call, so they run on a machine without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hybrid_mixer_decoding_b200 as hmd
+from hybrid_mixer_decoding_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # a 16-byte aligned non-null address that validation never dereferences
+ARG, SHAPE, DTYPE, UNSUP = 1, 2, 3, 6
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "hmd.h")) as f:
+        src = f.read()
+    return re.findall(r"^HMD_API\s+[\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M)
+
+
+def test_library_exports_every_declared_symbol():
+    L = hmd.lib()
+    names = _declared()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib._SIGS), "binding and header disagree"
+
+
+def test_status_strings_and_version():
+    assert hmd.hmd_version().startswith("hmd")
+    for s in range(8):
+        assert hmd.hmd_status_string(s)
+    assert hmd.hmd_status_string(99) == "unknown status"
+
+
+def _decode(kind=hmd.GDN, B=2, H=2, dk=64, dv=64, dtype=hmd.BF16, ptr=FAKE, n_slots=4):
+    return hmd.lib().delta_rule_decode(kind, B, H, dk, dv, dtype, ptr, ptr, ptr, ptr, ptr, ptr,
+                                       n_slots, None, ptr, 1.0, None)
+
+
+def test_delta_decode_validation():
+    assert _decode(kind=hmd.FA) == ARG
+    assert _decode(dtype=7) == DTYPE
+    assert _decode(B=-1) == SHAPE
+    assert _decode(ptr=None) == ARG
+    assert _decode(dk=96) == UNSUP
+    assert _decode(dv=6) == UNSUP
+    assert _decode(n_slots=1) == SHAPE          # B=2 sequences, no slot map, 1 slot
+    assert _decode(B=0) == 0                    # empty batch: nothing to do
+    assert hmd.hmd_last_error() == SHAPE        # the last failing status, cleared on read
+    assert hmd.hmd_last_error() == 0
+
+
+def _prefill(kind=hmd.KDA, B=1, T=64, H=1, dk=128, dv=128, dtype=hmd.BF16, chunk=64, ptr=FAKE):
+    return hmd.lib().delta_rule_prefill_chunked(kind, B, T, H, dk, dv, dtype, ptr, ptr, ptr, ptr,
+                                                ptr, ptr, 4, None, ptr, chunk, 1.0, None)
+
+
+def test_prefill_validation():
+    assert _prefill(kind=hmd.SWA) == ARG
+    assert _prefill(chunk=0) == SHAPE
+    assert _prefill(chunk=32) == UNSUP
+    assert _prefill(dk=200) == UNSUP
+    assert _prefill(ptr=None) == ARG
+    assert _prefill(T=0) == 0
+
+
+def _attn(kind=hmd.FA, window=0, B=2, Hq=8, Hkv=2, d=128, PT=64, max_pages=4, max_len=256,
+          ws=1 << 30, ptr=FAKE, n_pages=16):
+    return hmd.lib().attn_decode(kind, window, B, Hq, Hkv, d, PT, ptr, ptr, ptr, ptr, ptr, n_pages,
+                                 ptr, max_pages, ptr, max_len, ptr, ptr, ws, None)
+
+
+def test_attn_validation():
+    assert _attn(kind=hmd.KDA) == ARG
+    assert _attn(kind=hmd.SWA, window=0) == ARG
+    assert _attn(Hq=6, Hkv=4) == SHAPE           # Hq not a multiple of Hkv
+    assert _attn(d=96) == UNSUP
+    assert _attn(PT=32) == UNSUP
+    assert _attn(Hq=64, Hkv=2) == UNSUP          # GQA group of 32 > 16
+    assert _attn(max_pages=3) == SHAPE           # table too narrow for 256 tokens
+    assert _attn(ws=16) == SHAPE                 # workspace too small
+    assert _attn(ptr=None) == ARG
+
+
+def test_workspace_size_monotone():
+    f = hmd.attn_decode_workspace_size
+    a = f(hmd.FA, 0, 32, 32, 8, 128, 64, 8192)
+    b = f(hmd.FA, 0, 32, 32, 8, 128, 64, 16384)
+    assert a > 0 and b >= a
+    assert f(hmd.SWA, 4096, 32, 32, 8, 128, 64, 1 << 20) <= f(hmd.FA, 0, 32, 32, 8, 128, 64,
+                                                              1 << 20)
+
+
+def test_dispatcher_validation():
+    io = hmd.DecodeIO(B=1, H=4, Hkv=1, d=128, dtype=hmd.BF16)
+    pl = (ctypes.c_int8 * 3)(0, 9, 3)
+    L = hmd.lib()
+    assert L.mixer_decode_step(pl, 3, 1, ctypes.byref(io), None, None, None, 0, None) == ARG
+    assert L.mixer_decode_step(pl, 3, 3, ctypes.byref(io), None, None, None, 0, None) == ARG
+    # FA layer with no KV cache registered, GDN layer with no state cache registered
+    assert L.mixer_decode_step(pl, 3, 0, ctypes.byref(io), None, None, None, 0, None) == ARG
+    assert L.mixer_decode_step(pl, 3, 2, ctypes.byref(io), None, None, None, 0, None) == ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.lib()
