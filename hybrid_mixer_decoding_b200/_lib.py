@@ -39,6 +39,8 @@ _SIGS = {
     "attn_decode_workspace_size": (_sz, [_c_int] * 8),
     "attn_decode": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
                                                       _vp, _sz, _vp]),
+    "attn_decode_static_ws": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp,
+                                                                _c_int, _vp, _vp]),
     "state_cache_alloc": (_c_int, [_c_int] * 5 + [_vp, ctypes.POINTER(_vp)]),
     "state_cache_free": (_c_int, [_vp, _vp]),
     "state_cache_layer": (_c_int, [_vp, _c_int, ctypes.POINTER(_vp)]),
@@ -155,6 +157,20 @@ def attn_decode(kind, window, q, new_k, new_v, k_pool, v_pool, page_table, seq_l
                            _p(seq_lens), int(max_seq_len), _p(o), _p(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check("attn_decode", st)
+
+
+def attn_decode_static_ws(kind, window, q, new_k, new_v, k_pool, v_pool, page_table, seq_lens,
+                          max_seq_len, o, stream=None) -> None:
+    """attn_decode with its workspace taken from the library's fixed device array instead of a
+    caller buffer (for callers that cannot allocate device memory; see include/hmd.h)."""
+    _contig(q, new_k, new_v, k_pool, v_pool, page_table, seq_lens, o)
+    B, Hq, d = q.shape
+    n_pages, Hkv, PT, _ = k_pool.shape
+    st = lib().attn_decode_static_ws(kind, int(window), B, Hq, Hkv, d, PT, _p(q), _p(new_k),
+                                     _p(new_v), _p(k_pool), _p(v_pool), n_pages, _p(page_table),
+                                     page_table.shape[1], _p(seq_lens), int(max_seq_len), _p(o),
+                                     _stream(stream))
+    _check("attn_decode_static_ws", st)
 
 
 class StateCache:

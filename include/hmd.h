@@ -129,6 +129,26 @@ HMD_API hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int
                          int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
                          void *workspace, size_t ws_bytes, hmd_stream_t stream);
 
+/* attn_decode without a caller-provided workspace. The paper has no counterpart to this entry
+ * point: it exists for callers that cannot allocate device memory, such as a plugin whose host
+ * application owns all device memory through its own allocator, or a serving loop that forbids
+ * device allocation after start-up. Arguments, layouts and results are those of attn_decode.
+ * The split-K partials go to a fixed 16 MiB array compiled into the library (one per GPU that
+ * loads it, held until the process exits); the call allocates nothing.
+ *  - Returns HMD_ERR_UNSUPPORTED, before launching anything, when
+ *    attn_decode_workspace_size(...) for these sizes exceeds 16 MiB (16777216 bytes).
+ *  - The first call on each device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture.
+ *  - All calls share the one array and leave it holding the last call's partials; nothing needs
+ *    clearing, since each call writes every partial it reads. Calls that overlap on the GPU
+ *    (different streams, or unordered host threads) race on it and must not be issued.       */
+HMD_API hmd_status_t attn_decode_static_ws(hmd_kind_t kind, int window, int B, int Hq, int Hkv,
+                                           int d, int page_tokens, const void *q,
+                                           const void *new_k, const void *new_v, void *k_pool,
+                                           void *v_pool, int n_pages, const int32_t *page_table,
+                                           int max_pages, const int32_t *seq_lens,
+                                           int max_seq_len, void *o, hmd_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* Caches and the placement dispatcher.                                                       */
 /* A placement selects one mixer per layer and can change between requests without reloading */

@@ -1,0 +1,71 @@
+"""attn_decode_static_ws: the allocation-free variant of attn_decode.
+
+Some callers cannot allocate device memory (a plugin whose host application owns all device
+memory, a serving loop that forbids allocation after start-up), so they cannot provide the
+split-K workspace attn_decode needs. attn_decode_static_ws takes its workspace from a fixed
+16 MiB array inside the library instead. These tests call it through the C ABI twice in a row
+(the second call runs on whatever the first left in the shared array) and check each result
+against attn_decode with a caller workspace, at the tolerance used for bf16 outputs (2e-2
+normwise). This file is named to be collected last.
+"""
+import numpy as np
+import pytest
+import torch
+
+import hybrid_mixer_decoding_b200 as hmd
+from hybrid_mixer_decoding_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+def _bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _i32(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).cuda()
+
+
+def _both(a: I.AttnInputs):
+    """(output with a caller workspace, output from the static workspace), on separate pool
+    copies so the two appends do not interact."""
+    q, nk, nv = _bits(a.q), _bits(a.new_k), _bits(a.new_v)
+    table, lens = _i32(a.page_table), _i32(a.seq_lens)
+    msl = int(a.seq_lens.max())
+    kp1, vp1 = _bits(a.k_pool), _bits(a.v_pool)
+    kp2, vp2 = kp1.clone(), vp1.clone()
+    ws = torch.empty(hmd.attn_decode_workspace_size(a.kind, a.window, a.B, a.Hq, a.Hkv, a.d, 64,
+                                                    msl), dtype=torch.uint8, device="cuda")
+    o_ref = torch.empty(a.B, a.Hq, a.d, device="cuda", dtype=torch.bfloat16)
+    o_st = torch.full_like(o_ref, float("nan"))
+    hmd.attn_decode(a.kind, a.window, q, nk, nv, kp1, vp1, table, lens, msl, o_ref, ws)
+    hmd.attn_decode_static_ws(a.kind, a.window, q, nk, nv, kp2, vp2, table, lens, msl, o_st)
+    torch.cuda.synchronize()
+    assert torch.equal(kp1, kp2) and torch.equal(vp1, vp2)  # same append
+    return o_ref.float(), o_st.float()
+
+
+def _rel(x, y):
+    return float((x - y).abs().max() / y.abs().max())
+
+
+def test_static_workspace_matches_caller_workspace_twice():
+    first = I.attn_inputs(I.FA, 32, 32, 8, 128, 8192, seed=2)          # config-3 FA shape
+    second = I.attn_inputs(I.SWA, 7, 16, 4, 128, 700, window=300, seed=9,
+                           seq_lens=np.array([1, 64, 65, 299, 300, 301, 700], np.int32))
+    for a in (first, second):
+        o_ref, o_st = _both(a)
+        assert torch.isfinite(o_st).all()
+        assert _rel(o_st, o_ref) <= TOL
+    assert hmd.hmd_device_errors(clear=True) == 0
+
+
+def test_static_workspace_rejects_sizes_beyond_its_array():
+    # B=4096 sequences x 32 heads: the split-K partials need more than 16 MiB
+    need = hmd.attn_decode_workspace_size(I.FA, 0, 4096, 32, 8, 128, 64, 8192)
+    assert need > (16 << 20)
+    fake = 0x10000
+    st = hmd.lib().attn_decode_static_ws(I.FA, 0, 4096, 32, 8, 128, 64, fake, fake, fake, fake,
+                                         fake, 1 << 16, fake, 128, fake, 8192, fake, None)
+    assert st == 6  # HMD_ERR_UNSUPPORTED, returned before anything is launched
