@@ -369,6 +369,178 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------------------------------
+# single-kernel workloads (the per-mixer configurations) and the context sweep
+# ------------------------------------------------------------------------------------------
+def _events_time(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps * 1e-3  # seconds per launch
+
+
+def run_kernel_workload(args):
+    """One mixer kernel at its configuration:
+    attn_fa / attn_swa: B=32, Hq=32, Hkv=8, d=128, context 8192, SWA w=4096, paged bf16 KV
+      (pages of 64, random page permutation), one new token per sequence;
+    decode_kda / decode_gdn: one decode step at the stack's layer shape (B=64, H=32, d=128),
+      rotating over 4 state buffers (512 MiB) so every launch streams from HBM;
+    prefill_kda / prefill_gdn: B=4, H=16, d=128, T=4096, chunk 64, bf16 q/k/v, fp32 state."""
+    import torch
+
+    import hybrid_mixer_decoding_b200 as hmd
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    dev = "cuda"
+    bf = torch.bfloat16
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    w = args.workload
+    extra = {}
+    if w in ("attn_fa", "attn_swa"):
+        kind = I.FA if w == "attn_fa" else I.SWA
+        B, Hq, Hkv, d, L, win = 32, 32, 8, 128, 8192, 4096
+        pps = L // 64 if kind == I.FA else win // 64
+        P = B * pps
+        kp = torch.randn(P, Hkv, 64, d, device=dev, dtype=bf, generator=g)
+        vp = torch.randn(P, Hkv, 64, d, device=dev, dtype=bf, generator=g)
+        table = torch.randperm(P, device=dev, generator=g).to(torch.int32).view(B, pps).contiguous()
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        q = torch.randn(B, Hq, d, device=dev, dtype=bf, generator=g)
+        nk = torch.randn(B, Hkv, d, device=dev, dtype=bf, generator=g)
+        nv = torch.randn(B, Hkv, d, device=dev, dtype=bf, generator=g)
+        o = torch.empty(B, Hq, d, device=dev, dtype=bf)
+        ws = torch.empty(hmd.attn_decode_workspace_size(kind, win, B, Hq, Hkv, d, 64, L),
+                         dtype=torch.uint8, device=dev)
+
+        def fn():
+            hmd.attn_decode(kind, win, q, nk, nv, kp, vp, table, lens, L, o, ws)
+        sec = _events_time(fn, args.steps, args.warmup)
+        keys = L if kind == I.FA else win
+        byts = B * (keys * Hkv * d * 4 + 2 * Hq * d * 2 + 2 * Hkv * d * 2)
+        value, unit = B / sec, "tok/s"
+        desc = (f"{'FA' if kind == I.FA else 'SWA(w=4096)'} decode: B=32, Hq=32, Hkv=8, d=128, "
+                f"ctx 8192, paged bf16 KV (64-token pages, random permutation)")
+        roof = {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
+                "traffic": traffic_for(w), "algorithmic_bytes": byts}
+        launches = 2
+    elif w in ("decode_kda", "decode_gdn"):
+        kind = I.KDA if w == "decode_kda" else I.GDN
+        B, H, d = 64, 32, 128
+        states = [torch.randn(B, H, d, d, device=dev, generator=g) / math.sqrt(d) for _ in range(4)]
+        q = torch.randn(B, H, d, device=dev, dtype=bf, generator=g)
+        k = torch.nn.functional.normalize(torch.randn(B, H, d, device=dev, generator=g), dim=-1).to(bf)
+        v = torch.randn(B, H, d, device=dev, dtype=bf, generator=g)
+        beta = torch.sigmoid(torch.randn(B, H, device=dev, generator=g))
+        lg = (-0.05 * torch.rand(B, H, d, device=dev, generator=g) if kind == I.KDA
+              else -0.1 * torch.rand(B, H, device=dev, generator=g))
+        o = torch.empty(B, H, d, device=dev, dtype=bf)
+        it = [0]
+
+        def fn():
+            hmd.delta_rule_decode(kind, q, k, v, beta, lg, states[it[0] % 4], o)
+            it[0] += 1
+        sec = _events_time(fn, args.steps, args.warmup)
+        byts = B * H * (2 * d * d * 4 + 4 * d * 2 + 4 + (4 * d if kind == I.KDA else 4))
+        value, unit = B / sec, "tok/s"
+        desc = f"{I.KIND_NAMES[kind]} decode step, B=64, H=32, d=128, bf16 act, fp32 state"
+        roof = {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
+                "traffic": traffic_for(w), "algorithmic_bytes": byts}
+        launches = 1
+    elif w in ("prefill_kda", "prefill_gdn"):
+        kind = I.KDA if w == "prefill_kda" else I.GDN
+        B, T, H, d = 4, 4096, 16, 128
+        q = torch.randn(B, T, H, d, device=dev, dtype=bf, generator=g)
+        k = torch.nn.functional.normalize(torch.randn(B, T, H, d, device=dev, generator=g), dim=-1).to(bf)
+        v = torch.randn(B, T, H, d, device=dev, dtype=bf, generator=g)
+        beta = torch.sigmoid(torch.randn(B, T, H, device=dev, generator=g))
+        lg = (-0.05 * torch.rand(B, T, H, d, device=dev, generator=g) if kind == I.KDA
+              else -0.1 * torch.rand(B, T, H, device=dev, generator=g))
+        st = torch.zeros(B, H, d, d, device=dev)
+        o = torch.empty(B, T, H, d, device=dev, dtype=bf)
+
+        def fn():
+            hmd.delta_rule_prefill_chunked(kind, q, k, v, beta, lg, st, o)
+        sec = _events_time(fn, args.steps, args.warmup)
+        per_tok = 768 + 256 + 4 + (512 if kind == I.KDA else 4)
+        byts = B * T * H * per_tok + 2 * B * H * d * d * 4
+        flops = B * T * H * (10 * 64 * d + 6 * d * d)
+        tf = float(pk["bf16_tflops"])
+        value, unit = B * T / sec, "tok/s"
+        desc = f"{I.KIND_NAMES[kind]} chunked prefill: B=4, H=16, d=128, T=4096, chunk 64"
+        roof = {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 5),
+                "traffic": traffic_for(w), "algorithmic_bytes": byts}
+        extra["tensor"] = {"achieved_tflops": round(flops / sec / 1e12, 3), "peak": tf,
+                           "frac": round(flops / sec / 1e12 / tf, 5), "algorithmic_flops": flops}
+        launches = 1
+    else:
+        raise SystemExit(f"unknown workload {w}")
+    assert hmd.hmd_device_errors(clear=True) == 0
+    out = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded)", "config": {"workload": f"{w}: {desc}"},
+           "roofline": roof, "gpu_launches": launches * args.steps}
+    out.update(extra)
+    return out
+
+
+SWEEP_CTX = (4096, 16384, 65536, 131072)
+
+
+def sweep_placements():
+    return {
+        "all-FA": np.full(48, I.FA, np.int8),
+        "24FA+24GDN": I.placement({I.FA: 24, I.GDN: 24}, seed=0),
+        "8FA+20KDA+20GDN": I.placement({I.FA: 8, I.KDA: 20, I.GDN: 20}, seed=0),
+        "all-GDN": np.full(48, I.GDN, np.int8),
+    }
+
+
+def run_sweep(args):
+    """Context sweep: B=16, ctx in {4k, 16k, 64k, 128k}, 48-layer stack, placements all-FA,
+    24 FA + 24 GDN, 8 FA + 40 (20 KDA + 20 GDN), all-GDN; decode tok/s and speedup over all-FA.
+    KV pools are zero-filled (timing only); FA layers share physical pools round-robin when the
+    placement's KV exceeds device memory (each layer still streams its own full context)."""
+    import torch
+
+    from hybrid_mixer_decoding_b200.stack import MixerStack, StackShape, layer_bytes
+    pls = sweep_placements()
+    rows = []
+    for ctx in SWEEP_CTX:
+        shape = StackShape(16, 32, 8, 128, ctx, 4096)
+        st = MixerStack(pls, shape, seed=0, fill_kv=False)
+        res = {}
+        for name in pls:
+            sec = _events_time(lambda: st.step(name), args.steps, args.warmup)
+            byts = sum(layer_bytes(int(k), shape) for k in pls[name])
+            res[name] = {"tok_s": round(16 / sec, 1), "ms_per_step": round(sec * 1e3, 3),
+                         "achieved_gbs": round(byts / sec / 1e9, 1)}
+        fa_bytes = sum(layer_bytes(int(k), shape) for k in pls["all-FA"])
+        for name in pls:
+            res[name]["speedup_vs_all_fa"] = round(res[name]["tok_s"] / res["all-FA"]["tok_s"], 3)
+            res[name]["predicted_by_bytes"] = round(
+                fa_bytes / sum(layer_bytes(int(k), shape) for k in pls[name]), 3)
+        rows.append({"ctx": ctx, "aliased_fa_pools": st.n_fa_pools if st.aliased else None,
+                     "placements": res})
+        st.free()
+        del st
+        torch.cuda.empty_cache()
+    return {"metric": "decode tok/s per placement (BxCtx), context sweep", "workload":
+            "sweep: 48-layer mixer-only stack, B=16, H=32, Hkv=8, d=128, SWA-free placements",
+            "steps": args.steps, "warmup": args.warmup, "rows": rows}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -378,6 +550,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used for profiler runs)")
+    ap.add_argument("--workload", default="stack48",
+                    choices=["stack48", "attn_fa", "attn_swa", "decode_kda", "decode_gdn",
+                             "prefill_kda", "prefill_gdn", "sweep"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
@@ -385,8 +560,12 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         out = run_reference(args, rank, world)
-    else:
+    elif args.workload == "stack48":
         out = run_ours(args, rank, world, local_rank)
+    elif args.workload == "sweep":
+        out = run_sweep(args)
+    else:
+        out = run_kernel_workload(args)
     if rank == 0 and out is not None:
         print(json.dumps(out), flush=True)
 

@@ -48,7 +48,9 @@ def _gen(seed: int) -> torch.Generator:
 
 class MixerStack:
     def __init__(self, placements: dict[str, np.ndarray], shape: StackShape, seed: int = 0,
-                 mem_fraction: float = 0.9, stream: torch.cuda.Stream | None = None):
+                 mem_fraction: float = 0.9, fill_kv: bool = True):
+        """fill_kv=False leaves the KV pools zero-filled (as allocated), for timing runs whose
+        results are not checked: the data does not change the work done."""
         self.placements = {k: np.asarray(v, dtype=np.int8) for k, v in placements.items()}
         self.n_layers = len(next(iter(self.placements.values())))
         assert all(len(p) == self.n_layers for p in self.placements.values())
@@ -90,7 +92,8 @@ class MixerStack:
             for i, l in enumerate(swa_layers):
                 lp[l] = i
             self.kv_swa = L.KVCache(lp, len(swa_layers), self.pages_swa, Hkv, d, PAGE)
-        self._fill_pools(fa_layers, swa_layers, seed)
+        if fill_kv:
+            self._fill_pools(fa_layers, swa_layers, seed)
 
         # page tables (a seeded random permutation of each pool's pages) and lengths
         dev = "cuda"
