@@ -85,7 +85,7 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
     if (!bits) return fail(HMD_ERR_ARG);
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
     *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
-            hmd::delta_prefill_read_errors(clear != 0);
+            hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_mma_read_errors(clear != 0);
     return HMD_OK;
 }
 
@@ -121,7 +121,8 @@ hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, in
     if (!slots && n_slots < B) return fail(HMD_ERR_SHAPE);
     if (!hmd::delta_prefill_supported(dk, dv, dtype == HMD_BF16, chunk))
         return fail(HMD_ERR_UNSUPPORTED);
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+        !aligned16(log_gate))
         return fail(HMD_ERR_ARG);
     hmd::DeltaPrefillArgs a{};
     a.kind = kind; a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;

@@ -93,7 +93,8 @@ HMD_API hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, in
  *   one (slot slots[b], or b when slots == NULL).
  *   chunk: tokens per chunk; 64 is the supported value. T need not be a multiple of it.
  * Supported: bf16 with dk = dv = 128 on the tensor-core path; fp32 or other sizes (dk, dv in
- * {16..128}, multiples of 16) on the CUDA-core path.                                          */
+ * {16..128}, multiples of 16) on the CUDA-core path. q, k, v, o, log_gate and state must be
+ * 16-byte aligned (HMD_ERR_ARG otherwise).                                                     */
 HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
                                         hmd_dtype_t dtype, const void *q, const void *k,
                                         const void *v, const float *beta, const float *log_gate,

@@ -86,3 +86,26 @@ def test_config2_full_size(oracle_mod, kind):
     o_ref, st_ref = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
     assert O.rel_err(o, o_ref) < 2e-2
     assert O.rel_err(st, st_ref) < 2e-2
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_more_heads_than_sms(oracle_mod, kind):
+    """B*H = 200 (sequence, head) pairs: more CTAs than SMs, ragged T, random initial states."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 5, 70, 40, 128, 128, dtype="bf16", seed=33, state0="randn")
+    o, st = run_prefill(d)
+    o_ref, st_ref = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    assert O.rel_err(o, o_ref) < 2e-2
+    assert O.rel_err(st, st_ref) < 2e-2
+
+
+def test_prefill_bad_slot_sets_device_error():
+    hmd.hmd_device_errors(clear=True)
+    d = I.delta_inputs(I.KDA, 2, 64, 1, 128, 128, dtype="bf16", seed=34)
+    bf = torch.bfloat16
+    state = torch.zeros(2, 1, 128, 128, device="cuda")
+    o = torch.zeros(2, 64, 1, 128, device="cuda", dtype=bf)
+    slots = torch.tensor([0, 7], dtype=torch.int32, device="cuda")
+    hmd.delta_rule_prefill_chunked(I.KDA, _dev(d.q, bf), _dev(d.k, bf), _dev(d.v, bf),
+                                   _dev(d.beta), _dev(d.log_gate), state, o, slots=slots)
+    assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_SLOT
