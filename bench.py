@@ -117,6 +117,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------
+# replicas: every rank runs its own copy of the workload; the job's time is the slowest rank's
+# ------------------------------------------------------------------------------------------
+def max_over_ranks(ms: float, dist=None, device="cpu") -> float:
+    """The largest of every rank's device time (ms); the local value without a process group."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms * 1e-3)
+
+
+# ------------------------------------------------------------------------------------------
 # our arm
 # ------------------------------------------------------------------------------------------
 def traffic_for(kernel_key: str):
@@ -180,14 +198,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clocks = clk.stop()
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, "cuda")
     ms_per_step = ms / args.steps
     tokens = shape.B * args.steps * world
-    value = tokens / (ms * 1e-3)
+    value = job_throughput(shape.B * args.steps, world, ms)
 
     # per-mixer achieved bandwidth from the per-layer events
     pk, pk_kind = peaks()
@@ -247,11 +261,7 @@ def run_ours(args, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    ems = e0.elapsed_time(e1)
-    if dist is not None:
-        tt = torch.tensor([ems], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ems = float(tt.item())
+    ems = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     e2e = {"value": round(tokens / (ems * 1e-3), 2), "unit": "tok/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h}
 
