@@ -9,11 +9,15 @@
 // read of M gives both column reductions M'^T k and M'^T q, and one write stores the update:
 // the state crosses HBM exactly twice (read + write), which is the algorithmic minimum.
 //
-// Work split: one CTA of 128 threads per (sequence, head, 32-column slice of d_v). A thread
-// owns 4 adjacent columns (one 16-byte vector) of d_k/16 rows; the 8 threads of a row group
-// cover 128 contiguous bytes, so every warp-wide load or store is four full 128-byte lines.
-// Column sums are reduced over rows with warp shuffles (xor 8, 16), then across the 4 warps
-// through shared memory. No tensor cores: the step is ~1 flop per byte, far below any ridge.
+// Work split: one CTA of 128 threads per (sequence, head, 32-column slice of d_v). The slice
+// ([d_k][32] fp32, 16 KiB at d_k = 128) arrives by one 2-D TMA box into shared memory and leaves
+// by one TMA store after the in-place update, so each CTA holds few registers and many CTAs per
+// SM keep their slices in flight. A thread owns 4 adjacent columns (one 16-byte vector) of
+// d_k/16 rows; column sums are reduced over rows with warp shuffles (xor 8, 16), then across the
+// 4 warps through shared memory. No tensor cores: the step is ~1 flop per byte, far below any
+// ridge.
+#include <cuda.h>
+
 #include "kernels.h"
 #include "ptx.cuh"
 #include "../../include/hmd.h"
@@ -39,9 +43,15 @@ __device__ __forceinline__ float act(const void *p, size_t i) {
 }
 
 template <int DK, bool BF16>
-__global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecodeArgs a,
+__global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                const DeltaDecodeArgs a,
                                                                 int n_slices) {
     constexpr int RPT = DK / kRowThreads;  // rows per thread
+    __shared__ __align__(128) float S[DK][kSliceCols];
+    __shared__ float sk[DK], sq[DK], sa[DK];
+    __shared__ float red[kWarps][kColThreads][9];
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int s_ok;
     const int slice = blockIdx.x % n_slices;
     const int bh = blockIdx.x / n_slices;
     const int b = bh / a.H;
@@ -52,26 +62,20 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecod
     const int col = slice * kSliceCols + ct * 4;
     const bool active = col < a.dv;
 
-    const int slot = a.slots ? a.slots[b] : b;
-    if (slot < 0 || slot >= a.n_slots) {
-        if (tid == 0) atomicOr(&g_err, HMD_DEVERR_SLOT);
-        return;
-    }
-    float *M = a.state + ((size_t)slot * a.H + h) * (size_t)DK * a.dv;
-
-    // Issue every state load first: RPT independent 16-byte loads per thread in flight.
-    float4 m[RPT];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        if (active) {
-            m[r] = *reinterpret_cast<const float4 *>(M + (size_t)(rt + r * kRowThreads) * a.dv + col);
+    if (tid == 0) {
+        const int slot = a.slots ? a.slots[b] : b;
+        const bool ok = slot >= 0 && slot < a.n_slots;
+        s_ok = ok;
+        if (ok) {
+            const uint32_t bb = smem_u32(&bar);
+            mbar_init(bb, 1);
+            fence_barrier_init();
+            mbar_arrive_expect_tx(bb, DK * kSliceCols * 4);
+            tma_load_2d(smem_u32(&S[0][0]), &tm, bb, slice * kSliceCols, (slot * a.H + h) * DK);
         } else {
-            m[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            atomicOr(&g_err, HMD_DEVERR_SLOT);
         }
     }
-
-    __shared__ float sk[DK], sq[DK], sa[DK];
-    __shared__ float red[kWarps][kColThreads][9];
     const size_t tok = (size_t)b * a.H + h;
     if (a.kind == HMD_GDN) {
         const float g = expf(a.log_gate[tok]);
@@ -83,20 +87,31 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecod
         sk[i] = act<BF16>(a.k, tok * DK + i);
         sq[i] = act<BF16>(a.q, tok * DK + i);
     }
+    float vv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (active) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vv[c] = act<BF16>(a.v, tok * a.dv + col + c);
+    }
+    const float beta = a.beta[tok];
     __syncthreads();
+    if (!s_ok) return;
+    if (!mbar_wait_bounded(smem_u32(&bar), 0)) {
+        if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+        return;  // nothing was written; the state slice is left as it was
+    }
 
-    // M' = Diag(a) M in registers, and the partial column sums of M'^T k, M'^T q, k.q.
+    // M' = Diag(a) M and the partial column sums of M'^T k, M'^T q, k.q.
     float w[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f}, kq = 0.f;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = rt + r * kRowThreads;
         const float ai = sa[i], ki = sk[i], qi = sq[i];
-        m[r].x *= ai; m[r].y *= ai; m[r].z *= ai; m[r].w *= ai;
-        w[0] += ki * m[r].x; w[1] += ki * m[r].y; w[2] += ki * m[r].z; w[3] += ki * m[r].w;
-        pq[0] += qi * m[r].x; pq[1] += qi * m[r].y; pq[2] += qi * m[r].z; pq[3] += qi * m[r].w;
+        float4 m = *reinterpret_cast<const float4 *>(&S[i][ct * 4]);
+        m.x *= ai; m.y *= ai; m.z *= ai; m.w *= ai;
+        w[0] += ki * m.x; w[1] += ki * m.y; w[2] += ki * m.z; w[3] += ki * m.w;
+        pq[0] += qi * m.x; pq[1] += qi * m.y; pq[2] += qi * m.z; pq[3] += qi * m.w;
         kq += ki * qi;
     }
-    // Reduce over the 4 row groups of this warp (lanes differing in bits 3 and 4).
 #pragma unroll
     for (int off = 8; off < 32; off <<= 1) {
 #pragma unroll
@@ -126,28 +141,25 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecod
         }
         KQ += red[wi][ct][8];
     }
-    if (!active) return;
-
-    const float beta = a.beta[tok];
     float u[4], o[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        const float vc = act<BF16>(a.v, tok * a.dv + col + c);
-        u[c] = beta * (vc - W[c]);
+        u[c] = beta * (vv[c] - W[c]);
         o[c] = a.scale * (PQ[c] + u[c] * KQ);
     }
+    // M = M' + k u^T, in place
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int i = rt + r * kRowThreads;
-        const float ki = sk[i];
-        float4 nm;
-        nm.x = m[r].x + ki * u[0];
-        nm.y = m[r].y + ki * u[1];
-        nm.z = m[r].z + ki * u[2];
-        nm.w = m[r].w + ki * u[3];
-        *reinterpret_cast<float4 *>(M + (size_t)i * a.dv + col) = nm;
+        const float ai = sa[i], ki = sk[i];
+        float4 m = *reinterpret_cast<const float4 *>(&S[i][ct * 4]);
+        m.x = ai * m.x + ki * u[0];
+        m.y = ai * m.y + ki * u[1];
+        m.z = ai * m.z + ki * u[2];
+        m.w = ai * m.w + ki * u[3];
+        *reinterpret_cast<float4 *>(&S[i][ct * 4]) = m;
     }
-    if (rt == 0) {
+    if (rt == 0 && active) {
         if constexpr (BF16) {
             uint2 pk;
             pk.x = pack_bf16x2(o[0], o[1]);
@@ -158,6 +170,14 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const DeltaDecod
                 make_float4(o[0], o[1], o[2], o[3]);
         }
     }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        const int slot = a.slots ? a.slots[b] : b;
+        tma_store_2d(&tm, smem_u32(&S[0][0]), slice * kSliceCols, (slot * a.H + h) * DK);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+    }
 }
 
 template <int DK>
@@ -165,10 +185,15 @@ cudaError_t launch_dk(const DeltaDecodeArgs &a, cudaStream_t s) {
     const int n_slices = (a.dv + kSliceCols - 1) / kSliceCols;
     const long long grid = (long long)a.B * a.H * n_slices;
     if (grid <= 0) return cudaSuccess;
+    // the state cache as a 2-D tensor [n_slots*H*DK rows][dv] fp32, read in 32-column boxes
+    CUtensorMap tm;
+    if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.state, a.dv,
+                      (long long)a.n_slots * a.H * DK, kSliceCols, DK))
+        return cudaErrorInvalidValue;
     if (a.bf16) {
-        delta_decode_kernel<DK, true><<<(unsigned)grid, kThreads, 0, s>>>(a, n_slices);
+        delta_decode_kernel<DK, true><<<(unsigned)grid, kThreads, 0, s>>>(tm, a, n_slices);
     } else {
-        delta_decode_kernel<DK, false><<<(unsigned)grid, kThreads, 0, s>>>(a, n_slices);
+        delta_decode_kernel<DK, false><<<(unsigned)grid, kThreads, 0, s>>>(tm, a, n_slices);
     }
     return cudaGetLastError();
 }

@@ -1,11 +1,16 @@
 // Internal launchers shared between the C-ABI layer (hmd_api.cu) and the kernel files.
 // Every launcher validates nothing (the API layer already did) and returns the launch status.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace hmd {
+
+// TMA tensor map over a 2-D row-major tensor, boxes of [box_rows][box_cols], no swizzle.
+bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base, long long cols,
+                  long long rows, int box_cols, int box_rows);
 
 struct DeltaDecodeArgs {
     int kind;  // 2 = KDA (per-channel gate), 3 = GDN (scalar gate)

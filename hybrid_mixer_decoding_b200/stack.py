@@ -196,6 +196,22 @@ class MixerStack:
             if ev:
                 ev[1].record()
 
+    def capture(self, name: str, warmup: int = 2) -> "torch.cuda.CUDAGraph":
+        """Capture one step of placement `name` into a CUDA graph (the library's calls allocate
+        nothing and never synchronise, so the whole 48-layer step is one graph launch)."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for _ in range(warmup):
+                self.step(name)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step(name)
+        torch.cuda.synchronize()
+        return g
+
     def launches_per_step(self, name: str) -> int:
         pl = self.placements[name]
         return int(sum(2 if k in (FA, SWA) else 1 for k in pl))

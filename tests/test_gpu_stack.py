@@ -98,3 +98,40 @@ def test_stack48_full_size_sampled(oracle_mod):
     seqs = torch.tensor([0, 31, 63], device="cuda")
     check_step(O, st, "hybrid", seqs)
     st.free()
+
+
+def test_graph_replay_matches_eager_step():
+    """A CUDA graph of the 48-call step (as the sweep replays it) reproduces the eager step
+    bit for bit, starting from the same caches."""
+    shape = StackShape(B=3, H=8, Hkv=2, d=128, ctx=300, window=100)
+    pl = I.placement({I.FA: 2, I.SWA: 2, I.KDA: 2, I.GDN: 2}, seed=1)
+    st = MixerStack({"p": pl}, shape, seed=4)
+    g = st.capture("p")  # capture runs two warm-up steps first
+
+    def snap():
+        states = [st.state.layer_view(l).clone() for l in range(st.n_layers)]
+        pools = [tuple(p.clone() for p in st.pools_for(l)) if pl[l] in (I.FA, I.SWA) else None
+                 for l in range(st.n_layers)]
+        return states, pools
+
+    def restore(s):
+        for l in range(st.n_layers):
+            st.state.layer_view(l).copy_(s[0][l])
+            if s[1][l] is not None:
+                kp, vp = st.pools_for(l)
+                kp.copy_(s[1][l][0])
+                vp.copy_(s[1][l][1])
+
+    s0 = snap()
+    st.step("p")
+    torch.cuda.synchronize()
+    eager = [st.inputs[l]["o"].clone() for l in range(st.n_layers)]
+    eager_state = [st.state.layer_view(l).clone() for l in range(st.n_layers)]
+    restore(s0)
+    g.replay()
+    torch.cuda.synchronize()
+    for l in range(st.n_layers):
+        assert torch.equal(st.inputs[l]["o"], eager[l]), l
+        assert torch.equal(st.state.layer_view(l), eager_state[l]), l
+    del g
+    st.free()
