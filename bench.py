@@ -171,7 +171,7 @@ def run_ours(args, rank, world, local_rank):
     cfg = WORKLOADS["stack48"]
     shape = StackShape(cfg["B"], cfg["H"], cfg["Hkv"], cfg["d"], cfg["ctx"], cfg["window"])
     pl = stack_placement()
-    st = MixerStack({"hybrid": pl}, shape, seed=0)
+    st = MixerStack({"hybrid": pl}, shape, seed=0, io_sets=2)
 
     def barrier():
         if dist is not None:
@@ -226,39 +226,60 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": pk_kind}
     assert hmd.hmd_device_errors(clear=True) == 0
 
-    # end to end through the C ABI from pinned host buffers: per step, copy every layer's
-    # inputs host->device, run the step, copy every layer's output device->host
-    host_in, dev_in, host_out = [], [], []
+    # end to end through the C ABI from pinned host buffers. Every step copies that step's
+    # inputs host->device and reads every layer's output device->host. A copy stream moves the
+    # next step's inputs into the other buffer set while the current step computes, and drains
+    # the current step's outputs once it is done (events order every reuse of a buffer).
+    host_in, dev_in, dev_out = [], [[], []], [[], []]
     for l in range(n_layers):
-        t = st.inputs[l]
-        names = ["q", "k", "v", "beta", "lg_s", "lg_c"] if pl[l] in (I.GDN, I.KDA) else ["q", "nk", "nv"]
-        if pl[l] == I.GDN:
-            names.remove("lg_c")
-        if pl[l] == I.KDA:
-            names.remove("lg_s")
+        names = ["q", "k", "v", "beta", "lg_s" if pl[l] == I.GDN else "lg_c"] \
+            if pl[l] in (I.GDN, I.KDA) else ["q", "nk", "nv"]
         for nm in names:
-            host_in.append(torch.empty_like(t[nm], device="cpu").pin_memory().copy_(t[nm]))
-            dev_in.append(t[nm])
-        host_out.append(torch.empty_like(t["o"], device="cpu").pin_memory())
+            src = st.input_sets[0][l][nm]
+            host_in.append(torch.empty_like(src, device="cpu").pin_memory().copy_(src))
+            for b_ in range(2):
+                dev_in[b_].append(st.input_sets[b_][l][nm])
+        for b_ in range(2):
+            dev_out[b_].append(st.input_sets[b_][l]["o"])
+    host_out = [[torch.empty_like(o, device="cpu").pin_memory() for o in dev_out[b_]]
+                for b_ in range(2)]
     h2d = sum(h.numel() * h.element_size() for h in host_in)
-    d2h = sum(h.numel() * h.element_size() for h in host_out)
+    d2h = sum(h.numel() * h.element_size() for h in host_out[0])
+    comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_done = [torch.cuda.Event(), torch.cuda.Event()]
 
-    def e2e_step():
-        for h, dv in zip(host_in, dev_in):
-            dv.copy_(h, non_blocking=True)
-        st.step("hybrid")
-        for l in range(n_layers):
-            host_out[l].copy_(st.inputs[l]["o"], non_blocking=True)
+    def e2e_run(n_steps, e0=None, e1=None):
+        with torch.cuda.stream(copy):
+            if e0 is not None:
+                e0.record(copy)
+            for h, d in zip(host_in, dev_in[0]):
+                d.copy_(h, non_blocking=True)
+            ev_in[0].record(copy)
+        for k in range(n_steps):
+            b_ = k % 2
+            comp.wait_event(ev_in[b_])
+            st.step("hybrid", io_set=b_)
+            ev_done[b_].record(comp)
+            with torch.cuda.stream(copy):
+                if k + 1 < n_steps:
+                    if k >= 1:
+                        copy.wait_event(ev_done[1 - b_])
+                    for h, d in zip(host_in, dev_in[1 - b_]):
+                        d.copy_(h, non_blocking=True)
+                    ev_in[1 - b_].record(copy)
+                copy.wait_event(ev_done[b_])
+                for d, h in zip(dev_out[b_], host_out[b_]):
+                    h.copy_(d, non_blocking=True)
+        with torch.cuda.stream(copy):
+            if e1 is not None:
+                e1.record(copy)
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    e2e_run(max(2, args.warmup // 2))
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record()
+    e2e_run(args.steps, e0, e1)
     torch.cuda.synchronize()
     barrier()
     ems = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")

@@ -48,9 +48,11 @@ def _gen(seed: int) -> torch.Generator:
 
 class MixerStack:
     def __init__(self, placements: dict[str, np.ndarray], shape: StackShape, seed: int = 0,
-                 mem_fraction: float = 0.9, fill_kv: bool = True):
+                 mem_fraction: float = 0.9, fill_kv: bool = True, io_sets: int = 1):
         """fill_kv=False leaves the KV pools zero-filled (as allocated), for timing runs whose
-        results are not checked: the data does not change the work done."""
+        results are not checked: the data does not change the work done. io_sets > 1 keeps
+        that many independent sets of per-layer input/output buffers (same initial values), so
+        a caller can copy the next step's inputs into one set while a step runs on another."""
         self.placements = {k: np.asarray(v, dtype=np.int8) for k, v in placements.items()}
         self.n_layers = len(next(iter(self.placements.values())))
         assert all(len(p) == self.n_layers for p in self.placements.values())
@@ -131,26 +133,38 @@ class MixerStack:
                 t["nk"] = torch.randn(B, Hkv, d, generator=_gen(layer_seed(l, 6) + seed), device=dev).to(bf)
                 t["nv"] = torch.randn(B, Hkv, d, generator=_gen(layer_seed(l, 7) + seed), device=dev).to(bf)
             self.inputs.append(t)
-            ios = {}
-            for kind in kinds_of[l]:
-                io = L.DecodeIO(B=B, H=H, Hkv=Hkv, d=d, dtype=L.BF16)
-                io.q, io.o, io.scale = t["q"].data_ptr(), t["o"].data_ptr(), 1.0
-                if kind in (GDN, KDA):
-                    io.k, io.v = t["k"].data_ptr(), t["v"].data_ptr()
-                    io.beta = t["beta"].data_ptr()
-                    io.log_gate_scalar = t["lg_s"].data_ptr()
-                    io.log_gate_channel = t["lg_c"].data_ptr()
-                else:
-                    io.k, io.v = t["nk"].data_ptr(), t["nv"].data_ptr()
-                    io.seq_lens, io.max_seq_len, io.window = self.seq_lens.data_ptr(), s.ctx, s.window
-                    tab = self.table_for(l, kind)
-                    io.page_table, io.max_pages = tab.data_ptr(), tab.shape[1]
-                ios[kind] = io
-            self.io.append(ios)
+            self.io.append(self._make_io(l, t))
+        # further buffer sets: copies of the same inputs, their own outputs
+        self.input_sets = [self.inputs]
+        self.io_sets = [self.io]
+        for _ in range(1, io_sets):
+            ts = [{k: v.clone() for k, v in t.items()} for t in self.inputs]
+            self.input_sets.append(ts)
+            self.io_sets.append([self._make_io(l, ts[l]) for l in range(self.n_layers)])
         self.ws = torch.empty(max(16, L.attn_decode_workspace_size(FA, 0, B, H, Hkv, d, PAGE, s.ctx)),
                               dtype=torch.uint8, device=dev)
         self.c_placements = {k: (np.ctypeslib.as_ctypes(v)) for k, v in self.placements.items()}
         torch.cuda.synchronize()
+
+    def _make_io(self, l: int, t: dict) -> dict:
+        """hmd_decode_io_t for every kind layer l can take, pointing at the tensors in t."""
+        s = self.shape
+        ios = {}
+        for kind in self.kinds_of[l]:
+            io = L.DecodeIO(B=s.B, H=s.H, Hkv=s.Hkv, d=s.d, dtype=L.BF16)
+            io.q, io.o, io.scale = t["q"].data_ptr(), t["o"].data_ptr(), 1.0
+            if kind in (GDN, KDA):
+                io.k, io.v = t["k"].data_ptr(), t["v"].data_ptr()
+                io.beta = t["beta"].data_ptr()
+                io.log_gate_scalar = t["lg_s"].data_ptr()
+                io.log_gate_channel = t["lg_c"].data_ptr()
+            else:
+                io.k, io.v = t["nk"].data_ptr(), t["nv"].data_ptr()
+                io.seq_lens, io.max_seq_len, io.window = self.seq_lens.data_ptr(), s.ctx, s.window
+                tab = self.table_for(l, kind)
+                io.page_table, io.max_pages = tab.data_ptr(), tab.shape[1]
+            ios[kind] = io
+        return ios
 
     def _fill_pools(self, fa_layers, swa_layers, seed):
         done = set()
@@ -180,17 +194,19 @@ class MixerStack:
     def pools_for(self, layer: int):
         return self.kv_for(layer).layer_pools(layer)
 
-    def step(self, name: str, events: dict | None = None) -> None:
-        """One decode token for every sequence through all layers under placement `name`.
+    def step(self, name: str, events: dict | None = None, io_set: int = 0) -> None:
+        """One decode token for every sequence through all layers under placement `name`,
+        reading and writing the per-layer buffers of set `io_set`.
         events: optional {layer: (start_event, end_event)} recorded around that layer."""
         pl = self.placements[name]
         cpl = self.c_placements[name]
+        ios = self.io_sets[io_set]
         for l in range(self.n_layers):
             kind = int(pl[l])
             ev = events.get(l) if events else None
             if ev:
                 ev[0].record()
-            L.mixer_decode_step(cpl, l, self.io[l][kind], self.state,
+            L.mixer_decode_step(cpl, l, ios[l][kind], self.state,
                                 self.kv_for(l) if kind in (FA, SWA) else None,
                                 self.ws if kind in (FA, SWA) else None)
             if ev:
