@@ -11,9 +11,10 @@
 // or at ring page page_table[b][c mod R], R = ceil(w/64) (SWA) -- a ring holding exactly the
 // pages a window can touch, so logical pages map to whole ring pages.
 //
-// Kernel 1 (split): one CTA per (split, kv-head, sequence). It streams its range of pages
-// through a 3-stage TMA pipeline (two 64x64 bf16 boxes per page and operand, 128-byte
-// swizzle), and its 4 warps each take 16 keys of every page: S = Q K^T and O += P V run on
+// Kernel 1 (split): one CTA per work item (sequence, kv-head, key range), two resident per SM.
+// The plan either fits all items in one wave of long ranges or makes about eight waves of short
+// ones. A CTA streams its pages through a 3-stage TMA pipeline (two 64x64 bf16 boxes per page
+// and operand, 128-byte swizzle); its 4 warps each take 16 keys of every page: S = Q K^T and O += P V run on
 // mma.sync m16n8k16 (the GQA group's <=16 query heads fill the M=16 rows; tcgen05 needs M>=64),
 // with an online softmax in the log2 domain. The CTA whose range holds position L-1 patches the
 // new token into its shared-memory tile and writes it to the pool (the fused append). Keys
@@ -25,6 +26,7 @@
 #include <cuda.h>
 #include <float.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kernels.h"
@@ -41,7 +43,8 @@ constexpr int kStages = 3;    // pages in flight per CTA
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxGroup = 16;  // query heads per kv-head handled by one CTA (the MMA's M)
-constexpr int kTargetCtas = 148 * 2 * 8;  // about 8 waves of 2 resident CTAs per SM
+constexpr long long kWaves = 8;  // target waves of resident CTAs when ranges are split finely
+constexpr long long kMaxSplits = 256;  // key ranges per (sequence, kv-head), bounds the workspace
 
 struct SplitParams {
     const __nv_bfloat16 *q, *new_k, *new_v;
@@ -62,10 +65,62 @@ __device__ __forceinline__ uint32_t tile_off(int row, int dim) {
 }
 
 template <int D>
+constexpr int stage_bytes() {
+    return kStages * 2 * kPT * D * 2;
+}
+// stages + alignment slack (the cross-warp merge buffer reuses the stages after the last tile)
+template <int D>
 constexpr int smem_bytes() {
-    return kStages * 2 * kPT * D * 2 + 1024;  // + alignment slack
+    return stage_bytes<D>() + 1024;
 }
 
+// Work item i of the split-K plan: sequence b, kv-head g, key range `split` of that sequence.
+struct Item {
+    int b, g, split, L, lo, last_page, t_begin, n_tiles;
+    bool bad_len;
+};
+
+__device__ __forceinline__ Item item_info(const SplitParams &p, int i) {
+    Item it;
+    it.split = i % p.n_splits;
+    it.g = (i / p.n_splits) % p.Hkv;
+    it.b = i / (p.n_splits * p.Hkv);
+    it.L = p.seq_lens[it.b];
+    it.bad_len = it.L < 1 || it.L > p.max_seq_len;
+    it.lo = (p.swa && it.L > p.window) ? it.L - p.window : 0;
+    const int first_page = it.bad_len ? 0 : it.lo / kPT;
+    it.last_page = it.bad_len ? -1 : (it.L - 1) / kPT;
+    it.t_begin = first_page + it.split * p.pages_per_split;
+    const int t_end = min(it.t_begin + p.pages_per_split, it.last_page + 1);
+    it.n_tiles = max(0, t_end - it.t_begin);
+    return it;
+}
+
+__device__ __forceinline__ int phys_page(const SplitParams &p, int b, int c) {
+    const int idx = p.swa ? c % p.ring_pages : c;
+    return idx < p.max_pages ? p.page_table[(size_t)b * p.max_pages + idx] : -1;
+}
+
+// Q of one (sequence, kv-head) as mma.sync A fragments (rows = the group's query heads).
+template <int D>
+__device__ __forceinline__ void load_q(const SplitParams &p, int b, int g, int lane,
+                                       uint32_t (&qa)[D / 16][4]) {
+    const int G = p.group, r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2;
+    const uint32_t *q0 = r0 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + r0) * D) : nullptr;
+    const uint32_t *q1 = r1 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + r1) * D) : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        qa[kk][0] = q0 ? q0[(kk * 16 + cq) >> 1] : 0u;
+        qa[kk][1] = q1 ? q1[(kk * 16 + cq) >> 1] : 0u;
+        qa[kk][2] = q0 ? q0[(kk * 16 + 8 + cq) >> 1] : 0u;
+        qa[kk][3] = q1 ? q1[(kk * 16 + 8 + cq) >> 1] : 0u;
+    }
+}
+
+// Split-K kernel: CTA i processes work item i. Warp 0 produces: its lanes hold the physical
+// pages of 32 consecutive tiles (one coalesced page-table load per 32 tiles, fetched a chunk
+// ahead), and lane 0 issues each tile's TMA copies and records the tile's page in shared memory
+// before arming the stage's barrier. The tile loop itself reads no global memory.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -73,112 +128,108 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     constexpr int TB = kPT * D * 2;  // bytes of one page of one head (K or V)
     constexpr int NK = D / 16;       // k-steps of Q K^T
     constexpr int NN = D / 8;        // n-tiles of P V
+    constexpr int RS = D + 2;
+    static_assert(kWarps * kMaxGroup * RS * 4 <= stage_bytes<D>(), "merge buffer fits the stages");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[kStages];
-    __shared__ int s_abort;
+    __shared__ int stage_pg[kStages];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const uint32_t smem_base = smem_u32(smem);
 
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = p.group, h0 = g * G;
-
-    const int L = p.seq_lens[b];
-    const bool bad_len = (L < 1 || L > p.max_seq_len);
-    const int lo = (p.swa && L > p.window) ? L - p.window : 0;
-    const int first_page = bad_len ? 0 : lo / kPT;
-    const int last_page = bad_len ? -1 : (L - 1) / kPT;
-    const int t_begin = first_page + split * p.pages_per_split;
-    const int t_end = min(t_begin + p.pages_per_split, last_page + 1);
-    const int n_tiles = max(0, t_end - t_begin);
-    if (bad_len && split == 0 && tid == 0) atomicOr(&g_err, HMD_DEVERR_SEQLEN);
-    const int32_t *prow = p.page_table + (size_t)b * p.max_pages;
-    auto phys_page = [&](int c) -> int {
-        const int idx = p.swa ? c % p.ring_pages : c;
-        return idx < p.max_pages ? prow[idx] : -1;
-    };
-
+    const int G = p.group;
+    const Item it = item_info(p, blockIdx.x);
     if (tid == 0) {
+        if (it.bad_len && it.split == 0) atomicOr(&g_err, HMD_DEVERR_SEQLEN);
         for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&full_bar[s]), 1);
         fence_barrier_init();
-        s_abort = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
-    __syncthreads();
 
-    auto issue = [&](int t) {
-        const int c = t_begin + t;
-        const int pg = phys_page(c);
-        const int s = t % kStages;
-        const uint32_t bar = smem_u32(&full_bar[s]);
-        if (pg < 0 || pg >= p.n_pages) {
-            atomicOr(&g_err, HMD_DEVERR_PAGE);
-            mbar_arrive_expect_tx(bar, 0);  // complete the phase with no copy
-            return;
-        }
-        mbar_arrive_expect_tx(bar, 2 * TB);
-        const uint32_t kb = smem_base + s * 2 * TB, vb = kb + TB;
-        const int y = (pg * p.Hkv + g) * kPT;
-#pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-            tma_load_2d(kb + hf * kPT * 128, &tmk, bar, hf * 64, y);
-            tma_load_2d(vb + hf * kPT * 128, &tmv, bar, hf * 64, y);
-        }
+    // ---- producer (warp 0, warp-uniform calls; lane 0 issues) -----------------------------
+    auto table_entry = [&](int t) -> int {
+        return t < it.n_tiles ? phys_page(p, it.b, it.t_begin + t) : -1;
     };
-    if (tid == 0) {
-        for (int t = 0; t < kStages && t < n_tiles; ++t) issue(t);
+    int pt_cur = -1, pt_next = -1, issued = 0;
+    if (warp == 0) {
+        pt_cur = table_entry(lane);
+        pt_next = table_entry(32 + lane);
     }
-
-    // Q as the A operand (rows = the group's query heads, zero beyond G), kept in registers.
-    const int r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2;
-    uint32_t qa[NK][4];
-    {
-        const uint32_t *q0 = r0 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + h0 + r0) * D) : nullptr;
-        const uint32_t *q1 = r1 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + h0 + r1) * D) : nullptr;
-#pragma unroll
-        for (int kk = 0; kk < NK; ++kk) {
-            qa[kk][0] = q0 ? q0[(kk * 16 + cq) >> 1] : 0u;
-            qa[kk][1] = q1 ? q1[(kk * 16 + cq) >> 1] : 0u;
-            qa[kk][2] = q0 ? q0[(kk * 16 + 8 + cq) >> 1] : 0u;
-            qa[kk][3] = q1 ? q1[(kk * 16 + 8 + cq) >> 1] : 0u;
+    auto issue_next = [&]() {
+        if (issued >= it.n_tiles) return;
+        if (issued > 0 && (issued & 31) == 0) {
+            pt_cur = pt_next;
+            pt_next = table_entry(issued + 32 + lane);
         }
+        const int pg = __shfl_sync(0xffffffffu, pt_cur, issued & 31);
+        if (lane == 0) {
+            const int s = issued % kStages;
+            const uint32_t bar = smem_u32(&full_bar[s]);
+            if (pg < 0 || pg >= p.n_pages) {
+                stage_pg[s] = -1;
+                atomicOr(&g_err, HMD_DEVERR_PAGE);
+                mbar_arrive_expect_tx(bar, 0);  // complete the phase with no copy
+            } else {
+                stage_pg[s] = pg;
+                mbar_arrive_expect_tx(bar, 2 * TB);
+                const uint32_t kb = smem_base + s * 2 * TB, vb = kb + TB;
+                const int y = (pg * p.Hkv + it.g) * kPT;
+#pragma unroll
+                for (int hf = 0; hf < D / 64; ++hf) {
+                    tma_load_2d(kb + hf * kPT * 128, &tmk, bar, hf * 64, y);
+                    tma_load_2d(vb + hf * kPT * 128, &tmv, bar, hf * 64, y);
+                }
+            }
+        }
+        ++issued;
+    };
+    __syncthreads();  // barriers initialised
+    if (warp == 0) {
+        for (int t = 0; t < kStages; ++t) issue_next();
     }
 
+    const int r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2, mi = lane >> 3;
+    uint32_t qa[NK][4];
+    load_q<D>(p, it.b, it.g, lane, qa);
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
     float oacc[NN][4];
 #pragma unroll
     for (int n = 0; n < NN; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
 
-    int t = 0;
-    for (; t < n_tiles; ++t) {
+    for (int t = 0; t < it.n_tiles; ++t) {
         const int s = t % kStages;
         const bool ok = mbar_wait_bounded(smem_u32(&full_bar[s]), (t / kStages) & 1);
         if (__syncthreads_or(!ok)) {
-            if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
-            break;
+            if (tid == 0) {
+                atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+                // let the copies this CTA issued finish (bounded) before leaving
+                for (int u = t; u < issued; ++u)
+                    (void)mbar_wait_bounded(smem_u32(&full_bar[u % kStages]), (u / kStages) & 1);
+            }
+            return;  // no partials are written; the error word reports the step as failed
         }
-        const int c = t_begin + t;
-        const int pg = phys_page(c);
-        const bool tile_ok = pg >= 0 && pg < p.n_pages;
+        const int pg = stage_pg[s];
+        const bool tile_ok = pg >= 0;
+        const int c = it.t_begin + t;
         const int base = c * kPT;
         uint8_t *kb = smem + s * 2 * TB;
         uint8_t *vb = kb + TB;
-        const bool has_new = (c == last_page);
-        const bool partial = base < lo || base + kPT - 1 > L - 1;
+        const bool has_new = (c == it.last_page);
+        const bool partial = base < it.lo || base + kPT - 1 > it.L - 1;
         if (tile_ok && (has_new || partial)) {
             // zero V rows of masked positions; patch in the new token's K and V
             for (int idx = tid; idx < kPT * (D / 8); idx += kThreads) {
                 const int row = idx / (D / 8), ch = idx % (D / 8);
                 const int pos = base + row;
-                if (pos < lo || pos > L - 1)
+                if (pos < it.lo || pos > it.L - 1)
                     *reinterpret_cast<uint4 *>(vb + tile_off(row, ch * 8)) = make_uint4(0, 0, 0, 0);
             }
             if (has_new) {
-                const int rr = (L - 1) % kPT;
-                const size_t src = ((size_t)b * p.Hkv + g) * D;
+                const int rr = (it.L - 1) % kPT;
+                const size_t src = ((size_t)it.b * p.Hkv + it.g) * D;
                 for (int ch = tid; ch < 2 * (D / 8); ch += kThreads) {
                     const int cc = ch % (D / 8);
                     const uint4 val = ch < D / 8
@@ -188,18 +239,15 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     *reinterpret_cast<uint4 *>(dst) = val;
                     // the append itself: the pool slot of position L-1
                     __nv_bfloat16 *pool = ch < D / 8 ? p.k_pool : p.v_pool;
-                    *reinterpret_cast<uint4 *>(pool + (((size_t)pg * p.Hkv + g) * kPT + rr) * D + cc * 8) = val;
+                    *reinterpret_cast<uint4 *>(pool + (((size_t)pg * p.Hkv + it.g) * kPT + rr) * D + cc * 8) = val;
                 }
             }
+            fence_proxy_async_smem();  // these generic writes precede the stage's next TMA fill
             __syncthreads();
-        } else if (!tile_ok && has_new && tid == 0) {
-            atomicOr(&g_err, HMD_DEVERR_PAGE);
         }
 
         if (tile_ok) {
             const uint32_t kbu = smem_u32(kb), vbu = smem_u32(vb);
-            const int mi = lane >> 3;
-            // S^T block: this warp's 16 keys x the group's query heads
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             {
                 const int key = warp * 16 + ((mi >> 1) << 3) + (lane & 7);
@@ -217,7 +265,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int pos = base + warp * 16 + j * 8 + cq + (e & 1);
-                    const bool valid = pos >= lo && pos <= L - 1;
+                    const bool valid = pos >= it.lo && pos <= it.L - 1;
                     sc[j][e] = valid ? sc[j][e] * p.scale_log2 : -INFINITY;
                     mx[e >> 1] = fmaxf(mx[e >> 1], sc[j][e]);
                 }
@@ -265,24 +313,14 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             }
         }
         __syncthreads();  // every warp is done with stage s
-        if (tid == 0 && t + kStages < n_tiles) {
-            fence_proxy_async_smem();
-            issue(t + kStages);
+        if (warp == 0) {
+            if (lane == 0) fence_proxy_async_smem();
+            issue_next();
         }
-    }
-    if (t < n_tiles) {
-        // A wait gave up: drain the copies this CTA issued (bounded), then leave no partial.
-        if (tid == 0) {
-            for (int u = t; u < n_tiles && u < t + kStages; ++u)
-                (void)mbar_wait_bounded(smem_u32(&full_bar[u % kStages]), (u / kStages) & 1);
-            s_abort = 1;
-        }
-        __syncthreads();
     }
 
-    // Merge the 4 warps' partials through shared memory (the pipeline buffers are free now).
-    float *red = reinterpret_cast<float *>(smem);  // [kWarps][kMaxGroup][D + 2]
-    constexpr int RS = D + 2;
+    // ---- merge the 4 warps' partials (the stages are idle now: reuse them) -------------------
+    float *red = reinterpret_cast<float *>(smem);  // [kWarps][group][D + 2]
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         float l = l_run[r];
@@ -291,7 +329,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         l_run[r] = l;
     }
     if (r0 < G) {
-        float *dst = red + (warp * kMaxGroup + r0) * RS;
+        float *dst = red + (warp * G + r0) * RS;
 #pragma unroll
         for (int n = 0; n < NN; ++n) {
             dst[n * 8 + cq] = oacc[n][0];
@@ -300,7 +338,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if ((lane & 3) == 0) { dst[D] = m_run[0]; dst[D + 1] = l_run[0]; }
     }
     if (r1 < G) {
-        float *dst = red + (warp * kMaxGroup + r1) * RS;
+        float *dst = red + (warp * G + r1) * RS;
 #pragma unroll
         for (int n = 0; n < NN; ++n) {
             dst[n * 8 + cq] = oacc[n][2];
@@ -309,24 +347,21 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if ((lane & 3) == 0) { dst[D] = m_run[1]; dst[D + 1] = l_run[1]; }
     }
     __syncthreads();
-    const bool aborted = s_abort != 0;
     for (int idx = tid; idx < G * D; idx += kThreads) {
         const int r = idx / D, dim = idx % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * kMaxGroup + r) * RS + D]);
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * G + r) * RS + D]);
         float acc = 0.f, lsum = 0.f;
-        if (M != -INFINITY && !aborted) {
+        if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
-                const float f = exp2f(red[(w * kMaxGroup + r) * RS + D] - M);
-                acc += f * red[(w * kMaxGroup + r) * RS + dim];
-                lsum += f * red[(w * kMaxGroup + r) * RS + D + 1];
+                const float f = exp2f(red[(w * G + r) * RS + D] - M);
+                acc += f * red[(w * G + r) * RS + dim];
+                lsum += f * red[(w * G + r) * RS + D + 1];
             }
-        } else {
-            M = -INFINITY;
         }
-        const size_t row = ((size_t)b * p.Hq + h0 + r) * p.n_splits + split;
+        const size_t row = ((size_t)it.b * p.Hq + it.g * G + r) * p.n_splits + it.split;
         p.ws_acc[row * D + dim] = acc;
         if (dim == 0) {
             p.ws_ml[row * 2] = M;
@@ -391,6 +426,8 @@ bool make_pool_map(CUtensorMap *m, void *pool, int n_pages, int Hkv, int d) {
 
 template <int D>
 cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t s) {
+    const int group = a.Hq / a.Hkv;
+    constexpr int smem = smem_bytes<D>();
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -414,20 +451,36 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     const size_t rows = (size_t)a.B * a.Hq * plan.n_splits;
     p.ws_ml = static_cast<float *>(a.workspace);
     p.ws_acc = p.ws_ml + ((rows * 2 + 3) & ~static_cast<size_t>(3));
-    p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.group = a.Hq / a.Hkv;
+    p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.group = group;
     p.n_pages = a.n_pages; p.max_pages = a.max_pages;
     p.window = a.window; p.swa = a.swa ? 1 : 0;
     p.ring_pages = a.swa ? (a.window + kPT - 1) / kPT : 0;
     p.n_splits = plan.n_splits; p.pages_per_split = plan.pages_per_split;
     p.max_seq_len = a.max_seq_len;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    dim3 grid(plan.n_splits, a.Hkv, a.B);
-    attn_split_kernel<D><<<grid, kThreads, smem_bytes<D>(), s>>>(tmk, tmv, p);
+    attn_split_kernel<D><<<(unsigned)plan.n_ctas, kThreads, smem, s>>>(tmk, tmv, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_combine_kernel<D><<<(unsigned)(a.B * a.Hq), D, 0, s>>>(p.ws_ml, p.ws_acc, plan.n_splits,
                                                                static_cast<__nv_bfloat16 *>(a.o));
     return cudaGetLastError();
+}
+
+// SMs of the current device (148 when no device can be queried).
+int device_sms() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else {
+            cudaGetLastError();
+            n = 148;
+        }
+    });
+    return n;
 }
 
 }  // namespace
@@ -439,17 +492,29 @@ bool attn_decode_supported(int d, int page_tokens, int group) {
 AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, int page_tokens,
                           int max_seq_len) {
     (void)page_tokens;
+    (void)Hq;
     AttnPlan pl;
     long long tiles = (max_seq_len + kPT - 1) / kPT;
     if (swa) tiles = std::min<long long>(tiles, (window + kPT - 1) / kPT + 1);
     tiles = std::max<long long>(tiles, 1);
     const long long units = std::max<long long>(1, (long long)B * Hkv);
-    long long splits = (kTargetCtas + units - 1) / units;
-    splits = std::max<long long>(1, std::min(splits, (tiles + 1) / 2));  // >= 2 pages per split
-    long long pps = (tiles + splits - 1) / splits;
-    splits = (tiles + pps - 1) / pps;
+    // resident CTAs per SM from shared memory (228 KiB per SM, 1 KiB reserved per CTA)
+    const int smem = (d == 64 ? smem_bytes<64>() : smem_bytes<128>()) + 1024;
+    const long long slots = (long long)std::max(1, std::min(2, 233472 / smem)) * device_sms();
+    // One wave: the most key ranges that still fit every item in a resident slot, so each CTA
+    // streams one long range. Taken when it fills at least 3/4 of the slots; otherwise about
+    // kWaves waves of shorter ranges (>= 2 pages each), which the block scheduler balances.
+    long long s_one = std::max<long long>(1, std::min({tiles, slots / units, kMaxSplits}));
+    long long s_many = std::max<long long>(
+        1, std::min({(kWaves * slots + units - 1) / units, std::max<long long>(1, tiles / 2),
+                     kMaxSplits}));
+    const bool one_wave_fits = units * s_one <= slots && units * s_one * 4 >= slots * 3;
+    long long splits = (one_wave_fits || units * s_many <= slots) ? s_one : s_many;
+    const long long pps = (tiles + splits - 1) / splits;
+    splits = (tiles + pps - 1) / pps;  // no empty range
     pl.n_splits = (int)splits;
     pl.pages_per_split = (int)pps;
+    pl.n_ctas = (int)(units * splits);
     const size_t rows = (size_t)B * Hq * splits;
     pl.ws_bytes = (((rows * 2 + 3) & ~static_cast<size_t>(3)) + rows * d) * sizeof(float);
     return pl;

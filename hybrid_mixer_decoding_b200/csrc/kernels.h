@@ -44,8 +44,9 @@ struct AttnDecodeArgs {
     size_t ws_bytes;
 };
 struct AttnPlan {
-    int n_splits;
+    int n_splits;         // key ranges per (sequence, kv-head)
     int pages_per_split;
+    int n_ctas;           // grid size: one CTA per (sequence, kv-head, key range)
     size_t ws_bytes;
 };
 AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, int page_tokens,

@@ -141,8 +141,9 @@ class MixerStack:
             ts = [{k: v.clone() for k, v in t.items()} for t in self.inputs]
             self.input_sets.append(ts)
             self.io_sets.append([self._make_io(l, ts[l]) for l in range(self.n_layers)])
-        self.ws = torch.empty(max(16, L.attn_decode_workspace_size(FA, 0, B, H, Hkv, d, PAGE, s.ctx)),
-                              dtype=torch.uint8, device=dev)
+        ws_bytes = max(L.attn_decode_workspace_size(FA, 0, B, H, Hkv, d, PAGE, s.ctx),
+                       L.attn_decode_workspace_size(SWA, s.window, B, H, Hkv, d, PAGE, s.ctx))
+        self.ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
         self.c_placements = {k: (np.ctypeslib.as_ctypes(v)) for k, v in self.placements.items()}
         torch.cuda.synchronize()
 

@@ -114,7 +114,10 @@ HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, i
 /* i.e. (page_table[b][r / page_tokens], r % page_tokens).                                     */
 /* ------------------------------------------------------------------------------------------ */
 
-/* Workspace bytes attn_decode needs for these sizes (split-K partials; 0 is never returned).  */
+/* Workspace bytes attn_decode needs for these sizes (split-K partials; 0 is never returned).
+ * The figure follows the launch plan for exactly these arguments and is not monotone in them
+ * (a longer context may take fewer key ranges); size a shared workspace as the maximum over
+ * every (kind, window, sizes) it will serve. It never exceeds 4 * B * Hq * 256 * (d + 2) + 12. */
 HMD_API size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
                                   int page_tokens, int max_seq_len);
 
@@ -206,7 +209,8 @@ typedef struct {
 
 /* One decode token for layer `layer`: runs the mixer placement[layer] (host int8 array of
  * n_layers kinds) on that layer's registered caches. Attention layers need a workspace of
- * attn_decode_workspace_size(...) bytes. Returns HMD_ERR_ARG if the chosen mixer's cache is not
+ * attn_decode_workspace_size(...) bytes for the chosen kind; one workspace serving layers that
+ * can switch between FA and SWA takes the larger of the two sizes. Returns HMD_ERR_ARG if the chosen mixer's cache is not
  * registered for the layer (no pool for FA/SWA, no state block for GDN/KDA).                 */
 HMD_API hmd_status_t mixer_decode_step(const int8_t *placement, int n_layers, int layer,
                                const hmd_decode_io_t *io, hmd_state_cache_t *state_cache,

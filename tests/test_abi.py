@@ -88,13 +88,18 @@ def test_attn_validation():
     assert _attn(ptr=None) == ARG
 
 
-def test_workspace_size_monotone():
+def test_workspace_size_bounds():
+    """Partials are one (m, l) pair and one d-vector per query row and key range, with at most
+    256 key ranges and never more ranges than 64-token pages."""
     f = hmd.attn_decode_workspace_size
-    a = f(hmd.FA, 0, 32, 32, 8, 128, 64, 8192)
-    b = f(hmd.FA, 0, 32, 32, 8, 128, 64, 16384)
-    assert a > 0 and b >= a
-    assert f(hmd.SWA, 4096, 32, 32, 8, 128, 64, 1 << 20) <= f(hmd.FA, 0, 32, 32, 8, 128, 64,
-                                                              1 << 20)
+    for kind, w in ((hmd.FA, 0), (hmd.SWA, 4096)):
+        for B, Hq, Hkv, d, L in ((32, 32, 8, 128, 8192), (64, 32, 8, 128, 32768), (1, 8, 2, 64, 65),
+                                 (3, 8, 2, 128, 300), (16, 32, 8, 128, 1 << 20)):
+            n = f(kind, w, B, Hq, Hkv, d, 64, L)
+            pages = -(-L // 64) if kind == hmd.FA else min(-(-L // 64), -(-w // 64) + 1)
+            s_max = min(256, pages)
+            assert 4 * B * Hq * (d + 2) <= n <= 4 * B * Hq * s_max * (d + 2) + 12, (kind, B, L)
+            assert (n - 4 * B * Hq * (d + 2) * (n // (4 * B * Hq * (d + 2)))) <= 12
 
 
 def test_dispatcher_validation():
