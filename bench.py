@@ -513,7 +513,7 @@ def run_kernel_workload(args):
                 "traffic": traffic_for(w), "algorithmic_bytes": byts}
         extra["tensor"] = {"achieved_tflops": round(flops / sec / 1e12, 3), "peak": tf,
                            "frac": round(flops / sec / 1e12 / tf, 5), "algorithmic_flops": flops}
-        launches = 1
+        launches = 2  # chunk-parallel pass + state scan
     else:
         raise SystemExit(f"unknown workload {w}")
     assert hmd.hmd_device_errors(clear=True) == 0

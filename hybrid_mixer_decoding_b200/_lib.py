@@ -36,6 +36,9 @@ _SIGS = {
     "delta_rule_decode": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _c_float, _vp]),
     "delta_rule_prefill_chunked": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
                                                                       _c_float, _vp]),
+    "delta_rule_prefill_workspace_size": (_sz, [_c_int] * 8),
+    "delta_rule_prefill_chunked_ws": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
+                                                                         _c_float, _vp, _sz, _vp]),
     "attn_decode_workspace_size": (_sz, [_c_int] * 8),
     "attn_decode": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
                                                       _vp, _sz, _vp]),
@@ -137,6 +140,26 @@ def delta_rule_prefill_chunked(kind, q, k, v, beta, log_gate, state, o, slots=No
                                           state.shape[0], _p(slots), _p(o), int(chunk),
                                           float(scale), _stream(stream))
     _check("delta_rule_prefill_chunked", st)
+
+
+def delta_rule_prefill_workspace_size(kind, B, T, H, dk, dv, dtype, chunk=64) -> int:
+    return int(lib().delta_rule_prefill_workspace_size(kind, B, T, H, dk, dv, dtype, chunk))
+
+
+def delta_rule_prefill_chunked_ws(kind, q, k, v, beta, log_gate, state, o, workspace, slots=None,
+                                  chunk=64, scale=1.0, stream=None) -> None:
+    """delta_rule_prefill_chunked with caller-owned scratch `workspace` (a device tensor; its
+    byte size is passed, see include/hmd.h)."""
+    _contig(q, k, v, beta, log_gate, state, o, slots, workspace)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().delta_rule_prefill_chunked_ws(kind, B, T, H, dk, dv, _dtype_code(q), _p(q), _p(k),
+                                             _p(v), _p(beta), _p(log_gate), _p(state),
+                                             state.shape[0], _p(slots), _p(o), int(chunk),
+                                             float(scale), _p(workspace), ws_bytes,
+                                             _stream(stream))
+    _check("delta_rule_prefill_chunked_ws", st)
 
 
 def attn_decode_workspace_size(kind, window, B, Hq, Hkv, d, page_tokens, max_seq_len) -> int:

@@ -1,0 +1,625 @@
+// Chunked delta-rule prefill in two passes on tensor cores (mma.sync m16n8k16, bf16 operands,
+// fp32 accumulation), bf16 activations, d_k = d_v = 128, chunk C = 64.
+//
+// Chunk algebra: the standard WY / UT-transform rewriting of the gated delta rule for the GDN and
+// KDA mixers of "Super Apriel: One Checkpoint, Many Speeds" (abstract; gist.science technical
+// summary, section 2a). For a chunk with start state M ([d_k][d_v] fp32) and G the per-channel
+// cumulative log-gate inside the chunk (G_C its last row):
+//   Kt = k e^G, Kh = k e^-G, Qt = q e^G, Kc = k e^(G_C - G)
+//   A = beta_r (Kt Kh^T)_{rs} (s < r),  P = (Qt Kh^T)_{rs} (s <= r)
+//   T = (I + A)^-1 Diag(beta),  W = T Kt,  Ut = T V
+//   U = Ut - W M,  O = Qt M + P U,  M_next = Diag(e^{G_C}) M + Kc^T U
+// Everything up to W and Ut depends only on the chunk's own inputs; only the last line carries
+// the state from chunk to chunk.
+//
+// Pass A (prefill_prep_kernel): one CTA per (sequence, head, chunk), all chunks at once. It
+// computes the gate factors, A and P, the blocked UT solve, W and Ut, and writes one record per
+// chunk: Qt, -W, Kc, P (bf16, already in the 128-byte XOR-swizzled tile layout pass B reads with
+// ldmatrix), e^{G_C} and Ut (fp32).
+// Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks in
+// order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
+// the previous chunk computes; the state half lives in registers as MMA accumulator fragments.
+// Per chunk it does only the state-dependent products (U, O, state update): 7.3 MFLOP of the
+// chunk's 11.5 per head, split over two CTAs.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "kernels.h"
+#include "ptx.cuh"
+#include "../../include/hmd.h"
+
+namespace hmd {
+namespace {
+
+__device__ unsigned int g_err;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+constexpr int kSplitV = 2;             // pass B: CTAs per (sequence, head), each d_v / 2 columns
+constexpr int kDV = kD / kSplitV;      // 64 columns of d_v per pass-B CTA
+
+// ---- the per-chunk record (bytes) ----------------------------------------------------------
+constexpr uint32_t REC_QT = 0;         // Qt  bf16 [64][128], swizzled halves
+constexpr uint32_t REC_NW = 16384;     // -W  bf16 [64][128]
+constexpr uint32_t REC_KC = 32768;     // Kc  bf16 [64][128]
+constexpr uint32_t REC_P = 49152;      // P   bf16 [64][64]
+constexpr uint32_t REC_GAM = 57344;    // e^{G_C} fp32 [128]
+constexpr uint32_t REC_HEAD = 57856;   // bytes above, moved by one bulk copy
+constexpr uint32_t REC_UT = 57856;     // Ut  fp32 [64][128] row-major
+constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 4;  // 90624
+static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
+
+// ---- pass A shared memory (bytes from a 1024-aligned base) ---------------------------------
+constexpr uint32_t A_KT = 0;           // Kt  [64][128]
+constexpr uint32_t A_QT = 16384;       // q, then Qt  [64][128]
+constexpr uint32_t A_KH = 32768;       // k, then Kh  [64][128]
+constexpr uint32_t A_V = 49152;        // V   [64][128]
+constexpr uint32_t A_AS = 65536;       // A fp32 [64][68]; after the solve: T bf16 [64][64]
+constexpr uint32_t A_XS = 82944;       // X fp32 [64][68]
+constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
+constexpr uint32_t A_SMALL = 104192;
+constexpr uint32_t A_SMEM = A_SMALL + 3072 + 1024;
+constexpr uint32_t A_LG = A_AS;        // KDA raw log-gates fp32 [64][128] (before A exists)
+constexpr uint32_t A_T = A_AS;
+constexpr int AS_LD = 68;
+constexpr int YS_LD = 20;
+static_assert(A_LG + kC * kD * 4 <= A_YS, "log-gate staging fits the A/X region");
+
+// ---- pass B shared memory ----------------------------------------------------------------
+constexpr uint32_t B_STAGE = 58368;    // one record head, padded to 1 KiB
+constexpr uint32_t B_M = 2 * B_STAGE;  // M bf16 [128][64]
+constexpr uint32_t B_U = B_M + 16384;  // U bf16 [64][64]
+constexpr uint32_t B_BAR = B_U + 8192;
+constexpr uint32_t B_SMEM = B_BAR + 64 + 1024;
+
+// byte offset of element (row, col) of a tile whose halves (64 columns each) hold `rows` rows
+__device__ __forceinline__ uint32_t toff(int row, int col, int rows) {
+    return (uint32_t)((col >> 6) * rows * 128 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                      ((col & 7) << 1));
+}
+
+__device__ __forceinline__ void st_bf16x2(uint8_t *base, uint32_t off, float lo, float hi) {
+    *reinterpret_cast<uint32_t *>(base + off) = pack_bf16x2(lo, hi);
+}
+
+__device__ __forceinline__ uint8_t *record(const PrefillScanArgs &a, int bh, int c) {
+    return static_cast<uint8_t *>(a.ws) + ((size_t)bh * a.n_seg + c) * REC_BYTES;
+}
+
+// ================================ pass A ==================================================
+template <bool KDA>
+__global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const PrefillScanArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    float *As = reinterpret_cast<float *>(sm + A_AS);
+    float *Xs = reinterpret_cast<float *>(sm + A_XS);
+    float *Ys = reinterpret_cast<float *>(sm + A_YS);
+    float *sbeta = reinterpret_cast<float *>(sm + A_SMALL);  // [64]
+    float *hsum = sbeta + 64;                                 // [2][128] half-chunk gate sums
+    float *lgp = hsum + 256;                                  // [64] GDN log-gate prefix
+    float *etok = lgp + 64;                                   // [64] GDN e^G
+    float *ietok = etok + 64;                                 // [64] GDN e^-G
+    float *wsum = ietok + 64;                                 // [2]
+    float *gam = wsum + 2;                                    // [128] e^{G_C}
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int l7 = lane & 7, lb3 = (lane >> 3) & 1, lb4 = lane >> 4;
+    const int bh = blockIdx.x / a.n_seg, c = blockIdx.x - bh * a.n_seg;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int T = a.T;
+    const int t0 = (a.chunk_begin + c) * kC;
+    const int n = min(kC, T - t0);
+    uint8_t *rec = record(a, bh, c);
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v);
+
+    // ---- stage q (into the Qt slot), k (into the Kh slot), v, KDA log-gates; beta ----------
+    {
+        const size_t row0 = ((size_t)b * T + t0) * a.H + h;  // token t0's row in [B][T][H]
+        uint4 qv[4], kv[4], vv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = tid + j * kThreads, r = idx >> 4, ch = idx & 15;
+            qv[j] = kv[j] = vv[j] = make_uint4(0, 0, 0, 0);
+            if (r < n) {
+                const size_t off = (row0 + (size_t)r * a.H) * kD + ch * 8;
+                qv[j] = __ldg(reinterpret_cast<const uint4 *>(qg + off));
+                kv[j] = __ldg(reinterpret_cast<const uint4 *>(kg + off));
+                vv[j] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
+            }
+        }
+        float4 gv[8];
+        if constexpr (KDA) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int idx = tid + j * kThreads, r = idx >> 5, c4 = idx & 31;
+                gv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r < n)
+                    gv[j] = __ldg(reinterpret_cast<const float4 *>(a.log_gate + (row0 + (size_t)r * a.H) * kD + c4 * 4));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = tid + j * kThreads, r = idx >> 4, ch = idx & 15;
+            const uint32_t o = toff(r, ch * 8, 64);
+            *reinterpret_cast<uint4 *>(sm + A_QT + o) = qv[j];
+            *reinterpret_cast<uint4 *>(sm + A_KH + o) = kv[j];
+            *reinterpret_cast<uint4 *>(sm + A_V + o) = vv[j];
+        }
+        if constexpr (KDA) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int idx = tid + j * kThreads, r = idx >> 5, c4 = idx & 31;
+                *reinterpret_cast<float4 *>(sm + A_LG + r * 512 + c4 * 16) = gv[j];
+            }
+        }
+        if (tid < kC) {
+            const size_t tok = row0 + (size_t)tid * a.H;
+            sbeta[tid] = tid < n ? a.beta[tok] : 0.f;
+            if constexpr (!KDA) {
+                float x = tid < n ? a.log_gate[tok] : 0.f;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                if (lane == 31) wsum[warp] = x;
+                lgp[tid] = x;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- gate pass: Kt, Qt, Kh (shared memory), Kc (record), e^{G_C}; thread = (channel,
+    //      half of the chunk's rows) ------------------------------------------------------------
+    {
+        const int i = tid & (kD - 1), hf = tid >> 7;
+        const float *lgs = reinterpret_cast<const float *>(sm + A_LG) + i;
+        if constexpr (KDA) {
+            float part = 0.f;
+#pragma unroll 8
+            for (int r = 32 * hf; r < 32 * hf + 32; ++r) part += lgs[r * kD];
+            hsum[hf * kD + i] = part;
+        } else {
+            if (tid < kC) {
+                const float gc = lgp[tid] + (warp == 1 ? wsum[0] : 0.f);
+                lgp[tid] = gc;
+                etok[tid] = expf(gc);
+                ietok[tid] = expf(-gc);
+            }
+        }
+        __syncthreads();
+        const float gC = KDA ? hsum[i] + hsum[kD + i] : lgp[kC - 1];
+        float gsum = KDA ? (hf ? hsum[i] : 0.f) : 0.f;
+        uint8_t *kc = rec + REC_KC;
+#pragma unroll 4
+        for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
+            float e, ie, gr;
+            if constexpr (KDA) {
+                gsum += lgs[r * kD];
+                gr = gsum;
+                e = expf(gsum);
+                ie = expf(-gsum);
+            } else {
+                gr = lgp[r];
+                e = etok[r];
+                ie = ietok[r];
+            }
+            const uint32_t o = toff(r, i, 64);
+            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + A_KH + o));
+            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + A_QT + o));
+            *reinterpret_cast<__nv_bfloat16 *>(sm + A_KT + o) = __float2bfloat16_rn(kv * e);
+            *reinterpret_cast<__nv_bfloat16 *>(sm + A_QT + o) = __float2bfloat16_rn(qv * e);
+            *reinterpret_cast<__nv_bfloat16 *>(sm + A_KH + o) = __float2bfloat16_rn(kv * ie);
+            *reinterpret_cast<__nv_bfloat16 *>(kc + o) = __float2bfloat16_rn(kv * expf(gC - gr));
+        }
+        if (hf == 1) gam[i] = expf(gC);
+    }
+    __syncthreads();
+    // Qt -> record (16-byte copies); e^{G_C} -> record
+    {
+        const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_QT);
+        uint4 *dst = reinterpret_cast<uint4 *>(rec + REC_QT);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[tid + j * kThreads] = src[tid + j * kThreads];
+        if (tid < kD) reinterpret_cast<float *>(rec + REC_GAM)[tid] = gam[tid];
+    }
+
+    // ---- A (warps 0-3) and P (warps 4-7), 16 rows each: [Kt | Qt] Kh^T ----------------------
+    {
+        const int mat = warp >> 2, rt = warp & 3;
+        const uint32_t abase = sb + (mat ? A_QT : A_KT);
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            uint32_t af[4];
+            ldmatrix_x4(abase + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
+                        af[2], af[3]);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(sb + A_KH + toff(np * 16 + l7 + lb4 * 8, kk * 16 + lb3 * 8, 64), b0, b1,
+                            b2, b3);
+                mma_bf16_16816(acc[2 * np], af, b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+            }
+        }
+        const int r0 = 16 * rt + g, r1 = r0 + 8;
+        uint8_t *pr = rec + REC_P;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            const int s0 = nt * 8 + 2 * t4;
+            if (mat == 0) {
+                As[r0 * AS_LD + s0] = (s0 < r0 && r0 < n) ? sbeta[r0] * acc[nt][0] : 0.f;
+                As[r0 * AS_LD + s0 + 1] = (s0 + 1 < r0 && r0 < n) ? sbeta[r0] * acc[nt][1] : 0.f;
+                As[r1 * AS_LD + s0] = (s0 < r1 && r1 < n) ? sbeta[r1] * acc[nt][2] : 0.f;
+                As[r1 * AS_LD + s0 + 1] = (s0 + 1 < r1 && r1 < n) ? sbeta[r1] * acc[nt][3] : 0.f;
+            } else {
+                st_bf16x2(pr, toff(r0, s0, 64), (s0 <= r0 && r0 < n) ? acc[nt][0] : 0.f,
+                          (s0 + 1 <= r0 && r0 < n) ? acc[nt][1] : 0.f);
+                st_bf16x2(pr, toff(r1, s0, 64), (s0 <= r1 && r1 < n) ? acc[nt][2] : 0.f,
+                          (s0 + 1 <= r1 && r1 < n) ? acc[nt][3] : 0.f);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- X = (I + A)^-1 (16x16 blocks, fp32), T = X Diag(beta) ----------------------------
+    if (tid < 64) {  // diagonal blocks by forward substitution, one column per thread
+        const int bi = tid >> 4, c0 = tid & 15;
+        const float *ab = As + bi * 16 * AS_LD + bi * 16;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int s = 0; s < r; ++s) acc += ab[r * AS_LD + s] * x[s];
+            x[r] = r < c0 ? 0.f : (r == c0 ? 1.f : -acc);
+            Xs[(bi * 16 + r) * AS_LD + bi * 16 + c0] = x[r];
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int L = 1; L < 4; ++L) {
+        const int nb = 4 - L;  // blocks (i, j) with i - j = L
+        for (int it = tid; it < nb * 64; it += kThreads) {  // Y_ij = sum_{k=j}^{i-1} A_ik X_kj
+            const int j = it >> 6, r = (it >> 2) & 15, cg = it & 3, i = j + L;
+            const float *arow = As + (i * 16 + r) * AS_LD;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = j * 16; k < i * 16; ++k) {
+                const float av = arow[k];
+                const float4 xv = *reinterpret_cast<const float4 *>(Xs + k * AS_LD + j * 16 + cg * 4);
+                acc.x += av * xv.x; acc.y += av * xv.y; acc.z += av * xv.z; acc.w += av * xv.w;
+            }
+            *reinterpret_cast<float4 *>(Ys + (j * 16 + r) * YS_LD + cg * 4) = acc;
+        }
+        __syncthreads();
+        for (int it = tid; it < nb * 64; it += kThreads) {  // X_ij = -X_ii Y_ij
+            const int j = it >> 6, r = (it >> 2) & 15, cg = it & 3, i = j + L;
+            const float *xrow = Xs + (i * 16 + r) * AS_LD + i * 16;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s <= r; ++s) {
+                const float xv = xrow[s];
+                const float4 yv = *reinterpret_cast<const float4 *>(Ys + (j * 16 + s) * YS_LD + cg * 4);
+                acc.x += xv * yv.x; acc.y += xv * yv.y; acc.z += xv * yv.z; acc.w += xv * yv.w;
+            }
+            *reinterpret_cast<float4 *>(Xs + (i * 16 + r) * AS_LD + j * 16 + cg * 4) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        }
+        __syncthreads();
+    }
+    // T overwrites A (no longer read)
+    for (int idx = tid; idx < 64 * 32; idx += kThreads) {
+        const int r = idx >> 5, s0 = (idx & 31) * 2;
+        const float v0 = s0 <= r ? Xs[r * AS_LD + s0] * sbeta[s0] : 0.f;
+        const float v1 = s0 + 1 <= r ? Xs[r * AS_LD + s0 + 1] * sbeta[s0 + 1] : 0.f;
+        st_bf16x2(sm + A_T, toff(r, s0, 64), v0, v1);
+    }
+    __syncthreads();
+
+    // ---- Ut = T V (warps 0-3, fp32 -> record) and W = T Kt (warps 4-7, -W bf16 -> record) ---
+    {
+        const int mat = warp >> 2, rt = warp & 3;
+        float acc[16][4];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        const uint32_t bbase = sb + (mat ? A_KT : A_V);
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk) {
+            uint32_t af[4];
+            ldmatrix_x4(sb + A_T + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
+                        af[2], af[3]);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(bbase + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64), b0, b1,
+                                  b2, b3);
+                mma_bf16_16816(acc[2 * np], af, b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+            }
+        }
+        const int r0 = 16 * rt + g, r1 = r0 + 8;
+        if (mat == 1) {
+            uint8_t *nw = rec + REC_NW;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const int cc = nt * 8 + 2 * t4;
+                st_bf16x2(nw, toff(r0, cc, 64), -acc[nt][0], -acc[nt][1]);
+                st_bf16x2(nw, toff(r1, cc, 64), -acc[nt][2], -acc[nt][3]);
+            }
+        } else {
+            float *ut = reinterpret_cast<float *>(rec + REC_UT);
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const int cc = nt * 8 + 2 * t4;
+                *reinterpret_cast<float2 *>(ut + r0 * kD + cc) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2 *>(ut + r1 * kD + cc) = make_float2(acc[nt][2], acc[nt][3]);
+            }
+        }
+    }
+}
+
+// ================================ pass B ==================================================
+__global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const PrefillScanArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + B_BAR);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int l7 = lane & 7, lb3 = (lane >> 3) & 1, lb4 = lane >> 4;
+    const int bh = blockIdx.x / kSplitV, sv = blockIdx.x - bh * kSplitV;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int col0 = sv * kDV;  // this CTA's first d_v column
+    const int T = a.T;
+    const int slot = a.slots ? a.slots[b] : b;
+    if (slot < 0 || slot >= a.n_slots) {
+        if (tid == 0) atomicOr(&g_err, HMD_DEVERR_SLOT);
+        return;
+    }
+    float *Mg = a.state + ((size_t)slot * a.H + h) * kD * kD;
+    __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto issue = [&](int c) {  // thread 0: chunk c's record head -> stage c & 1
+        const uint32_t bar = smem_u32(&bars[c & 1]);
+        mbar_arrive_expect_tx(bar, REC_HEAD);
+        bulk_load(sb + (c & 1) * B_STAGE, record(a, bh, c), REC_HEAD, bar);
+    };
+    if (tid == 0) {
+        issue(0);
+        if (a.n_seg > 1) issue(1);
+    }
+
+    // state strip of this warp: rows 16*warp + g (+8), slice columns 8*nt + 2*t4 (+1)
+    const int sr0 = 16 * warp + g, sr1 = sr0 + 8;
+    float st[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int cc = col0 + nt * 8 + 2 * t4;
+        const float2 x0 = *reinterpret_cast<const float2 *>(Mg + (size_t)sr0 * kD + cc);
+        const float2 x1 = *reinterpret_cast<const float2 *>(Mg + (size_t)sr1 * kD + cc);
+        st[nt][0] = x0.x; st[nt][1] = x0.y; st[nt][2] = x1.x; st[nt][3] = x1.y;
+    }
+    // U / O role: chunk rows 16*rt + g (+8), slice columns 32*chh + 8*j + 2*t4 (+1)
+    const int rt = warp & 3, chh = warp >> 2;
+    const int ur0 = 16 * rt + g, ur1 = ur0 + 8;
+    float un[4][4];  // Ut of the next chunk, prefetched
+    auto load_ut = [&](int c) {
+        const float *ut = reinterpret_cast<const float *>(record(a, bh, c) + REC_UT);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
+            const float2 x0 = *reinterpret_cast<const float2 *>(ut + ur0 * kD + cc);
+            const float2 x1 = *reinterpret_cast<const float2 *>(ut + ur1 * kD + cc);
+            un[j][0] = x0.x; un[j][1] = x0.y; un[j][2] = x1.x; un[j][3] = x1.y;
+        }
+    };
+    load_ut(0);
+
+    int aborted_at = -1;
+    for (int c = 0; c < a.n_seg; ++c) {
+        const int s = c & 1;
+        const uint32_t stg = sb + s * B_STAGE;
+        const int t0 = (a.chunk_begin + c) * kC;
+        const int n = min(kC, T - t0);
+        const bool ok = mbar_wait_bounded(smem_u32(&bars[s]), (c >> 1) & 1);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+            aborted_at = c;
+            break;
+        }
+        // ---- phase 1: bf16 copy of M (the B operand of U and O); st <- e^{G_C} st ---------
+        {
+            const float *gm = reinterpret_cast<const float *>(sm + s * B_STAGE + REC_GAM);
+            const float g0 = gm[sr0], g1 = gm[sr1];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int cc = nt * 8 + 2 * t4;
+                st_bf16x2(sm + B_M, toff(sr0, cc, 128), st[nt][0], st[nt][1]);
+                st_bf16x2(sm + B_M, toff(sr1, cc, 128), st[nt][2], st[nt][3]);
+                st[nt][0] *= g0; st[nt][1] *= g0; st[nt][2] *= g1; st[nt][3] *= g1;
+            }
+        }
+        float u[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[j][e] = un[j][e];
+        __syncthreads();
+
+        // ---- phase 2: U = Ut + (-W) M (16 rows x 32 columns per warp) ----------------------
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            uint32_t af[4];
+            ldmatrix_x4(stg + REC_NW + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
+                        af[2], af[3]);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(sb + B_M + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 128),
+                                  b0, b1, b2, b3);
+                mma_bf16_16816(u[2 * np], af, b0, b1);
+                mma_bf16_16816(u[2 * np + 1], af, b2, b3);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int cc = 32 * chh + 8 * j + 2 * t4;
+            st_bf16x2(sm + B_U, toff(ur0, cc, 64), u[j][0], u[j][1]);
+            st_bf16x2(sm + B_U, toff(ur1, cc, 64), u[j][2], u[j][3]);
+        }
+        if (c + 1 < a.n_seg) load_ut(c + 1);
+        __syncthreads();
+
+        // ---- phase 3: O = Qt M + P U (16 rows x 32 columns per warp), then the state ------
+        {
+            float o[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                uint32_t af[4];
+                ldmatrix_x4(stg + REC_QT + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0],
+                            af[1], af[2], af[3]);
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(sb + B_M + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 128),
+                                      b0, b1, b2, b3);
+                    mma_bf16_16816(o[2 * np], af, b0, b1);
+                    mma_bf16_16816(o[2 * np + 1], af, b2, b3);
+                }
+            }
+#pragma unroll
+            for (int kk = 0; kk < kC / 16; ++kk) {
+                uint32_t af[4];
+                ldmatrix_x4(stg + REC_P + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0],
+                            af[1], af[2], af[3]);
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(sb + B_U + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 64),
+                                      b0, b1, b2, b3);
+                    mma_bf16_16816(o[2 * np], af, b0, b1);
+                    mma_bf16_16816(o[2 * np + 1], af, b2, b3);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
+                if (ur0 < n)
+                    *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur0) * a.H + h) * kD + cc) =
+                        pack_bf16x2(a.scale * o[j][0], a.scale * o[j][1]);
+                if (ur1 < n)
+                    *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur1) * a.H + h) * kD + cc) =
+                        pack_bf16x2(a.scale * o[j][2], a.scale * o[j][3]);
+            }
+        }
+        // st += Kc^T U (this warp's 16 rows of d_k, all 64 slice columns)
+#pragma unroll
+        for (int kk = 0; kk < kC / 16; ++kk) {
+            uint32_t af[4];
+            ldmatrix_x4_trans(stg + REC_KC + toff(kk * 16 + l7 + lb4 * 8, 16 * warp + lb3 * 8, 64), af[0],
+                              af[1], af[2], af[3]);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(sb + B_U + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64), b0, b1,
+                                  b2, b3);
+                mma_bf16_16816(st[2 * np], af, b0, b1);
+                mma_bf16_16816(st[2 * np + 1], af, b2, b3);
+            }
+        }
+        __syncthreads();  // stage s, M and U are free
+        if (tid == 0 && c + 2 < a.n_seg) issue(c + 2);
+    }
+    if (aborted_at >= 0) {
+        // a wait gave up: let this CTA's bulk copies in flight (chunks aborted_at and the one
+        // after it) finish, bounded; the state is left as it was at the start of this segment
+        if (tid == 0)
+            for (int c = aborted_at; c < aborted_at + 2 && c < a.n_seg; ++c)
+                (void)mbar_wait_bounded(smem_u32(&bars[c & 1]), (c >> 1) & 1);
+        return;
+    }
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int cc = col0 + nt * 8 + 2 * t4;
+        *reinterpret_cast<float2 *>(Mg + (size_t)sr0 * kD + cc) = make_float2(st[nt][0], st[nt][1]);
+        *reinterpret_cast<float2 *>(Mg + (size_t)sr1 * kD + cc) = make_float2(st[nt][2], st[nt][3]);
+    }
+}
+
+}  // namespace
+
+bool delta_prefill_scan_supported(int dk, int dv, bool bf16, int chunk) {
+    return bf16 && dk == kD && dv == kD && chunk == kC;
+}
+
+size_t delta_prefill_scan_record_bytes() { return REC_BYTES; }
+
+cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_t ws_bytes,
+                                      cudaStream_t s) {
+    static cudaError_t attr = [] {
+        cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_prep_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)B_SMEM);
+        return e;
+    }();
+    if (attr != cudaSuccess) return attr;
+    const long long bhs = (long long)a.B * a.H;
+    const int n_chunks = (a.T + kC - 1) / kC;
+    if (bhs <= 0 || n_chunks <= 0) return cudaSuccess;
+    const long long fit = (long long)(ws_bytes / ((size_t)bhs * REC_BYTES));
+    if (fit < 1 || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
+    const int seg = (int)std::min<long long>(n_chunks, fit);
+    PrefillScanArgs p;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.beta = a.beta; p.log_gate = a.log_gate;
+    p.state = a.state; p.slots = a.slots; p.n_slots = a.n_slots; p.o = a.o;
+    p.B = a.B; p.T = a.T; p.H = a.H; p.scale = a.scale; p.ws = ws;
+    for (int cb = 0; cb < n_chunks; cb += seg) {
+        p.chunk_begin = cb;
+        p.n_seg = std::min(seg, n_chunks - cb);
+        const unsigned grid_a = (unsigned)(bhs * p.n_seg);
+        if (a.kind == HMD_KDA)
+            prefill_prep_kernel<true><<<grid_a, kThreads, A_SMEM, s>>>(p);
+        else
+            prefill_prep_kernel<false><<<grid_a, kThreads, A_SMEM, s>>>(p);
+        prefill_scan_kernel<<<(unsigned)(bhs * kSplitV), kThreads, B_SMEM, s>>>(p);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+uint32_t delta_prefill_scan_read_errors(bool clear) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err, sizeof v) != cudaSuccess) return 0;
+    if (clear && v) {
+        const unsigned int z = 0;
+        cudaMemcpyToSymbol(g_err, &z, sizeof z);
+    }
+    return v;
+}
+
+}  // namespace hmd

@@ -8,7 +8,10 @@
 // their whole life, so a switch is a different placement array: nothing is copied.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
+#include <map>
+#include <mutex>
 #include <vector>
 
 #include "kernels.h"
@@ -85,7 +88,8 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
     if (!bits) return fail(HMD_ERR_ARG);
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
     *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
-            hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_mma_read_errors(clear != 0);
+            hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_mma_read_errors(clear != 0) |
+            hmd::delta_prefill_scan_read_errors(clear != 0);
     return HMD_OK;
 }
 
@@ -107,28 +111,131 @@ hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hm
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of the two-pass prefill when the caller passes none: a stream-ordered allocation from
+// a library-owned pool per device that keeps up to kPrefillPoolKeep bytes cached between calls.
+constexpr size_t kPrefillWsCap = size_t(1) << 30;   // per call: longer inputs run in segments
+constexpr uint64_t kPrefillPoolKeep = uint64_t(1) << 30;
+
+cudaMemPool_t prefill_pool() {
+    static std::mutex mu;
+    static std::map<int, cudaMemPool_t> pools;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = pools.find(dev);
+    if (it != pools.end()) return it->second;
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = kPrefillPoolKeep;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+    return pool;
+}
+
+hmd_status_t check_prefill(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                           hmd_dtype_t dtype, const void *q, const void *k, const void *v,
+                           const float *beta, const float *log_gate, const float *state,
+                           int n_slots, const int32_t *slots, const void *o, int chunk) {
+    if (kind != HMD_GDN && kind != HMD_KDA) return HMD_ERR_ARG;
+    if (dtype != HMD_F32 && dtype != HMD_BF16) return HMD_ERR_DTYPE;
+    if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || n_slots < 0 || chunk < 1)
+        return HMD_ERR_SHAPE;
+    if (B == 0 || T == 0) return HMD_OK;
+    if (!q || !k || !v || !beta || !log_gate || !state || !o) return HMD_ERR_ARG;
+    if (!slots && n_slots < B) return HMD_ERR_SHAPE;
+    if (!hmd::delta_prefill_supported(dk, dv, dtype == HMD_BF16, chunk)) return HMD_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
+        !aligned16(log_gate))
+        return HMD_ERR_ARG;
+    return HMD_OK;
+}
+
+hmd::DeltaPrefillArgs prefill_args(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                   hmd_dtype_t dtype, const void *q, const void *k, const void *v,
+                                   const float *beta, const float *log_gate, float *state,
+                                   int n_slots, const int32_t *slots, void *o, int chunk,
+                                   float scale) {
+    hmd::DeltaPrefillArgs a{};
+    a.kind = kind; a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
+    a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
+    a.n_slots = n_slots; a.slots = slots; a.o = o; a.chunk = chunk; a.scale = scale;
+    return a;
+}
+
+// bytes of one chunk record for every (sequence, head): the smallest usable workspace
+size_t prefill_min_ws(int B, int H) {
+    return (size_t)B * H * hmd::delta_prefill_scan_record_bytes();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t delta_rule_prefill_workspace_size(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                         hmd_dtype_t dtype, int chunk) {
+    (void)kind;
+    if (B < 1 || T < 1 || H < 1 || chunk < 1) return 0;
+    if (!hmd::delta_prefill_scan_supported(dk, dv, dtype == HMD_BF16, chunk)) return 0;
+    const size_t n_chunks = (size_t)(T + chunk - 1) / chunk;
+    return prefill_min_ws(B, H) * n_chunks;
+}
+
+hmd_status_t delta_rule_prefill_chunked_ws(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                           hmd_dtype_t dtype, const void *q, const void *k,
+                                           const void *v, const float *beta,
+                                           const float *log_gate, float *state, int n_slots,
+                                           const int32_t *slots, void *o, int chunk, float scale,
+                                           void *workspace, size_t ws_bytes,
+                                           hmd_stream_t stream) {
+    const hmd_status_t st = check_prefill(kind, B, T, H, dk, dv, dtype, q, k, v, beta, log_gate,
+                                          state, n_slots, slots, o, chunk);
+    if (st != HMD_OK) return fail(st);
+    if (B == 0 || T == 0) return HMD_OK;
+    const hmd::DeltaPrefillArgs a = prefill_args(kind, B, T, H, dk, dv, dtype, q, k, v, beta,
+                                                 log_gate, state, n_slots, slots, o, chunk, scale);
+    if (!hmd::delta_prefill_scan_supported(dk, dv, dtype == HMD_BF16, chunk))
+        return from_cuda(hmd::launch_delta_prefill(a, as_stream(stream)));
+    if (!workspace || !aligned16(workspace)) return fail(HMD_ERR_ARG);
+    if (ws_bytes < prefill_min_ws(B, H)) return fail(HMD_ERR_SHAPE);
+    return from_cuda(hmd::launch_delta_prefill_scan(a, workspace, ws_bytes, as_stream(stream)));
+}
+
 hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
                                         hmd_dtype_t dtype, const void *q, const void *k,
                                         const void *v, const float *beta, const float *log_gate,
                                         float *state, int n_slots, const int32_t *slots, void *o,
                                         int chunk, float scale, hmd_stream_t stream) {
-    if (kind != HMD_GDN && kind != HMD_KDA) return fail(HMD_ERR_ARG);
-    if (dtype != HMD_F32 && dtype != HMD_BF16) return fail(HMD_ERR_DTYPE);
-    if (B < 0 || T < 0 || H < 1 || dk < 1 || dv < 1 || n_slots < 0 || chunk < 1)
-        return fail(HMD_ERR_SHAPE);
+    const hmd_status_t st = check_prefill(kind, B, T, H, dk, dv, dtype, q, k, v, beta, log_gate,
+                                          state, n_slots, slots, o, chunk);
+    if (st != HMD_OK) return fail(st);
     if (B == 0 || T == 0) return HMD_OK;
-    if (!q || !k || !v || !beta || !log_gate || !state || !o) return fail(HMD_ERR_ARG);
-    if (!slots && n_slots < B) return fail(HMD_ERR_SHAPE);
-    if (!hmd::delta_prefill_supported(dk, dv, dtype == HMD_BF16, chunk))
-        return fail(HMD_ERR_UNSUPPORTED);
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state) ||
-        !aligned16(log_gate))
-        return fail(HMD_ERR_ARG);
-    hmd::DeltaPrefillArgs a{};
-    a.kind = kind; a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
-    a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
-    a.n_slots = n_slots; a.slots = slots; a.o = o; a.chunk = chunk; a.scale = scale;
-    return from_cuda(hmd::launch_delta_prefill(a, as_stream(stream)));
+    const hmd::DeltaPrefillArgs a = prefill_args(kind, B, T, H, dk, dv, dtype, q, k, v, beta,
+                                                 log_gate, state, n_slots, slots, o, chunk, scale);
+    if (!hmd::delta_prefill_scan_supported(dk, dv, dtype == HMD_BF16, chunk))
+        return from_cuda(hmd::launch_delta_prefill(a, as_stream(stream)));
+    const size_t full = delta_rule_prefill_workspace_size(kind, B, T, H, dk, dv, dtype, chunk);
+    const size_t bytes = full <= kPrefillWsCap ? full : std::max(prefill_min_ws(B, H), kPrefillWsCap);
+    cudaMemPool_t pool = prefill_pool();
+    if (!pool) return fail(HMD_ERR_CUDA);
+    const cudaStream_t s = as_stream(stream);
+    void *ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, bytes, pool, s) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HMD_ERR_OOM);
+    }
+    const cudaError_t e = hmd::launch_delta_prefill_scan(a, ws, bytes, s);
+    const cudaError_t f = cudaFreeAsync(ws, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(f);
 }
 
 // ---- attention mixers --------------------------------------------------------------------

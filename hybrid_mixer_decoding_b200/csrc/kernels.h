@@ -76,5 +76,28 @@ bool delta_prefill_mma_supported(int dk, int dv, bool bf16, int chunk);
 cudaError_t launch_delta_prefill_mma(const DeltaPrefillArgs &a, cudaStream_t s);
 uint32_t delta_prefill_mma_read_errors(bool clear);
 
+// two-pass tensor-core path (bf16, d_k = d_v = 128, chunk 64): a chunk-parallel pass writes one
+// record per chunk to a workspace, a scan pass carries the state through the chunks
+struct PrefillScanArgs {
+    const void *q, *k, *v;
+    const float *beta, *log_gate;
+    float *state;
+    const int32_t *slots;
+    int n_slots;
+    void *o;
+    int B, T, H;
+    float scale;
+    void *ws;         // records [B*H][n_seg][record bytes]
+    int chunk_begin;  // first chunk of this segment
+    int n_seg;        // chunks in this segment
+};
+bool delta_prefill_scan_supported(int dk, int dv, bool bf16, int chunk);
+size_t delta_prefill_scan_record_bytes();
+// Runs the sequence in segments of as many chunks as ws_bytes holds for all B*H heads
+// (cudaErrorInvalidValue if not even one chunk fits or ws is not 16-byte aligned).
+cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_t ws_bytes,
+                                      cudaStream_t s);
+uint32_t delta_prefill_scan_read_errors(bool clear);
+
 
 }  // namespace hmd

@@ -92,14 +92,41 @@ HMD_API hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, in
  *   state [n_slots][H][dk][dv] fp32: read as the initial state and overwritten with the final
  *   one (slot slots[b], or b when slots == NULL).
  *   chunk: tokens per chunk; 64 is the supported value. T need not be a multiple of it.
- * Supported: bf16 with dk = dv = 128 on the tensor-core path; fp32 or other sizes (dk, dv in
- * {16..128}, multiples of 16) on the CUDA-core path. q, k, v, o, log_gate and state must be
- * 16-byte aligned (HMD_ERR_ARG otherwise).                                                     */
+ * Supported: bf16 with dk = dv = 128 and chunk 64 on the tensor-core path; fp32 or other
+ * sizes (dk, dv in {16..128}, multiples of 16) on the CUDA-core path. q, k, v, o, log_gate and
+ * state must be 16-byte aligned (HMD_ERR_ARG otherwise).
+ * The tensor-core path runs in two passes that exchange one record per chunk and head through
+ * device scratch (delta_rule_prefill_workspace_size bytes for the whole input). This entry point
+ * takes that scratch, up to 1 GiB per call (longer inputs run in segments), as a stream-ordered
+ * allocation from a pool the library keeps per device (up to 1 GiB stays cached between calls);
+ * HMD_ERR_OOM if it cannot. Under stream capture, or to own the memory, call
+ * delta_rule_prefill_chunked_ws instead.                                                       */
 HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
                                         hmd_dtype_t dtype, const void *q, const void *k,
                                         const void *v, const float *beta, const float *log_gate,
                                         float *state, int n_slots, const int32_t *slots, void *o,
                                         int chunk, float scale, hmd_stream_t stream);
+
+/* Scratch bytes for delta_rule_prefill_chunked_ws to run these sizes in one segment: one record
+ * (90,624 bytes at dk = dv = 128, chunk 64) per chunk and (sequence, head). 0 when the call
+ * needs no scratch (the CUDA-core path) or the sizes are empty or invalid.                    */
+HMD_API size_t delta_rule_prefill_workspace_size(hmd_kind_t kind, int B, int T, int H, int dk,
+                                                 int dv, hmd_dtype_t dtype, int chunk);
+
+/* delta_rule_prefill_chunked with caller-owned scratch: `workspace` (device, 16-byte aligned)
+ * of ws_bytes. Any size from one chunk's records for all B*H heads up works; with less than
+ * delta_rule_prefill_workspace_size(...) bytes the call runs the sequence in segments of as many
+ * chunks as fit (same results, bit for bit). HMD_ERR_SHAPE if not even one chunk fits. The
+ * scratch must not be in use by another call while this one runs. Allocates nothing, so it
+ * can be captured in a CUDA graph. Paths that need no scratch ignore workspace and ws_bytes. */
+HMD_API hmd_status_t delta_rule_prefill_chunked_ws(hmd_kind_t kind, int B, int T, int H, int dk,
+                                                   int dv, hmd_dtype_t dtype, const void *q,
+                                                   const void *k, const void *v,
+                                                   const float *beta, const float *log_gate,
+                                                   float *state, int n_slots,
+                                                   const int32_t *slots, void *o, int chunk,
+                                                   float scale, void *workspace,
+                                                   size_t ws_bytes, hmd_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------ */
 /* Attention mixers (FA, SWA) over a paged bf16 KV cache.                                     */

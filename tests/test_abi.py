@@ -70,6 +70,28 @@ def test_prefill_validation():
     assert _prefill(T=0) == 0
 
 
+def _prefill_ws(ws, ws_bytes, B=2, T=300, H=3, dtype=hmd.BF16, dk=128):
+    return hmd.lib().delta_rule_prefill_chunked_ws(hmd.GDN, B, T, H, dk, dk, dtype, FAKE, FAKE,
+                                                   FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, 64,
+                                                   1.0, ws, ws_bytes, None)
+
+
+def test_prefill_workspace_size_and_validation():
+    f = hmd.delta_rule_prefill_workspace_size
+    rec = 90624  # Qt, -W, Kc (bf16 64x128), P (bf16 64x64), e^{G_C} (128 fp32), Ut (fp32 64x128)
+    assert rec == 3 * 64 * 128 * 2 + 64 * 64 * 2 + 128 * 4 + 64 * 128 * 4
+    assert f(hmd.KDA, 4, 4096, 16, 128, 128, hmd.BF16, 64) == 4 * 16 * 64 * rec
+    assert f(hmd.GDN, 2, 65, 3, 128, 128, hmd.BF16, 64) == 2 * 3 * 2 * rec   # ragged: 2 chunks
+    assert f(hmd.GDN, 2, 65, 3, 64, 64, hmd.BF16, 64) == 0     # CUDA-core path: no scratch
+    assert f(hmd.GDN, 2, 65, 3, 128, 128, hmd.F32, 64) == 0
+    assert f(hmd.GDN, 0, 65, 3, 128, 128, hmd.BF16, 64) == 0
+    one = 2 * 3 * rec                                          # one chunk for all heads
+    assert _prefill_ws(None, one) == ARG                       # tensor-core path needs scratch
+    assert _prefill_ws(FAKE + 8, one) == ARG                   # not 16-byte aligned
+    assert _prefill_ws(FAKE, one - 16) == SHAPE                # not even one chunk fits
+    assert _prefill_ws(FAKE, one, T=0) == 0                    # nothing to do
+
+
 def _attn(kind=hmd.FA, window=0, B=2, Hq=8, Hkv=2, d=128, PT=64, max_pages=4, max_len=256,
           ws=1 << 30, ptr=FAKE, n_pages=16):
     return hmd.lib().attn_decode(kind, window, B, Hq, Hkv, d, PT, ptr, ptr, ptr, ptr, ptr, n_pages,

@@ -109,3 +109,34 @@ def test_prefill_bad_slot_sets_device_error():
     hmd.delta_rule_prefill_chunked(I.KDA, _dev(d.q, bf), _dev(d.k, bf), _dev(d.v, bf),
                                    _dev(d.beta), _dev(d.log_gate), state, o, slots=slots)
     assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_SLOT
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_caller_workspace_segments_are_bit_exact(oracle_mod, kind):
+    """delta_rule_prefill_chunked_ws with scratch for one chunk (5 segments of T=300) and for two
+    chunks (3 segments, the last ragged) gives the same bits as the one-segment call, and both
+    match the recurrence."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 2, 300, 3, 128, 128, dtype="bf16", seed=40, state0="randn")
+    bf = torch.bfloat16
+    args = (_dev(d.q, bf), _dev(d.k, bf), _dev(d.v, bf), _dev(d.beta), _dev(d.log_gate))
+    full = hmd.delta_rule_prefill_workspace_size(kind, 2, 300, 3, 128, 128, hmd.BF16, 64)
+    one = full // 5
+    results = []
+    for ws_bytes in (None, one, 2 * one, full):
+        state = _dev(d.state0)
+        o = torch.empty(2, 300, 3, 128, device="cuda", dtype=bf)
+        if ws_bytes is None:
+            hmd.delta_rule_prefill_chunked(kind, *args, state, o)
+        else:
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+            hmd.delta_rule_prefill_chunked_ws(kind, *args, state, o, ws)
+        torch.cuda.synchronize()
+        results.append((o, state))
+    assert hmd.hmd_device_errors(clear=True) == 0
+    for o, state in results[1:]:
+        assert torch.equal(o, results[0][0])
+        assert torch.equal(state, results[0][1])
+    o_ref, st_ref = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    assert O.rel_err(results[0][0].float().cpu().numpy(), o_ref) < 2e-2
+    assert O.rel_err(results[0][1].cpu().numpy(), st_ref) < 2e-2
