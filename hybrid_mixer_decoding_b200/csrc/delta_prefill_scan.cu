@@ -18,7 +18,7 @@
 // ldmatrix), e^{G_C} and Ut (fp32).
 // Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks in
 // order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
-// the previous chunk computes; the state half lives in registers as MMA accumulator fragments.
+// the chunk before it computes; the state half lives in registers as MMA accumulator fragments.
 // Per chunk it does only the state-dependent products (U, O, state update): 7.3 MFLOP of the
 // chunk's 11.5 per head, split over two CTAs.
 #include <cuda_runtime.h>
@@ -36,7 +36,8 @@ __device__ unsigned int g_err;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;       // pass B
+constexpr int kPrepThreads = 256;   // pass A: 8 warps, two CTAs per SM
 constexpr int kSplitV = 2;             // pass B: CTAs per (sequence, head), each d_v / 2 columns
 constexpr int kDV = kD / kSplitV;      // 64 columns of d_v per pass-B CTA
 
@@ -47,31 +48,31 @@ constexpr uint32_t REC_KC = 32768;     // Kc  bf16 [64][128]
 constexpr uint32_t REC_P = 49152;      // P   bf16 [64][64]
 constexpr uint32_t REC_GAM = 57344;    // e^{G_C} fp32 [128]
 constexpr uint32_t REC_HEAD = 57856;   // bytes above, moved by one bulk copy
-constexpr uint32_t REC_UT = 57856;     // Ut  fp32 [64][128] row-major
+constexpr uint32_t REC_UT = 57856;     // Ut  fp32 [64][128], rows of 128 words (see ut_idx)
 constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 4;  // 90624
 static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
 
 // ---- pass A shared memory (bytes from a 1024-aligned base) ---------------------------------
-constexpr uint32_t A_KT = 0;           // Kt  [64][128]
-constexpr uint32_t A_QT = 16384;       // q, then Qt  [64][128]
-constexpr uint32_t A_KH = 32768;       // k, then Kh  [64][128]
-constexpr uint32_t A_V = 49152;        // V   [64][128]
-constexpr uint32_t A_AS = 65536;       // A fp32 [64][68]; after the solve: T bf16 [64][64]
+constexpr uint32_t A_KT = 0;           // Kt [64][128]; at the end -W (bf16, record layout)
+constexpr uint32_t A_QT = 16384;       // q, then Qt [64][128]
+constexpr uint32_t A_KH = 32768;       // k, then Kh [64][128]; then P + e^{G_C}; at the end
+constexpr uint32_t A_V = 49152;        //   Ut fp32 across Kh and V (32 KiB, record layout)
+constexpr uint32_t A_G = 65536;        // KDA log-gates -> in-chunk prefix, fp32 [64][128]
+constexpr uint32_t A_AS = 65536;       // after the gate pass: A fp32 [64][68], then T bf16
 constexpr uint32_t A_XS = 82944;       // X fp32 [64][68]
 constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
 constexpr uint32_t A_SMALL = 104192;
-constexpr uint32_t A_SMEM = A_SMALL + 3072 + 1024;
-constexpr uint32_t A_LG = A_AS;        // KDA raw log-gates fp32 [64][128] (before A exists)
+constexpr uint32_t A_SMEM = A_SMALL + 3584 + 1024;
 constexpr uint32_t A_T = A_AS;
 constexpr int AS_LD = 68;
 constexpr int YS_LD = 20;
-static_assert(A_LG + kC * kD * 4 <= A_YS, "log-gate staging fits the A/X region");
+static_assert(A_G + kC * kD * 4 <= A_YS, "log-gate staging fits the A/X region");
 
 // ---- pass B shared memory ----------------------------------------------------------------
-constexpr uint32_t B_STAGE = 58368;    // one record head, padded to 1 KiB
-constexpr uint32_t B_M = 2 * B_STAGE;  // M bf16 [128][64]
-constexpr uint32_t B_U = B_M + 16384;  // U bf16 [64][64]
-constexpr uint32_t B_BAR = B_U + 8192;
+constexpr uint32_t B_STAGE = 58368;        // one record head, padded to 1 KiB
+constexpr uint32_t B_M = 2 * B_STAGE;      // M bf16 [128][64], two buffers (chunk parity)
+constexpr uint32_t B_U = B_M + 2 * 16384;  // U bf16 [64][64], two buffers
+constexpr uint32_t B_BAR = B_U + 2 * 8192;
 constexpr uint32_t B_SMEM = B_BAR + 64 + 1024;
 
 // byte offset of element (row, col) of a tile whose halves (64 columns each) hold `rows` rows
@@ -79,6 +80,10 @@ __device__ __forceinline__ uint32_t toff(int row, int col, int rows) {
     return (uint32_t)((col >> 6) * rows * 128 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
                       ((col & 7) << 1));
 }
+
+// word index of fp32 element (row, col) of the Ut block: rows of 128 words, the 8-word groups
+// XOR-permuted by row so that a warp's (row, even column) fragment stores hit distinct banks
+__device__ __forceinline__ int ut_idx(int row, int col) { return row * kD + (col ^ ((row & 7) << 3)); }
 
 __device__ __forceinline__ void st_bf16x2(uint8_t *base, uint32_t off, float lo, float hi) {
     *reinterpret_cast<uint32_t *>(base + off) = pack_bf16x2(lo, hi);
@@ -89,23 +94,86 @@ __device__ __forceinline__ uint8_t *record(const PrefillScanArgs &a, int bh, int
 }
 
 // ================================ pass A ==================================================
+constexpr int pow2_floor(int x) { return x >= 2 ? 2 * pow2_floor(x / 2) : 1; }
+
+// One level of the blocked inverse X = (I + A)^-1 (16x16 blocks): the blocks (i, j) with
+// i - j = L. Y_ij = sum_{k=j}^{i-1} A_ik X_kj, then X_ij = -X_ii Y_ij. Each (block, row,
+// 4-column group) is shared by as many threads as the block has to spare (a power of two);
+// they split the sums and combine them by shuffles.
+template <int L>
+__device__ __forceinline__ void solve_level(const float *As, float *Xs, float *Ys, int tid) {
+    constexpr int NB = 4 - L;                                  // blocks on this diagonal
+    constexpr int TPI = pow2_floor(kPrepThreads / (NB * 64));  // threads per (block, row, group)
+    constexpr int KPT = 16 * L / TPI;  // terms of Y per thread
+    constexpr int XPT = 16 / TPI;      // terms of X_ii Y_ij per thread
+    const bool active = tid < NB * 64 * TPI;  // whole warps
+    const int item = tid / TPI, part = tid % TPI;
+    const int j = item >> 6, r = (item >> 2) & 15, cg = item & 3, i = j + L;
+    if (active) {
+        const float *arow = As + (i * 16 + r) * AS_LD;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int kk = 0; kk < KPT; ++kk) {
+            const int k = j * 16 + part * KPT + kk;
+            const float av = arow[k];
+            const float4 xv = *reinterpret_cast<const float4 *>(Xs + k * AS_LD + j * 16 + cg * 4);
+            acc.x += av * xv.x; acc.y += av * xv.y; acc.z += av * xv.z; acc.w += av * xv.w;
+        }
+#pragma unroll
+        for (int m = 1; m < TPI; m <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+        }
+        if (part == 0) *reinterpret_cast<float4 *>(Ys + (j * 16 + r) * YS_LD + cg * 4) = acc;
+    }
+    __syncthreads();
+    if (active) {
+        const float *xrow = Xs + (i * 16 + r) * AS_LD + i * 16;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int ss = 0; ss < XPT; ++ss) {
+            const int s2 = part * XPT + ss;
+            const float xv = s2 <= r ? xrow[s2] : 0.f;  // X_ii is lower triangular
+            const float4 yv = *reinterpret_cast<const float4 *>(Ys + (j * 16 + s2) * YS_LD + cg * 4);
+            acc.x += xv * yv.x; acc.y += xv * yv.y; acc.z += xv * yv.z; acc.w += xv * yv.w;
+        }
+#pragma unroll
+        for (int m = 1; m < TPI; m <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+        }
+        if (part == 0)
+            *reinterpret_cast<float4 *>(Xs + (i * 16 + r) * AS_LD + j * 16 + cg * 4) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    __syncthreads();
+}
+
 template <bool KDA>
-__global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const PrefillScanArgs a) {
+__global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const PrefillScanArgs a) {
+    constexpr int NT = kPrepThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
+    float *Gs = reinterpret_cast<float *>(sm + A_G);
     float *As = reinterpret_cast<float *>(sm + A_AS);
     float *Xs = reinterpret_cast<float *>(sm + A_XS);
     float *Ys = reinterpret_cast<float *>(sm + A_YS);
     float *sbeta = reinterpret_cast<float *>(sm + A_SMALL);  // [64]
-    float *hsum = sbeta + 64;                                 // [2][128] half-chunk gate sums
-    float *lgp = hsum + 256;                                  // [64] GDN log-gate prefix
-    float *etok = lgp + 64;                                   // [64] GDN e^G
-    float *ietok = etok + 64;                                 // [64] GDN e^-G
-    float *wsum = ietok + 64;                                 // [2]
-    float *gam = wsum + 2;                                    // [128] e^{G_C}
+    float *qoff = sbeta + 64;                                 // [NQ][128] KDA: gate sums of
+                                                              //   the row parts, then their
+                                                              //   exclusive prefix
+    float *lgp = qoff + 512;                                  // [64] GDN log-gate prefix
+    float *wsum = lgp + 64;                                   // [2]
+    float *egc = wsum + 2;                                    // [128] e^{G_C}
 
+    constexpr int NQ = NT / kD;       // KDA gate prefix: row parts per channel
+    constexpr int RPQ = kC / NQ;      // rows per part
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     const int l7 = lane & 7, lb3 = (lane >> 3) & 1, lb4 = lane >> 4;
@@ -121,11 +189,13 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
 
     // ---- stage q (into the Qt slot), k (into the Kh slot), v, KDA log-gates; beta ----------
     {
+        constexpr int J16 = kC * kD / 8 / NT;  // 16-byte pieces of a bf16 tile per thread
+        constexpr int JG = kC * kD / 4 / NT;   // float4 pieces of the KDA gate tile per thread
         const size_t row0 = ((size_t)b * T + t0) * a.H + h;  // token t0's row in [B][T][H]
-        uint4 qv[4], kv[4], vv[4];
+        uint4 qv[J16], kv[J16], vv[J16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int idx = tid + j * kThreads, r = idx >> 4, ch = idx & 15;
+        for (int j = 0; j < J16; ++j) {
+            const int idx = tid + j * NT, r = idx >> 4, ch = idx & 15;
             qv[j] = kv[j] = vv[j] = make_uint4(0, 0, 0, 0);
             if (r < n) {
                 const size_t off = (row0 + (size_t)r * a.H) * kD + ch * 8;
@@ -134,19 +204,19 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
                 vv[j] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
             }
         }
-        float4 gv[8];
+        float4 gv[JG];
         if constexpr (KDA) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int idx = tid + j * kThreads, r = idx >> 5, c4 = idx & 31;
+            for (int j = 0; j < JG; ++j) {
+                const int idx = tid + j * NT, r = idx >> 5, c4 = idx & 31;
                 gv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (r < n)
                     gv[j] = __ldg(reinterpret_cast<const float4 *>(a.log_gate + (row0 + (size_t)r * a.H) * kD + c4 * 4));
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int idx = tid + j * kThreads, r = idx >> 4, ch = idx & 15;
+        for (int j = 0; j < J16; ++j) {
+            const int idx = tid + j * NT, r = idx >> 4, ch = idx & 15;
             const uint32_t o = toff(r, ch * 8, 64);
             *reinterpret_cast<uint4 *>(sm + A_QT + o) = qv[j];
             *reinterpret_cast<uint4 *>(sm + A_KH + o) = kv[j];
@@ -154,9 +224,9 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
         }
         if constexpr (KDA) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int idx = tid + j * kThreads, r = idx >> 5, c4 = idx & 31;
-                *reinterpret_cast<float4 *>(sm + A_LG + r * 512 + c4 * 16) = gv[j];
+            for (int j = 0; j < JG; ++j) {
+                const int idx = tid + j * NT, r = idx >> 5, c4 = idx & 31;
+                *reinterpret_cast<float4 *>(Gs + r * kD + c4 * 4) = gv[j];
             }
         }
         if (tid < kC) {
@@ -176,101 +246,132 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
     }
     __syncthreads();
 
-    // ---- gate pass: Kt, Qt, Kh (shared memory), Kc (record), e^{G_C}; thread = (channel,
-    //      half of the chunk's rows) ------------------------------------------------------------
-    {
-        const int i = tid & (kD - 1), hf = tid >> 7;
-        const float *lgs = reinterpret_cast<const float *>(sm + A_LG) + i;
-        if constexpr (KDA) {
-            float part = 0.f;
-#pragma unroll 8
-            for (int r = 32 * hf; r < 32 * hf + 32; ++r) part += lgs[r * kD];
-            hsum[hf * kD + i] = part;
-        } else {
-            if (tid < kC) {
-                const float gc = lgp[tid] + (warp == 1 ? wsum[0] : 0.f);
-                lgp[tid] = gc;
-                etok[tid] = expf(gc);
-                ietok[tid] = expf(-gc);
-            }
+    // ---- gate prefix G (log domain): KDA per channel in place within NQ row parts, plus the
+    //      parts' exclusive prefix; GDN per token -------------------------------------------------
+    if constexpr (KDA) {
+        const int i = tid & (kD - 1), qr = tid >> 7;
+        float run = 0.f;
+#pragma unroll
+        for (int r = RPQ * qr; r < RPQ * qr + RPQ; ++r) {
+            run += Gs[r * kD + i];
+            Gs[r * kD + i] = run;
         }
+        qoff[qr * kD + i] = run;
         __syncthreads();
-        const float gC = KDA ? hsum[i] + hsum[kD + i] : lgp[kC - 1];
-        float gsum = KDA ? (hf ? hsum[i] : 0.f) : 0.f;
-        uint8_t *kc = rec + REC_KC;
-#pragma unroll 4
-        for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
-            float e, ie, gr;
-            if constexpr (KDA) {
-                gsum += lgs[r * kD];
-                gr = gsum;
-                e = expf(gsum);
-                ie = expf(-gsum);
-            } else {
-                gr = lgp[r];
-                e = etok[r];
-                ie = ietok[r];
+        if (qr == 0) {
+            float acc = 0.f;
+#pragma unroll
+            for (int q2 = 0; q2 < NQ; ++q2) {
+                const float part = qoff[q2 * kD + i];
+                qoff[q2 * kD + i] = acc;
+                acc += part;
             }
-            const uint32_t o = toff(r, i, 64);
-            const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + A_KH + o));
-            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + A_QT + o));
-            *reinterpret_cast<__nv_bfloat16 *>(sm + A_KT + o) = __float2bfloat16_rn(kv * e);
-            *reinterpret_cast<__nv_bfloat16 *>(sm + A_QT + o) = __float2bfloat16_rn(qv * e);
-            *reinterpret_cast<__nv_bfloat16 *>(sm + A_KH + o) = __float2bfloat16_rn(kv * ie);
-            *reinterpret_cast<__nv_bfloat16 *>(kc + o) = __float2bfloat16_rn(kv * expf(gC - gr));
+            egc[i] = __expf(acc);
         }
-        if (hf == 1) gam[i] = expf(gC);
+    } else {
+        if (tid < kC) lgp[tid] += (warp == 1 ? wsum[0] : 0.f);
+        __syncthreads();
+        if (tid < kD) egc[tid] = __expf(lgp[kC - 1]);
     }
     __syncthreads();
-    // Qt -> record (16-byte copies); e^{G_C} -> record
+
+    // ---- gate factors, 8 channels of one row per item: Kt, Qt, Kh (shared memory), Kc -------
+    //      (record), with e^{G_C - G} = e^{G_C} e^-G <= 1
     {
-        const uint4 *src = reinterpret_cast<const uint4 *>(sm + A_QT);
-        uint4 *dst = reinterpret_cast<uint4 *>(rec + REC_QT);
+        uint8_t *kc = rec + REC_KC;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) dst[tid + j * kThreads] = src[tid + j * kThreads];
-        if (tid < kD) reinterpret_cast<float *>(rec + REC_GAM)[tid] = gam[tid];
+        for (int j = 0; j < kC * kD / 8 / NT; ++j) {
+            const int idx = tid + j * NT, r = idx >> 4, c0 = (idx & 15) * 8;
+            const uint32_t o = toff(r, c0, 64);
+            const uint4 qr = *reinterpret_cast<const uint4 *>(sm + A_QT + o);
+            const uint4 kr = *reinterpret_cast<const uint4 *>(sm + A_KH + o);
+            float G[8];
+            if constexpr (KDA) {
+                const float4 g0 = *reinterpret_cast<const float4 *>(Gs + r * kD + c0);
+                const float4 g1 = *reinterpret_cast<const float4 *>(Gs + r * kD + c0 + 4);
+                const float4 f0 = *reinterpret_cast<const float4 *>(qoff + (r / RPQ) * kD + c0);
+                const float4 f1 = *reinterpret_cast<const float4 *>(qoff + (r / RPQ) * kD + c0 + 4);
+                G[0] = g0.x + f0.x; G[1] = g0.y + f0.y; G[2] = g0.z + f0.z; G[3] = g0.w + f0.w;
+                G[4] = g1.x + f1.x; G[5] = g1.y + f1.y; G[6] = g1.z + f1.z; G[7] = g1.w + f1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) G[e] = lgp[r];
+            }
+            const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w};
+            const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+            uint32_t kt[4], qt[4], kh[4], kcw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float ea = __expf(G[2 * e]), eb = __expf(G[2 * e + 1]);
+                const float ia = __expf(-G[2 * e]), ib = __expf(-G[2 * e + 1]);
+                const float ka = bf16_lo(kw[e]), kb = bf16_hi(kw[e]);
+                const float qa = bf16_lo(qw[e]), qb = bf16_hi(qw[e]);
+                kt[e] = pack_bf16x2(ka * ea, kb * eb);
+                qt[e] = pack_bf16x2(qa * ea, qb * eb);
+                kh[e] = pack_bf16x2(ka * ia, kb * ib);
+                kcw[e] = pack_bf16x2(ka * (egc[c0 + 2 * e] * ia), kb * (egc[c0 + 2 * e + 1] * ib));
+            }
+            *reinterpret_cast<uint4 *>(sm + A_KT + o) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+            *reinterpret_cast<uint4 *>(sm + A_QT + o) = make_uint4(qt[0], qt[1], qt[2], qt[3]);
+            *reinterpret_cast<uint4 *>(sm + A_KH + o) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
+            *reinterpret_cast<uint4 *>(kc + o) = make_uint4(kcw[0], kcw[1], kcw[2], kcw[3]);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {  // Qt -> record
+        bulk_store(rec + REC_QT, sb + A_QT, 16384);
+        bulk_commit_group();
     }
 
-    // ---- A (warps 0-3) and P (warps 4-7), 16 rows each: [Kt | Qt] Kh^T ----------------------
+    // ---- A and P: [Kt | Qt] Kh^T; each warp 16 rows x (64 / NH) columns -------------------
     {
-        const int mat = warp >> 2, rt = warp & 3;
+        constexpr int NH = NT / 256;  // warps per 16-row strip of A or P
+        constexpr int NP = 4 / NH;    // 16-column pairs per warp (n-tiles = 2 NP)
+        const int mat = warp / (4 * NH), rt = (warp / NH) & 3, nh = warp % NH;
         const uint32_t abase = sb + (mat ? A_QT : A_KT);
-        float acc[8][4];
+        float acc[2 * NP][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        for (int i = 0; i < 2 * NP; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
             uint32_t af[4];
             ldmatrix_x4(abase + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
                         af[2], af[3]);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
+            for (int np = 0; np < NP; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(sb + A_KH + toff(np * 16 + l7 + lb4 * 8, kk * 16 + lb3 * 8, 64), b0, b1,
-                            b2, b3);
+                ldmatrix_x4(sb + A_KH + toff(16 * NP * nh + np * 16 + l7 + lb4 * 8, kk * 16 + lb3 * 8, 64),
+                            b0, b1, b2, b3);
                 mma_bf16_16816(acc[2 * np], af, b0, b1);
                 mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
             }
         }
+        __syncthreads();  // Kh is read by every warp above; P and e^{G_C} take its place below
         const int r0 = 16 * rt + g, r1 = r0 + 8;
-        uint8_t *pr = rec + REC_P;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int s0 = nt * 8 + 2 * t4;
+        for (int nt = 0; nt < 2 * NP; ++nt) {
+            const int s0 = 16 * NP * nh + nt * 8 + 2 * t4;
             if (mat == 0) {
                 As[r0 * AS_LD + s0] = (s0 < r0 && r0 < n) ? sbeta[r0] * acc[nt][0] : 0.f;
                 As[r0 * AS_LD + s0 + 1] = (s0 + 1 < r0 && r0 < n) ? sbeta[r0] * acc[nt][1] : 0.f;
                 As[r1 * AS_LD + s0] = (s0 < r1 && r1 < n) ? sbeta[r1] * acc[nt][2] : 0.f;
                 As[r1 * AS_LD + s0 + 1] = (s0 + 1 < r1 && r1 < n) ? sbeta[r1] * acc[nt][3] : 0.f;
             } else {
-                st_bf16x2(pr, toff(r0, s0, 64), (s0 <= r0 && r0 < n) ? acc[nt][0] : 0.f,
+                st_bf16x2(sm + A_KH, toff(r0, s0, 64), (s0 <= r0 && r0 < n) ? acc[nt][0] : 0.f,
                           (s0 + 1 <= r0 && r0 < n) ? acc[nt][1] : 0.f);
-                st_bf16x2(pr, toff(r1, s0, 64), (s0 <= r1 && r1 < n) ? acc[nt][2] : 0.f,
+                st_bf16x2(sm + A_KH, toff(r1, s0, 64), (s0 <= r1 && r1 < n) ? acc[nt][2] : 0.f,
                           (s0 + 1 <= r1 && r1 < n) ? acc[nt][3] : 0.f);
             }
         }
+        if (tid < kD) reinterpret_cast<float *>(sm + A_KH + 8192)[tid] = egc[tid];
     }
+    fence_proxy_async_smem();
     __syncthreads();
+    if (tid == 0) {  // P and e^{G_C} (contiguous in the record) -> record
+        bulk_store(rec + REC_P, sb + A_KH, 8192 + 512);
+        bulk_commit_group();
+    }
 
     // ---- X = (I + A)^-1 (16x16 blocks, fp32), T = X Diag(beta) ----------------------------
     if (tid < 64) {  // diagonal blocks by forward substitution, one column per thread
@@ -281,43 +382,17 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
         for (int r = 0; r < 16; ++r) {
             float acc = 0.f;
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc += ab[r * AS_LD + s] * x[s];
+            for (int s2 = 0; s2 < r; ++s2) acc += ab[r * AS_LD + s2] * x[s2];
             x[r] = r < c0 ? 0.f : (r == c0 ? 1.f : -acc);
             Xs[(bi * 16 + r) * AS_LD + bi * 16 + c0] = x[r];
         }
     }
     __syncthreads();
-#pragma unroll 1
-    for (int L = 1; L < 4; ++L) {
-        const int nb = 4 - L;  // blocks (i, j) with i - j = L
-        for (int it = tid; it < nb * 64; it += kThreads) {  // Y_ij = sum_{k=j}^{i-1} A_ik X_kj
-            const int j = it >> 6, r = (it >> 2) & 15, cg = it & 3, i = j + L;
-            const float *arow = As + (i * 16 + r) * AS_LD;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = j * 16; k < i * 16; ++k) {
-                const float av = arow[k];
-                const float4 xv = *reinterpret_cast<const float4 *>(Xs + k * AS_LD + j * 16 + cg * 4);
-                acc.x += av * xv.x; acc.y += av * xv.y; acc.z += av * xv.z; acc.w += av * xv.w;
-            }
-            *reinterpret_cast<float4 *>(Ys + (j * 16 + r) * YS_LD + cg * 4) = acc;
-        }
-        __syncthreads();
-        for (int it = tid; it < nb * 64; it += kThreads) {  // X_ij = -X_ii Y_ij
-            const int j = it >> 6, r = (it >> 2) & 15, cg = it & 3, i = j + L;
-            const float *xrow = Xs + (i * 16 + r) * AS_LD + i * 16;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s <= r; ++s) {
-                const float xv = xrow[s];
-                const float4 yv = *reinterpret_cast<const float4 *>(Ys + (j * 16 + s) * YS_LD + cg * 4);
-                acc.x += xv * yv.x; acc.y += xv * yv.y; acc.z += xv * yv.z; acc.w += xv * yv.w;
-            }
-            *reinterpret_cast<float4 *>(Xs + (i * 16 + r) * AS_LD + j * 16 + cg * 4) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        }
-        __syncthreads();
-    }
+    solve_level<1>(As, Xs, Ys, tid);
+    solve_level<2>(As, Xs, Ys, tid);
+    solve_level<3>(As, Xs, Ys, tid);
     // T overwrites A (no longer read)
-    for (int idx = tid; idx < 64 * 32; idx += kThreads) {
+    for (int idx = tid; idx < 64 * 32; idx += NT) {
         const int r = idx >> 5, s0 = (idx & 31) * 2;
         const float v0 = s0 <= r ? Xs[r * AS_LD + s0] * sbeta[s0] : 0.f;
         const float v1 = s0 + 1 <= r ? Xs[r * AS_LD + s0 + 1] * sbeta[s0 + 1] : 0.f;
@@ -325,12 +400,14 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
     }
     __syncthreads();
 
-    // ---- Ut = T V (warps 0-3, fp32 -> record) and W = T Kt (warps 4-7, -W bf16 -> record) ---
+    // ---- Ut = T V and W = T Kt; each warp 16 rows x (128 / NH) columns ---------------------
     {
-        const int mat = warp >> 2, rt = warp & 3;
-        float acc[16][4];
+        constexpr int NH = NT / 256;
+        constexpr int NP = 8 / NH;    // 16-column pairs per warp (n-tiles = 2 NP)
+        const int mat = warp / (4 * NH), rt = (warp / NH) & 3, nh = warp % NH;
+        float acc[2 * NP][4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        for (int i = 0; i < 2 * NP; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
         const uint32_t bbase = sb + (mat ? A_KT : A_V);
 #pragma unroll
         for (int kk = 0; kk < kC / 16; ++kk) {
@@ -338,36 +415,50 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_prep_kernel(const Prefill
             ldmatrix_x4(sb + A_T + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
                         af[2], af[3]);
 #pragma unroll
-            for (int np = 0; np < 8; ++np) {
+            for (int np = 0; np < NP; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(bbase + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64), b0, b1,
-                                  b2, b3);
+                ldmatrix_x4_trans(bbase + toff(kk * 16 + l7 + lb3 * 8, 16 * NP * nh + np * 16 + lb4 * 8, 64),
+                                  b0, b1, b2, b3);
                 mma_bf16_16816(acc[2 * np], af, b0, b1);
                 mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
             }
         }
+        if (tid == 0) bulk_wait_group_read0();  // P's bulk store has left the Kh region
+        __syncthreads();  // Kt and V are no longer read: -W and Ut take their place
         const int r0 = 16 * rt + g, r1 = r0 + 8;
         if (mat == 1) {
-            uint8_t *nw = rec + REC_NW;
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const int cc = nt * 8 + 2 * t4;
-                st_bf16x2(nw, toff(r0, cc, 64), -acc[nt][0], -acc[nt][1]);
-                st_bf16x2(nw, toff(r1, cc, 64), -acc[nt][2], -acc[nt][3]);
+            for (int nt = 0; nt < 2 * NP; ++nt) {
+                const int cc = 16 * NP * nh + nt * 8 + 2 * t4;
+                st_bf16x2(sm + A_KT, toff(r0, cc, 64), -acc[nt][0], -acc[nt][1]);
+                st_bf16x2(sm + A_KT, toff(r1, cc, 64), -acc[nt][2], -acc[nt][3]);
             }
         } else {
-            float *ut = reinterpret_cast<float *>(rec + REC_UT);
+            float *ut = reinterpret_cast<float *>(sm + A_KH);
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const int cc = nt * 8 + 2 * t4;
-                *reinterpret_cast<float2 *>(ut + r0 * kD + cc) = make_float2(acc[nt][0], acc[nt][1]);
-                *reinterpret_cast<float2 *>(ut + r1 * kD + cc) = make_float2(acc[nt][2], acc[nt][3]);
+            for (int nt = 0; nt < 2 * NP; ++nt) {
+                const int cc = 16 * NP * nh + nt * 8 + 2 * t4;
+                *reinterpret_cast<float2 *>(ut + ut_idx(r0, cc)) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2 *>(ut + ut_idx(r1, cc)) = make_float2(acc[nt][2], acc[nt][3]);
             }
         }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(rec + REC_NW, sb + A_KT, 16384);
+        bulk_store(rec + REC_UT, sb + A_KH, 32768);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // shared memory must outlive the copies' reads
     }
 }
 
 // ================================ pass B ==================================================
+// Per chunk c (p = c & 1 picks the stage, the M buffer and the U buffer):
+//   phase 1  bf16 copy of M -> M[p]; st <- e^{G_C} st                 | barrier; issue chunk c+1
+//   phase 2  U = Ut - W M and O = Qt M, sharing M's fragments; U -> U[p] | barrier
+//   phase 3  O += P U, store O; st += Kc^T U
+// Two barriers per chunk: the buffers a chunk writes were last read two phases earlier.
 __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const PrefillScanArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -401,10 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
         mbar_arrive_expect_tx(bar, REC_HEAD);
         bulk_load(sb + (c & 1) * B_STAGE, record(a, bh, c), REC_HEAD, bar);
     };
-    if (tid == 0) {
-        issue(0);
-        if (a.n_seg > 1) issue(1);
-    }
+    if (tid == 0) issue(0);
 
     // state strip of this warp: rows 16*warp + g (+8), slice columns 8*nt + 2*t4 (+1)
     const int sr0 = 16 * warp + g, sr1 = sr0 + 8;
@@ -425,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
-            const float2 x0 = *reinterpret_cast<const float2 *>(ut + ur0 * kD + cc);
-            const float2 x1 = *reinterpret_cast<const float2 *>(ut + ur1 * kD + cc);
+            const float2 x0 = *reinterpret_cast<const float2 *>(ut + ut_idx(ur0, cc));
+            const float2 x1 = *reinterpret_cast<const float2 *>(ut + ut_idx(ur1, cc));
             un[j][0] = x0.x; un[j][1] = x0.y; un[j][2] = x1.x; un[j][3] = x1.y;
         }
     };
@@ -434,102 +522,94 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
 
     int aborted_at = -1;
     for (int c = 0; c < a.n_seg; ++c) {
-        const int s = c & 1;
-        const uint32_t stg = sb + s * B_STAGE;
+        const int p = c & 1;
+        const uint32_t stg = sb + p * B_STAGE;
+        const uint32_t mb = sb + B_M + p * 16384, ub = sb + B_U + p * 8192;
         const int t0 = (a.chunk_begin + c) * kC;
         const int n = min(kC, T - t0);
-        const bool ok = mbar_wait_bounded(smem_u32(&bars[s]), (c >> 1) & 1);
+        const bool ok = mbar_wait_bounded(smem_u32(&bars[p]), (c >> 1) & 1);
+        // ---- phase 1: bf16 copy of M (the B operand of U and O); st <- e^{G_C} st ---------
+        if (ok) {
+            const float *gm = reinterpret_cast<const float *>(sm + p * B_STAGE + REC_GAM);
+            const float g0 = gm[sr0], g1 = gm[sr1];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int cc = nt * 8 + 2 * t4;
+                st_bf16x2(sm + B_M + p * 16384, toff(sr0, cc, 128), st[nt][0], st[nt][1]);
+                st_bf16x2(sm + B_M + p * 16384, toff(sr1, cc, 128), st[nt][2], st[nt][3]);
+                st[nt][0] *= g0; st[nt][1] *= g0; st[nt][2] *= g1; st[nt][3] *= g1;
+            }
+        }
         if (__syncthreads_or(!ok)) {
             if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
             aborted_at = c;
             break;
         }
-        // ---- phase 1: bf16 copy of M (the B operand of U and O); st <- e^{G_C} st ---------
-        {
-            const float *gm = reinterpret_cast<const float *>(sm + s * B_STAGE + REC_GAM);
-            const float g0 = gm[sr0], g1 = gm[sr1];
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const int cc = nt * 8 + 2 * t4;
-                st_bf16x2(sm + B_M, toff(sr0, cc, 128), st[nt][0], st[nt][1]);
-                st_bf16x2(sm + B_M, toff(sr1, cc, 128), st[nt][2], st[nt][3]);
-                st[nt][0] *= g0; st[nt][1] *= g0; st[nt][2] *= g1; st[nt][3] *= g1;
-            }
+        if (tid == 0 && c + 1 < a.n_seg) {  // every warp is past chunk c-1: its stage is free
+            fence_proxy_async_smem();
+            issue(c + 1);
         }
-        float u[4][4];
+
+        // ---- phase 2: U = Ut + (-W) M and O = Qt M (16 rows x 32 columns per warp) -------
+        float u[4][4], o[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) u[j][e] = un[j][e];
-        __syncthreads();
-
-        // ---- phase 2: U = Ut + (-W) M (16 rows x 32 columns per warp) ----------------------
+            for (int e = 0; e < 4; ++e) {
+                u[j][e] = un[j][e];
+                o[j][e] = 0.f;
+            }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-            uint32_t af[4];
-            ldmatrix_x4(stg + REC_NW + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
-                        af[2], af[3]);
+            uint32_t aw[4], aq[4];
+            ldmatrix_x4(stg + REC_NW + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), aw[0], aw[1],
+                        aw[2], aw[3]);
+            ldmatrix_x4(stg + REC_QT + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), aq[0], aq[1],
+                        aq[2], aq[3]);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(sb + B_M + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 128),
+                ldmatrix_x4_trans(mb + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 128),
                                   b0, b1, b2, b3);
-                mma_bf16_16816(u[2 * np], af, b0, b1);
-                mma_bf16_16816(u[2 * np + 1], af, b2, b3);
+                mma_bf16_16816(u[2 * np], aw, b0, b1);
+                mma_bf16_16816(u[2 * np + 1], aw, b2, b3);
+                mma_bf16_16816(o[2 * np], aq, b0, b1);
+                mma_bf16_16816(o[2 * np + 1], aq, b2, b3);
             }
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int cc = 32 * chh + 8 * j + 2 * t4;
-            st_bf16x2(sm + B_U, toff(ur0, cc, 64), u[j][0], u[j][1]);
-            st_bf16x2(sm + B_U, toff(ur1, cc, 64), u[j][2], u[j][3]);
+            st_bf16x2(sm + B_U + p * 8192, toff(ur0, cc, 64), u[j][0], u[j][1]);
+            st_bf16x2(sm + B_U + p * 8192, toff(ur1, cc, 64), u[j][2], u[j][3]);
         }
         if (c + 1 < a.n_seg) load_ut(c + 1);
         __syncthreads();
 
-        // ---- phase 3: O = Qt M + P U (16 rows x 32 columns per warp), then the state ------
-        {
-            float o[4][4];
+        // ---- phase 3: O += P U and store it; st += Kc^T U ------------------------------------
 #pragma unroll
-            for (int j = 0; j < 4; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        for (int kk = 0; kk < kC / 16; ++kk) {
+            uint32_t af[4];
+            ldmatrix_x4(stg + REC_P + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0],
+                        af[1], af[2], af[3]);
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                uint32_t af[4];
-                ldmatrix_x4(stg + REC_QT + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0],
-                            af[1], af[2], af[3]);
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(sb + B_M + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 128),
-                                      b0, b1, b2, b3);
-                    mma_bf16_16816(o[2 * np], af, b0, b1);
-                    mma_bf16_16816(o[2 * np + 1], af, b2, b3);
-                }
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(ub + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 64),
+                                  b0, b1, b2, b3);
+                mma_bf16_16816(o[2 * np], af, b0, b1);
+                mma_bf16_16816(o[2 * np + 1], af, b2, b3);
             }
+        }
 #pragma unroll
-            for (int kk = 0; kk < kC / 16; ++kk) {
-                uint32_t af[4];
-                ldmatrix_x4(stg + REC_P + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0],
-                            af[1], af[2], af[3]);
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(sb + B_U + toff(kk * 16 + l7 + lb3 * 8, 32 * chh + np * 16 + lb4 * 8, 64),
-                                      b0, b1, b2, b3);
-                    mma_bf16_16816(o[2 * np], af, b0, b1);
-                    mma_bf16_16816(o[2 * np + 1], af, b2, b3);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
-                if (ur0 < n)
-                    *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur0) * a.H + h) * kD + cc) =
-                        pack_bf16x2(a.scale * o[j][0], a.scale * o[j][1]);
-                if (ur1 < n)
-                    *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur1) * a.H + h) * kD + cc) =
-                        pack_bf16x2(a.scale * o[j][2], a.scale * o[j][3]);
-            }
+        for (int j = 0; j < 4; ++j) {
+            const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
+            if (ur0 < n)
+                *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur0) * a.H + h) * kD + cc) =
+                    pack_bf16x2(a.scale * o[j][0], a.scale * o[j][1]);
+            if (ur1 < n)
+                *reinterpret_cast<uint32_t *>(og + (((size_t)b * T + t0 + ur1) * a.H + h) * kD + cc) =
+                    pack_bf16x2(a.scale * o[j][2], a.scale * o[j][3]);
         }
         // st += Kc^T U (this warp's 16 rows of d_k, all 64 slice columns)
 #pragma unroll
@@ -540,21 +620,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
 #pragma unroll
             for (int np = 0; np < 4; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(sb + B_U + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64), b0, b1,
-                                  b2, b3);
+                ldmatrix_x4_trans(ub + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64), b0, b1, b2, b3);
                 mma_bf16_16816(st[2 * np], af, b0, b1);
                 mma_bf16_16816(st[2 * np + 1], af, b2, b3);
             }
         }
-        __syncthreads();  // stage s, M and U are free
-        if (tid == 0 && c + 2 < a.n_seg) issue(c + 2);
     }
     if (aborted_at >= 0) {
-        // a wait gave up: let this CTA's bulk copies in flight (chunks aborted_at and the one
-        // after it) finish, bounded; the state is left as it was at the start of this segment
+        // a wait gave up: let this CTA's one bulk copy in flight (chunk aborted_at) finish,
+        // bounded; the state is left as it was at the start of this segment
         if (tid == 0)
-            for (int c = aborted_at; c < aborted_at + 2 && c < a.n_seg; ++c)
-                (void)mbar_wait_bounded(smem_u32(&bars[c & 1]), (c >> 1) & 1);
+            (void)mbar_wait_bounded(smem_u32(&bars[aborted_at & 1]), (aborted_at >> 1) & 1);
         return;
     }
 #pragma unroll
@@ -602,9 +678,9 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
         p.n_seg = std::min(seg, n_chunks - cb);
         const unsigned grid_a = (unsigned)(bhs * p.n_seg);
         if (a.kind == HMD_KDA)
-            prefill_prep_kernel<true><<<grid_a, kThreads, A_SMEM, s>>>(p);
+            prefill_prep_kernel<true><<<grid_a, kPrepThreads, A_SMEM, s>>>(p);
         else
-            prefill_prep_kernel<false><<<grid_a, kThreads, A_SMEM, s>>>(p);
+            prefill_prep_kernel<false><<<grid_a, kPrepThreads, A_SMEM, s>>>(p);
         prefill_scan_kernel<<<(unsigned)(bhs * kSplitV), kThreads, B_SMEM, s>>>(p);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -227,6 +227,13 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src, int
         "r"(x), "r"(y), "r"(src)
         : "memory");
 }
+// Untiled bulk copy shared -> global (both 16-byte aligned, bytes a multiple of 16), completed
+// through this thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(src), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
