@@ -11,7 +11,8 @@
 //   O = Qt M0 + P U
 //   M_C = Diag(exp(G_C)) M0 + (Kh Diag(exp(G_C)))^T U,  G_C = G of the chunk's last token.
 //
-// bf16 inputs with d_k = d_v = 128 run on the tensor cores (delta_prefill_mma.cu).
+// bf16 inputs with d_k = d_v = 128 and C = 64 run on the tensor cores in two passes
+// (delta_prefill_scan.cu).
 // This file holds the generic path: one CTA per (sequence, head, 32-column slice of d_v) runs
 // the chunks in order with the slice of the state resident in shared memory, all arithmetic in
 // fp32 on CUDA cores (so fp32 inputs keep fp32 accuracy). The k-side products (A, T, W, P) do
@@ -199,7 +200,6 @@ bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk) {
 }
 
 cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s) {
-    if (delta_prefill_mma_supported(a.dk, a.dv, a.bf16, a.chunk)) return launch_delta_prefill_mma(a, s);
     const int dvs = a.dv < kSlice ? a.dv : kSlice;
     const int n_slices = (a.dv + dvs - 1) / dvs;
     const size_t smem = generic_smem_bytes(a.dk, dvs);

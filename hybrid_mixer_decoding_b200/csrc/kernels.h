@@ -71,11 +71,6 @@ struct DeltaPrefillArgs {
 cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s);
 bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk);
 uint32_t delta_prefill_read_errors(bool clear);
-// tensor-core path (bf16, d_k = d_v = 128, chunk 64); launch_delta_prefill dispatches to it
-bool delta_prefill_mma_supported(int dk, int dv, bool bf16, int chunk);
-cudaError_t launch_delta_prefill_mma(const DeltaPrefillArgs &a, cudaStream_t s);
-uint32_t delta_prefill_mma_read_errors(bool clear);
-
 // two-pass tensor-core path (bf16, d_k = d_v = 128, chunk 64): a chunk-parallel pass writes one
 // record per chunk to a workspace, a scan pass carries the state through the chunks
 struct PrefillScanArgs {
