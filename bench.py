@@ -535,12 +535,33 @@ def sweep_placements():
         "24FA+24GDN": I.placement({I.FA: 24, I.GDN: 24}, seed=0),
         "8FA+20KDA+20GDN": I.placement({I.FA: 8, I.KDA: 20, I.GDN: 20}, seed=0),
         "all-GDN": np.full(48, I.GDN, np.int8),
+        "all-KDA": np.full(48, I.KDA, np.int8),
     }
+
+
+PURE = {I.FA: "all-FA", I.KDA: "all-KDA", I.GDN: "all-GDN"}
+
+
+def linear_cost_model(pls, res):
+    """The pages' cost model: a placement's step time is the sum of its layers' costs. Per-layer
+    costs come from the single-kind placements (step / 48); the mixed placements are predicted
+    from their mixer counts and compared with their measured step times."""
+    per_layer = {k: res[name]["ms_per_step"] / len(pls[name]) for k, name in PURE.items()}
+    out = {"per_layer_us": {I.KIND_NAMES[k]: round(v * 1e3, 2) for k, v in per_layer.items()},
+           "predicted_ms": {}, "error_pct": {}}
+    for name, pl in pls.items():
+        if name in PURE.values():
+            continue
+        pred = sum(per_layer[int(k)] for k in pl)
+        out["predicted_ms"][name] = round(pred, 3)
+        out["error_pct"][name] = round(100.0 * (res[name]["ms_per_step"] / pred - 1.0), 2)
+    return out
 
 
 def run_sweep(args):
     """Context sweep: B=16, ctx in {4k, 16k, 64k, 128k}, 48-layer stack, placements all-FA,
-    24 FA + 24 GDN, 8 FA + 40 (20 KDA + 20 GDN), all-GDN; decode tok/s and speedup over all-FA.
+    24 FA + 24 GDN, 8 FA + 40 (20 KDA + 20 GDN), all-GDN, all-KDA; decode tok/s, speedup over
+    all-FA, and the linear per-layer cost model checked against the mixed placements.
     KV pools are zero-filled (timing only); FA layers share physical pools round-robin when the
     placement's KV exceeds device memory (each layer still streams its own full context)."""
     import torch
@@ -564,7 +585,7 @@ def run_sweep(args):
             res[name]["predicted_by_bytes"] = round(
                 fa_bytes / sum(layer_bytes(int(k), shape) for k in pls[name]), 3)
         rows.append({"ctx": ctx, "aliased_fa_pools": st.n_fa_pools if st.aliased else None,
-                     "placements": res})
+                     "placements": res, "linear_cost_model": linear_cost_model(pls, res)})
         del graphs
         st.free()
         del st
