@@ -139,14 +139,16 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = p.group;
-    const Item it = item_info(p, blockIdx.x);
     if (tid == 0) {
-        if (it.bad_len && it.split == 0) atomicOr(&g_err, HMD_DEVERR_SEQLEN);
         for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&full_bar[s]), 1);
         fence_barrier_init();
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
+    griddep_launch_dependents();
+    griddep_wait();  // q, the new token, the pools and the tables may come from the previous kernel
+    const Item it = item_info(p, blockIdx.x);
+    if (tid == 0 && it.bad_len && it.split == 0) atomicOr(&g_err, HMD_DEVERR_SEQLEN);
 
     // ---- producer (warp 0, warp-uniform calls; lane 0 issues) -----------------------------
     auto table_entry = [&](int t) -> int {
@@ -375,6 +377,8 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const float *ws_ml, con
                                                          int n_splits, __nv_bfloat16 *o) {
     const size_t bh = blockIdx.x;
     const int dim = threadIdx.x;
+    griddep_launch_dependents();
+    griddep_wait();  // the partials are the split kernel's output
     const float *ml = ws_ml + bh * n_splits * 2;
     float M = -INFINITY;
     for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[2 * s]);
@@ -458,12 +462,12 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     p.n_splits = plan.n_splits; p.pages_per_split = plan.pages_per_split;
     p.max_seq_len = a.max_seq_len;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    attn_split_kernel<D><<<(unsigned)plan.n_ctas, kThreads, smem, s>>>(tmk, tmv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(attn_split_kernel<D>, dim3((unsigned)plan.n_ctas), dim3(kThreads),
+                               smem, s, tmk, tmv, p);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<D><<<(unsigned)(a.B * a.Hq), D, 0, s>>>(p.ws_ml, p.ws_acc, plan.n_splits,
-                                                               static_cast<__nv_bfloat16 *>(a.o));
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(a.B * a.Hq)), dim3(D), 0, s,
+                      (const float *)p.ws_ml, (const float *)p.ws_acc, plan.n_splits,
+                      static_cast<__nv_bfloat16 *>(a.o));
 }
 
 // SMs of the current device (148 when no device can be queried).

@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     const int col = slice * kSliceCols + ct * 4;
     const bool active = col < a.dv;
 
+    if (tid == 0) prefetch_tmap(&tm);
+    griddep_launch_dependents();
+    griddep_wait();  // q, k, v, gates and the state may come from the previous kernel
     if (tid == 0) {
         const int slot = a.slots ? a.slots[b] : b;
         const bool ok = slot >= 0 && slot < a.n_slots;
@@ -190,12 +193,11 @@ cudaError_t launch_dk(const DeltaDecodeArgs &a, cudaStream_t s) {
     if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.state, a.dv,
                       (long long)a.n_slots * a.H * DK, kSliceCols, DK))
         return cudaErrorInvalidValue;
-    if (a.bf16) {
-        delta_decode_kernel<DK, true><<<(unsigned)grid, kThreads, 0, s>>>(tm, a, n_slices);
-    } else {
-        delta_decode_kernel<DK, false><<<(unsigned)grid, kThreads, 0, s>>>(tm, a, n_slices);
-    }
-    return cudaGetLastError();
+    if (a.bf16)
+        return launch_pdl(delta_decode_kernel<DK, true>, dim3((unsigned)grid), dim3(kThreads), 0, s,
+                          tm, a, n_slices);
+    return launch_pdl(delta_decode_kernel<DK, false>, dim3((unsigned)grid), dim3(kThreads), 0, s, tm,
+                      a, n_slices);
 }
 
 }  // namespace

@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
     const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
     const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
     const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v);
+    griddep_launch_dependents();
+    griddep_wait();  // the inputs may come from the previous kernel
 
     // ---- stage q (into the Qt slot), k (into the Kh slot), v, KDA log-gates; beta ----------
     {
@@ -473,6 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
     const int b = bh / a.H, h = bh - b * a.H;
     const int col0 = sv * kDV;  // this CTA's first d_v column
     const int T = a.T;
+    griddep_launch_dependents();
+    griddep_wait();  // the records are the prep pass's output
     const int slot = a.slots ? a.slots[b] : b;
     if (slot < 0 || slot >= a.n_slots) {
         if (tid == 0) atomicOr(&g_err, HMD_DEVERR_SLOT);
@@ -677,12 +681,11 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
         p.chunk_begin = cb;
         p.n_seg = std::min(seg, n_chunks - cb);
         const unsigned grid_a = (unsigned)(bhs * p.n_seg);
-        if (a.kind == HMD_KDA)
-            prefill_prep_kernel<true><<<grid_a, kPrepThreads, A_SMEM, s>>>(p);
-        else
-            prefill_prep_kernel<false><<<grid_a, kPrepThreads, A_SMEM, s>>>(p);
-        prefill_scan_kernel<<<(unsigned)(bhs * kSplitV), kThreads, B_SMEM, s>>>(p);
-        const cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_pdl(a.kind == HMD_KDA ? prefill_prep_kernel<true> : prefill_prep_kernel<false>,
+                                   dim3(grid_a), dim3(kPrepThreads), A_SMEM, s, p);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(prefill_scan_kernel, dim3((unsigned)(bhs * kSplitV)), dim3(kThreads), B_SMEM, s,
+                       p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -6,7 +6,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace hmd {
+
+// Launches `kernel` on stream s with programmatic stream serialisation: it may be scheduled
+// while the previous kernel in the stream drains, and waits for it (griddep_wait) before its
+// first global-memory access, so results are those of an ordinary launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // TMA tensor map over a 2-D row-major tensor, boxes of [box_rows][box_cols], no swizzle.
 bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base, long long cols,

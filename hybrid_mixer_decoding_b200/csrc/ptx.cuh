@@ -85,6 +85,15 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
+// Programmatic dependent launch. griddep_wait: block until the grids this launch depends on
+// have completed and their writes are visible (a no-op for a launch without such a dependency);
+// every kernel calls it before its first global-memory access. griddep_launch_dependents: allow
+// the next kernel in the stream to be scheduled (it still waits in its own griddep_wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

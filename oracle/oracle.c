@@ -355,6 +355,54 @@ int oracle_attn_decode(int kind, int window, int B, int Hq, int Hkv, int d, int 
     return bad ? -1 : 0;
 }
 
+/* Prefill of FA or SWA over T new tokens per sequence, starting from an empty cache. Token t
+ * sits at logical position t and attends keys j in [lo_t, t], lo_t = 0 (FA) or
+ * max(0, t + 1 - window) (SWA): the decode step above with L = t + 1, for every t at once.
+ *   q [B][T][Hq][d], k, v [B][T][Hkv][d], o [B][T][Hq][d] (double).
+ * Returns 0, or -1 on bad arguments.                                                          */
+int oracle_attn_prefill(int kind, int window, int B, int T, int Hq, int Hkv, int d,
+                        const double *q, const double *k, const double *v, double *o,
+                        int n_threads) {
+    if ((kind != OR_FA && kind != OR_SWA) || Hkv < 1 || Hq % Hkv || T < 0 || d < 1) return -1;
+    if (kind == OR_SWA && window < 1) return -1;
+    set_threads(n_threads);
+    const int group = Hq / Hkv;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+    for (int bh = 0; bh < B * Hq; ++bh) {
+        const int b = bh / Hq, h = bh % Hq, kvh = h / group;
+        double *s = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        if (!s) { bad |= 1; continue; }
+        for (int t = 0; t < T; ++t) {
+            const int lo = (kind == OR_SWA && t + 1 > window) ? t + 1 - window : 0;
+            const double *qv = q + (((size_t)b * T + t) * Hq + h) * d;
+            double mx = -INFINITY;
+            for (int j = lo; j <= t; ++j) {
+                const double *kv = k + (((size_t)b * T + j) * Hkv + kvh) * d;
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c) acc += qv[c] * kv[c];
+                s[j - lo] = inv_sqrt_d * acc;
+                if (s[j - lo] > mx) mx = s[j - lo];
+            }
+            double denom = 0.0;
+            for (int j = lo; j <= t; ++j) {
+                s[j - lo] = exp(s[j - lo] - mx);
+                denom += s[j - lo];
+            }
+            double *ov = o + (((size_t)b * T + t) * Hq + h) * d;
+            for (int c = 0; c < d; ++c) ov[c] = 0.0;
+            for (int j = lo; j <= t; ++j) {
+                const double p = s[j - lo] / denom;
+                const double *vv = v + (((size_t)b * T + j) * Hkv + kvh) * d;
+                for (int c = 0; c < d; ++c) ov[c] += p * vv[c];
+            }
+        }
+        free(s);
+    }
+    return bad ? -1 : 0;
+}
+
 /* The oracle's thread count after set-up (for reporting). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -51,9 +51,10 @@ def _load():
         lib.oracle_kv_slot.argtypes = [c_int, c_int, c_int, I32, c_int, c_int, I32, I32]
         lib.oracle_attn_decode.argtypes = ([c_int] * 8 + [D, D, D, U16, U16, I32, c_int, I32, D,
                                                           c_int])
+        lib.oracle_attn_prefill.argtypes = [c_int] * 7 + [D, D, D, D, c_int]
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_delta_recurrent", "oracle_delta_chunked", "oracle_kv_slot",
-                  "oracle_attn_decode", "oracle_max_threads"):
+                  "oracle_attn_decode", "oracle_attn_prefill", "oracle_max_threads"):
             getattr(lib, f).restype = c_int
         _lib = lib
     return _lib
@@ -148,6 +149,23 @@ def attn_decode(kind, window, q_bits, new_k_bits, new_v_bits, k_pool, v_pool, pa
                                     _p(o, ctypes.c_double), int(n_threads))
     if rc:
         raise ValueError("oracle_attn_decode failed (bad arguments or page id)")
+    return o
+
+
+def attn_prefill(kind, window, q, k, v, n_threads=0):
+    """FA/SWA prefill from an empty cache (see oracle.c): q [B,T,Hq,d], k, v [B,T,Hkv,d]
+    (float64; pass the exact values the GPU receives). Returns o [B,T,Hq,d] float64."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    o = np.zeros((B, T, Hq, d), dtype=np.float64)
+    rc = _load().oracle_attn_prefill(kind, int(window), B, T, Hq, Hkv, d, _p(q, ctypes.c_double),
+                                     _p(k, ctypes.c_double), _p(v, ctypes.c_double),
+                                     _p(o, ctypes.c_double), int(n_threads))
+    if rc:
+        raise ValueError("oracle_attn_prefill: bad arguments")
     return o
 
 

@@ -346,3 +346,91 @@ def test_swa_ring_injective_over_every_window(oracle_mod, w):
             # is older than the window
             prev = [p for p in range(L - 1) if slots[p] == slots[L - 1]]
             assert all(p < lo for p in prev)
+
+
+# ---- attention prefill from an empty cache (token t attends [lo_t, t]) ------------------------
+
+def _prefill_qkv(B, T, Hq, Hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, T, Hq, d)), rng.standard_normal((B, T, Hkv, d)),
+            rng.standard_normal((B, T, Hkv, d)))
+
+
+def _masked_softmax_attention(q, k, v, window):
+    """Brute force with an explicit T x T mask: allowed[t, j] = j <= t and t - j < window."""
+    B, T, Hq, d = q.shape
+    grp = Hq // k.shape[2]
+    t = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    allowed = (j <= t) & (t - j < window)
+    out = np.zeros_like(q)
+    for b in range(B):
+        for h in range(Hq):
+            s = (q[b, :, h] @ k[b, :, h // grp].T) / math.sqrt(d)
+            s = np.where(allowed, s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            out[b, :, h] = (p / p.sum(axis=1, keepdims=True)) @ v[b, :, h // grp]
+    return out
+
+
+@pytest.mark.parametrize("kind,window", [(I.FA, 0), (I.SWA, 5), (I.SWA, 16)])
+def test_prefill_attention_matches_masked_softmax_and_sdpa(oracle_mod, kind, window):
+    O = oracle_mod
+    q, k, v = _prefill_qkv(2, 37, 4, 2, 8, seed=30 + window)
+    o = O.attn_prefill(kind, window, q, k, v)
+    ref = _masked_softmax_attention(q, k, v, window if kind == I.SWA else 10 ** 9)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+    if kind == I.FA:  # torch's fp64 causal attention on the same data
+        qt = torch.from_numpy(q.transpose(0, 2, 1, 3))
+        kt = torch.from_numpy(np.repeat(k, 2, axis=2).transpose(0, 2, 1, 3))
+        vt = torch.from_numpy(np.repeat(v, 2, axis=2).transpose(0, 2, 1, 3))
+        st = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+        np.testing.assert_allclose(o, st.numpy().transpose(0, 2, 1, 3), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind,window", [(I.FA, 0), (I.SWA, 7)])
+def test_prefill_rows_equal_decode_steps(oracle_mod, kind, window):
+    """Row t of the prefill is the decode step with L = t + 1 over a paged cache holding tokens
+    0..t-1 (the decode oracle is pinned on its own above)."""
+    O = oracle_mod
+    B, T, Hq, Hkv, d, PT = 2, 21, 4, 2, 8, 4
+    bits = lambda x: I.bf16_bits(x)
+    q, k, v = _prefill_qkv(B, T, Hq, Hkv, d, seed=41)
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    o = O.attn_prefill(kind, window, O.bf16_bits_to_f64(qb), O.bf16_bits_to_f64(kb),
+                       O.bf16_bits_to_f64(vb))
+    n_pg = -(-T // PT) if kind == I.FA else -(-window // PT)  # FA pages / SWA ring pages
+    table = np.arange(B * n_pg, dtype=np.int32).reshape(B, n_pg)
+    for t in range(T):
+        # the cache as t decode steps leave it: positions 0..t-1 written in order at their
+        # slots (for SWA the ring keeps the latest position of each slot)
+        kp = np.zeros((B * n_pg, Hkv, PT, d), np.uint16)
+        vp = np.zeros_like(kp)
+        for b in range(B):
+            for p in range(t):
+                pg, off = O.kv_slot(kind, window, PT, table[b], p)
+                kp[pg, :, off], vp[pg, :, off] = kb[b, p], vb[b, p]
+        dec = O.attn_decode(kind, window, qb[:, t], kb[:, t], vb[:, t], kp, vp, table,
+                            np.full(B, t + 1, np.int32))
+        np.testing.assert_allclose(o[:, t], dec, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_attention_closed_forms(oracle_mod):
+    O = oracle_mod
+    q, k, v = _prefill_qkv(2, 12, 4, 1, 8, seed=50)
+    # the first token sees only itself; a window of 1 gives every token its own value
+    o = O.attn_prefill(I.FA, 0, q, k, v)
+    np.testing.assert_array_equal(o[:, 0], np.repeat(v[:, 0], 4, axis=1))
+    o1 = O.attn_prefill(I.SWA, 1, q, k, v)
+    np.testing.assert_array_equal(o1, np.repeat(v, 4, axis=2))
+    # a window covering the whole prompt is FA, bit for bit
+    np.testing.assert_array_equal(O.attn_prefill(I.SWA, 12, q, k, v), o)
+    np.testing.assert_array_equal(O.attn_prefill(I.SWA, 500, q, k, v), o)
+    # equal keys: uniform weights, so each row is the mean of the values in its window
+    ke = np.repeat(k[:, :1], 12, axis=1)
+    w = 3
+    oe = O.attn_prefill(I.SWA, w, q, ke, v)
+    for t in range(12):
+        lo = max(0, t + 1 - w)
+        np.testing.assert_allclose(oe[:, t], np.repeat(v[:, lo:t + 1].mean(axis=1), 4, axis=1),
+                                   rtol=1e-12, atol=1e-13)

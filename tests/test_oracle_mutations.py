@@ -37,6 +37,11 @@ MUTANTS = [
     ("gqa_map_interleaved", [("g = h / group", "g = h % Hkv")]),
     ("ring_not_wrapped", [("idx = pos % (R * page_tokens);", "idx = pos;")]),
     ("new_token_ignored", [("if (j == L - 1) {", "if (0) {")]),
+    ("prefill_window_off_by_one", [("? t + 1 - window : 0", "? t - window : 0")]),
+    ("prefill_gqa_interleaved", [("kvh = h / group", "kvh = h % Hkv")]),
+    ("prefill_scale_missing", [("s[j - lo] = inv_sqrt_d * acc;", "s[j - lo] = acc;")]),
+    ("prefill_value_row_shifted", [("const double *vv = v + (((size_t)b * T + j) * Hkv + kvh) * d;",
+                                    "const double *vv = v + (((size_t)b * T + (j > lo ? j - 1 : j)) * Hkv + kvh) * d;")]),
 ]
 
 
