@@ -2,8 +2,8 @@
 """Decode throughput of the 48-layer mixer-only stack, one B200 per rank.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload stack48|attn_fa|attn_swa|decode_kda|decode_gdn|prefill_kda|
-                                prefill_gdn|sweep]
+                    [--workload stack48|attn_fa|attn_swa|prefill_fa|prefill_swa|decode_kda|
+                                decode_gdn|prefill_kda|prefill_gdn|sweep]
 
 Default workload ("stack48"): 48 layers, placement 12 FA / 12 SWA (w=4096) / 12 KDA / 12 GDN
 randomly interleaved (seed 0), B=64 sequences at context 32768, H=32 query/delta heads, 8 KV
@@ -421,6 +421,8 @@ def run_kernel_workload(args):
     """One mixer kernel at its configuration:
     attn_fa / attn_swa: B=32, Hq=32, Hkv=8, d=128, context 8192, SWA w=4096, paged bf16 KV
       (pages of 64, random page permutation), one new token per sequence;
+    prefill_fa / prefill_swa: B=2, T=8192, Hq=32, Hkv=8, d=128, SWA w=4096, prompts written into
+      an empty paged cache;
     decode_kda / decode_gdn: one decode step at the stack's layer shape (B=64, H=32, d=128),
       rotating over 4 state buffers (512 MiB) so every launch streams from HBM;
     prefill_kda / prefill_gdn: B=4, H=16, d=128, T=4096, chunk 64, bf16 q/k/v, fp32 state."""
@@ -463,6 +465,33 @@ def run_kernel_workload(args):
                 "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
                 "traffic": traffic_for(w), "algorithmic_bytes": byts}
         launches = 2
+    elif w in ("prefill_fa", "prefill_swa"):
+        kind = I.FA if w == "prefill_fa" else I.SWA
+        B, T, Hq, Hkv, d, win = 2, 8192, 32, 8, 128, 4096
+        pps = T // 64 if kind == I.FA else win // 64
+        P = B * pps
+        kp = torch.empty(P, Hkv, 64, d, device=dev, dtype=bf)
+        vp = torch.empty(P, Hkv, 64, d, device=dev, dtype=bf)
+        table = torch.randperm(P, device=dev, generator=g).to(torch.int32).view(B, pps).contiguous()
+        q = torch.randn(B, T, Hq, d, device=dev, dtype=bf, generator=g)
+        k = torch.randn(B, T, Hkv, d, device=dev, dtype=bf, generator=g)
+        v = torch.randn(B, T, Hkv, d, device=dev, dtype=bf, generator=g)
+        o = torch.empty(B, T, Hq, d, device=dev, dtype=bf)
+
+        def fn():
+            hmd.attn_prefill(kind, win, q, k, v, kp, vp, table, o)
+        sec = _events_time(fn, args.steps, args.warmup)
+        keys = sum(min(t + 1, win) if kind == I.SWA else t + 1 for t in range(T))
+        flops = 4 * d * Hq * B * keys  # S = q K^T and O = P V over the attended keys
+        tf = float(pk["bf16_tflops"])
+        value, unit = B * T / sec, "tok/s"
+        desc = (f"{'FA' if kind == I.FA else 'SWA(w=4096)'} prefill from an empty cache: B=2, "
+                f"T=8192, Hq=32, Hkv=8, d=128, K/V written to a paged bf16 cache "
+                f"(64-token pages, random permutation)")
+        roof = {"bound": "tensor", "achieved": round(flops / sec / 1e12, 2), "peak": tf,
+                "unit": "TFLOP/s", "frac": round(flops / sec / 1e12 / tf, 5),
+                "traffic": traffic_for(w), "algorithmic_flops": flops}
+        launches = 1
     elif w in ("decode_kda", "decode_gdn"):
         kind = I.KDA if w == "decode_kda" else I.GDN
         B, H, d = 64, 32, 128
@@ -606,7 +635,8 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used for profiler runs)")
     ap.add_argument("--workload", default="stack48",
-                    choices=["stack48", "attn_fa", "attn_swa", "decode_kda", "decode_gdn",
+                    choices=["stack48", "attn_fa", "attn_swa", "prefill_fa", "prefill_swa",
+                             "decode_kda", "decode_gdn",
                              "prefill_kda", "prefill_gdn", "sweep"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -42,6 +42,7 @@ _SIGS = {
     "attn_decode_workspace_size": (_sz, [_c_int] * 8),
     "attn_decode": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
                                                       _vp, _sz, _vp]),
+    "attn_prefill": (_c_int, [_c_int] * 8 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _vp]),
     "attn_decode_static_ws": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp,
                                                                 _c_int, _vp, _vp]),
     "state_cache_alloc": (_c_int, [_c_int] * 5 + [_vp, ctypes.POINTER(_vp)]),
@@ -194,6 +195,19 @@ def attn_decode_static_ws(kind, window, q, new_k, new_v, k_pool, v_pool, page_ta
                                      page_table.shape[1], _p(seq_lens), int(max_seq_len), _p(o),
                                      _stream(stream))
     _check("attn_decode_static_ws", st)
+
+
+def attn_prefill(kind, window, q, k, v, k_pool, v_pool, page_table, o, stream=None) -> None:
+    """FA/SWA prefill of a prompt into an empty paged cache (see include/hmd.h).
+    q,o [B,T,Hq,d]; k,v [B,T,Hkv,d] bf16; pools [n_pages,Hkv,page_tokens,d];
+    page_table [B,max_pages] int32."""
+    _contig(q, k, v, k_pool, v_pool, page_table, o)
+    B, T, Hq, d = q.shape
+    n_pages, Hkv, PT, _ = k_pool.shape
+    st = lib().attn_prefill(kind, int(window), B, T, Hq, Hkv, d, PT, _p(q), _p(k), _p(v),
+                            _p(k_pool), _p(v_pool), n_pages, _p(page_table), page_table.shape[1],
+                            _p(o), _stream(stream))
+    _check("attn_prefill", st)
 
 
 class StateCache:

@@ -20,7 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhmd.so")
 SOURCES = ["hmd_api.cu", "delta_decode.cu", "attn_decode.cu", "delta_prefill.cu",
-           "attn_decode_static.cu", "delta_prefill_scan.cu", "tmap.cu"]
+           "attn_decode_static.cu", "delta_prefill_scan.cu", "attn_prefill.cu",
+           "tmap.cu"]
 HEADERS = ["ptx.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",

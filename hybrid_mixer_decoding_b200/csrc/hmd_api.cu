@@ -88,7 +88,8 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
     if (!bits) return fail(HMD_ERR_ARG);
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
     *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
-            hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_scan_read_errors(clear != 0);
+            hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_scan_read_errors(clear != 0) |
+            hmd::attn_prefill_read_errors(clear != 0);
     return HMD_OK;
 }
 
@@ -238,6 +239,32 @@ hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, in
 }
 
 // ---- attention mixers --------------------------------------------------------------------
+
+hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv, int d,
+                          int page_tokens, const void *q, const void *k, const void *v,
+                          void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
+                          int max_pages, void *o, hmd_stream_t stream) {
+    if (kind != HMD_FA && kind != HMD_SWA) return fail(HMD_ERR_ARG);
+    if (kind == HMD_SWA && window < 1) return fail(HMD_ERR_ARG);
+    if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
+        max_pages < 1)
+        return fail(HMD_ERR_SHAPE);
+    if (Hq % Hkv) return fail(HMD_ERR_SHAPE);
+    if (B == 0 || T == 0) return HMD_OK;
+    if (!q || !k || !v || !k_pool || !v_pool || !page_table || !o) return fail(HMD_ERR_ARG);
+    if (!hmd::attn_prefill_supported(d, page_tokens, Hq / Hkv)) return fail(HMD_ERR_UNSUPPORTED);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_pool) ||
+        !aligned16(v_pool))
+        return fail(HMD_ERR_ARG);
+    const long long need = kind == HMD_SWA ? (window + page_tokens - 1) / page_tokens
+                                           : ((long long)T + page_tokens - 1) / page_tokens;
+    if (max_pages < need) return fail(HMD_ERR_SHAPE);
+    hmd::AttnPrefillArgs a{};
+    a.swa = kind == HMD_SWA; a.window = window; a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.page_tokens = page_tokens; a.q = q; a.k = k; a.v = v; a.k_pool = k_pool; a.v_pool = v_pool;
+    a.n_pages = n_pages; a.page_table = page_table; a.max_pages = max_pages; a.o = o;
+    return from_cuda(hmd::launch_attn_prefill(a, as_stream(stream)));
+}
 
 size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
                                   int page_tokens, int max_seq_len) {

@@ -33,6 +33,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base, long long cols,
                   long long rows, int box_cols, int box_rows);
 
+// [n_tok][heads][d] bf16 as (d, heads, n_tok) in 64 x 1 x 64 boxes, 128-byte swizzle.
+bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int heads, int d);
+
 struct DeltaDecodeArgs {
     int kind;  // 2 = KDA (per-channel gate), 3 = GDN (scalar gate)
     int B, H, dk, dv;
@@ -92,6 +95,22 @@ struct DeltaPrefillArgs {
 cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s);
 bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk);
 uint32_t delta_prefill_read_errors(bool clear);
+// FA / SWA prefill from an empty cache (attn_prefill.cu)
+struct AttnPrefillArgs {
+    bool swa;
+    int window;
+    int B, T, Hq, Hkv, d, page_tokens;
+    const void *q, *k, *v;
+    void *k_pool, *v_pool;
+    int n_pages;
+    const int32_t *page_table;
+    int max_pages;
+    void *o;
+};
+bool attn_prefill_supported(int d, int page_tokens, int group);
+cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s);
+uint32_t attn_prefill_read_errors(bool clear);
+
 // two-pass tensor-core path (bf16, d_k = d_v = 128, chunk 64): a chunk-parallel pass writes one
 // record per chunk to a workspace, a scan pass carries the state through the chunks
 struct PrefillScanArgs {

@@ -44,4 +44,20 @@ bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The K or V input of a prompt, [n_tok][heads][d] bf16 (n_tok = B*T), as a 3-D tensor
+// (d, heads, n_tok) read in boxes of (64 dims, 1 head, 64 tokens) with the 128-byte swizzle:
+// one box is a [64 tokens][128 B] tile. Tokens past n_tok read as zero.
+bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int heads, int d) {
+    EncodeTiledFn enc = encode();
+    if (!enc) return false;
+    const cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)n_tok};
+    const cuuint64_t gstride[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, gdim, gstride, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 }  // namespace hmd

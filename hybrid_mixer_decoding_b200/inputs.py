@@ -179,6 +179,47 @@ def attn_inputs(kind: int, B: int, Hq: int, Hkv: int, d: int, ctx: int, window: 
                       seq_lens, q, new_k, new_v)
 
 
+@dataclass
+class AttnPrefillInputs:
+    """Inputs of one FA or SWA prefill of T prompt tokens per sequence into an empty cache.
+
+    q: bf16 bits [B][T][Hq][d]; k, v: bf16 bits [B][T][Hkv][d].
+    page_table: int32 [B][max_pages] (FA: ceil(T/64) pages per sequence; SWA: the ring's
+    R = ceil(window/64) pages), physical ids a seeded permutation of the pool when permute.
+    n_pages: pool size (the caller allocates [n_pages][Hkv][page_tokens][d] pools).
+    """
+    kind: int
+    window: int
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    d: int
+    page_tokens: int
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    page_table: np.ndarray
+    n_pages: int
+
+
+def attn_prefill_inputs(kind: int, B: int, T: int, Hq: int, Hkv: int, d: int, window: int = 0,
+                        page_tokens: int = 64, seed: int = 0,
+                        permute: bool = True) -> AttnPrefillInputs:
+    """Draw one seeded attention-prefill problem: q, k, v ~ N(0, 1) rounded to bf16."""
+    assert kind in (FA, SWA)
+    g = rng(seed)
+    max_pages = -(-window // page_tokens) if kind == SWA else -(-T // page_tokens)
+    max_pages = max(max_pages, 1)
+    P = B * max_pages
+    perm = g.permutation(P).astype(np.int32) if permute else np.arange(P, dtype=np.int32)
+    table = perm.reshape(B, max_pages).copy()
+    q = bf16_bits(g.standard_normal((B, T, Hq, d), dtype=np.float32))
+    k = bf16_bits(g.standard_normal((B, T, Hkv, d), dtype=np.float32))
+    v = bf16_bits(g.standard_normal((B, T, Hkv, d), dtype=np.float32))
+    return AttnPrefillInputs(kind, window, B, T, Hq, Hkv, d, page_tokens, q, k, v, table, P)
+
+
 def placement(counts: dict[int, int], seed: int = 0) -> np.ndarray:
     """A placement vector (int8, one mixer kind per layer) with the given count of each kind,
     positions shuffled by a seeded permutation ("randomly interleaved")."""

@@ -160,6 +160,22 @@ HMD_API hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int
                          int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
                          void *workspace, size_t ws_bytes, hmd_stream_t stream);
 
+/* FA / SWA prefill of T prompt tokens per sequence into an empty paged cache. Token t of
+ * sequence b is logical position t and attends keys j in [lo_t, t], lo_t = 0 (FA) or
+ * max(0, t + 1 - window) (SWA): the attn_decode step with L = t + 1 for every t at once. The
+ * prompt's K and V are written to the cache at the slots attn_decode reads (FA: every position;
+ * SWA: the positions the ring keeps, t >= T - R*page_tokens), so decoding can follow directly.
+ *   q, o [B][T][Hq][d] bf16; k, v [B][T][Hkv][d] bf16 (the prompt's own keys and values, which
+ *   must hold finite values); k_pool, v_pool, page_table, n_pages as in attn_decode, with
+ *   max_pages >= ceil(T / page_tokens) (FA) or R (SWA).
+ * Supported: d in {64, 128}; page_tokens == 64; Hq / Hkv in {1, 2, 4, 8, 16}. q, k, v, o and
+ * the pools must be 16-byte aligned (HMD_ERR_ARG). Allocates nothing.                          */
+HMD_API hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv,
+                                  int d, int page_tokens, const void *q, const void *k,
+                                  const void *v, void *k_pool, void *v_pool, int n_pages,
+                                  const int32_t *page_table, int max_pages, void *o,
+                                  hmd_stream_t stream);
+
 /* attn_decode without a caller-provided workspace. The paper has no counterpart to this entry
  * point: it exists for callers that cannot allocate device memory, such as a plugin whose host
  * application owns all device memory through its own allocator, or a serving loop that forbids

@@ -140,3 +140,22 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _lib.lib()
+
+
+def _attn_prefill(kind=hmd.FA, window=0, B=2, T=100, Hq=8, Hkv=2, d=128, pt=64, n_pages=8,
+                  max_pages=2, ptr=FAKE):
+    return hmd.lib().attn_prefill(kind, window, B, T, Hq, Hkv, d, pt, ptr, ptr, ptr, ptr, ptr,
+                                  n_pages, ptr, max_pages, ptr, None)
+
+
+def test_attn_prefill_validation():
+    assert _attn_prefill(kind=hmd.GDN) == ARG
+    assert _attn_prefill(kind=hmd.SWA, window=0) == ARG
+    assert _attn_prefill(Hq=6, Hkv=4) == SHAPE          # Hq not a multiple of Hkv
+    assert _attn_prefill(Hq=24, Hkv=8) == UNSUP         # group of 3
+    assert _attn_prefill(d=96) == UNSUP
+    assert _attn_prefill(pt=32) == UNSUP
+    assert _attn_prefill(max_pages=1) == SHAPE          # 100 tokens need 2 pages
+    assert _attn_prefill(kind=hmd.SWA, window=200, max_pages=3) == SHAPE  # ring of 4 pages
+    assert _attn_prefill(ptr=None) == ARG
+    assert _attn_prefill(T=0) == 0 and _attn_prefill(B=0) == 0
