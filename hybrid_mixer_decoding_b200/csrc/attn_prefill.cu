@@ -10,8 +10,10 @@
 // One CTA per (sequence, kv-head, block of query tokens): its 128 query rows are the GQA
 // group's G heads x 128/G tokens, so every K/V tile it loads serves all heads of the group. The
 // tiles (64 keys) come from the prompt's own K and V by 3-D TMA boxes with the 128-byte swizzle
-// through a 3-stage ring; each of the 8 warps takes 16 query rows: S = Q K^T and O += P V on
-// mma.sync m16n8k16 (bf16, fp32 accumulate) with an online softmax in the log2 domain. Only
+// through a 2-stage ring (two CTAs per SM); each of the 4 warps takes 32 query rows as two m16
+// tiles that share every K and V fragment it loads (half the shared-memory reads per flop of
+// one tile per warp): S = Q K^T and O += P V on mma.sync m16n8k16 (bf16, fp32 accumulate) with
+// an online softmax in the log2 domain; Q sits in shared memory. Only
 // tiles on the causal diagonal or the window's lower edge are masked; a warp skips a tile none
 // of its rows can see. Query blocks are scheduled longest first.
 // The cache write is fused: each CTA copies its own tokens' K and V of its kv-head to their
@@ -33,9 +35,10 @@ namespace {
 __device__ unsigned int g_err;
 
 constexpr int kPT = 64;        // tokens per page = keys per tile
-constexpr int kStages = 3;     // K/V tiles in flight per CTA
-constexpr int kThreads = 256;  // 8 warps x 16 query rows
+constexpr int kStages = 2;     // K/V tiles in flight per CTA (two CTAs per SM)
+constexpr int kThreads = 128;  // 4 warps x 32 query rows
 constexpr int kRows = 128;     // query rows per CTA: G heads x (128 / G) tokens
+constexpr int kMT = 2;         // m16 tiles per warp
 
 struct PrefillParams {
     const __nv_bfloat16 *q, *k, *v;
@@ -46,15 +49,19 @@ struct PrefillParams {
     float scale_log2;  // log2(e) / sqrt(d)
 };
 
-// Byte offset of the 16-byte chunk holding (row, dim..dim+7) in a tile stored as D/64 halves of
-// [64 rows][128 B] with the TMA 128-byte swizzle (chunk index ^= row % 8).
-__device__ __forceinline__ uint32_t tile_off(int row, int dim) {
-    return (uint32_t)((dim >> 6) * (kPT * 128) + row * 128 + ((((dim & 63) >> 3) ^ (row & 7)) << 4));
+// Byte offset of the 16-byte chunk holding (row, dim..dim+7) in a tile of `rows` rows stored as
+// D/64 halves of [rows][128 B] with the 128-byte swizzle (chunk index ^= row % 8).
+__device__ __forceinline__ uint32_t tile_off(int row, int dim, int rows) {
+    return (uint32_t)((dim >> 6) * (rows * 128) + row * 128 + ((((dim & 63) >> 3) ^ (row & 7)) << 4));
 }
 
 template <int D>
+constexpr int q_bytes() {
+    return kRows * D * 2;
+}
+template <int D>
 constexpr int smem_bytes() {
-    return kStages * 2 * kPT * D * 2 + 1024;
+    return kStages * 2 * kPT * D * 2 + q_bytes<D>() + 1024;
 }
 
 // first key of token t's window
@@ -63,7 +70,7 @@ __device__ __forceinline__ int key_lo(const PrefillParams &p, int t) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                     const PrefillParams p) {
     constexpr int TB = kPT * D * 2;  // bytes of one tile of K or V
@@ -74,6 +81,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const uint32_t smem_base = smem_u32(smem);
+    const uint32_t qs = smem_base + kStages * 2 * TB;  // Q tile [128 rows][D]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // the longest query blocks (the last ones) first
@@ -110,11 +118,25 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
     if (tid == 0)
         for (int i = 0; i < kStages && i < n_tiles; ++i) issue(i);
 
+    // ---- Q tile: row r is head g*G + r / QT, token t_first + r % QT (zero past the prompt) ---
+    {
+        constexpr int CH = D / 8;  // 16-byte chunks per row
+        for (int idx = tid; idx < kRows * CH; idx += kThreads) {
+            const int r = idx / CH, ch = idx - r * CH;
+            const int t = t_first + r % p.QT;
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (t <= t_last)
+                val = *reinterpret_cast<const uint4 *>(
+                    p.q + (((size_t)b * p.T + t) * p.Hq + g * p.G + r / p.QT) * D + ch * 8);
+            *reinterpret_cast<uint4 *>(smem + kStages * 2 * TB + tile_off(r, ch * 8, kRows)) = val;
+        }
+    }
+
     // ---- fused cache write: this block's tokens of kv-head g --------------------------------
     {
         const int ring = p.ring_pages * kPT;
         const int n_tok = t_last - t_first + 1;
-        constexpr int CH = D / 8;  // 16-byte chunks per row
+        constexpr int CH = D / 8;
         for (int idx = tid; idx < n_tok * 2 * CH; idx += kThreads) {
             const int tt = idx / (2 * CH), rem = idx - tt * 2 * CH;
             const bool is_v = rem >= CH;
@@ -134,38 +156,44 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
             *reinterpret_cast<uint4 *>((is_v ? p.v_pool : p.k_pool) + dst) = val;
         }
     }
+    __syncthreads();  // Q tile complete
 
-    // ---- this warp's 16 query rows: row r is head g*G + r / QT, token t_first + r % QT --------
-    const int r0 = 16 * warp + (lane >> 2), r1 = r0 + 8;
-    const int tq0 = t_first + r0 % p.QT, tq1 = t_first + r1 % p.QT;
-    const bool ok0 = tq0 <= t_last, ok1 = tq1 <= t_last;  // rows past the prompt see nothing
-    const int lo0 = key_lo(p, tq0), lo1 = key_lo(p, tq1);
-    const int hq0 = g * p.G + r0 / p.QT, hq1 = g * p.G + r1 / p.QT;
-    // the warp's token range (rows past the prompt excluded)
-    const int t_lo_w = __reduce_min_sync(0xffffffffu, min(ok0 ? tq0 : INT_MAX, ok1 ? tq1 : INT_MAX));
-    const int t_hi_w = __reduce_max_sync(0xffffffffu, max(ok0 ? tq0 : -1, ok1 ? tq1 : -1));
-    const bool all_ok = __all_sync(0xffffffffu, ok0 && ok1);
+    // ---- this warp's 32 rows: m-tile mt holds rows 32 warp + 16 mt + (lane / 4) (+ 8) --------
+    const int cq = (lane & 3) * 2, mi = lane >> 3, l7 = lane & 7;
+    int tq[kMT][2];  // token of each of this thread's 4 rows (rows past the prompt see nothing)
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+            tq[mt][h2] = t_first + (32 * warp + 16 * mt + (lane >> 2) + 8 * h2) % p.QT;
+    int my_lo = INT_MAX, my_hi = -1;
+    bool my_ok = true;
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            if (tq[mt][h2] <= t_last) {
+                my_lo = min(my_lo, tq[mt][h2]);
+                my_hi = max(my_hi, tq[mt][h2]);
+            } else {
+                my_ok = false;
+            }
+        }
+    const int t_lo_w = __reduce_min_sync(0xffffffffu, my_lo);
+    const int t_hi_w = __reduce_max_sync(0xffffffffu, my_hi);
+    const bool all_ok = __all_sync(0xffffffffu, my_ok);
     const int lo_w = t_hi_w >= 0 ? key_lo(p, t_lo_w) : 0;
     const int lo_w_hi = t_hi_w >= 0 ? key_lo(p, t_hi_w) : 0;
 
-    const int cq = (lane & 3) * 2, mi = lane >> 3;
-    uint32_t qa[NK][4];
-    {
-        const uint32_t *q0 = ok0 ? reinterpret_cast<const uint32_t *>(p.q + (((size_t)b * p.T + tq0) * p.Hq + hq0) * D) : nullptr;
-        const uint32_t *q1 = ok1 ? reinterpret_cast<const uint32_t *>(p.q + (((size_t)b * p.T + tq1) * p.Hq + hq1) * D) : nullptr;
+    float m_run[kMT][2], l_run[kMT][2];
+    float oacc[kMT][NN][4];
 #pragma unroll
-        for (int kk = 0; kk < NK; ++kk) {
-            qa[kk][0] = q0 ? q0[(kk * 16 + cq) >> 1] : 0u;
-            qa[kk][1] = q1 ? q1[(kk * 16 + cq) >> 1] : 0u;
-            qa[kk][2] = q0 ? q0[(kk * 16 + 8 + cq) >> 1] : 0u;
-            qa[kk][3] = q1 ? q1[(kk * 16 + 8 + cq) >> 1] : 0u;
-        }
+    for (int mt = 0; mt < kMT; ++mt) {
+        m_run[mt][0] = m_run[mt][1] = -INFINITY;
+        l_run[mt][0] = l_run[mt][1] = 0.f;
+#pragma unroll
+        for (int n = 0; n < NN; ++n) oacc[mt][n][0] = oacc[mt][n][1] = oacc[mt][n][2] = oacc[mt][n][3] = 0.f;
     }
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-    float oacc[NN][4];
-#pragma unroll
-    for (int n = 0; n < NN; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
 
     for (int i = 0; i < n_tiles; ++i) {
         const int s = i % kStages;
@@ -184,75 +212,94 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
         if (needed) {
             const bool masked = !all_ok || j0 + kPT - 1 > t_lo_w || j0 < lo_w_hi;
             const uint32_t kbu = smem_base + s * 2 * TB, vbu = kbu + TB;
-            float sc[8][4];
+            float sc[kMT][8][4];
 #pragma unroll
-            for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+            for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+                for (int n = 0; n < 8; ++n) sc[mt][n][0] = sc[mt][n][1] = sc[mt][n][2] = sc[mt][n][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < NK; ++kk) {
+                uint32_t qa[kMT][4];
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt)
+                    ldmatrix_x4(qs + tile_off(32 * warp + 16 * mt + l7 + ((mi & 1) << 3), kk * 16 + ((mi >> 1) << 3), kRows),
+                                qa[mt][0], qa[mt][1], qa[mt][2], qa[mt][3]);
 #pragma unroll
                 for (int np = 0; np < 4; ++np) {
                     uint32_t b00, b01, b10, b11;
-                    ldmatrix_x4(kbu + tile_off(np * 16 + ((mi >> 1) << 3) + (lane & 7), kk * 16 + ((mi & 1) << 3)),
+                    ldmatrix_x4(kbu + tile_off(np * 16 + ((mi >> 1) << 3) + l7, kk * 16 + ((mi & 1) << 3), kPT),
                                 b00, b01, b10, b11);
-                    mma_bf16_16816(sc[2 * np], qa[kk], b00, b01);
-                    mma_bf16_16816(sc[2 * np + 1], qa[kk], b10, b11);
-                }
-            }
-            float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    bool valid = true;
-                    if (masked) {
-                        const int key = j0 + n * 8 + cq + (e & 1);
-                        valid = (e < 2) ? (ok0 && key >= lo0 && key <= tq0)
-                                        : (ok1 && key >= lo1 && key <= tq1);
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        mma_bf16_16816(sc[mt][2 * np], qa[mt], b00, b01);
+                        mma_bf16_16816(sc[mt][2 * np + 1], qa[mt], b10, b11);
                     }
-                    sc[n][e] = valid ? sc[n][e] * p.scale_log2 : -INFINITY;
-                    mx[e >> 1] = fmaxf(mx[e >> 1], sc[n][e]);
                 }
             }
-            float corr[2], mu[2];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-                mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-                const float mnew = fmaxf(m_run[r], mx[r]);
-                mu[r] = (mnew == -INFINITY) ? 0.f : mnew;
-                corr[r] = exp2f(m_run[r] - mu[r]);
-                m_run[r] = mnew;
-            }
-            float ls[2] = {0.f, 0.f};
+            for (int mt = 0; mt < kMT; ++mt) {
+                float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
+                for (int n = 0; n < 8; ++n) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    sc[n][e] = exp2f(sc[n][e] - mu[e >> 1]);
-                    ls[e >> 1] += sc[n][e];
+                    for (int e = 0; e < 4; ++e) {
+                        bool valid = true;
+                        if (masked) {
+                            const int key = j0 + n * 8 + cq + (e & 1);
+                            const int t = tq[mt][e >> 1];
+                            valid = t <= t_last && key <= t && key >= key_lo(p, t);
+                        }
+                        sc[mt][n][e] = valid ? sc[mt][n][e] * p.scale_log2 : -INFINITY;
+                        mx[e >> 1] = fmaxf(mx[e >> 1], sc[mt][n][e]);
+                    }
                 }
-            }
-            l_run[0] = l_run[0] * corr[0] + ls[0];
-            l_run[1] = l_run[1] * corr[1] + ls[1];
+                float corr[2], mu[2];
 #pragma unroll
-            for (int n = 0; n < NN; ++n) {
-                oacc[n][0] *= corr[0]; oacc[n][1] *= corr[0];
-                oacc[n][2] *= corr[1]; oacc[n][3] *= corr[1];
+                for (int r = 0; r < 2; ++r) {
+                    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+                    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+                    const float mnew = fmaxf(m_run[mt][r], mx[r]);
+                    mu[r] = (mnew == -INFINITY) ? 0.f : mnew;
+                    corr[r] = exp2f(m_run[mt][r] - mu[r]);
+                    m_run[mt][r] = mnew;
+                }
+                float ls[2] = {0.f, 0.f};
+#pragma unroll
+                for (int n = 0; n < 8; ++n) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        sc[mt][n][e] = exp2f(sc[mt][n][e] - mu[e >> 1]);
+                        ls[e >> 1] += sc[mt][n][e];
+                    }
+                }
+                l_run[mt][0] = l_run[mt][0] * corr[0] + ls[0];
+                l_run[mt][1] = l_run[mt][1] * corr[1] + ls[1];
+#pragma unroll
+                for (int n = 0; n < NN; ++n) {
+                    oacc[mt][n][0] *= corr[0]; oacc[mt][n][1] *= corr[0];
+                    oacc[mt][n][2] *= corr[1]; oacc[mt][n][3] *= corr[1];
+                }
             }
 #pragma unroll
             for (int kk2 = 0; kk2 < kPT / 16; ++kk2) {
-                uint32_t pa[4];
-                pa[0] = pack_bf16x2(sc[2 * kk2][0], sc[2 * kk2][1]);
-                pa[1] = pack_bf16x2(sc[2 * kk2][2], sc[2 * kk2][3]);
-                pa[2] = pack_bf16x2(sc[2 * kk2 + 1][0], sc[2 * kk2 + 1][1]);
-                pa[3] = pack_bf16x2(sc[2 * kk2 + 1][2], sc[2 * kk2 + 1][3]);
-                const int key = kk2 * 16 + ((mi & 1) << 3) + (lane & 7);
+                uint32_t pa[kMT][4];
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    pa[mt][0] = pack_bf16x2(sc[mt][2 * kk2][0], sc[mt][2 * kk2][1]);
+                    pa[mt][1] = pack_bf16x2(sc[mt][2 * kk2][2], sc[mt][2 * kk2][3]);
+                    pa[mt][2] = pack_bf16x2(sc[mt][2 * kk2 + 1][0], sc[mt][2 * kk2 + 1][1]);
+                    pa[mt][3] = pack_bf16x2(sc[mt][2 * kk2 + 1][2], sc[mt][2 * kk2 + 1][3]);
+                }
+                const int key = kk2 * 16 + ((mi & 1) << 3) + l7;
 #pragma unroll
                 for (int nn = 0; nn < D / 16; ++nn) {
                     uint32_t v0, v1, v2, v3;
-                    ldmatrix_x4_trans(vbu + tile_off(key, nn * 16 + ((mi >> 1) << 3)), v0, v1, v2, v3);
-                    mma_bf16_16816(oacc[2 * nn], pa, v0, v1);
-                    mma_bf16_16816(oacc[2 * nn + 1], pa, v2, v3);
+                    ldmatrix_x4_trans(vbu + tile_off(key, nn * 16 + ((mi >> 1) << 3), kPT), v0, v1, v2, v3);
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        mma_bf16_16816(oacc[mt][2 * nn], pa[mt], v0, v1);
+                        mma_bf16_16816(oacc[mt][2 * nn + 1], pa[mt], v2, v3);
+                    }
                 }
             }
         }
@@ -265,22 +312,22 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
 
     // ---- normalise and store ------------------------------------------------------------------
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        float l = l_run[r];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        l_run[r] = l > 0.f ? 1.f / l : 0.f;
-    }
-    __nv_bfloat16 *o0 = p.o + (((size_t)b * p.T + tq0) * p.Hq + hq0) * D;
-    __nv_bfloat16 *o1 = p.o + (((size_t)b * p.T + tq1) * p.Hq + hq1) * D;
+    for (int mt = 0; mt < kMT; ++mt) {
 #pragma unroll
-    for (int n = 0; n < NN; ++n) {
-        if (ok0)
-            *reinterpret_cast<uint32_t *>(o0 + n * 8 + cq) =
-                pack_bf16x2(oacc[n][0] * l_run[0], oacc[n][1] * l_run[0]);
-        if (ok1)
-            *reinterpret_cast<uint32_t *>(o1 + n * 8 + cq) =
-                pack_bf16x2(oacc[n][2] * l_run[1], oacc[n][3] * l_run[1]);
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float l = l_run[mt][h2];
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            if (tq[mt][h2] > t_last) continue;
+            const int r = 32 * warp + 16 * mt + (lane >> 2) + 8 * h2;
+            __nv_bfloat16 *orow =
+                p.o + (((size_t)b * p.T + tq[mt][h2]) * p.Hq + g * p.G + r / p.QT) * D;
+#pragma unroll
+            for (int n = 0; n < NN; ++n)
+                *reinterpret_cast<uint32_t *>(orow + n * 8 + cq) =
+                    pack_bf16x2(oacc[mt][n][2 * h2] * inv, oacc[mt][n][2 * h2 + 1] * inv);
+        }
     }
 }
 
