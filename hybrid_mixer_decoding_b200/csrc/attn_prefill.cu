@@ -376,6 +376,7 @@ bool attn_prefill_supported(int d, int page_tokens, int group) {
 
 cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
+    if (attn_prefill_tc_supported(a.d, a.page_tokens, a.Hq / a.Hkv)) return launch_attn_prefill_tc(a, s);
     if (a.d == 128) return launch_d<128>(a, s);
     if (a.d == 64) return launch_d<64>(a, s);
     return cudaErrorInvalidValue;

@@ -89,7 +89,7 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
     *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
             hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_scan_read_errors(clear != 0) |
-            hmd::attn_prefill_read_errors(clear != 0);
+            hmd::attn_prefill_read_errors(clear != 0) | hmd::attn_prefill_tc_read_errors(clear != 0);
     return HMD_OK;
 }
 

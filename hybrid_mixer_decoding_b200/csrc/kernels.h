@@ -110,6 +110,10 @@ struct AttnPrefillArgs {
 bool attn_prefill_supported(int d, int page_tokens, int group);
 cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s);
 uint32_t attn_prefill_read_errors(bool clear);
+// tcgen05 path (d = 128); launch_attn_prefill dispatches to it
+bool attn_prefill_tc_supported(int d, int page_tokens, int group);
+cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s);
+uint32_t attn_prefill_tc_read_errors(bool clear);
 
 // two-pass tensor-core path (bf16, d_k = d_v = 128, chunk 64): a chunk-parallel pass writes one
 // record per chunk to a workspace, a scan pass carries the state through the chunks
