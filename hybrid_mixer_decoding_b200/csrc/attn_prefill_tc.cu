@@ -4,20 +4,22 @@
 // technical summary of "Super Apriel: One Checkpoint, Many Speeds", sections 1 and 2a): token t
 // attends keys [lo_t, t], lo_t = 0 (FA) or max(0, t + 1 - w) (SWA).
 //
-// One CTA of 8 warps per (sequence, kv-head, block of 128/G tokens). Query row r (head
-// g*G + r / QT, token t_first + r % QT) is TMEM lane r of every accumulator; threads r and
-// r + 128 (warps w and w + 4 read the same TMEM lanes) split its columns: each takes half of the
-// row's scores and half of its output, and they exchange one partial maximum per tile. Per
-// 64-key tile i:
-//   S_i = Q K_i^T   tcgen05.mma M=128 N=64 K=128 (Q and K K-major, 128-byte swizzle) into one
-//                   of two TMEM buffers; issued one tile ahead so it overlaps the softmax
-//   softmax         tcgen05.ld of the row, online max / sum in the log2 domain, P_i in bf16 to
-//                   shared memory in the swizzled K-major layout (two buffers)
-//   PV_i = P_i V_i  tcgen05.mma M=128 N=128 K=64 (V MN-major) into TMEM; the next tile reads it
-//                   back and folds it into the fp32 O accumulator held in registers.
-// The accumulators are only ever read from TMEM (tcgen05.ld), never written by the threads. One
-// thread issues the TMA copies (3-stage K/V ring, 3-D boxes from the prompt) and the MMAs;
-// every mbarrier wait is bounded.
+// One CTA per (sequence, kv-head, block of 128/G tokens), warp-specialised:
+//   warp 8 (one lane) issues the TMA copies of the K/V tiles (4-stage ring, 3-D boxes from the
+//     prompt, 128-byte swizzle) and the tcgen05.mma products:
+//       S_i = Q K_i^T   M=128 N=64 K=128 (Q and K K-major) into TMEM buffer i & 1
+//       PV_i = P_i V_i  M=128 N=128 K=64 (P K-major, V MN-major) into TMEM
+//     in the order PV_{i-1}, S_{i+1}, so the tensor core works on them while the softmax warps
+//     process tile i;
+//   warps 0-7 run the softmax: query row r (head g*G + r / QT, token t_first + r % QT) is TMEM
+//     lane r; threads r and r + 128 split its columns (half of the scores, half of the output)
+//     and exchange one partial maximum per tile through a 64-thread named barrier. They read S
+//     and PV with tcgen05.ld, write P (bf16) to shared memory in the swizzled K-major layout,
+//     and keep the fp32 output in registers.
+// The roles hand over through mbarriers only (S full / free, P full, PV full / free), so no
+// CTA-wide barrier sits in the tile loop. Accumulators are only read from TMEM (never written
+// by the threads). Every wait is bounded; a wait that gives up raises a shared abort flag that
+// ends every other wait of the CTA, and the error word reports the call as failed.
 #include <cuda.h>
 #include <float.h>
 
@@ -33,9 +35,10 @@ namespace {
 __device__ unsigned int g_err;
 
 constexpr int kD = 128;
-constexpr int kPT = 64;        // keys per tile = tokens per page
-constexpr int kStages = 3;     // K/V tiles in flight
-constexpr int kThreads = 256;  // threads r and r + 128 share query row r = TMEM lane r
+constexpr int kPT = 64;          // keys per tile = tokens per page
+constexpr int kStages = 4;       // K/V tiles in flight
+constexpr int kSoftmax = 256;    // softmax threads (warps 0-7)
+constexpr int kThreads = kSoftmax + 32;  // + the TMA / MMA warp
 constexpr int kRows = 128;
 constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, PV at 128
 
@@ -45,9 +48,17 @@ constexpr uint32_t OFF_KV = 32768;             // stage s: K at +0, V at +16384 
 constexpr uint32_t STAGE = 32768;
 constexpr uint32_t OFF_P = OFF_KV + kStages * STAGE;  // P [128 rows][64 keys] x 2 buffers
 constexpr uint32_t P_BYTES = 16384;
-constexpr uint32_t OFF_RED = OFF_P + 2 * P_BYTES;     // partial row maxima [2][128] fp32
-constexpr uint32_t OFF_BAR = OFF_RED + 1024;          // full[3], s_done[2], pv_done, tmem slot
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;
+constexpr uint32_t OFF_RED = OFF_P + 2 * P_BYTES;     // partial row maxima [2 tiles][2][128]
+constexpr uint32_t OFF_BAR = OFF_RED + 2048;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+// barrier indices
+constexpr int B_FULL = 0;    // [4] K/V tile landed (TMA)
+constexpr int B_SFULL = 4;   // [2] S_i computed (commit)
+constexpr int B_SFREE = 6;   // [2] S_i read by the 8 softmax warps
+constexpr int B_PFULL = 8;   // [2] P_i written by the 8 softmax warps
+constexpr int B_PVFULL = 10; // PV_i computed (commit)
+constexpr int B_PVFREE = 11; // PV_i read by the 8 softmax warps
+constexpr int N_BARS = 12;
 
 constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);    // A = Q (K-major), B = K (K-major)
 constexpr uint32_t ID_PV = idesc_bf16(128, 128, 0, 1);  // A = P (K-major), B = V (MN-major)
@@ -70,6 +81,24 @@ __device__ __forceinline__ int key_lo(const TcParams &p, int t) {
     return (p.swa && t + 1 > p.window) ? t + 1 - p.window : 0;
 }
 
+// Bounded wait that also gives up as soon as another thread of the CTA raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void pair_barrier(int id) {  // warps w and w + 4 (64 threads)
+    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                        const TcParams p) {
@@ -78,11 +107,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                                               ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    const uint32_t bar_full = smem_u32(&bars[0]);    // + 8 * stage
-    const uint32_t bar_s = smem_u32(&bars[3]);       // + 8 * (tile & 1)
-    const uint32_t bar_pv = smem_u32(&bars[5]);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 48);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * N_BARS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int bg = blockIdx.x % (p.B * p.Hkv);
     const int qb = p.n_qb - 1 - (int)(blockIdx.x / (p.B * p.Hkv));  // longest blocks first
@@ -91,52 +119,33 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     const int t_last = min(p.T, t_first + p.QT) - 1;
 
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&bars[i]), 1);
+        for (int i = 0; i < N_BARS; ++i) {
+            const bool by_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL ||
+                                  i == B_PFULL + 1 || i == B_PVFREE;
+            mbar_init(bar(i), by_warps ? 8 : 1);
+        }
         fence_barrier_init();
+        *abort_flag = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
-    if (warp == 0) {
+    if (warp == 8) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
     griddep_launch_dependents();
     griddep_wait();  // the prompt and the cache may come from the previous kernel
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
 
     const int kb_lo = key_lo(p, t_first) / kPT, kb_hi = t_last / kPT;
     const int n_tiles = kb_hi - kb_lo + 1;
-    auto issue_tile = [&](int i) {  // thread 0
-        const int s = i % kStages;
-        const uint32_t bar = bar_full + 8 * s;
-        mbar_arrive_expect_tx(bar, STAGE);  // K and V tiles: 4 boxes of 8 KiB
-        const uint32_t kb = sb + OFF_KV + s * STAGE, vb = kb + 16384;
-        const int z = b * p.T + (kb_lo + i) * kPT;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(kb + hf * 8192, &tmk, bar, hf * 64, g, z);
-            tma_load_3d(vb + hf * 8192, &tmv, bar, hf * 64, g, z);
-        }
-    };
-    int tiles_issued = 0, s_issued = 0, pv_issued = 0;  // thread 0's bookkeeping
-    if (tid == 0)
-        for (; tiles_issued < 2 && tiles_issued < n_tiles; ++tiles_issued) issue_tile(tiles_issued);
 
-    // ---- row r = tid % 128 (its token, head and window); column half ch = tid / 128 ---------
-    const int row = tid & (kRows - 1), ch = tid >> 7;
+    // ---- Q rows -> shared memory (half a row per softmax thread); fused cache write ----------
+    const int row = tid & (kRows - 1), ch = (tid >> 7) & 1;
     const int t_row = t_first + row % p.QT;
     const bool row_ok = t_row <= t_last;
     const int lo_row = key_lo(p, t_row);
     const int h_row = g * p.G + row / p.QT;
-    float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [2][128]
-
-    // Q row -> shared memory (swizzled K-major A operand), half a row per thread; zero past the
-    // prompt
-    {
+    if (tid < kSoftmax) {
         const uint4 *src = reinterpret_cast<const uint4 *>(
             p.q + (((size_t)b * p.T + (row_ok ? t_row : 0)) * p.Hq + h_row) * kD);
 #pragma unroll
@@ -144,18 +153,15 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             const uint4 v = row_ok ? src[c] : make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(sm + OFF_Q + swz(row, c * 8, kRows)) = v;
         }
-    }
-    // ---- fused cache write: this block's tokens of kv-head g (as attn_prefill.cu) -------------
-    {
         const int ring = p.ring_pages * kPT;
         const int n_tok = t_last - t_first + 1;
         constexpr int CH = kD / 8;
-        for (int idx = tid; idx < n_tok * 2 * CH; idx += kThreads) {
+        for (int idx = tid; idx < n_tok * 2 * CH; idx += kSoftmax) {
             const int tt = idx / (2 * CH), rem = idx - tt * 2 * CH;
             const bool is_v = rem >= CH;
-            const int ch = is_v ? rem - CH : rem;
+            const int chk = is_v ? rem - CH : rem;
             const int t = t_first + tt;
-            if (p.swa && t < p.T - ring) continue;
+            if (p.swa && t < p.T - ring) continue;  // overwritten later in the ring
             const int li = p.swa ? t % ring : t;
             const int lp = li / kPT;
             const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
@@ -163,151 +169,193 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                 atomicOr(&g_err, HMD_DEVERR_PAGE);
                 continue;
             }
-            const size_t srco = (((size_t)b * p.T + t) * p.Hkv + g) * kD + ch * 8;
-            const size_t dsto = (((size_t)pg * p.Hkv + g) * kPT + (li % kPT)) * kD + ch * 8;
+            const size_t srco = (((size_t)b * p.T + t) * p.Hkv + g) * kD + chk * 8;
+            const size_t dsto = (((size_t)pg * p.Hkv + g) * kPT + (li % kPT)) * kD + chk * 8;
             *reinterpret_cast<uint4 *>((is_v ? p.v_pool : p.k_pool) + dsto) =
                 *reinterpret_cast<const uint4 *>((is_v ? p.v : p.k) + srco);
         }
+        fence_proxy_async_smem();  // Q is read by the tensor cores
     }
-    fence_proxy_async_smem();  // Q is read by the tensor cores
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    auto issue_s = [&](int i) {  // thread 0: S_i = Q K_i^T -> TMEM buffer i & 1
-        const uint32_t kbase = sb + OFF_KV + (i % kStages) * STAGE;
+    if (warp == 8) {
+        // ================= TMA and MMA issue (one lane) ================================
+        if (lane == 0) {
+            int tiles_issued = 0, s_issued = 0, pv_issued = 0;
+            auto issue_tile = [&](int i) {
+                const int st = i % kStages;
+                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: 4 boxes of 8 KiB
+                const uint32_t kb = sb + OFF_KV + st * STAGE, vb = kb + 16384;
+                const int z = b * p.T + (kb_lo + i) * kPT;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sb + OFF_Q + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-            umma_bf16(tmem + (i & 1) * 64, ad, bd, ID_S, kk > 0);
-        }
-        umma_commit(bar_s + 8 * (i & 1));
-    };
-    auto issue_pv = [&](int i) {  // thread 0: PV_i = P_i V_i -> TMEM columns 128..255
-        const uint32_t pbase = sb + OFF_P + (i & 1) * P_BYTES;
-        const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + 16384;
-#pragma unroll
-        for (int kk = 0; kk < kPT / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-            umma_bf16(tmem + 128, ad, bd, ID_PV, kk > 0);
-        }
-        umma_commit(bar_pv);
-    };
-
-    bool fail = false;
-    if (tid == 0) {
-        if (mbar_wait_bounded(bar_full, 0)) {
-            tc_fence_after();
-            issue_s(0);
-            s_issued = 1;
-        } else {
-            fail = true;
-        }
-    }
-
-    float o[kD / 2];  // this thread's half of the row's output
-#pragma unroll
-    for (int j = 0; j < kD / 2; ++j) o[j] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
-
-    int i = 0;
-    for (; i < n_tiles; ++i) {
-        // ---- this thread's 32 scores of S_i -> registers ------------------------------------
-        float s[kPT / 2];
-        if (!fail) {
-            if (!mbar_wait_bounded(bar_s + 8 * (i & 1), (i >> 1) & 1)) fail = true;
-        }
-        if (!fail) {
-            tc_fence_after();
-            uint32_t r[32];
-            tmem_ld32(lane_base + (i & 1) * 64 + ch * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
-        }
-        // ---- thread 0: S_{i+1} into the other buffer (read by every thread last iteration) ---
-        if (tid == 0 && !fail && i + 1 < n_tiles) {
-            const int n1 = i + 1;
-            if (mbar_wait_bounded(bar_full + 8 * (n1 % kStages), (n1 / kStages) & 1)) {
-                tc_fence_after();
-                issue_s(n1);
-                ++s_issued;
-            } else {
-                fail = true;
-            }
-        }
-        // ---- mask, scale, partial maximum of this half row -----------------------------------
-        const int j0 = (kb_lo + i) * kPT + ch * 32;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kPT / 2; ++j) {
-            const int key = j0 + j;
-            const bool valid = row_ok && key >= lo_row && key <= t_row;
-            s[j] = valid ? s[j] * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, s[j]);
-        }
-        red[ch * kRows + row] = mx;
-        __syncthreads();
-        // ---- softmax with the row's maximum; P_i half row -> shared memory -------------------
-        const float m_new = fmaxf(m_run, fmaxf(red[row], red[kRows + row]));
-        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        const float corr = exp2f(m_run - mu);
-        m_run = m_new;
-        {
-            float ls = 0.f;
-            uint8_t *prow = sm + OFF_P + (i & 1) * P_BYTES;
-#pragma unroll
-            for (int c = 0; c < kPT / 16; ++c) {
-                float e[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    e[u] = exp2f(s[c * 8 + u] - mu);
-                    ls += e[u];
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_3d(kb + hf * 8192, &tmk, bar(B_FULL + st), hf * 64, g, z);
+                    tma_load_3d(vb + hf * 8192, &tmv, bar(B_FULL + st), hf * 64, g, z);
                 }
-                *reinterpret_cast<uint4 *>(prow + swz(row, ch * 32 + c * 8, kRows)) =
-                    make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
-                               pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
-            }
-            l_run = l_run * corr + ls;
-        }
-        // ---- PV_{i-1} (scale of tile i-1) joins O; then O takes this tile's scale ------------
-        if (i > 0 && !fail) {
-            if (!mbar_wait_bounded(bar_pv, (i - 1) & 1)) fail = true;
-        }
-        if (i > 0 && !fail) {
-            tc_fence_after();
+            };
+            auto issue_s = [&](int i) {
+                const uint32_t kbase = sb + OFF_KV + (i % kStages) * STAGE;
 #pragma unroll
-            for (int c4 = 0; c4 < kD / 64; ++c4) {
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(sb + OFF_Q + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    umma_bf16(tmem + (i & 1) * 64, ad, bd, ID_S, kk > 0);
+                }
+                umma_commit(bar(B_SFULL + (i & 1)));
+            };
+            auto issue_pv = [&](int i) {
+                const uint32_t pbase = sb + OFF_P + (i & 1) * P_BYTES;
+                const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + 16384;
+#pragma unroll
+                for (int kk = 0; kk < kPT / 16; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
+                    umma_bf16(tmem + 128, ad, bd, ID_PV, kk > 0);
+                }
+                umma_commit(bar(B_PVFULL));
+            };
+            bool ok = true;
+            for (; tiles_issued < kStages && tiles_issued < n_tiles; ++tiles_issued) issue_tile(tiles_issued);
+            for (; s_issued < 2 && s_issued < n_tiles && ok; ++s_issued) {
+                ok = wait_or_abort(bar(B_FULL + s_issued % kStages), (s_issued / kStages) & 1, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(s_issued);
+                }
+            }
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                // PV_i: P_i written, PV_{i-1} read
+                ok = wait_or_abort(bar(B_PFULL + (i & 1)), (i >> 1) & 1, abort_flag);
+                if (ok && i > 0) ok = wait_or_abort(bar(B_PVFREE), (i - 1) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(i);
+                pv_issued = i + 1;
+                // S_{i+2} into the buffer S_i used: tile landed, S_i read
+                if (i + 2 < n_tiles) {
+                    ok = wait_or_abort(bar(B_FULL + (i + 2) % kStages), ((i + 2) / kStages) & 1, abort_flag);
+                    if (ok) ok = wait_or_abort(bar(B_SFREE + (i & 1)), (i >> 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(i + 2);
+                    s_issued = i + 3;
+                }
+                // tile i+kStages into the stage tile i used, once PV_i (hence S_i) is done
+                if (tiles_issued < n_tiles) {
+                    ok = wait_or_abort(bar(B_PVFULL), i & 1, abort_flag);
+                    if (!ok) break;
+                    issue_tile(tiles_issued);
+                    ++tiles_issued;
+                }
+            }
+            if (!ok) {
+                // let what this CTA started finish (bounded) before TMEM is freed
+                atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+                if (s_issued > 0)
+                    (void)mbar_wait_bounded(bar(B_SFULL + ((s_issued - 1) & 1)), ((s_issued - 1) >> 1) & 1);
+                if (pv_issued > 0) (void)mbar_wait_bounded(bar(B_PVFULL), (pv_issued - 1) & 1);
+                for (int u = max(0, tiles_issued - kStages); u < tiles_issued; ++u)
+                    (void)mbar_wait_bounded(bar(B_FULL + u % kStages), (u / kStages) & 1);
+            }
+        }
+    } else {
+        // ================= softmax warps ==============================================
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int pair_id = 1 + (warp & 3);
+        float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [2 tiles][2 halves][128]
+        float o[kD / 2];
+#pragma unroll
+        for (int j = 0; j < kD / 2; ++j) o[j] = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
+        // After an abort the loop keeps its shape (every wait then fails at once and the work
+        // and arrivals are skipped), so the two warps of a pair always meet the same barriers.
+        bool ok = true;
+        for (int i = 0; i < n_tiles; ++i) {
+            // ---- this thread's 32 scores of S_i; then hand the buffer back --------------------
+            if (ok) ok = wait_or_abort(bar(B_SFULL + (i & 1)), (i >> 1) & 1, abort_flag);
+            float s[kPT / 2];
+            if (ok) {
+                tc_fence_after();
                 uint32_t r[32];
-                tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
+                tmem_ld32(lane_base + (i & 1) * 64 + ch * 32, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * corr;
+                for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
+                tc_fence_before();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) s[j] = 0.f;
+            }
+            __syncwarp();
+            if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
+            // ---- mask, scale, partial maximum; the row's maximum from the partner thread ------
+            const int j0 = (kb_lo + i) * kPT + ch * 32;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kPT / 2; ++j) {
+                const int key = j0 + j;
+                const bool valid = row_ok && key >= lo_row && key <= t_row;
+                s[j] = valid ? s[j] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, s[j]);
+            }
+            float *rb = red + (i & 1) * 2 * kRows;
+            rb[ch * kRows + row] = mx;
+            pair_barrier(pair_id);
+            const float m_new = fmaxf(m_run, fmaxf(rb[row], rb[kRows + row]));
+            const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+            const float corr = exp2f(m_run - mu);
+            m_run = m_new;
+            // ---- P_i half row -> shared memory (its buffer's last reader, PV_{i-2}, is done) ---
+            {
+                float ls = 0.f;
+                uint8_t *prow = sm + OFF_P + (i & 1) * P_BYTES;
+#pragma unroll
+                for (int c = 0; c < kPT / 16; ++c) {
+                    float e[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        e[u] = exp2f(s[c * 8 + u] - mu);
+                        ls += e[u];
+                    }
+                    if (ok)
+                        *reinterpret_cast<uint4 *>(prow + swz(row, ch * 32 + c * 8, kRows)) =
+                            make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
+                                       pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
+                }
+                l_run = l_run * corr + ls;
+            }
+            fence_proxy_async_smem();  // P is read by the tensor cores
+            __syncwarp();
+            if (ok && lane == 0) mbar_arrive(bar(B_PFULL + (i & 1)));
+            // ---- PV_{i-1} (scale of tile i-1) joins O; O takes this tile's scale --------------
+            if (i > 0) {
+                if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int c4 = 0; c4 < kD / 64; ++c4) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * corr;
+                    }
+                    tc_fence_before();
+                }
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(bar(B_PVFREE));
             }
         }
-        // ---- thread 0: tile i+2 into the stage tile i-1 used (its S and PV are done) ----------
-        if (tid == 0 && !fail && tiles_issued < n_tiles && tiles_issued <= i + 2) {
-            issue_tile(tiles_issued);
-            ++tiles_issued;
-        }
-        // ---- every thread has written P_i and read S_i, PV_{i-1} and the maxima --------------
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(fail)) break;
-        if (tid == 0) {
-            tc_fence_after();
-            issue_pv(i);
-            ++pv_issued;
-        }
-    }
-    const bool aborted = i < n_tiles;
-    if (!aborted) {
+        if (ok) ok = wait_or_abort(bar(B_PVFULL), (n_tiles - 1) & 1, abort_flag);
         // the last PV joins O; the two halves' sums make the row's; normalise and store
-        bool ok = mbar_wait_bounded(bar_pv, (n_tiles - 1) & 1);
-        red[ch * kRows + row] = l_run;
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
-        } else {
+        float *lb = red + (n_tiles & 1) * 2 * kRows;
+        lb[ch * kRows + row] = l_run;
+        pair_barrier(pair_id);
+        if (ok) {
             tc_fence_after();
 #pragma unroll
             for (int c4 = 0; c4 < kD / 64; ++c4) {
@@ -318,7 +366,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                 for (int j = 0; j < 32; ++j) o[c4 * 32 + j] += __uint_as_float(r[j]);
             }
             if (row_ok) {
-                const float l = red[row] + red[kRows + row];
+                const float l = lb[row] + lb[kRows + row];
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 uint4 *dst = reinterpret_cast<uint4 *>(
                     p.o + (((size_t)b * p.T + t_row) * p.Hq + h_row) * kD + ch * 64);
@@ -329,19 +377,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                                         pack_bf16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv),
                                         pack_bf16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv));
             }
+        } else if (lane == 0) {
+            atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
         }
-    } else if (tid == 0) {
-        // a wait gave up: let what this CTA started finish (bounded) before freeing TMEM
-        atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
-        if (s_issued > 0)
-            (void)mbar_wait_bounded(bar_s + 8 * ((s_issued - 1) & 1), ((s_issued - 1) >> 1) & 1);
-        if (pv_issued > 0) (void)mbar_wait_bounded(bar_pv, (pv_issued - 1) & 1);
-        for (int u = max(0, tiles_issued - kStages); u < tiles_issued; ++u)
-            (void)mbar_wait_bounded(bar_full + 8 * (u % kStages), (u / kStages) & 1);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
