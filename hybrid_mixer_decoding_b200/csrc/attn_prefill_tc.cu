@@ -13,11 +13,14 @@
 //     process tile i;
 //   warps 0-7 run the softmax: query row r (head g*G + r / QT, token t_first + r % QT) is TMEM
 //     lane r; threads r and r + 128 split its columns (half of the scores, half of the output)
-//     and exchange one partial maximum per tile through a 64-thread named barrier. They read S
-//     and PV with tcgen05.ld, write P (bf16) to shared memory in the swizzled K-major layout,
-//     and keep the fp32 output in registers.
-// The roles hand over through mbarriers only (S full / free, P full, PV full / free), so no
-// CTA-wide barrier sits in the tile loop. Accumulators are only read from TMEM (never written
+//     and exchange partial maxima through one 256-thread named barrier per tile. They read S
+//     with tcgen05.ld and write P (bf16) to shared memory in the swizzled K-major layout.
+// Lazy rescaling: PV accumulates in TMEM across tiles at a fixed exponent base per row, which
+// moves only when some row's maximum exceeds its base by more than 8 (P stays below 2^8). On
+// such a tile every row folds the TMEM accumulator into an fp32 register accumulator at the new
+// base and the tile's PV restarts the TMEM sum, so the threads never write TMEM.
+// The roles hand over through mbarriers only (S full / free, P full, PV full), so no CTA-wide
+// barrier sits in the tile loop. Accumulators are only read from TMEM (never written
 // by the threads). Every wait is bounded; a wait that gives up raises a shared abort flag that
 // ends every other wait of the CTA, and the error word reports the call as failed.
 #include <cuda.h>
@@ -57,8 +60,8 @@ constexpr int B_SFULL = 4;   // [2] S_i computed (commit)
 constexpr int B_SFREE = 6;   // [2] S_i read by the 8 softmax warps
 constexpr int B_PFULL = 8;   // [2] P_i written by the 8 softmax warps
 constexpr int B_PVFULL = 10; // PV_i computed (commit)
-constexpr int B_PVFREE = 11; // PV_i read by the 8 softmax warps
-constexpr int N_BARS = 12;
+constexpr int N_BARS = 11;
+constexpr float kLazy = 8.f;  // log2 headroom before the exponent base moves
 
 constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);    // A = Q (K-major), B = K (K-major)
 constexpr uint32_t ID_PV = idesc_bf16(128, 128, 0, 1);  // A = P (K-major), B = V (MN-major)
@@ -95,8 +98,8 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     }
 }
 
-__device__ __forceinline__ void pair_barrier(int id) {  // warps w and w + 4 (64 threads)
-    asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+__device__ __forceinline__ void softmax_barrier() {  // warps 0-7 only (named barrier 1)
+    asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -110,6 +113,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * N_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 4);
+    volatile int *restart = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 8);  // [2]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int bg = blockIdx.x % (p.B * p.Hkv);
@@ -121,11 +125,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     if (tid == 0) {
         for (int i = 0; i < N_BARS; ++i) {
             const bool by_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL ||
-                                  i == B_PFULL + 1 || i == B_PVFREE;
+                                  i == B_PFULL + 1;
             mbar_init(bar(i), by_warps ? 8 : 1);
         }
         fence_barrier_init();
         *abort_flag = 0;
+        restart[0] = restart[1] = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
     }
@@ -206,14 +211,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                 }
                 umma_commit(bar(B_SFULL + (i & 1)));
             };
-            auto issue_pv = [&](int i) {
+            auto issue_pv = [&](int i, bool fresh) {  // fresh: restart the TMEM sum
                 const uint32_t pbase = sb + OFF_P + (i & 1) * P_BYTES;
                 const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + 16384;
 #pragma unroll
                 for (int kk = 0; kk < kPT / 16; ++kk) {
                     const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-                    umma_bf16(tmem + 128, ad, bd, ID_PV, kk > 0);
+                    umma_bf16(tmem + 128, ad, bd, ID_PV, (kk > 0 || !fresh) ? 1u : 0u);
                 }
                 umma_commit(bar(B_PVFULL));
             };
@@ -227,12 +232,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                 }
             }
             for (int i = 0; i < n_tiles && ok; ++i) {
-                // PV_i: P_i written, PV_{i-1} read
+                // PV_i: P_i written (and, on a restart tile, the TMEM sum folded into registers)
                 ok = wait_or_abort(bar(B_PFULL + (i & 1)), (i >> 1) & 1, abort_flag);
-                if (ok && i > 0) ok = wait_or_abort(bar(B_PVFREE), (i - 1) & 1, abort_flag);
                 if (!ok) break;
+                const bool fresh = restart[i & 1] != 0;
+                restart[i & 1] = 0;  // every softmax thread read it before arriving
                 tc_fence_after();
-                issue_pv(i);
+                issue_pv(i, fresh || i == 0);
                 pv_issued = i + 1;
                 // S_{i+2} into the buffer S_i used: tile landed, S_i read
                 if (i + 2 < n_tiles) {
@@ -264,14 +270,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     } else {
         // ================= softmax warps ==============================================
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        const int pair_id = 1 + (warp & 3);
         float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [2 tiles][2 halves][128]
-        float o[kD / 2];
+        float o[kD / 2];  // this thread's half of the row's output, at exponent base m_base
 #pragma unroll
         for (int j = 0; j < kD / 2; ++j) o[j] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
+        float m_base = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
         // After an abort the loop keeps its shape (every wait then fails at once and the work
-        // and arrivals are skipped), so the two warps of a pair always meet the same barriers.
+        // and arrivals are skipped), so every softmax thread meets the same barriers.
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             // ---- this thread's 32 scores of S_i; then hand the buffer back --------------------
@@ -291,7 +296,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             }
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
-            // ---- mask, scale, partial maximum; the row's maximum from the partner thread ------
+            // ---- mask, scale, partial maximum; a restart if it outgrows the base ---------------
             const int j0 = (kb_lo + i) * kPT + ch * 32;
             float mx = -INFINITY;
 #pragma unroll
@@ -303,11 +308,34 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             }
             float *rb = red + (i & 1) * 2 * kRows;
             rb[ch * kRows + row] = mx;
-            pair_barrier(pair_id);
-            const float m_new = fmaxf(m_run, fmaxf(rb[row], rb[kRows + row]));
-            const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-            const float corr = exp2f(m_run - mu);
-            m_run = m_new;
+            if (mx > m_base + kLazy) restart[i & 1] = 1;
+            softmax_barrier();
+            const bool fold = restart[i & 1] != 0;
+            if (fold) {
+                // new base per row; the TMEM sum (PV up to i-1) joins the register sum there
+                const float m_new = fmaxf(m_base, fmaxf(rb[row], rb[kRows + row]));
+                const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+                const float f = exp2f(m_base - mu);
+                if (i > 0) {
+                    if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c4 = 0; c4 < kD / 64; ++c4) {
+                            uint32_t r[32];
+                            tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * f;
+                        }
+                        tc_fence_before();
+                    }
+                }
+                l_run *= f;
+                m_base = m_new;
+            }
+            const float mu = (m_base == -INFINITY) ? 0.f : m_base;
             // ---- P_i half row -> shared memory (its buffer's last reader, PV_{i-2}, is done) ---
             {
                 float ls = 0.f;
@@ -325,36 +353,17 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                             make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
                                        pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
                 }
-                l_run = l_run * corr + ls;
+                l_run += ls;
             }
             fence_proxy_async_smem();  // P is read by the tensor cores
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(B_PFULL + (i & 1)));
-            // ---- PV_{i-1} (scale of tile i-1) joins O; O takes this tile's scale --------------
-            if (i > 0) {
-                if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int c4 = 0; c4 < kD / 64; ++c4) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * corr;
-                    }
-                    tc_fence_before();
-                }
-                __syncwarp();
-                if (ok && lane == 0) mbar_arrive(bar(B_PVFREE));
-            }
         }
         if (ok) ok = wait_or_abort(bar(B_PVFULL), (n_tiles - 1) & 1, abort_flag);
-        // the last PV joins O; the two halves' sums make the row's; normalise and store
+        // the TMEM sum joins O (same base); the two halves' sums make the row's; normalise, store
         float *lb = red + (n_tiles & 1) * 2 * kRows;
         lb[ch * kRows + row] = l_run;
-        pair_barrier(pair_id);
+        softmax_barrier();
         if (ok) {
             tc_fence_after();
 #pragma unroll
