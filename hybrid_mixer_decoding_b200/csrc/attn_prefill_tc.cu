@@ -296,16 +296,22 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             }
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
-            // ---- mask, scale, partial maximum; a restart if it outgrows the base ---------------
+            // ---- mask (edge tiles only), partial maximum; a restart if it outgrows the base ----
             const int j0 = (kb_lo + i) * kPT + ch * 32;
             float mx = -INFINITY;
+            if (row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= t_row) {
 #pragma unroll
-            for (int j = 0; j < kPT / 2; ++j) {
-                const int key = j0 + j;
-                const bool valid = row_ok && key >= lo_row && key <= t_row;
-                s[j] = valid ? s[j] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
+                for (int j = 0; j < kPT / 2; ++j) mx = fmaxf(mx, s[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kPT / 2; ++j) {
+                    const int key = j0 + j;
+                    const bool valid = row_ok && key >= lo_row && key <= t_row;
+                    s[j] = valid ? s[j] : -INFINITY;
+                    mx = fmaxf(mx, s[j]);
+                }
             }
+            mx *= p.scale_log2;  // scores and maxima in the log2 domain from here on
             float *rb = red + (i & 1) * 2 * kRows;
             rb[ch * kRows + row] = mx;
             if (mx > m_base + kLazy) restart[i & 1] = 1;
@@ -345,7 +351,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     float e[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        e[u] = exp2f(s[c * 8 + u] - mu);
+                        e[u] = ex2_approx(fmaf(s[c * 8 + u], p.scale_log2, -mu));
                         ls += e[u];
                     }
                     if (ok)
