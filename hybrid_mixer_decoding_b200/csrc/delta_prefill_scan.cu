@@ -15,7 +15,7 @@
 // Pass A (prefill_prep_kernel): one CTA per (sequence, head, chunk), all chunks at once. It
 // computes the gate factors, A and P, the blocked UT solve, W and Ut, and writes one record per
 // chunk: Qt, -W, Kc, P (bf16, already in the 128-byte XOR-swizzled tile layout pass B reads with
-// ldmatrix), e^{G_C} and Ut (fp32).
+// ldmatrix), e^{G_C} and Ut^T (fp32, rows of d_v).
 // Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks in
 // order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
 // the chunk before it computes; the state half lives in registers as MMA accumulator fragments.
@@ -48,7 +48,7 @@ constexpr uint32_t REC_KC = 32768;     // Kc  bf16 [64][128]
 constexpr uint32_t REC_P = 49152;      // P   bf16 [64][64]
 constexpr uint32_t REC_GAM = 57344;    // e^{G_C} fp32 [128]
 constexpr uint32_t REC_HEAD = 57856;   // bytes above, moved by one bulk copy
-constexpr uint32_t REC_UT = 57856;     // Ut  fp32 [64][128], rows of 128 words (see ut_idx)
+constexpr uint32_t REC_UT = 57856;     // Ut^T fp32 [128 d_v][64 tokens] (see utt_idx)
 constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 4;  // 90624
 static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
 
@@ -81,9 +81,9 @@ __device__ __forceinline__ uint32_t toff(int row, int col, int rows) {
                       ((col & 7) << 1));
 }
 
-// word index of fp32 element (row, col) of the Ut block: rows of 128 words, the 8-word groups
-// XOR-permuted by row so that a warp's (row, even column) fragment stores hit distinct banks
-__device__ __forceinline__ int ut_idx(int row, int col) { return row * kD + (col ^ ((row & 7) << 3)); }
+// word index of Ut[token][dv] in the Ut^T block: rows of 64 tokens per d_v column, the 8-word
+// groups XOR-permuted by row so that a warp's fragment stores hit distinct banks
+__device__ __forceinline__ int utt_idx(int dv, int tok) { return dv * kC + (tok ^ ((dv & 7) << 3)); }
 
 __device__ __forceinline__ void st_bf16x2(uint8_t *base, uint32_t off, float lo, float hi) {
     *reinterpret_cast<uint32_t *>(base + off) = pack_bf16x2(lo, hi);
@@ -402,46 +402,74 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
     }
     __syncthreads();
 
-    // ---- Ut = T V and W = T Kt; each warp 16 rows x (128 / NH) columns ---------------------
+    // ---- W = T Kt (warps 4-7, 16 token rows x 128 each) and Ut^T = V^T T^T (warps 0-3,
+    //      32 d_v rows x 64 tokens each) ---------------------------------------------------
     {
-        constexpr int NH = NT / 256;
-        constexpr int NP = 8 / NH;    // 16-column pairs per warp (n-tiles = 2 NP)
-        const int mat = warp / (4 * NH), rt = (warp / NH) & 3, nh = warp % NH;
-        float acc[2 * NP][4];
+        static_assert(NT == 256, "one warp per 16 rows of W, per 32 rows of Ut^T");
+        const int rt = warp & 3;
+        float acc[16][4];
 #pragma unroll
-        for (int i = 0; i < 2 * NP; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-        const uint32_t bbase = sb + (mat ? A_KT : A_V);
+        for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        if (warp >= 4) {
 #pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk) {
-            uint32_t af[4];
-            ldmatrix_x4(sb + A_T + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
-                        af[2], af[3]);
+            for (int kk = 0; kk < kC / 16; ++kk) {
+                uint32_t af[4];
+                ldmatrix_x4(sb + A_T + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
+                            af[2], af[3]);
 #pragma unroll
-            for (int np = 0; np < NP; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(bbase + toff(kk * 16 + l7 + lb3 * 8, 16 * NP * nh + np * 16 + lb4 * 8, 64),
-                                  b0, b1, b2, b3);
-                mma_bf16_16816(acc[2 * np], af, b0, b1);
-                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+                for (int np = 0; np < 8; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(sb + A_KT + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64),
+                                      b0, b1, b2, b3);
+                    mma_bf16_16816(acc[2 * np], af, b0, b1);
+                    mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
+                }
+            }
+        } else {
+            // A = V^T (rows d_v) by transposed loads of V [token][d_v]; B = T^T from T [r][s]
+#pragma unroll
+            for (int kk = 0; kk < kC / 16; ++kk) {
+                uint32_t af[2][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+                    ldmatrix_x4_trans(sb + A_V + toff(kk * 16 + l7 + lb4 * 8, 32 * rt + 16 * mt + lb3 * 8, 64),
+                                      af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(sb + A_T + toff(np * 16 + lb4 * 8 + l7, kk * 16 + lb3 * 8, 64), b0, b1,
+                                b2, b3);
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        mma_bf16_16816(acc[8 * mt + 2 * np], af[mt], b0, b1);
+                        mma_bf16_16816(acc[8 * mt + 2 * np + 1], af[mt], b2, b3);
+                    }
+                }
             }
         }
         if (tid == 0) bulk_wait_group_read0();  // P's bulk store has left the Kh region
-        __syncthreads();  // Kt and V are no longer read: -W and Ut take their place
-        const int r0 = 16 * rt + g, r1 = r0 + 8;
-        if (mat == 1) {
+        __syncthreads();  // Kt and V are no longer read: -W and Ut^T take their place
+        if (warp >= 4) {
+            const int r0 = 16 * rt + g, r1 = r0 + 8;
 #pragma unroll
-            for (int nt = 0; nt < 2 * NP; ++nt) {
-                const int cc = 16 * NP * nh + nt * 8 + 2 * t4;
+            for (int nt = 0; nt < 16; ++nt) {
+                const int cc = nt * 8 + 2 * t4;
                 st_bf16x2(sm + A_KT, toff(r0, cc, 64), -acc[nt][0], -acc[nt][1]);
                 st_bf16x2(sm + A_KT, toff(r1, cc, 64), -acc[nt][2], -acc[nt][3]);
             }
         } else {
             float *ut = reinterpret_cast<float *>(sm + A_KH);
 #pragma unroll
-            for (int nt = 0; nt < 2 * NP; ++nt) {
-                const int cc = 16 * NP * nh + nt * 8 + 2 * t4;
-                *reinterpret_cast<float2 *>(ut + ut_idx(r0, cc)) = make_float2(acc[nt][0], acc[nt][1]);
-                *reinterpret_cast<float2 *>(ut + ut_idx(r1, cc)) = make_float2(acc[nt][2], acc[nt][3]);
+            for (int mt = 0; mt < 2; ++mt) {
+                const int d0 = 32 * rt + 16 * mt + g, d1 = d0 + 8;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    const int tk = nt * 8 + 2 * t4;
+                    *reinterpret_cast<float2 *>(ut + utt_idx(d0, tk)) =
+                        make_float2(acc[8 * mt + nt][0], acc[8 * mt + nt][1]);
+                    *reinterpret_cast<float2 *>(ut + utt_idx(d1, tk)) =
+                        make_float2(acc[8 * mt + nt][2], acc[8 * mt + nt][3]);
+                }
             }
         }
     }
@@ -517,9 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
-            const float2 x0 = *reinterpret_cast<const float2 *>(ut + ut_idx(ur0, cc));
-            const float2 x1 = *reinterpret_cast<const float2 *>(ut + ut_idx(ur1, cc));
-            un[j][0] = x0.x; un[j][1] = x0.y; un[j][2] = x1.x; un[j][3] = x1.y;
+            un[j][0] = ut[utt_idx(cc, ur0)];
+            un[j][1] = ut[utt_idx(cc + 1, ur0)];
+            un[j][2] = ut[utt_idx(cc, ur1)];
+            un[j][3] = ut[utt_idx(cc + 1, ur1)];
         }
     };
     load_ut(0);
