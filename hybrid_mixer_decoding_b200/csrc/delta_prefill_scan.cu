@@ -53,20 +53,32 @@ constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 4;  // 90624
 static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
 
 // ---- pass A shared memory (bytes from a 1024-aligned base) ---------------------------------
-constexpr uint32_t A_KT = 0;           // Kt [64][128]; at the end -W (bf16, record layout)
-constexpr uint32_t A_QT = 16384;       // q, then Qt [64][128]
-constexpr uint32_t A_KH = 32768;       // k, then Kh [64][128]; then P + e^{G_C}; at the end
-constexpr uint32_t A_V = 49152;        //   Ut fp32 across Kh and V (32 KiB, record layout)
-constexpr uint32_t A_G = 65536;        // KDA log-gates -> in-chunk prefix, fp32 [64][128]
+constexpr uint32_t A_KQ = 0;           // [Kt; Qt], the K-major A operand of one M = 128 product:
+                                       //   two 64-column halves of 128 rows (16 KiB each), Kt in
+                                       //   rows 0-63, q then Qt in rows 64-127; at the end -W
+                                       //   (record layout) in the Kt rows; Kt is also read
+                                       //   MN-major (halves 16 KiB apart)
+constexpr uint32_t A_KH = 32768;       // k, then Kh [64][128] (K-major B operand); then P, e^{G_C}
+constexpr uint32_t A_V = 49152;        // v [64][128] (MN-major A operand)
+constexpr uint32_t A_G = 65536;        // KDA log-gates -> in-chunk prefix, fp32 [4][64][32]
 constexpr uint32_t A_AS = 65536;       // after the gate pass: A fp32 [64][68], then T bf16
 constexpr uint32_t A_XS = 82944;       // X fp32 [64][68]
 constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
+constexpr uint32_t A_UT = 65536;       // at the end: Ut^T fp32 (record layout, 32 KiB)
 constexpr uint32_t A_SMALL = 104192;
-constexpr uint32_t A_SMEM = A_SMALL + 3584 + 1024;
+constexpr uint32_t S_BETA = 0, S_QOFF = 256, S_LGP = 1280, S_WSUM = 1536, S_EGC = 1552,
+                   S_BAR = 2064, S_TMEM = 2080, S_SIZE = 2112;
+constexpr uint32_t A_SMEM = A_SMALL + S_SIZE + 1024;
 constexpr uint32_t A_T = A_AS;
 constexpr int AS_LD = 68;
 constexpr int YS_LD = 20;
+constexpr uint32_t kPrepTmemCols = 128;
+constexpr uint32_t ID_AP = idesc_bf16(128, 64, 0, 0);  // [Kt; Qt] Kh^T: both operands K-major
+constexpr uint32_t ID_WU = idesc_bf16(128, 64, 1, 0);  // Kt^T T^T, V^T T^T: A MN-major
 static_assert(A_G + kC * kD * 4 <= A_YS, "log-gate staging fits the A/X region");
+static_assert(A_UT + kC * kD * 4 <= A_YS, "Ut^T fits the A/X region");
+static_assert(S_QOFF + (kPrepThreads / kD) * kD * 4 <= S_LGP, "gate part sums fit");
+static_assert(S_BAR % 8 == 0 && S_TMEM + 4 <= S_SIZE, "small area");
 
 // ---- pass B shared memory ----------------------------------------------------------------
 constexpr uint32_t B_STAGE = 58368;        // one record head, padded to 1 KiB
@@ -84,6 +96,10 @@ __device__ __forceinline__ uint32_t toff(int row, int col, int rows) {
 // word index of Ut[token][dv] in the Ut^T block: rows of 64 tokens per d_v column, the 8-word
 // groups XOR-permuted by row so that a warp's fragment stores hit distinct banks
 __device__ __forceinline__ int utt_idx(int dv, int tok) { return dv * kC + (tok ^ ((dv & 7) << 3)); }
+
+// float index of log-gate (row r, channel i) in the staged KDA gate tile: four TMA boxes of
+// [64 rows][32 channels]
+__device__ __forceinline__ int gidx(int r, int i) { return (i >> 5) * 2048 + r * 32 + (i & 31); }
 
 __device__ __forceinline__ void st_bf16x2(uint8_t *base, uint32_t off, float lo, float hi) {
     *reinterpret_cast<uint32_t *>(base + off) = pack_bf16x2(lo, hi);
@@ -154,7 +170,10 @@ __device__ __forceinline__ void solve_level(const float *As, float *Xs, float *Y
 }
 
 template <bool KDA>
-__global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const PrefillScanArgs a) {
+__global__ void __launch_bounds__(kPrepThreads, 2)
+prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmg,
+                    const PrefillScanArgs a) {
     constexpr int NT = kPrepThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,99 +183,109 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
     float *As = reinterpret_cast<float *>(sm + A_AS);
     float *Xs = reinterpret_cast<float *>(sm + A_XS);
     float *Ys = reinterpret_cast<float *>(sm + A_YS);
-    float *sbeta = reinterpret_cast<float *>(sm + A_SMALL);  // [64]
-    float *qoff = sbeta + 64;                                 // [NQ][128] KDA: gate sums of
-                                                              //   the row parts, then their
-                                                              //   exclusive prefix
-    float *lgp = qoff + 512;                                  // [64] GDN log-gate prefix
-    float *wsum = lgp + 64;                                   // [2]
-    float *egc = wsum + 2;                                    // [128] e^{G_C}
+    float *sbeta = reinterpret_cast<float *>(sm + A_SMALL + S_BETA);  // [64]
+    float *qoff = reinterpret_cast<float *>(sm + A_SMALL + S_QOFF);   // [NQ][128] KDA: gate sums
+                                                                       //   of the row parts, then
+                                                                       //   their exclusive prefix
+    float *lgp = reinterpret_cast<float *>(sm + A_SMALL + S_LGP);     // [64] GDN log-gate prefix
+    float *wsum = reinterpret_cast<float *>(sm + A_SMALL + S_WSUM);   // [2]
+    float *egc = reinterpret_cast<float *>(sm + A_SMALL + S_EGC);     // [128] e^{G_C}
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + A_SMALL + S_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + A_SMALL + S_TMEM);
 
     constexpr int NQ = NT / kD;       // KDA gate prefix: row parts per channel
     constexpr int RPQ = kC / NQ;      // rows per part
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t4 = lane & 3;
-    const int l7 = lane & 7, lb3 = (lane >> 3) & 1, lb4 = lane >> 4;
     const int bh = blockIdx.x / a.n_seg, c = blockIdx.x - bh * a.n_seg;
     const int b = bh / a.H, h = bh - b * a.H;
     const int T = a.T;
     const int t0 = (a.chunk_begin + c) * kC;
     const int n = min(kC, T - t0);
     uint8_t *rec = record(a, bh, c);
-    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
-    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
-    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v);
+    const uint32_t bar_in = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_mma, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmq);
+        prefetch_tmap(&tmk);
+        prefetch_tmap(&tmv);
+        if constexpr (KDA) prefetch_tmap(&tmg);
+    }
     griddep_launch_dependents();
     griddep_wait();  // the inputs may come from the previous kernel
+    if (warp == 0) {
+        __syncwarp();
+        tmem_alloc(smem_u32(tmem_slot), kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    // ---- stage q (into the Qt slot), k (into the Kh slot), v, KDA log-gates; beta ----------
-    {
-        constexpr int J16 = kC * kD / 8 / NT;  // 16-byte pieces of a bf16 tile per thread
-        constexpr int JG = kC * kD / 4 / NT;   // float4 pieces of the KDA gate tile per thread
-        const size_t row0 = ((size_t)b * T + t0) * a.H + h;  // token t0's row in [B][T][H]
-        uint4 qv[J16], kv[J16], vv[J16];
-#pragma unroll
-        for (int j = 0; j < J16; ++j) {
-            const int idx = tid + j * NT, r = idx >> 4, ch = idx & 15;
-            qv[j] = kv[j] = vv[j] = make_uint4(0, 0, 0, 0);
-            if (r < n) {
-                const size_t off = (row0 + (size_t)r * a.H) * kD + ch * 8;
-                qv[j] = __ldg(reinterpret_cast<const uint4 *>(qg + off));
-                kv[j] = __ldg(reinterpret_cast<const uint4 *>(kg + off));
-                vv[j] = __ldg(reinterpret_cast<const uint4 *>(vg + off));
-            }
+    // Abort after a wait gave up: let the copies and products in flight end (bounded), free
+    // the tensor memory, report. Every thread of the CTA takes this path together.
+    auto abort_cta = [&](uint32_t bar, uint32_t parity) {
+        if (tid == 0) {
+            atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+            (void)mbar_wait_bounded(bar, parity);
+            bulk_wait_group_read0();
         }
-        float4 gv[JG];
-        if constexpr (KDA) {
-#pragma unroll
-            for (int j = 0; j < JG; ++j) {
-                const int idx = tid + j * NT, r = idx >> 5, c4 = idx & 31;
-                gv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r < n)
-                    gv[j] = __ldg(reinterpret_cast<const float4 *>(a.log_gate + (row0 + (size_t)r * a.H) * kD + c4 * 4));
-            }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) {
+            __syncwarp();
+            tc_fence_after();
+            tmem_dealloc(tmem, kPrepTmemCols);
         }
+    };
+
+    // ---- inputs: q (into the Qt rows), k (into the Kh slot), v, KDA log-gates by TMA; rows
+    //      past the end of the sequence read as zero. beta and the GDN log-gates by plain loads.
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_in, (KDA ? 10u : 6u) * 8192u);
 #pragma unroll
-        for (int j = 0; j < J16; ++j) {
-            const int idx = tid + j * NT, r = idx >> 4, ch = idx & 15;
-            const uint32_t o = toff(r, ch * 8, 64);
-            *reinterpret_cast<uint4 *>(sm + A_QT + o) = qv[j];
-            *reinterpret_cast<uint4 *>(sm + A_KH + o) = kv[j];
-            *reinterpret_cast<uint4 *>(sm + A_V + o) = vv[j];
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(sb + A_KQ + hf * 16384 + 8192, &tmq, bar_in, hf * 64, h, t0, b);
+            tma_load_4d(sb + A_KH + hf * 8192, &tmk, bar_in, hf * 64, h, t0, b);
+            tma_load_4d(sb + A_V + hf * 8192, &tmv, bar_in, hf * 64, h, t0, b);
         }
         if constexpr (KDA) {
 #pragma unroll
-            for (int j = 0; j < JG; ++j) {
-                const int idx = tid + j * NT, r = idx >> 5, c4 = idx & 31;
-                *reinterpret_cast<float4 *>(Gs + r * kD + c4 * 4) = gv[j];
-            }
-        }
-        if (tid < kC) {
-            const size_t tok = row0 + (size_t)tid * a.H;
-            sbeta[tid] = tid < n ? a.beta[tok] : 0.f;
-            if constexpr (!KDA) {
-                float x = tid < n ? a.log_gate[tok] : 0.f;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if (lane >= off) x += y;
-                }
-                if (lane == 31) wsum[warp] = x;
-                lgp[tid] = x;
-            }
+            for (int j = 0; j < 4; ++j) tma_load_4d(sb + A_G + j * 8192, &tmg, bar_in, j * 32, h, t0, b);
         }
     }
-    __syncthreads();
+    if (tid < kC) {
+        const size_t tok = ((size_t)b * T + t0 + tid) * a.H + h;
+        sbeta[tid] = tid < n ? a.beta[tok] : 0.f;
+        if constexpr (!KDA) {
+            float x = tid < n ? a.log_gate[tok] : 0.f;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (lane == 31) wsum[warp] = x;
+            lgp[tid] = x;
+        }
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(bar_in, 0))) {
+        abort_cta(bar_in, 0);
+        return;
+    }
 
     // ---- gate prefix G (log domain): KDA per channel in place within NQ row parts, plus the
     //      parts' exclusive prefix; GDN per token -------------------------------------------------
     if constexpr (KDA) {
         const int i = tid & (kD - 1), qr = tid >> 7;
+        float *gcol = Gs + gidx(0, i);
         float run = 0.f;
 #pragma unroll
         for (int r = RPQ * qr; r < RPQ * qr + RPQ; ++r) {
-            run += Gs[r * kD + i];
-            Gs[r * kD + i] = run;
+            run += gcol[r * 32];
+            gcol[r * 32] = run;
         }
         qoff[qr * kD + i] = run;
         __syncthreads();
@@ -285,12 +314,13 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
         for (int j = 0; j < kC * kD / 8 / NT; ++j) {
             const int idx = tid + j * NT, r = idx >> 4, c0 = (idx & 15) * 8;
             const uint32_t o = toff(r, c0, 64);
-            const uint4 qr = *reinterpret_cast<const uint4 *>(sm + A_QT + o);
+            const uint32_t okt = A_KQ + toff(r, c0, 128), oqt = A_KQ + toff(64 + r, c0, 128);
+            const uint4 qr = *reinterpret_cast<const uint4 *>(sm + oqt);
             const uint4 kr = *reinterpret_cast<const uint4 *>(sm + A_KH + o);
             float G[8];
             if constexpr (KDA) {
-                const float4 g0 = *reinterpret_cast<const float4 *>(Gs + r * kD + c0);
-                const float4 g1 = *reinterpret_cast<const float4 *>(Gs + r * kD + c0 + 4);
+                const float4 g0 = *reinterpret_cast<const float4 *>(Gs + gidx(r, c0));
+                const float4 g1 = *reinterpret_cast<const float4 *>(Gs + gidx(r, c0) + 4);
                 const float4 f0 = *reinterpret_cast<const float4 *>(qoff + (r / RPQ) * kD + c0);
                 const float4 f1 = *reinterpret_cast<const float4 *>(qoff + (r / RPQ) * kD + c0 + 4);
                 G[0] = g0.x + f0.x; G[1] = g0.y + f0.y; G[2] = g0.z + f0.z; G[3] = g0.w + f0.w;
@@ -313,61 +343,71 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
                 kh[e] = pack_bf16x2(ka * ia, kb * ib);
                 kcw[e] = pack_bf16x2(ka * (egc[c0 + 2 * e] * ia), kb * (egc[c0 + 2 * e + 1] * ib));
             }
-            *reinterpret_cast<uint4 *>(sm + A_KT + o) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
-            *reinterpret_cast<uint4 *>(sm + A_QT + o) = make_uint4(qt[0], qt[1], qt[2], qt[3]);
+            *reinterpret_cast<uint4 *>(sm + okt) = make_uint4(kt[0], kt[1], kt[2], kt[3]);
+            *reinterpret_cast<uint4 *>(sm + oqt) = make_uint4(qt[0], qt[1], qt[2], qt[3]);
             *reinterpret_cast<uint4 *>(sm + A_KH + o) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
             *reinterpret_cast<uint4 *>(kc + o) = make_uint4(kcw[0], kcw[1], kcw[2], kcw[3]);
         }
     }
-    fence_proxy_async_smem();
+    fence_proxy_async_smem();  // the tiles are read by the tensor cores and the bulk copies
     __syncthreads();
-    if (tid == 0) {  // Qt -> record
-        bulk_store(rec + REC_QT, sb + A_QT, 16384);
-        bulk_commit_group();
-    }
 
-    // ---- A and P: [Kt | Qt] Kh^T; each warp 16 rows x (64 / NH) columns -------------------
-    {
-        constexpr int NH = NT / 256;  // warps per 16-row strip of A or P
-        constexpr int NP = 4 / NH;    // 16-column pairs per warp (n-tiles = 2 NP)
-        const int mat = warp / (4 * NH), rt = (warp / NH) & 3, nh = warp % NH;
-        const uint32_t abase = sb + (mat ? A_QT : A_KT);
-        float acc[2 * NP][4];
-#pragma unroll
-        for (int i = 0; i < 2 * NP; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    // ---- [A_raw; P] = [Kt; Qt] Kh^T: one M = 128, N = 64, K = 128 product into TMEM columns
+    //      0-63 (lanes 0-63 the rows of Kt Kh^T, lanes 64-127 those of Qt Kh^T); Qt -> record
+    if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-            uint32_t af[4];
-            ldmatrix_x4(abase + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
-                        af[2], af[3]);
-#pragma unroll
-            for (int np = 0; np < NP; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(sb + A_KH + toff(16 * NP * nh + np * 16 + l7 + lb4 * 8, kk * 16 + lb3 * 8, 64),
-                            b0, b1, b2, b3);
-                mma_bf16_16816(acc[2 * np], af, b0, b1);
-                mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
-            }
+            const uint64_t ad = smem_desc_sw128(sb + A_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + A_KH + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+            umma_bf16(tmem, ad, bd, ID_AP, kk > 0 ? 1u : 0u);
         }
-        __syncthreads();  // Kh is read by every warp above; P and e^{G_C} take its place below
-        const int r0 = 16 * rt + g, r1 = r0 + 8;
+        umma_commit(bar_mma);
+        bulk_store(rec + REC_QT, sb + A_KQ + 8192, 8192);
+        bulk_store(rec + REC_QT + 8192, sb + A_KQ + 16384 + 8192, 8192);
+        bulk_commit_group();
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(bar_mma, 0))) {
+        abort_cta(bar_mma, 0);
+        return;
+    }
+    tc_fence_after();
+    {
+        // warp w reads TMEM lanes 32 (w & 3) .. +31 (one row each), columns 32 (w >> 2) .. +31
+        const int quad = warp & 3, s0 = 32 * (warp >> 2);
+        uint32_t d[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + s0, d);
+        tmem_wait_ld();
+        if (quad < 2) {  // A_rs = beta_r (Kt Kh^T)_rs, s < r, fp32 for the solve
+            const int r = 32 * quad + lane;
+            const float br = r < n ? sbeta[r] : 0.f;
+            float *arow = As + r * AS_LD + s0;
 #pragma unroll
-        for (int nt = 0; nt < 2 * NP; ++nt) {
-            const int s0 = 16 * NP * nh + nt * 8 + 2 * t4;
-            if (mat == 0) {
-                As[r0 * AS_LD + s0] = (s0 < r0 && r0 < n) ? sbeta[r0] * acc[nt][0] : 0.f;
-                As[r0 * AS_LD + s0 + 1] = (s0 + 1 < r0 && r0 < n) ? sbeta[r0] * acc[nt][1] : 0.f;
-                As[r1 * AS_LD + s0] = (s0 < r1 && r1 < n) ? sbeta[r1] * acc[nt][2] : 0.f;
-                As[r1 * AS_LD + s0 + 1] = (s0 + 1 < r1 && r1 < n) ? sbeta[r1] * acc[nt][3] : 0.f;
-            } else {
-                st_bf16x2(sm + A_KH, toff(r0, s0, 64), (s0 <= r0 && r0 < n) ? acc[nt][0] : 0.f,
-                          (s0 + 1 <= r0 && r0 < n) ? acc[nt][1] : 0.f);
-                st_bf16x2(sm + A_KH, toff(r1, s0, 64), (s0 <= r1 && r1 < n) ? acc[nt][2] : 0.f,
-                          (s0 + 1 <= r1 && r1 < n) ? acc[nt][3] : 0.f);
+            for (int j4 = 0; j4 < 8; ++j4) {
+                float v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    v[e] = (s0 + 4 * j4 + e < r) ? br * __uint_as_float(d[4 * j4 + e]) : 0.f;
+                *reinterpret_cast<float4 *>(arow + 4 * j4) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+        } else {  // P_rs = (Qt Kh^T)_rs, s <= r, bf16 into the (now free) Kh slot
+            const int r = 32 * (quad - 2) + lane;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int s = s0 + 8 * u + 2 * e;
+                    w[e] = pack_bf16x2((s <= r && r < n) ? __uint_as_float(d[8 * u + 2 * e]) : 0.f,
+                                       (s + 1 <= r && r < n) ? __uint_as_float(d[8 * u + 2 * e + 1]) : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(sm + A_KH + toff(r, s0 + 8 * u, 64)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
         if (tid < kD) reinterpret_cast<float *>(sm + A_KH + 8192)[tid] = egc[tid];
     }
+    tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {  // P and e^{G_C} (contiguous in the record) -> record
@@ -393,93 +433,77 @@ __global__ void __launch_bounds__(kPrepThreads, 2) prefill_prep_kernel(const Pre
     solve_level<1>(As, Xs, Ys, tid);
     solve_level<2>(As, Xs, Ys, tid);
     solve_level<3>(As, Xs, Ys, tid);
-    // T overwrites A (no longer read)
+    // T overwrites A (no longer read): [r][s] bf16, the K-major B operand below
     for (int idx = tid; idx < 64 * 32; idx += NT) {
         const int r = idx >> 5, s0 = (idx & 31) * 2;
         const float v0 = s0 <= r ? Xs[r * AS_LD + s0] * sbeta[s0] : 0.f;
         const float v1 = s0 + 1 <= r ? Xs[r * AS_LD + s0 + 1] * sbeta[s0 + 1] : 0.f;
         st_bf16x2(sm + A_T, toff(r, s0, 64), v0, v1);
     }
+    fence_proxy_async_smem();
     __syncthreads();
 
-    // ---- W = T Kt (warps 4-7, 16 token rows x 128 each) and Ut^T = V^T T^T (warps 0-3,
-    //      32 d_v rows x 64 tokens each) ---------------------------------------------------
-    {
-        static_assert(NT == 256, "one warp per 16 rows of W, per 32 rows of Ut^T");
-        const int rt = warp & 3;
-        float acc[16][4];
+    // ---- W^T = Kt^T T^T and Ut^T = V^T T^T: M = 128 (d), N = 64 (r), K = 64 (s), with Kt and V
+    //      read MN-major; W^T into TMEM columns 64-127, Ut^T into columns 0-63 -----------------
+    if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-        if (warp >= 4) {
-#pragma unroll
-            for (int kk = 0; kk < kC / 16; ++kk) {
-                uint32_t af[4];
-                ldmatrix_x4(sb + A_T + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), af[0], af[1],
-                            af[2], af[3]);
-#pragma unroll
-                for (int np = 0; np < 8; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(sb + A_KT + toff(kk * 16 + l7 + lb3 * 8, np * 16 + lb4 * 8, 64),
-                                      b0, b1, b2, b3);
-                    mma_bf16_16816(acc[2 * np], af, b0, b1);
-                    mma_bf16_16816(acc[2 * np + 1], af, b2, b3);
-                }
-            }
-        } else {
-            // A = V^T (rows d_v) by transposed loads of V [token][d_v]; B = T^T from T [r][s]
-#pragma unroll
-            for (int kk = 0; kk < kC / 16; ++kk) {
-                uint32_t af[2][4];
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-                    ldmatrix_x4_trans(sb + A_V + toff(kk * 16 + l7 + lb4 * 8, 32 * rt + 16 * mt + lb3 * 8, 64),
-                                      af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(sb + A_T + toff(np * 16 + lb4 * 8 + l7, kk * 16 + lb3 * 8, 64), b0, b1,
-                                b2, b3);
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        mma_bf16_16816(acc[8 * mt + 2 * np], af[mt], b0, b1);
-                        mma_bf16_16816(acc[8 * mt + 2 * np + 1], af[mt], b2, b3);
-                    }
-                }
-            }
+        for (int kk = 0; kk < kC / 16; ++kk) {
+            const uint64_t bd = smem_desc_sw128(sb + A_T + kk * 32, 16, 1024);
+            const uint64_t aw = smem_desc_sw128(sb + A_KQ + kk * 2048, 16384, 1024);
+            const uint64_t au = smem_desc_sw128(sb + A_V + kk * 2048, 8192, 1024);
+            umma_bf16(tmem + 64, aw, bd, ID_WU, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem, au, bd, ID_WU, kk > 0 ? 1u : 0u);
         }
-        if (tid == 0) bulk_wait_group_read0();  // P's bulk store has left the Kh region
-        __syncthreads();  // Kt and V are no longer read: -W and Ut^T take their place
-        if (warp >= 4) {
-            const int r0 = 16 * rt + g, r1 = r0 + 8;
+        umma_commit(bar_mma);
+    }
+    if (__syncthreads_or(!mbar_wait_bounded(bar_mma, 1))) {
+        abort_cta(bar_mma, 1);
+        return;
+    }
+    tc_fence_after();
+    {
+        const int quad = warp & 3, dd = 32 * quad + lane;  // this thread's row of d_k or d_v
+        uint32_t d[32];
+        if (warp < 4) {  // -W [r][d_k] bf16 (record layout) into the Kt rows of both halves
+            uint8_t *wb = sm + A_KQ + (dd >> 6) * 16384;
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const int cc = nt * 8 + 2 * t4;
-                st_bf16x2(sm + A_KT, toff(r0, cc, 64), -acc[nt][0], -acc[nt][1]);
-                st_bf16x2(sm + A_KT, toff(r1, cc, 64), -acc[nt][2], -acc[nt][3]);
+            for (int hr = 0; hr < 2; ++hr) {
+                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 64 + 32 * hr, d);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    *reinterpret_cast<__nv_bfloat16 *>(wb + toff(32 * hr + j, dd & 63, 64)) =
+                        __float2bfloat16_rn(-__uint_as_float(d[j]));
             }
-        } else {
-            float *ut = reinterpret_cast<float *>(sm + A_KH);
+        } else {  // Ut^T fp32 [d_v][64 tokens] (record layout)
+            float *ut = reinterpret_cast<float *>(sm + A_UT);
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const int d0 = 32 * rt + 16 * mt + g, d1 = d0 + 8;
+            for (int hr = 0; hr < 2; ++hr) {
+                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * hr, d);
+                tmem_wait_ld();
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                    const int tk = nt * 8 + 2 * t4;
-                    *reinterpret_cast<float2 *>(ut + utt_idx(d0, tk)) =
-                        make_float2(acc[8 * mt + nt][0], acc[8 * mt + nt][1]);
-                    *reinterpret_cast<float2 *>(ut + utt_idx(d1, tk)) =
-                        make_float2(acc[8 * mt + nt][2], acc[8 * mt + nt][3]);
-                }
+                for (int j4 = 0; j4 < 8; ++j4)
+                    *reinterpret_cast<float4 *>(ut + utt_idx(dd, 32 * hr + 4 * j4)) =
+                        make_float4(__uint_as_float(d[4 * j4]), __uint_as_float(d[4 * j4 + 1]),
+                                    __uint_as_float(d[4 * j4 + 2]), __uint_as_float(d[4 * j4 + 3]));
             }
         }
     }
+    tc_fence_before();
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_store(rec + REC_NW, sb + A_KT, 16384);
-        bulk_store(rec + REC_UT, sb + A_KH, 32768);
+        bulk_store(rec + REC_NW, sb + A_KQ, 8192);
+        bulk_store(rec + REC_NW + 8192, sb + A_KQ + 16384, 8192);
+        bulk_store(rec + REC_UT, sb + A_UT, 32768);
         bulk_commit_group();
         bulk_wait_group_read0();  // shared memory must outlive the copies' reads
+    }
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kPrepTmemCols);
     }
 }
 
@@ -702,6 +726,18 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
     const long long fit = (long long)(ws_bytes / ((size_t)bhs * REC_BYTES));
     if (fit < 1 || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
     const int seg = (int)std::min<long long>(n_chunks, fit);
+    CUtensorMap tmq, tmk, tmv, tmg;
+    if (!make_tmap_bthd(&tmq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.q, a.B, a.T, a.H, kD, 64, true) ||
+        !make_tmap_bthd(&tmk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.k, a.B, a.T, a.H, kD, 64, true) ||
+        !make_tmap_bthd(&tmv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.v, a.B, a.T, a.H, kD, 64, true))
+        return cudaErrorInvalidValue;
+    if (a.kind == HMD_KDA) {
+        if (!make_tmap_bthd(&tmg, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.log_gate, a.B, a.T, a.H, kD,
+                            32, false))
+            return cudaErrorInvalidValue;
+    } else {
+        tmg = tmq;  // not read
+    }
     PrefillScanArgs p;
     p.q = a.q; p.k = a.k; p.v = a.v; p.beta = a.beta; p.log_gate = a.log_gate;
     p.state = a.state; p.slots = a.slots; p.n_slots = a.n_slots; p.o = a.o;
@@ -711,7 +747,7 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
         p.n_seg = std::min(seg, n_chunks - cb);
         const unsigned grid_a = (unsigned)(bhs * p.n_seg);
         cudaError_t e = launch_pdl(a.kind == HMD_KDA ? prefill_prep_kernel<true> : prefill_prep_kernel<false>,
-                                   dim3(grid_a), dim3(kPrepThreads), A_SMEM, s, p);
+                                   dim3(grid_a), dim3(kPrepThreads), A_SMEM, s, tmq, tmk, tmv, tmg, p);
         if (e != cudaSuccess) return e;
         e = launch_pdl(prefill_scan_kernel, dim3((unsigned)(bhs * kSplitV)), dim3(kThreads), B_SMEM, s,
                        p);

@@ -35,6 +35,8 @@ bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base,
 
 // [n_tok][heads][d] bf16 as (d, heads, n_tok) in 64 x 1 x 64 boxes, 128-byte swizzle.
 bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int heads, int d);
+bool make_tmap_bthd(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int B,
+                    int T, int H, int d, int box_d, bool sw128);
 
 struct DeltaDecodeArgs {
     int kind;  // 2 = KDA (per-channel gate), 3 = GDN (scalar gate)

@@ -60,4 +60,24 @@ bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int hea
            CUDA_SUCCESS;
 }
 
+// A [B][T][H][d] activation (bf16 or fp32) as a 4-D tensor (d, H, T, B) read in boxes of
+// (box_d channels, 1 head, 64 tokens, 1 sequence): one box is a [64 tokens][box_d] tile,
+// 128-byte swizzled if sw128. Tokens past T read as zero, so a chunk never reaches into the
+// next sequence.
+bool make_tmap_bthd(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int B,
+                    int T, int H, int d, int box_d, bool sw128) {
+    EncodeTiledFn enc = encode();
+    if (!enc) return false;
+    const cuuint64_t gdim[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t gstride[3] = {(cuuint64_t)d * esize, (cuuint64_t)H * d * esize,
+                                   (cuuint64_t)T * H * d * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)box_d, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, dt, 4, const_cast<void *>(base), gdim, gstride, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 }  // namespace hmd
