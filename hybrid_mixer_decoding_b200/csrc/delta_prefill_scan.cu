@@ -1,5 +1,5 @@
-// Chunked delta-rule prefill in two passes on tensor cores (mma.sync m16n8k16, bf16 operands,
-// fp32 accumulation), bf16 activations, d_k = d_v = 128, chunk C = 64.
+// Chunked delta-rule prefill in two passes, bf16 activations, fp32 state and accumulation,
+// d_k = d_v = 128, chunk C = 64.
 //
 // Chunk algebra: the standard WY / UT-transform rewriting of the gated delta rule for the GDN and
 // KDA mixers of "Super Apriel: One Checkpoint, Many Speeds" (abstract; gist.science technical
@@ -12,12 +12,15 @@
 // Everything up to W and Ut depends only on the chunk's own inputs; only the last line carries
 // the state from chunk to chunk.
 //
-// Pass A (prefill_prep_kernel): one CTA per (sequence, head, chunk), all chunks at once. It
-// computes the gate factors, A and P, the blocked UT solve, W and Ut, and writes one record per
-// chunk: Qt, -W, Kc, P (bf16, already in the 128-byte XOR-swizzled tile layout pass B reads with
-// ldmatrix), e^{G_C} and Ut^T (fp32, rows of d_v).
-// Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks in
-// order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
+// Pass A (prefill_prep_kernel): one CTA per (sequence, head, chunk), all chunks at once, on the
+// 5th-generation tensor cores. TMA brings the chunk's q, k, v (and KDA log-gates) into shared
+// memory in the 128-byte swizzled layout the tensor cores read; the CTA forms the gate factors,
+// then [Kt; Qt] Kh^T as ONE M = 128 tcgen05.mma product into TMEM (rows 0-63 give A, rows 64-127
+// give P), the blocked fp32 UT solve on the CUDA cores, and W^T, Ut^T as two M = 128 products
+// that read Kt and V MN-major. It writes one record per chunk: Qt, -W, Kc, P, Ut (bf16, in the
+// 128-byte XOR-swizzled tile layout pass B reads with ldmatrix) and e^{G_C} (fp32).
+// Pass B (prefill_scan_kernel, mma.sync m16n8k16): one CTA per (sequence, head, half of d_v)
+// walks the chunks in order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
 // the chunk before it computes; the state half lives in registers as MMA accumulator fragments.
 // Per chunk it does only the state-dependent products (U, O, state update): 7.3 MFLOP of the
 // chunk's 11.5 per head, split over two CTAs.
@@ -48,8 +51,8 @@ constexpr uint32_t REC_KC = 32768;     // Kc  bf16 [64][128]
 constexpr uint32_t REC_P = 49152;      // P   bf16 [64][64]
 constexpr uint32_t REC_GAM = 57344;    // e^{G_C} fp32 [128]
 constexpr uint32_t REC_HEAD = 57856;   // bytes above, moved by one bulk copy
-constexpr uint32_t REC_UT = 57856;     // Ut^T fp32 [128 d_v][64 tokens] (see utt_idx)
-constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 4;  // 90624
+constexpr uint32_t REC_UT = 57856;     // Ut  bf16 [64][128], swizzled halves
+constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 2;  // 74240
 static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
 
 // ---- pass A shared memory (bytes from a 1024-aligned base) ---------------------------------
@@ -64,7 +67,7 @@ constexpr uint32_t A_G = 65536;        // KDA log-gates -> in-chunk prefix, fp32
 constexpr uint32_t A_AS = 65536;       // after the gate pass: A fp32 [64][68], then T bf16
 constexpr uint32_t A_XS = 82944;       // X fp32 [64][68]
 constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
-constexpr uint32_t A_UT = 65536;       // at the end: Ut^T fp32 (record layout, 32 KiB)
+constexpr uint32_t A_UT = 65536;       // at the end: Ut bf16 (record layout, 16 KiB)
 constexpr uint32_t A_SMALL = 104192;
 constexpr uint32_t S_BETA = 0, S_QOFF = 256, S_LGP = 1280, S_WSUM = 1536, S_EGC = 1552,
                    S_BAR = 2064, S_TMEM = 2080, S_SIZE = 2112;
@@ -76,7 +79,7 @@ constexpr uint32_t kPrepTmemCols = 128;
 constexpr uint32_t ID_AP = idesc_bf16(128, 64, 0, 0);  // [Kt; Qt] Kh^T: both operands K-major
 constexpr uint32_t ID_WU = idesc_bf16(128, 64, 1, 0);  // Kt^T T^T, V^T T^T: A MN-major
 static_assert(A_G + kC * kD * 4 <= A_YS, "log-gate staging fits the A/X region");
-static_assert(A_UT + kC * kD * 4 <= A_YS, "Ut^T fits the A/X region");
+static_assert(A_UT + kC * kD * 2 <= A_YS, "Ut fits the A/X region");
 static_assert(S_QOFF + (kPrepThreads / kD) * kD * 4 <= S_LGP, "gate part sums fit");
 static_assert(S_BAR % 8 == 0 && S_TMEM + 4 <= S_SIZE, "small area");
 
@@ -92,10 +95,6 @@ __device__ __forceinline__ uint32_t toff(int row, int col, int rows) {
     return (uint32_t)((col >> 6) * rows * 128 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
                       ((col & 7) << 1));
 }
-
-// word index of Ut[token][dv] in the Ut^T block: rows of 64 tokens per d_v column, the 8-word
-// groups XOR-permuted by row so that a warp's fragment stores hit distinct banks
-__device__ __forceinline__ int utt_idx(int dv, int tok) { return dv * kC + (tok ^ ((dv & 7) << 3)); }
 
 // float index of log-gate (row r, channel i) in the staged KDA gate tile: four TMA boxes of
 // [64 rows][32 channels]
@@ -476,17 +475,15 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     *reinterpret_cast<__nv_bfloat16 *>(wb + toff(32 * hr + j, dd & 63, 64)) =
                         __float2bfloat16_rn(-__uint_as_float(d[j]));
             }
-        } else {  // Ut^T fp32 [d_v][64 tokens] (record layout)
-            float *ut = reinterpret_cast<float *>(sm + A_UT);
+        } else {  // Ut [r][d_v] bf16 (record layout)
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * hr, d);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4)
-                    *reinterpret_cast<float4 *>(ut + utt_idx(dd, 32 * hr + 4 * j4)) =
-                        make_float4(__uint_as_float(d[4 * j4]), __uint_as_float(d[4 * j4 + 1]),
-                                    __uint_as_float(d[4 * j4 + 2]), __uint_as_float(d[4 * j4 + 3]));
+                for (int j = 0; j < 32; ++j)
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + A_UT + toff(32 * hr + j, dd, 64)) =
+                        __float2bfloat16_rn(__uint_as_float(d[j]));
             }
         }
     }
@@ -496,7 +493,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     if (tid == 0) {
         bulk_store(rec + REC_NW, sb + A_KQ, 8192);
         bulk_store(rec + REC_NW + 8192, sb + A_KQ + 16384, 8192);
-        bulk_store(rec + REC_UT, sb + A_UT, 32768);
+        bulk_store(rec + REC_UT, sb + A_UT, 16384);
         bulk_commit_group();
         bulk_wait_group_read0();  // shared memory must outlive the copies' reads
     }
@@ -563,16 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
     // U / O role: chunk rows 16*rt + g (+8), slice columns 32*chh + 8*j + 2*t4 (+1)
     const int rt = warp & 3, chh = warp >> 2;
     const int ur0 = 16 * rt + g, ur1 = ur0 + 8;
-    float un[4][4];  // Ut of the next chunk, prefetched
+    uint32_t un[4][2];  // Ut of the next chunk (bf16 pairs), prefetched
     auto load_ut = [&](int c) {
-        const float *ut = reinterpret_cast<const float *>(record(a, bh, c) + REC_UT);
+        const uint8_t *ut = record(a, bh, c) + REC_UT;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
-            un[j][0] = ut[utt_idx(cc, ur0)];
-            un[j][1] = ut[utt_idx(cc + 1, ur0)];
-            un[j][2] = ut[utt_idx(cc, ur1)];
-            un[j][3] = ut[utt_idx(cc + 1, ur1)];
+            un[j][0] = __ldg(reinterpret_cast<const unsigned int *>(ut + toff(ur0, cc, 64)));
+            un[j][1] = __ldg(reinterpret_cast<const unsigned int *>(ut + toff(ur1, cc, 64)));
         }
     };
     load_ut(0);
@@ -610,12 +605,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
         // ---- phase 2: U = Ut + (-W) M and O = Qt M (16 rows x 32 columns per warp) -------
         float u[4][4], o[4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < 4; ++j) {
+            u[j][0] = bf16_lo(un[j][0]); u[j][1] = bf16_hi(un[j][0]);
+            u[j][2] = bf16_lo(un[j][1]); u[j][3] = bf16_hi(un[j][1]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                u[j][e] = un[j][e];
-                o[j][e] = 0.f;
-            }
+            for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
+        }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
             uint32_t aw[4], aq[4];

@@ -108,7 +108,7 @@ HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, i
                                         int chunk, float scale, hmd_stream_t stream);
 
 /* Scratch bytes for delta_rule_prefill_chunked_ws to run these sizes in one segment: one record
- * (90,624 bytes at dk = dv = 128, chunk 64) per chunk and (sequence, head). 0 when the call
+ * (74,240 bytes at dk = dv = 128, chunk 64) per chunk and (sequence, head). 0 when the call
  * needs no scratch (the CUDA-core path) or the sizes are empty or invalid.                    */
 HMD_API size_t delta_rule_prefill_workspace_size(hmd_kind_t kind, int B, int T, int H, int dk,
                                                  int dv, hmd_dtype_t dtype, int chunk);

@@ -78,8 +78,8 @@ def _prefill_ws(ws, ws_bytes, B=2, T=300, H=3, dtype=hmd.BF16, dk=128):
 
 def test_prefill_workspace_size_and_validation():
     f = hmd.delta_rule_prefill_workspace_size
-    rec = 90624  # Qt, -W, Kc (bf16 64x128), P (bf16 64x64), e^{G_C} (128 fp32), Ut (fp32 64x128)
-    assert rec == 3 * 64 * 128 * 2 + 64 * 64 * 2 + 128 * 4 + 64 * 128 * 4
+    rec = 74240  # Qt, -W, Kc (bf16 64x128), P (bf16 64x64), e^{G_C} (128 fp32), Ut (bf16 64x128)
+    assert rec == 4 * 64 * 128 * 2 + 64 * 64 * 2 + 128 * 4
     assert f(hmd.KDA, 4, 4096, 16, 128, 128, hmd.BF16, 64) == 4 * 16 * 64 * rec
     assert f(hmd.GDN, 2, 65, 3, 128, 128, hmd.BF16, 64) == 2 * 3 * 2 * rec   # ragged: 2 chunks
     assert f(hmd.GDN, 2, 65, 3, 64, 64, hmd.BF16, 64) == 0     # CUDA-core path: no scratch
