@@ -180,6 +180,67 @@ def attn_inputs(kind: int, B: int, Hq: int, Hkv: int, d: int, ctx: int, window: 
 
 
 @dataclass
+class AttnVerifyInputs:
+    """Inputs of one FA or SWA verification pass: n_q new tokens per sequence on top of a paged
+    cache that already holds positions 0..seq_len-n_q-1.
+
+    q: bf16 bits [B][n_q][Hq][d]; new_k, new_v: bf16 bits [B][n_q][Hkv][d].
+    k_pool, v_pool: bf16 bits [P][Hkv][page_tokens][d], N(0,1) in every slot (the cached
+    positions are whatever the slot mapping reads there). page_table: int32 [B][max_pages]
+    (FA: ceil(ctx/64) pages; SWA: ring_pages), a seeded permutation of the pool when permute.
+    seq_lens: int32 [B], counting the n_q new tokens.
+    """
+    kind: int
+    window: int
+    ring_pages: int
+    n_q: int
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    page_tokens: int
+    k_pool: np.ndarray
+    v_pool: np.ndarray
+    page_table: np.ndarray
+    seq_lens: np.ndarray
+    q: np.ndarray
+    new_k: np.ndarray
+    new_v: np.ndarray
+
+
+def verify_inputs(kind: int, B: int, n_q: int, Hq: int, Hkv: int, d: int, ctx: int,
+                  window: int = 0, ring_pages: int = 0, page_tokens: int = 64, seed: int = 0,
+                  permute: bool = True, seq_lens: np.ndarray | None = None) -> AttnVerifyInputs:
+    """Draw one seeded verification problem (same distributions as attn_inputs). ctx is the
+    longest sequence length counting the new tokens; for SWA ring_pages (0: the smallest ring a
+    verifier of n_q tokens may use, ceil((window + n_q - 1) / 64)) sets the pages per sequence."""
+    assert kind in (FA, SWA) and n_q >= 1
+    g = rng(seed)
+    if seq_lens is None:
+        seq_lens = np.full(B, ctx, dtype=np.int32)
+    seq_lens = np.asarray(seq_lens, dtype=np.int32)
+    assert int(seq_lens.min()) >= n_q
+    if kind == SWA:
+        assert window >= 1
+        if ring_pages == 0:
+            ring_pages = -(-(window + n_q - 1) // page_tokens)
+        max_pages = ring_pages
+    else:
+        max_pages = -(-int(seq_lens.max()) // page_tokens)
+    P = B * max_pages
+    perm = g.permutation(P).astype(np.int32) if permute else np.arange(P, dtype=np.int32)
+    table = perm.reshape(B, max_pages).copy()
+    shape = (P, Hkv, page_tokens, d)
+    k_pool = bf16_bits(g.standard_normal(shape, dtype=np.float32))
+    v_pool = bf16_bits(g.standard_normal(shape, dtype=np.float32))
+    q = bf16_bits(g.standard_normal((B, n_q, Hq, d), dtype=np.float32))
+    new_k = bf16_bits(g.standard_normal((B, n_q, Hkv, d), dtype=np.float32))
+    new_v = bf16_bits(g.standard_normal((B, n_q, Hkv, d), dtype=np.float32))
+    return AttnVerifyInputs(kind, window, ring_pages, n_q, B, Hq, Hkv, d, page_tokens, k_pool,
+                            v_pool, table, seq_lens, q, new_k, new_v)
+
+
+@dataclass
 class AttnPrefillInputs:
     """Inputs of one FA or SWA prefill of T prompt tokens per sequence into an empty cache.
 

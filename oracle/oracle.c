@@ -403,6 +403,106 @@ int oracle_attn_prefill(int kind, int window, int B, int T, int Hq, int Hkv, int
     return bad ? -1 : 0;
 }
 
+/* Cache slot of logical position pos when SWA keeps a ring of ring_pages pages (a verifier of
+ * n_q tokens needs at least window + n_q - 1 positions in its ring, see below). FA ignores
+ * ring_pages. Returns 0, or -1 on bad arguments.                                              */
+int oracle_kv_slot_ring(int kind, int ring_pages, int page_tokens, const int32_t *page_row,
+                        int max_pages, int pos, int32_t *page, int32_t *offset) {
+    if (page_tokens < 1 || pos < 0) return -1;
+    long ring_idx = pos;
+    if (kind == OR_SWA) {
+        if (ring_pages < 1) return -1;
+        ring_idx = pos % ((long)ring_pages * page_tokens);
+    } else if (kind != OR_FA) {
+        return -1;
+    }
+    const long logical_page = ring_idx / page_tokens;
+    if (logical_page >= max_pages) return -1;
+    *page = page_row[logical_page];
+    *offset = (int32_t)(ring_idx % page_tokens);
+    return 0;
+}
+
+/* Verification pass of speculative decoding: n_q new tokens per sequence, which is exactly n_q
+ * decode steps in a row (each appends its token, then attends). Token i of sequence b sits at
+ * logical position P = L - n_q + i (L = seq_lens[b] counts all n_q) and query head h attends
+ * keys j in [lo, P], lo = 0 (FA) or max(0, P + 1 - window) (SWA), with kv-head h / (Hq / Hkv).
+ * Keys j < L - n_q are read from the pools (bf16 bits [P][Hkv][PT][d], SWA ring of ring_pages
+ * pages); keys j >= L - n_q are the new tokens themselves.
+ *   q [B][n_q][Hq][d]; new_k, new_v [B][n_q][Hkv][d]; o [B][n_q][Hq][d] (double).
+ * Returns 0, or -1 on bad arguments or a bad page id.                                          */
+int oracle_attn_verify(int kind, int window, int ring_pages, int n_q, int B, int Hq, int Hkv,
+                       int d, int page_tokens, int n_pages, const double *q, const double *new_k,
+                       const double *new_v, const uint16_t *k_pool, const uint16_t *v_pool,
+                       const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                       double *o, int n_threads) {
+    if ((kind != OR_FA && kind != OR_SWA) || Hkv < 1 || Hq % Hkv || n_q < 1) return -1;
+    if (kind == OR_SWA && window < 1) return -1;
+    set_threads(n_threads);
+    const int heads_per_kv = Hq / Hkv;
+    const double rsqrt_d = 1.0 / sqrt((double)d);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+    for (int row = 0; row < B * n_q * Hq; ++row) {
+        const int b = row / (n_q * Hq), i = (row / Hq) % n_q, h = row % Hq;
+        const int kvh_v = h / heads_per_kv;
+        const int L = seq_lens[b];
+        const int first_new = L - n_q;  /* logical position of new token 0 */
+        const int P_pos = first_new + i;
+        if (first_new < 0) { bad |= 1; continue; }
+        const int lo = (kind == OR_SWA && P_pos + 1 > window) ? P_pos + 1 - window : 0;
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(P_pos - lo + 1));
+        if (!sc) { bad |= 1; continue; }
+        const double *qv = q + (size_t)row * d;
+        double mx = -INFINITY;
+        for (int j = lo; j <= P_pos; ++j) {
+            double dot = 0.0;
+            if (j >= first_new) {
+                const double *kv = new_k + (((size_t)b * n_q + (j - first_new)) * Hkv + kvh_v) * d;
+                for (int c = 0; c < d; ++c) dot += qv[c] * kv[c];
+            } else {
+                int32_t pg, off;
+                if (oracle_kv_slot_ring(kind, ring_pages, page_tokens,
+                                        page_table + (size_t)b * max_pages, max_pages, j, &pg,
+                                        &off) || pg < 0 || pg >= n_pages) {
+                    bad |= 1;
+                } else {
+                    const uint16_t *kv = k_pool + (((size_t)pg * Hkv + kvh_v) * page_tokens + off) * d;
+                    for (int c = 0; c < d; ++c) dot += qv[c] * bf16_to_double(kv[c]);
+                }
+            }
+            sc[j - lo] = dot * rsqrt_d;
+            if (sc[j - lo] > mx) mx = sc[j - lo];
+        }
+        double denom = 0.0;
+        for (int j = lo; j <= P_pos; ++j) {
+            sc[j - lo] = exp(sc[j - lo] - mx);
+            denom += sc[j - lo];
+        }
+        double *ov = o + (size_t)row * d;
+        for (int c = 0; c < d; ++c) ov[c] = 0.0;
+        for (int j = lo; j <= P_pos; ++j) {
+            const double w = sc[j - lo] / denom;
+            if (j >= first_new) {
+                const double *vv = new_v + (((size_t)b * n_q + (j - first_new)) * Hkv + kvh_v) * d;
+                for (int c = 0; c < d; ++c) ov[c] += w * vv[c];
+            } else {
+                int32_t pg, off;
+                if (oracle_kv_slot_ring(kind, ring_pages, page_tokens,
+                                        page_table + (size_t)b * max_pages, max_pages, j, &pg,
+                                        &off) || pg < 0 || pg >= n_pages) {
+                    bad |= 1;
+                } else {
+                    const uint16_t *vv = v_pool + (((size_t)pg * Hkv + kvh_v) * page_tokens + off) * d;
+                    for (int c = 0; c < d; ++c) ov[c] += w * bf16_to_double(vv[c]);
+                }
+            }
+        }
+        free(sc);
+    }
+    return bad ? -1 : 0;
+}
+
 /* The oracle's thread count after set-up (for reporting). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -52,9 +52,13 @@ def _load():
         lib.oracle_attn_decode.argtypes = ([c_int] * 8 + [D, D, D, U16, U16, I32, c_int, I32, D,
                                                           c_int])
         lib.oracle_attn_prefill.argtypes = [c_int] * 7 + [D, D, D, D, c_int]
+        lib.oracle_kv_slot_ring.argtypes = [c_int, c_int, c_int, I32, c_int, c_int, I32, I32]
+        lib.oracle_attn_verify.argtypes = ([c_int] * 10 + [D, D, D, U16, U16, I32, c_int, I32, D,
+                                                           c_int])
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_delta_recurrent", "oracle_delta_chunked", "oracle_kv_slot",
-                  "oracle_attn_decode", "oracle_attn_prefill", "oracle_max_threads"):
+                  "oracle_attn_decode", "oracle_attn_prefill", "oracle_kv_slot_ring",
+                  "oracle_attn_verify", "oracle_max_threads"):
             getattr(lib, f).restype = c_int
         _lib = lib
     return _lib
@@ -166,6 +170,44 @@ def attn_prefill(kind, window, q, k, v, n_threads=0):
                                      _p(o, ctypes.c_double), int(n_threads))
     if rc:
         raise ValueError("oracle_attn_prefill: bad arguments")
+    return o
+
+
+def kv_slot_ring(kind, ring_pages, page_tokens, page_row, pos):
+    """(physical page, offset) of logical position pos with an SWA ring of ring_pages pages."""
+    row = np.ascontiguousarray(page_row, dtype=np.int32)
+    pg, off = ctypes.c_int32(), ctypes.c_int32()
+    rc = _load().oracle_kv_slot_ring(kind, int(ring_pages), int(page_tokens),
+                                     _p(row, ctypes.c_int32), int(row.shape[0]), int(pos),
+                                     ctypes.byref(pg), ctypes.byref(off))
+    if rc:
+        raise ValueError("oracle_kv_slot_ring: bad arguments")
+    return int(pg.value), int(off.value)
+
+
+def attn_verify(kind, window, ring_pages, q_bits, new_k_bits, new_v_bits, k_pool, v_pool,
+                page_table, seq_lens, n_threads=0):
+    """Verification of n_q tokens per sequence (see oracle.c): q_bits [B,n_q,Hq,d] and
+    new_k/new_v_bits [B,n_q,Hkv,d] bf16 bit patterns; pools uint16 [P,Hkv,PT,d] holding
+    positions 0..L-n_q-1. Returns o [B,n_q,Hq,d] float64."""
+    q = bf16_bits_to_f64(q_bits)
+    nk = bf16_bits_to_f64(new_k_bits)
+    nv = bf16_bits_to_f64(new_v_bits)
+    kp = np.ascontiguousarray(k_pool, dtype=np.uint16)
+    vp = np.ascontiguousarray(v_pool, dtype=np.uint16)
+    pt_ = np.ascontiguousarray(page_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, n_q, Hq, d = q.shape
+    P, Hkv, PT, _ = kp.shape
+    o = np.zeros((B, n_q, Hq, d), dtype=np.float64)
+    rc = _load().oracle_attn_verify(kind, int(window), int(ring_pages), n_q, B, Hq, Hkv, d, PT, P,
+                                    _p(q, ctypes.c_double), _p(nk, ctypes.c_double),
+                                    _p(nv, ctypes.c_double), _p(kp, ctypes.c_uint16),
+                                    _p(vp, ctypes.c_uint16), _p(pt_, ctypes.c_int32),
+                                    int(pt_.shape[1]), _p(sl, ctypes.c_int32),
+                                    _p(o, ctypes.c_double), int(n_threads))
+    if rc:
+        raise ValueError("oracle_attn_verify failed (bad arguments or page id)")
     return o
 
 

@@ -434,3 +434,111 @@ def test_prefill_attention_closed_forms(oracle_mod):
         lo = max(0, t + 1 - w)
         np.testing.assert_allclose(oe[:, t], np.repeat(v[:, lo:t + 1].mean(axis=1), 4, axis=1),
                                    rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------------------------
+# verification pass (speculative decoding): n_q new tokens, each a decode step
+# --------------------------------------------------------------------------------------------
+
+def _verify_brute(a: I.AttnVerifyInputs, O):
+    """Brute force over the logical sequence: positions below L - n_q are gathered from the
+    pools with the slot formula written out here (ring index p mod (R * PT) for SWA), the
+    last n_q are the new tokens; row i attends [lo, L - n_q + i]."""
+    PT, R = a.page_tokens, a.ring_pages
+    q = O.bf16_bits_to_f64(a.q)
+    nk, nv = O.bf16_bits_to_f64(a.new_k), O.bf16_bits_to_f64(a.new_v)
+    kp, vp = O.bf16_bits_to_f64(a.k_pool), O.bf16_bits_to_f64(a.v_pool)
+    grp = a.Hq // a.Hkv
+    out = np.zeros(q.shape)
+    for b in range(a.B):
+        L = int(a.seq_lens[b])
+        first = L - a.n_q
+        K = np.zeros((L, a.Hkv, a.d))
+        V = np.zeros_like(K)
+        for p in range(first):
+            r = p % (R * PT) if a.kind == I.SWA else p
+            pg = a.page_table[b, r // PT]
+            K[p], V[p] = kp[pg, :, r % PT], vp[pg, :, r % PT]
+        K[first:], V[first:] = nk[b], nv[b]
+        for i in range(a.n_q):
+            P_ = first + i
+            lo = max(0, P_ + 1 - a.window) if a.kind == I.SWA else 0
+            for h in range(a.Hq):
+                s = K[lo:P_ + 1, h // grp] @ q[b, i, h] / math.sqrt(a.d)
+                w = np.exp(s - s.max())
+                out[b, i, h] = (w / w.sum()) @ V[lo:P_ + 1, h // grp]
+    return out
+
+
+@pytest.mark.parametrize("kind,window,n_q,ring_extra", [
+    (I.FA, 0, 1, 0), (I.FA, 0, 3, 0), (I.FA, 0, 4, 0),
+    (I.SWA, 9, 1, 0), (I.SWA, 9, 4, 0), (I.SWA, 8, 3, 0), (I.SWA, 5, 2, 2), (I.SWA, 1, 4, 0)])
+def test_verify_matches_brute_force(oracle_mod, kind, window, n_q, ring_extra):
+    O = oracle_mod
+    PT = 4
+    ring = -(-(window + n_q - 1) // PT) + ring_extra if kind == I.SWA else 0
+    a = I.verify_inputs(kind, 3, n_q, 4, 2, 8, 30, window=window, ring_pages=ring,
+                        page_tokens=PT, seed=60 + n_q, seq_lens=np.array([30, n_q, 17]))
+    o = O.attn_verify(kind, window, a.ring_pages, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool,
+                      a.page_table, a.seq_lens)
+    np.testing.assert_allclose(o, _verify_brute(a, O), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("kind,window", [(I.FA, 0), (I.SWA, 9)])
+def test_verify_single_token_is_the_decode_step(oracle_mod, kind, window):
+    O = oracle_mod
+    PT = 4
+    a = I.verify_inputs(kind, 3, 1, 4, 2, 8, 30, window=window,
+                        ring_pages=-(-window // PT) if kind == I.SWA else 0, page_tokens=PT,
+                        seed=70, seq_lens=np.array([30, 1, 13]))
+    o = O.attn_verify(kind, window, a.ring_pages, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool,
+                      a.page_table, a.seq_lens)
+    dec = O.attn_decode(kind, window, a.q[:, 0], a.new_k[:, 0], a.new_v[:, 0], a.k_pool,
+                        a.v_pool, a.page_table, a.seq_lens)
+    np.testing.assert_allclose(o[:, 0], dec, rtol=1e-12, atol=1e-13)
+
+
+def test_verify_rows_equal_successive_decode_steps(oracle_mod):
+    """FA: row i of a verify pass is the decode step of token i after tokens 0..i-1 have been
+    appended at their slots (the decode oracle is pinned on its own)."""
+    O = oracle_mod
+    PT, n_q = 4, 4
+    a = I.verify_inputs(I.FA, 2, n_q, 4, 2, 8, 23, page_tokens=PT, seed=71,
+                        seq_lens=np.array([23, 9]))
+    o = O.attn_verify(I.FA, 0, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                      a.seq_lens)
+    kp, vp = a.k_pool.copy(), a.v_pool.copy()
+    for i in range(n_q):
+        L_i = a.seq_lens - n_q + i + 1
+        dec = O.attn_decode(I.FA, 0, a.q[:, i], a.new_k[:, i], a.new_v[:, i], kp, vp,
+                            a.page_table, L_i)
+        np.testing.assert_allclose(o[:, i], dec, rtol=1e-12, atol=1e-13)
+        for b in range(a.B):  # append token i for the next step
+            pg, off = O.kv_slot(I.FA, 0, PT, a.page_table[b], int(L_i[b]) - 1)
+            kp[pg, :, off], vp[pg, :, off] = a.new_k[b, i], a.new_v[b, i]
+
+
+def test_verify_from_empty_cache_is_prefill(oracle_mod):
+    """FA with L = n_q (nothing cached): the verify pass is the prefill of those n_q tokens."""
+    O = oracle_mod
+    n_q = 5
+    a = I.verify_inputs(I.FA, 2, n_q, 4, 2, 8, n_q, page_tokens=4, seed=72)
+    o = O.attn_verify(I.FA, 0, 0, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool, a.page_table,
+                      a.seq_lens)
+    pre = O.attn_prefill(I.FA, 0, O.bf16_bits_to_f64(a.q), O.bf16_bits_to_f64(a.new_k),
+                         O.bf16_bits_to_f64(a.new_v))
+    np.testing.assert_allclose(o, pre, rtol=1e-12, atol=1e-13)
+
+
+def test_ring_slot_formula_cases(oracle_mod):
+    """kv_slot_ring: FA ignores the ring; SWA wraps at ring_pages * PT; the default ring of
+    ceil(w / PT) pages agrees with kv_slot."""
+    O = oracle_mod
+    row = np.array([7, 3, 9, 1, 4], np.int32)
+    assert O.kv_slot_ring(I.FA, 2, 4, row, 13) == (1, 1)   # page 13 // 4 = 3
+    assert O.kv_slot_ring(I.SWA, 2, 4, row, 13) == (3, 1)   # 13 mod 8 = 5: page 1, offset 1
+    assert O.kv_slot_ring(I.SWA, 3, 4, row, 13) == (7, 1)   # 13 mod 12 = 1
+    assert O.kv_slot_ring(I.SWA, 5, 4, row, 19) == (4, 3)
+    for w in (1, 4, 5, 9):
+        for p in range(40):
+            assert O.kv_slot_ring(I.SWA, -(-w // 4), 4, row, p) == O.kv_slot(I.SWA, w, 4, row, p)

@@ -42,6 +42,12 @@ MUTANTS = [
     ("prefill_scale_missing", [("s[j - lo] = inv_sqrt_d * acc;", "s[j - lo] = acc;")]),
     ("prefill_value_row_shifted", [("const double *vv = v + (((size_t)b * T + j) * Hkv + kvh) * d;",
                                     "const double *vv = v + (((size_t)b * T + (j > lo ? j - 1 : j)) * Hkv + kvh) * d;")]),
+    ("verify_window_off_by_one", [("? P_pos + 1 - window : 0", "? P_pos - window : 0")]),
+    ("verify_gqa_interleaved", [("kvh_v = h / heads_per_kv", "kvh_v = h % Hkv")]),
+    ("verify_ring_not_wrapped", [("ring_idx = pos % ((long)ring_pages * page_tokens);",
+                                  "ring_idx = pos;")]),
+    ("verify_first_new_key_from_pool", [("if (j >= first_new) {", "if (j > first_new) {")]),
+    ("verify_rows_shifted", [("const int P_pos = first_new + i;", "const int P_pos = first_new + i - (i > 0);")]),
 ]
 
 
