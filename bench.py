@@ -465,6 +465,41 @@ def run_kernel_workload(args):
                 "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
                 "traffic": traffic_for(w), "algorithmic_bytes": byts}
         launches = 2
+    elif w in ("verify_fa", "verify_swa"):
+        kind = I.FA if w == "verify_fa" else I.SWA
+        B, Hq, Hkv, d, L, win, nq_max = 32, 32, 8, 128, 8192, 4096, 4
+        ring = -(-(win + nq_max - 1) // 64)
+        pps = L // 64 if kind == I.FA else ring
+        P = B * pps
+        kp = torch.randn(P, Hkv, 64, d, device=dev, dtype=bf, generator=g)
+        vp = torch.randn(P, Hkv, 64, d, device=dev, dtype=bf, generator=g)
+        table = torch.randperm(P, device=dev, generator=g).to(torch.int32).view(B, pps).contiguous()
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        per_nq = {}
+        for nq in range(1, nq_max + 1):
+            q = torch.randn(B, nq, Hq, d, device=dev, dtype=bf, generator=g)
+            nk = torch.randn(B, nq, Hkv, d, device=dev, dtype=bf, generator=g)
+            nv = torch.randn(B, nq, Hkv, d, device=dev, dtype=bf, generator=g)
+            o = torch.empty(B, nq, Hq, d, device=dev, dtype=bf)
+            ws = torch.empty(hmd.attn_verify_workspace_size(kind, win, nq, B, Hq, Hkv, d, 64, L),
+                             dtype=torch.uint8, device=dev)
+
+            def fn():
+                hmd.attn_verify(kind, win, ring, q, nk, nv, kp, vp, table, lens, L, o, ws)
+            per_nq[nq] = _events_time(fn, args.steps, args.warmup)
+        sec = per_nq[nq_max]
+        keys = L if kind == I.FA else win + nq_max - 1
+        byts = B * (keys * Hkv * d * 4 + nq_max * (2 * Hq * d * 2 + 2 * Hkv * d * 2))
+        value, unit = B * nq_max / sec, "tok/s"
+        desc = (f"{'FA' if kind == I.FA else 'SWA(w=4096, ring 65 pages)'} verification pass of "
+                f"4 new tokens per sequence: B=32, Hq=32, Hkv=8, d=128, ctx 8192 counting them, "
+                f"paged bf16 KV (64-token pages, random permutation); value = tokens checked/s")
+        roof = {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
+                "traffic": None, "algorithmic_bytes": byts}
+        extra["verify"] = {"us_per_pass_by_n_q": {str(n): round(t * 1e6, 2) for n, t in per_nq.items()},
+                           "cost_vs_one_token": round(per_nq[nq_max] / per_nq[1], 4)}
+        launches = 2
     elif w in ("prefill_fa", "prefill_swa"):
         kind = I.FA if w == "prefill_fa" else I.SWA
         B, T, Hq, Hkv, d, win = 2, 8192, 32, 8, 128, 4096
@@ -555,6 +590,94 @@ def run_kernel_workload(args):
     return out
 
 
+def run_spec(args):
+    """Self-speculative decoding on the 48-layer mixer-only stack: B=32, context 32768, H=32,
+    Hkv=8, d=128, target placement 12 FA / 12 SWA(w=4096) / 12 KDA / 12 GDN (the stack48
+    placement), drafter all-GDN, k=3 drafts per round (4 positions verified), each draft kept
+    with probability 0.8 until the first rejection (seeded). Every round is two CUDA-graph
+    replays (draft, verify); the plain decode step of the target placement is timed alongside."""
+    import torch
+
+    import hybrid_mixer_decoding_b200 as hmd
+    from hybrid_mixer_decoding_b200.spec import SpecStack, make_schedule
+    from hybrid_mixer_decoding_b200.stack import StackShape, layer_bytes
+
+    pk, _ = peaks()
+    hbm = float(pk["hbm_gbs"])
+    k, alpha = 3, 0.8
+    shape = StackShape(B=32, H=32, Hkv=8, d=128, ctx=32768, window=4096)
+    rounds = args.warmup + args.steps
+    target = stack_placement()
+    sp = SpecStack(target, shape, k, max_rounds=rounds + 2)
+    sched = make_schedule(shape.B, k, rounds, sp.L0, alpha, seed=1)
+    slots_dev = torch.from_numpy(sched.slots).cuda()
+    lens_dev = torch.from_numpy(sched.lens).cuda()
+    g_draft, g_verify, g_plain = sp.capture(sp.draft), sp.capture(sp.verify), sp.capture(sp.plain_step)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(n):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e-3
+
+    for _ in range(args.warmup):
+        g_plain.replay()
+    plain_s = timed(lambda i: g_plain.replay(), args.steps) / args.steps
+    # phase times (on the first round's chain; the work does not depend on it)
+    sp.set_round(sched, 0, slots_dev, lens_dev)
+    draft_s = timed(lambda i: g_draft.replay(), args.steps) / args.steps
+    verify_s = timed(lambda i: g_verify.replay(), args.steps) / args.steps
+
+    def round_(r):
+        sp.set_round(sched, r, slots_dev, lens_dev)
+        g_draft.replay()
+        g_verify.replay()
+    for r in range(args.warmup):
+        round_(r)
+    spec_s = timed(lambda i: round_(args.warmup + i), args.steps)
+    assert hmd.hmd_device_errors(clear=True) == 0
+    tokens = int(sched.tokens[args.warmup:].sum())
+    value = tokens / spec_s
+    plain_tok_s = shape.B / plain_s
+    # algorithmic bytes of one round: the drafter's k+1 steps, the target's verify pass
+    B, H, Hkv, d, ctx, w = shape.B, shape.H, shape.Hkv, shape.d, shape.ctx, shape.window
+    nq = k + 1
+    lin = lambda kind: layer_bytes(kind, shape)  # noqa: E731
+    draft_bytes = nq * sum(lin(int(x)) for x in sp.drafter)
+    attn = lambda keys: B * (keys * Hkv * d * 4 + nq * (2 * H * d * 2 + 2 * Hkv * d * 2))  # noqa: E731
+    verify_bytes = sum(attn(ctx) if x == I.FA else attn(w + k) if x == I.SWA else nq * lin(int(x))
+                       for x in target)
+    round_s = spec_s / args.steps
+    byts = draft_bytes + verify_bytes
+    la = sp.launches()
+    sp.free()
+    return {"metric": METRIC, "value": round(value, 2), "unit": "tok/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(round_s * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded); acceptance drawn from a seeded model, not a sampler",
+            "config": {"workload": ("spec_stack: self-speculative decode on the 48-layer "
+                                    "mixer-only stack, B=32, ctx 32768, H=32, Hkv=8, d=128; "
+                                    "target 12 FA/12 SWA(w=4096)/12 KDA/12 GDN, drafter all-GDN, "
+                                    "k=3 drafts, acceptance 0.8 per draft; a step is one round"),
+                       "inputs": "KV larger than L2 (48 GiB), states 22 GiB"},
+            "roofline": {"bound": "hbm", "achieved": round(byts / round_s / 1e9, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(byts / round_s / 1e9 / hbm, 4),
+                         "traffic": None, "algorithmic_bytes": byts,
+                         "scope": "whole round (draft + verify kernels)"},
+            "spec": {"k": k, "alpha": alpha,
+                     "mean_drafts_kept": round(float(sched.accepted[args.warmup:].mean()), 4),
+                     "tokens_per_round": round(tokens / args.steps, 3),
+                     "round_ms": round(round_s * 1e3, 4), "draft_ms": round(draft_s * 1e3, 4),
+                     "verify_ms": round(verify_s * 1e3, 4),
+                     "plain_step_ms": round(plain_s * 1e3, 4), "plain_tok_s": round(plain_tok_s, 2),
+                     "speedup_vs_plain": round(value / plain_tok_s, 4)},
+            "gpu_launches": (la["draft"] + la["verify"]) * args.steps}
+
+
 SWEEP_CTX = (4096, 16384, 65536, 131072)
 
 
@@ -637,7 +760,8 @@ def main():
     ap.add_argument("--workload", default="stack48",
                     choices=["stack48", "attn_fa", "attn_swa", "prefill_fa", "prefill_swa",
                              "decode_kda", "decode_gdn",
-                             "prefill_kda", "prefill_gdn", "sweep"])
+                             "prefill_kda", "prefill_gdn", "verify_fa", "verify_swa",
+                             "spec_stack", "sweep"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
@@ -649,6 +773,8 @@ def main():
         out = run_ours(args, rank, world, local_rank)
     elif args.workload == "sweep":
         out = run_sweep(args)
+    elif args.workload == "spec_stack":
+        out = run_spec(args)
     else:
         out = run_kernel_workload(args)
     if rank == 0 and out is not None:

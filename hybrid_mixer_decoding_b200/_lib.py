@@ -34,12 +34,17 @@ class DecodeIO(ctypes.Structure):
 
 _SIGS = {
     "delta_rule_decode": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _c_float, _vp]),
+    "delta_rule_decode_to": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _vp, _c_float,
+                                                                _vp]),
     "delta_rule_prefill_chunked": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
                                                                       _c_float, _vp]),
     "delta_rule_prefill_workspace_size": (_sz, [_c_int] * 8),
     "delta_rule_prefill_chunked_ws": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
                                                                          _c_float, _vp, _sz, _vp]),
     "attn_decode_workspace_size": (_sz, [_c_int] * 8),
+    "attn_verify_workspace_size": (_sz, [_c_int] * 9),
+    "attn_verify": (_c_int, [_c_int] * 9 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
+                                             _vp, _sz, _vp]),
     "attn_decode": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
                                                       _vp, _sz, _vp]),
     "attn_prefill": (_c_int, [_c_int] * 8 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _vp]),
@@ -129,6 +134,19 @@ def delta_rule_decode(kind, q, k, v, beta, log_gate, state, o, slots=None, scale
     _check("delta_rule_decode", st)
 
 
+def delta_rule_decode_to(kind, q, k, v, beta, log_gate, state, o, slots, dst_slots, scale=1.0,
+                         stream=None) -> None:
+    """delta_rule_decode reading slot slots[b] and writing the updated state to dst_slots[b]
+    (see include/hmd.h); slots, dst_slots int32 [B] on the device."""
+    _contig(q, k, v, beta, log_gate, state, o, slots, dst_slots)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    st = lib().delta_rule_decode_to(kind, B, H, dk, dv, _dtype_code(q), _p(q), _p(k), _p(v),
+                                    _p(beta), _p(log_gate), _p(state), state.shape[0], _p(slots),
+                                    _p(dst_slots), _p(o), float(scale), _stream(stream))
+    _check("delta_rule_decode_to", st)
+
+
 def delta_rule_prefill_chunked(kind, q, k, v, beta, log_gate, state, o, slots=None, chunk=64,
                                scale=1.0, stream=None) -> None:
     """Chunked GDN/KDA prefill (see include/hmd.h). q,k [B,T,H,dk]; v,o [B,T,H,dv];
@@ -181,6 +199,27 @@ def attn_decode(kind, window, q, new_k, new_v, k_pool, v_pool, page_table, seq_l
                            _p(seq_lens), int(max_seq_len), _p(o), _p(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check("attn_decode", st)
+
+
+def attn_verify_workspace_size(kind, window, n_q, B, Hq, Hkv, d, page_tokens, max_seq_len) -> int:
+    return int(lib().attn_verify_workspace_size(kind, window, n_q, B, Hq, Hkv, d, page_tokens,
+                                                max_seq_len))
+
+
+def attn_verify(kind, window, ring_pages, q, new_k, new_v, k_pool, v_pool, page_table, seq_lens,
+                max_seq_len, o, workspace, stream=None) -> None:
+    """Verification pass of n_q new tokens per sequence (see include/hmd.h).
+    q,o [B,n_q,Hq,d]; new_k,new_v [B,n_q,Hkv,d]; the rest as in attn_decode; ring_pages is the
+    SWA ring's size in pages (ignored for FA)."""
+    _contig(q, new_k, new_v, k_pool, v_pool, page_table, seq_lens, o, workspace)
+    B, n_q, Hq, d = q.shape
+    n_pages, Hkv, PT, _ = k_pool.shape
+    st = lib().attn_verify(kind, int(window), int(ring_pages), n_q, B, Hq, Hkv, d, PT, _p(q),
+                           _p(new_k), _p(new_v), _p(k_pool), _p(v_pool), n_pages, _p(page_table),
+                           page_table.shape[1], _p(seq_lens), int(max_seq_len), _p(o),
+                           _p(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check("attn_verify", st)
 
 
 def attn_decode_static_ws(kind, window, q, new_k, new_v, k_pool, v_pool, page_table, seq_lens,

@@ -20,6 +20,10 @@
 // new token into its shared-memory tile and writes it to the pool (the fused append). Keys
 // outside [lo, L-1] are masked and their V rows zeroed in shared memory, so stale or
 // uninitialised slots never reach the output. Partials (m, l, acc) go to the workspace.
+// Verification (speculative decoding) is the same kernel with n_q >= 1 new tokens per sequence:
+// token i sits at position P_i = L - n_q + i and attends [lo_i, P_i]; the n_q * G query rows of
+// a kv-head share the MMA's 16 rows (and the one pass over the pages), each row with its own
+// causal limit, and every new token is appended. n_q = 1 is the decode step.
 // Kernel 2 (combine): log-sum-exp merge of the splits into bf16 o.
 // The step is HBM-bound (K and V are read once: ~4 flop per byte); the design goal is to keep
 // enough page copies in flight to stream at the HBM rate.
@@ -51,9 +55,9 @@ struct SplitParams {
     __nv_bfloat16 *k_pool, *v_pool;
     const int32_t *page_table;
     const int32_t *seq_lens;
-    float *ws_ml;   // [B*Hq][n_splits][2]: running max (log2 domain), sum of exponentials
-    float *ws_acc;  // [B*Hq][n_splits][D]
-    int B, Hq, Hkv, group, n_pages, max_pages, window, swa, ring_pages;
+    float *ws_ml;   // [B*nq*Hq][n_splits][2]: running max (log2 domain), sum of exponentials
+    float *ws_acc;  // [B*nq*Hq][n_splits][D]
+    int B, Hq, Hkv, group, nq, n_pages, max_pages, window, swa, ring_pages;
     int n_splits, pages_per_split, max_seq_len;
     float scale_log2;  // log2(e) / sqrt(d)
 };
@@ -86,8 +90,9 @@ __device__ __forceinline__ Item item_info(const SplitParams &p, int i) {
     it.g = (i / p.n_splits) % p.Hkv;
     it.b = i / (p.n_splits * p.Hkv);
     it.L = p.seq_lens[it.b];
-    it.bad_len = it.L < 1 || it.L > p.max_seq_len;
-    it.lo = (p.swa && it.L > p.window) ? it.L - p.window : 0;
+    it.bad_len = it.L < p.nq || it.L > p.max_seq_len;
+    // the earliest key any row reads: that of the first new token, at position L - nq
+    it.lo = (p.swa && it.L - p.nq + 1 > p.window) ? it.L - p.nq + 1 - p.window : 0;
     const int first_page = it.bad_len ? 0 : it.lo / kPT;
     it.last_page = it.bad_len ? -1 : (it.L - 1) / kPT;
     it.t_begin = first_page + it.split * p.pages_per_split;
@@ -101,13 +106,21 @@ __device__ __forceinline__ int phys_page(const SplitParams &p, int b, int c) {
     return idx < p.max_pages ? p.page_table[(size_t)b * p.max_pages + idx] : -1;
 }
 
-// Q of one (sequence, kv-head) as mma.sync A fragments (rows = the group's query heads).
+// Q of one (sequence, kv-head) as mma.sync A fragments: row r = i * G + j is query head
+// g * G + j of new token i (rows past nq * G are zero).
+template <int D>
+__device__ __forceinline__ const uint32_t *q_row(const SplitParams &p, int b, int g, int r) {
+    const int G = p.group;
+    if (r >= p.nq * G) return nullptr;
+    const int i = r / G, j = r - i * G;
+    return reinterpret_cast<const uint32_t *>(p.q + (((size_t)b * p.nq + i) * p.Hq + g * G + j) * D);
+}
 template <int D>
 __device__ __forceinline__ void load_q(const SplitParams &p, int b, int g, int lane,
                                        uint32_t (&qa)[D / 16][4]) {
-    const int G = p.group, r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2;
-    const uint32_t *q0 = r0 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + r0) * D) : nullptr;
-    const uint32_t *q1 = r1 < G ? reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + r1) * D) : nullptr;
+    const int r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2;
+    const uint32_t *q0 = q_row<D>(p, b, g, r0);
+    const uint32_t *q1 = q_row<D>(p, b, g, r1);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         qa[kk][0] = q0 ? q0[(kk * 16 + cq) >> 1] : 0u;
@@ -195,6 +208,16 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     const int r0 = lane >> 2, r1 = r0 + 8, cq = (lane & 3) * 2, mi = lane >> 3;
     uint32_t qa[NK][4];
     load_q<D>(p, it.b, it.g, lane, qa);
+    // keys [lo_r, hi_r] of this thread's two rows (token r / G sits at L - nq + r / G); rows past
+    // nq * G read nothing
+    const int rows = p.nq * G, first_new = it.L - p.nq;
+    int row_lo[2], row_hi[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int r = rr ? r1 : r0;
+        row_hi[rr] = r < rows ? first_new + r / G : -1;
+        row_lo[rr] = (p.swa && row_hi[rr] + 1 > p.window) ? row_hi[rr] + 1 - p.window : 0;
+    }
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f};
     float oacc[NN][4];
@@ -219,7 +242,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         const int base = c * kPT;
         uint8_t *kb = smem + s * 2 * TB;
         uint8_t *vb = kb + TB;
-        const bool has_new = (c == it.last_page);
+        const bool has_new = base <= it.L - 1 && base + kPT - 1 >= first_new;
         const bool partial = base < it.lo || base + kPT - 1 > it.L - 1;
         if (tile_ok && (has_new || partial)) {
             // zero V rows of masked positions; patch in the new token's K and V
@@ -230,16 +253,19 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                     *reinterpret_cast<uint4 *>(vb + tile_off(row, ch * 8)) = make_uint4(0, 0, 0, 0);
             }
             if (has_new) {
-                const int rr = (it.L - 1) % kPT;
-                const size_t src = ((size_t)it.b * p.Hkv + it.g) * D;
-                for (int ch = tid; ch < 2 * (D / 8); ch += kThreads) {
+                for (int idx = tid; idx < p.nq * 2 * (D / 8); idx += kThreads) {
+                    const int i = idx / (2 * (D / 8)), ch = idx - i * (2 * (D / 8));
+                    const int pos = first_new + i;
+                    if (pos < base || pos >= base + kPT) continue;  // token i is in another tile
+                    const int rr = pos - base;
+                    const size_t src = (((size_t)it.b * p.nq + i) * p.Hkv + it.g) * D;
                     const int cc = ch % (D / 8);
                     const uint4 val = ch < D / 8
                         ? *reinterpret_cast<const uint4 *>(p.new_k + src + cc * 8)
                         : *reinterpret_cast<const uint4 *>(p.new_v + src + cc * 8);
                     uint8_t *dst = (ch < D / 8 ? kb : vb) + tile_off(rr, cc * 8);
                     *reinterpret_cast<uint4 *>(dst) = val;
-                    // the append itself: the pool slot of position L-1
+                    // the append itself: the pool slot of position L - nq + i
                     __nv_bfloat16 *pool = ch < D / 8 ? p.k_pool : p.v_pool;
                     *reinterpret_cast<uint4 *>(pool + (((size_t)pg * p.Hkv + it.g) * kPT + rr) * D + cc * 8) = val;
                 }
@@ -267,7 +293,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int pos = base + warp * 16 + j * 8 + cq + (e & 1);
-                    const bool valid = pos >= it.lo && pos <= it.L - 1;
+                    const bool valid = pos >= row_lo[e >> 1] && pos <= row_hi[e >> 1];
                     sc[j][e] = valid ? sc[j][e] * p.scale_log2 : -INFINITY;
                     mx[e >> 1] = fmaxf(mx[e >> 1], sc[j][e]);
                 }
@@ -322,7 +348,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     }
 
     // ---- merge the 4 warps' partials (the stages are idle now: reuse them) -------------------
-    float *red = reinterpret_cast<float *>(smem);  // [kWarps][group][D + 2]
+    float *red = reinterpret_cast<float *>(smem);  // [kWarps][rows][D + 2]
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         float l = l_run[r];
@@ -330,8 +356,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         l += __shfl_xor_sync(0xffffffffu, l, 2);
         l_run[r] = l;
     }
-    if (r0 < G) {
-        float *dst = red + (warp * G + r0) * RS;
+    if (r0 < rows) {
+        float *dst = red + (warp * rows + r0) * RS;
 #pragma unroll
         for (int n = 0; n < NN; ++n) {
             dst[n * 8 + cq] = oacc[n][0];
@@ -339,8 +365,8 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         }
         if ((lane & 3) == 0) { dst[D] = m_run[0]; dst[D + 1] = l_run[0]; }
     }
-    if (r1 < G) {
-        float *dst = red + (warp * G + r1) * RS;
+    if (r1 < rows) {
+        float *dst = red + (warp * rows + r1) * RS;
 #pragma unroll
         for (int n = 0; n < NN; ++n) {
             dst[n * 8 + cq] = oacc[n][2];
@@ -349,21 +375,22 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         if ((lane & 3) == 0) { dst[D] = m_run[1]; dst[D + 1] = l_run[1]; }
     }
     __syncthreads();
-    for (int idx = tid; idx < G * D; idx += kThreads) {
+    for (int idx = tid; idx < rows * D; idx += kThreads) {
         const int r = idx / D, dim = idx % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * G + r) * RS + D]);
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * rows + r) * RS + D]);
         float acc = 0.f, lsum = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) {
-                const float f = exp2f(red[(w * G + r) * RS + D] - M);
-                acc += f * red[(w * G + r) * RS + dim];
-                lsum += f * red[(w * G + r) * RS + D + 1];
+                const float f = exp2f(red[(w * rows + r) * RS + D] - M);
+                acc += f * red[(w * rows + r) * RS + dim];
+                lsum += f * red[(w * rows + r) * RS + D + 1];
             }
         }
-        const size_t row = ((size_t)it.b * p.Hq + it.g * G + r) * p.n_splits + it.split;
+        const int ti = r / G;  // new token ti, query head g * G + (r - ti * G)
+        const size_t row = (((size_t)it.b * p.nq + ti) * p.Hq + it.g * G + (r - ti * G)) * p.n_splits + it.split;
         p.ws_acc[row * D + dim] = acc;
         if (dim == 0) {
             p.ws_ml[row * 2] = M;
@@ -452,20 +479,20 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     p.v_pool = static_cast<__nv_bfloat16 *>(a.v_pool);
     p.page_table = a.page_table;
     p.seq_lens = a.seq_lens;
-    const size_t rows = (size_t)a.B * a.Hq * plan.n_splits;
+    const size_t rows = (size_t)a.B * a.nq * a.Hq * plan.n_splits;
     p.ws_ml = static_cast<float *>(a.workspace);
     p.ws_acc = p.ws_ml + ((rows * 2 + 3) & ~static_cast<size_t>(3));
-    p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.group = group;
+    p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.group = group; p.nq = a.nq;
     p.n_pages = a.n_pages; p.max_pages = a.max_pages;
     p.window = a.window; p.swa = a.swa ? 1 : 0;
-    p.ring_pages = a.swa ? (a.window + kPT - 1) / kPT : 0;
+    p.ring_pages = a.swa ? a.ring_pages : 0;
     p.n_splits = plan.n_splits; p.pages_per_split = plan.pages_per_split;
     p.max_seq_len = a.max_seq_len;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     cudaError_t e = launch_pdl(attn_split_kernel<D>, dim3((unsigned)plan.n_ctas), dim3(kThreads),
                                smem, s, tmk, tmv, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(a.B * a.Hq)), dim3(D), 0, s,
+    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(a.B * a.nq * a.Hq)), dim3(D), 0, s,
                       (const float *)p.ws_ml, (const float *)p.ws_acc, plan.n_splits,
                       static_cast<__nv_bfloat16 *>(a.o));
 }
@@ -489,17 +516,18 @@ int device_sms() {
 
 }  // namespace
 
-bool attn_decode_supported(int d, int page_tokens, int group) {
-    return (d == 64 || d == 128) && page_tokens == kPT && group >= 1 && group <= kMaxGroup;
+bool attn_decode_supported(int d, int page_tokens, int group, int nq) {
+    return (d == 64 || d == 128) && page_tokens == kPT && group >= 1 && nq >= 1 &&
+           (long long)group * nq <= kMaxGroup;
 }
 
 AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, int page_tokens,
-                          int max_seq_len) {
+                          int max_seq_len, int nq) {
     (void)page_tokens;
     (void)Hq;
     AttnPlan pl;
     long long tiles = (max_seq_len + kPT - 1) / kPT;
-    if (swa) tiles = std::min<long long>(tiles, (window + kPT - 1) / kPT + 1);
+    if (swa) tiles = std::min<long long>(tiles, ((long long)window + nq - 1 + kPT - 1) / kPT + 1);
     tiles = std::max<long long>(tiles, 1);
     const long long units = std::max<long long>(1, (long long)B * Hkv);
     // resident CTAs per SM from shared memory (228 KiB per SM, 1 KiB reserved per CTA)
@@ -519,14 +547,14 @@ AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, i
     pl.n_splits = (int)splits;
     pl.pages_per_split = (int)pps;
     pl.n_ctas = (int)(units * splits);
-    const size_t rows = (size_t)B * Hq * splits;
+    const size_t rows = (size_t)B * nq * Hq * splits;
     pl.ws_bytes = (((rows * 2 + 3) & ~static_cast<size_t>(3)) + rows * d) * sizeof(float);
     return pl;
 }
 
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s) {
     const AttnPlan plan = attn_decode_plan(a.swa, a.window, a.B, a.Hq, a.Hkv, a.d, a.page_tokens,
-                                           a.max_seq_len);
+                                           a.max_seq_len, a.nq);
     if (a.d == 128) return launch_d<128>(a, plan, s);
     if (a.d == 64) return launch_d<64>(a, plan, s);
     return cudaErrorInvalidValue;

@@ -11,7 +11,8 @@
 //
 // Work split: one CTA of 128 threads per (sequence, head, 32-column slice of d_v). The slice
 // ([d_k][32] fp32, 16 KiB at d_k = 128) arrives by one 2-D TMA box into shared memory and leaves
-// by one TMA store after the in-place update, so each CTA holds few registers and many CTAs per
+// by one TMA store after the update (in place, or to another slot: a speculative draft step
+// writes a fresh slot so that rejecting it is a choice of slot, not a copy), so each CTA holds few registers and many CTAs per
 // SM keep their slices in flight. A thread owns 4 adjacent columns (one 16-byte vector) of
 // d_k/16 rows; column sums are reduced over rows with warp shuffles (xor 8, 16), then across the
 // 4 warps through shared memory. No tensor cores: the step is ~1 flop per byte, far below any
@@ -67,7 +68,8 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     griddep_wait();  // q, k, v, gates and the state may come from the previous kernel
     if (tid == 0) {
         const int slot = a.slots ? a.slots[b] : b;
-        const bool ok = slot >= 0 && slot < a.n_slots;
+        const int dst = a.dst_slots ? a.dst_slots[b] : slot;
+        const bool ok = slot >= 0 && slot < a.n_slots && dst >= 0 && dst < a.n_slots;
         s_ok = ok;
         if (ok) {
             const uint32_t bb = smem_u32(&bar);
@@ -177,7 +179,8 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     __syncthreads();
     if (tid == 0) {
         const int slot = a.slots ? a.slots[b] : b;
-        tma_store_2d(&tm, smem_u32(&S[0][0]), slice * kSliceCols, (slot * a.H + h) * DK);
+        const int dst = a.dst_slots ? a.dst_slots[b] : slot;
+        tma_store_2d(&tm, smem_u32(&S[0][0]), slice * kSliceCols, (dst * a.H + h) * DK);
         bulk_commit_group();
         bulk_wait_group_read0();
     }

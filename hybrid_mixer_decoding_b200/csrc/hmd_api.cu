@@ -95,10 +95,11 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
 
 // ---- delta-rule mixers -------------------------------------------------------------------
 
-hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
-                               const void *q, const void *k, const void *v, const float *beta,
-                               const float *log_gate, float *state, int n_slots,
-                               const int32_t *slots, void *o, float scale, hmd_stream_t stream) {
+hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk, int dv,
+                                  hmd_dtype_t dtype, const void *q, const void *k, const void *v,
+                                  const float *beta, const float *log_gate, float *state,
+                                  int n_slots, const int32_t *slots, const int32_t *dst_slots,
+                                  void *o, float scale, hmd_stream_t stream) {
     const hmd_status_t st = check_delta_decode(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate,
                                                state, n_slots, o);
     if (st != HMD_OK) return fail(st);
@@ -107,8 +108,16 @@ hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hm
     hmd::DeltaDecodeArgs a{};
     a.kind = kind; a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
-    a.n_slots = n_slots; a.slots = slots; a.o = o; a.scale = scale;
+    a.n_slots = n_slots; a.slots = slots; a.dst_slots = dst_slots; a.o = o; a.scale = scale;
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
+}
+
+hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
+                               const void *q, const void *k, const void *v, const float *beta,
+                               const float *log_gate, float *state, int n_slots,
+                               const int32_t *slots, void *o, float scale, hmd_stream_t stream) {
+    return delta_rule_decode_to(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate, state,
+                                n_slots, slots, nullptr, o, scale, stream);
 }
 
 }  // extern "C"
@@ -266,22 +275,28 @@ hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int Hq, int
     return from_cuda(hmd::launch_attn_prefill(a, as_stream(stream)));
 }
 
-size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
-                                  int page_tokens, int max_seq_len) {
-    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || max_seq_len < 1) return 16;
+size_t attn_verify_workspace_size(hmd_kind_t kind, int window, int n_q, int B, int Hq, int Hkv,
+                                  int d, int page_tokens, int max_seq_len) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || max_seq_len < 1 || n_q < 1) return 16;
     const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, B, Hq, Hkv, d,
-                                                   page_tokens, max_seq_len);
+                                                   page_tokens, max_seq_len, n_q);
     return pl.ws_bytes < 16 ? 16 : pl.ws_bytes;
 }
 
-hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
-                         int page_tokens, const void *q, const void *new_k, const void *new_v,
-                         void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
-                         int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
-                         void *workspace, size_t ws_bytes, hmd_stream_t stream) {
+size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                                  int page_tokens, int max_seq_len) {
+    return attn_verify_workspace_size(kind, window, 1, B, Hq, Hkv, d, page_tokens, max_seq_len);
+}
+
+hmd_status_t attn_verify(hmd_kind_t kind, int window, int ring_pages, int n_q, int B, int Hq,
+                         int Hkv, int d, int page_tokens, const void *q, const void *new_k,
+                         const void *new_v, void *k_pool, void *v_pool, int n_pages,
+                         const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                         int max_seq_len, void *o, void *workspace, size_t ws_bytes,
+                         hmd_stream_t stream) {
     if (kind != HMD_FA && kind != HMD_SWA) return fail(HMD_ERR_ARG);
     if (kind == HMD_SWA && window < 1) return fail(HMD_ERR_ARG);
-    if (B < 0 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
+    if (B < 0 || n_q < 1 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
         max_pages < 1 || max_seq_len < 1)
         return fail(HMD_ERR_SHAPE);
     if (Hq % Hkv) return fail(HMD_ERR_SHAPE);
@@ -289,28 +304,45 @@ hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, in
     if (!q || !new_k || !new_v || !k_pool || !v_pool || !page_table || !seq_lens || !o ||
         !workspace)
         return fail(HMD_ERR_ARG);
-    if (!hmd::attn_decode_supported(d, page_tokens, Hq / Hkv)) return fail(HMD_ERR_UNSUPPORTED);
-    // the table must be wide enough for the longest sequence (FA) or for the ring (SWA)
-    const long long need = kind == HMD_SWA
-        ? (window + page_tokens - 1) / page_tokens < (max_seq_len + page_tokens - 1) / page_tokens
-              ? (window + page_tokens - 1) / page_tokens
-              : (max_seq_len + page_tokens - 1) / page_tokens
-        : (max_seq_len + page_tokens - 1) / page_tokens;
+    if (!hmd::attn_decode_supported(d, page_tokens, Hq / Hkv, n_q)) return fail(HMD_ERR_UNSUPPORTED);
+    const long long seq_pages = ((long long)max_seq_len + page_tokens - 1) / page_tokens;
+    long long need = seq_pages;  // FA: the table covers the longest sequence
+    if (kind == HMD_SWA) {
+        // the ring must hold every key of the n_q rows at once: window + n_q - 1 positions
+        const long long min_ring = ((long long)window + n_q - 1 + page_tokens - 1) / page_tokens;
+        if (ring_pages < min_ring) return fail(HMD_ERR_SHAPE);
+        need = ring_pages < seq_pages ? ring_pages : seq_pages;
+    }
     if (max_pages < need) return fail(HMD_ERR_SHAPE);
     if ((long long)n_pages * Hkv * page_tokens >= (1LL << 31)) return fail(HMD_ERR_UNSUPPORTED);
     if (!aligned16(q) || !aligned16(new_k) || !aligned16(new_v) || !aligned16(k_pool) ||
         !aligned16(v_pool) || !aligned16(workspace))
         return fail(HMD_ERR_ARG);
     const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, B, Hq, Hkv, d,
-                                                   page_tokens, max_seq_len);
+                                                   page_tokens, max_seq_len, n_q);
     if (ws_bytes < pl.ws_bytes) return fail(HMD_ERR_SHAPE);
     hmd::AttnDecodeArgs a{};
-    a.swa = kind == HMD_SWA; a.window = window; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.swa = kind == HMD_SWA; a.window = window; a.ring_pages = ring_pages; a.nq = n_q;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
     a.page_tokens = page_tokens; a.q = q; a.new_k = new_k; a.new_v = new_v;
     a.k_pool = k_pool; a.v_pool = v_pool; a.n_pages = n_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seq_lens = seq_lens; a.max_seq_len = max_seq_len; a.o = o;
     a.workspace = workspace; a.ws_bytes = ws_bytes;
     return from_cuda(hmd::launch_attn_decode(a, as_stream(stream)));
+}
+
+hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
+                         int page_tokens, const void *q, const void *new_k, const void *new_v,
+                         void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
+                         int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
+                         void *workspace, size_t ws_bytes, hmd_stream_t stream) {
+    // the decode step is the one-token verification pass on the ring of ceil(window / 64) pages
+    const int ring = (kind == HMD_SWA && window >= 1 && page_tokens >= 1)
+                         ? (int)(((long long)window + page_tokens - 1) / page_tokens)
+                         : 0;
+    return attn_verify(kind, window, ring, 1, B, Hq, Hkv, d, page_tokens, q, new_k, new_v, k_pool,
+                       v_pool, n_pages, page_table, max_pages, seq_lens, max_seq_len, o,
+                       workspace, ws_bytes, stream);
 }
 
 // ---- caches ------------------------------------------------------------------------------

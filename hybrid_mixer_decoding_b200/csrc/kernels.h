@@ -47,6 +47,7 @@ struct DeltaDecodeArgs {
     float *state;
     int n_slots;
     const int32_t *slots;
+    const int32_t *dst_slots;  // where the updated state goes (NULL: back to slots, in place)
     void *o;
     float scale;
 };
@@ -57,6 +58,8 @@ uint32_t delta_decode_read_errors(bool clear);
 struct AttnDecodeArgs {
     bool swa;
     int window;
+    int ring_pages;  // SWA ring size in pages (>= ceil((window + nq - 1) / page_tokens))
+    int nq = 1;      // new tokens per sequence (1: decode step; more: verification pass)
     int B, Hq, Hkv, d, page_tokens;
     const void *q, *new_k, *new_v;
     void *k_pool, *v_pool;
@@ -76,9 +79,9 @@ struct AttnPlan {
     size_t ws_bytes;
 };
 AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, int page_tokens,
-                          int max_seq_len);
+                          int max_seq_len, int nq);
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s);
-bool attn_decode_supported(int d, int page_tokens, int group);
+bool attn_decode_supported(int d, int page_tokens, int group, int nq);
 uint32_t attn_decode_read_errors(bool clear);
 
 struct DeltaPrefillArgs {

@@ -85,6 +85,19 @@ HMD_API hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, in
                                const float *log_gate, float *state, int n_slots,
                                const int32_t *slots, void *o, float scale, hmd_stream_t stream);
 
+/* delta_rule_decode that writes the updated state of sequence b to slot dst_slots[b] (device
+ * int32 [B]) and leaves slot slots[b] as it was (dst_slots == NULL: in place). A speculative
+ * draft of k tokens steps slot s0 -> s1 -> ... -> sk; keeping the first j accepted tokens is
+ * then the choice of slot s_j, with nothing copied or recomputed. Slots must lie in
+ * [0, n_slots) (else the device error word reports HMD_DEVERR_SLOT and that sequence is
+ * skipped); no destination slot may be another sequence's source or destination in this call. */
+HMD_API hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk, int dv,
+                                          hmd_dtype_t dtype, const void *q, const void *k,
+                                          const void *v, const float *beta,
+                                          const float *log_gate, float *state, int n_slots,
+                                          const int32_t *slots, const int32_t *dst_slots,
+                                          void *o, float scale, hmd_stream_t stream);
+
 /* Chunked (WY / UT-transform) prefill over T tokens per sequence for one layer: the same
  * recurrence as delta_rule_decode applied to tokens 0..T-1 in order, computed chunk by chunk.
  *   q, k [B][T][H][dk]; v, o [B][T][H][dv] (dtype); beta [B][T][H] fp32;
@@ -159,6 +172,34 @@ HMD_API hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int
                          void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
                          int max_pages, const int32_t *seq_lens, int max_seq_len, void *o,
                          void *workspace, size_t ws_bytes, hmd_stream_t stream);
+
+/* Verification pass of speculative decoding (and multi-token decoding): n_q new tokens per
+ * sequence in one pass, equal to n_q attn_decode steps in a row. Token i of sequence b sits at
+ * logical position P = L - n_q + i (L = seq_lens[b] counts all n_q, each L >= n_q) and attends
+ * keys j in [lo, P], lo = 0 (FA) or max(0, P + 1 - window) (SWA); all n_q tokens' k, v are
+ * appended at their slots. Self-speculative decoding drafts tokens with a cheap placement of
+ * the supernet and checks them with a better one ("Super Apriel: One Checkpoint, Many Speeds",
+ * gist.science summary, sections 1 and 4); on a memory-bound decode step the n_q * (Hq / Hkv)
+ * query rows of a kv-head share one pass over its pages, so checking n_q tokens costs about
+ * one decode step. Rejected tokens need no undo: the next call's seq_lens decide what is read.
+ *   q, o [B][n_q][Hq][d] bf16; new_k, new_v [B][n_q][Hkv][d] bf16; the rest as in attn_decode.
+ *   ring_pages (SWA; ignored for FA): the ring's size in pages. Positions are kept at ring index
+ *   p mod (ring_pages * page_tokens); it must hold window + n_q - 1 positions
+ *   (ring_pages >= ceil((window + n_q - 1) / page_tokens), else HMD_ERR_SHAPE), so that the new
+ *   tokens never overwrite a key an earlier row or the next step still reads. A cache verified
+ *   this way must be decoded with attn_verify(n_q = 1) on the same ring_pages (attn_decode
+ *   assumes ceil(window / page_tokens)).
+ *   workspace: at least attn_verify_workspace_size(...) bytes.
+ * Supported: d in {64, 128}; page_tokens == 64; n_q * (Hq / Hkv) <= 16 (HMD_ERR_UNSUPPORTED).
+ * Allocates nothing. attn_decode is this call with n_q = 1 on the default ring.               */
+HMD_API size_t attn_verify_workspace_size(hmd_kind_t kind, int window, int n_q, int B, int Hq,
+                                          int Hkv, int d, int page_tokens, int max_seq_len);
+HMD_API hmd_status_t attn_verify(hmd_kind_t kind, int window, int ring_pages, int n_q, int B,
+                                 int Hq, int Hkv, int d, int page_tokens, const void *q,
+                                 const void *new_k, const void *new_v, void *k_pool,
+                                 void *v_pool, int n_pages, const int32_t *page_table,
+                                 int max_pages, const int32_t *seq_lens, int max_seq_len,
+                                 void *o, void *workspace, size_t ws_bytes, hmd_stream_t stream);
 
 /* FA / SWA prefill of T prompt tokens per sequence into an empty paged cache. Token t of
  * sequence b is logical position t and attends keys j in [lo_t, t], lo_t = 0 (FA) or

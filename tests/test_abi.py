@@ -110,6 +110,41 @@ def test_attn_validation():
     assert _attn(ptr=None) == ARG
 
 
+def _verify(kind=hmd.SWA, window=100, ring=2, n_q=4, B=2, Hq=8, Hkv=2, d=128, PT=64, max_pages=4,
+            max_len=256, ws=1 << 30, ptr=FAKE, n_pages=16):
+    return hmd.lib().attn_verify(kind, window, ring, n_q, B, Hq, Hkv, d, PT, ptr, ptr, ptr, ptr,
+                                 ptr, n_pages, ptr, max_pages, ptr, max_len, ptr, ptr, ws, None)
+
+
+def test_verify_validation():
+    assert _verify(n_q=0) == SHAPE
+    assert _verify(n_q=5) == UNSUP               # 5 tokens x GQA group 4 > 16 MMA rows
+    assert _verify(n_q=4, Hq=16, Hkv=2) == UNSUP  # 4 x 8 > 16
+    assert _verify(n_q=16, Hq=8, Hkv=8) != UNSUP  # 16 x 1 rows fit
+    # SWA ring must hold window + n_q - 1 = 103 positions: 2 pages of 64
+    assert _verify(window=128, ring=2) == SHAPE  # 131 positions need 3 pages
+    assert _verify(window=128, ring=3, max_pages=3) != SHAPE
+    assert _verify(window=128, ring=3, max_pages=2, max_len=256) == SHAPE  # table < ring
+    assert _verify(window=128, ring=3, max_pages=2, max_len=100) != SHAPE  # short sequences
+    assert _verify(kind=hmd.FA, ring=0, max_pages=3) == SHAPE  # FA table < 256 tokens
+    assert _verify(ws=16) == SHAPE
+    assert _verify(ptr=None) == ARG
+    assert _verify(B=0) == 0
+    # one token on the default ring is the decode step's validation
+    assert _verify(window=4096, ring=64, n_q=1, max_pages=64, max_len=8192) != SHAPE
+    assert _verify(window=4096, ring=64, n_q=2, max_pages=64, max_len=8192) == SHAPE
+
+
+def test_verify_workspace_is_decode_workspace_times_rows():
+    for kind, w in ((hmd.FA, 0), (hmd.SWA, 4096)):
+        for n_q in (1, 2, 4):
+            v = hmd.attn_verify_workspace_size(kind, w, n_q, 64, 32, 8, 128, 64, 32768)
+            d1 = hmd.attn_decode_workspace_size(kind, w, 64, 32, 8, 128, 64, 32768)
+            if n_q == 1:
+                assert v == d1
+            assert v >= 4 * 64 * n_q * 32 * 130
+
+
 def test_workspace_size_bounds():
     """Partials are one (m, l) pair and one d-vector per query row and key range, with at most
     256 key ranges and never more ranges than 64-token pages."""

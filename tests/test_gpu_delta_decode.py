@@ -130,3 +130,54 @@ def test_full_size_stack_layer_sampled(oracle_mod, kind):
                                           d.log_gate[sl], d.state0[sl])
         assert O.rel_err(o[b].float().cpu().numpy(), o_ref[0, 0]) < 2e-2
         assert O.rel_err(state[b].cpu().numpy(), st_ref[0]) < 2e-2
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_out_of_place_draft_chain_and_rollback(oracle_mod, kind):
+    """A speculative draft of 3 tokens steps slots s0 -> s1 -> s2 -> s3 with
+    delta_rule_decode_to: each slot holds the state after its token, bit-identical to the
+    in-place path, the source slots are never written, and every slot matches the oracle's
+    recurrence after that many tokens (so rejecting tokens is a choice of slot)."""
+    O = oracle_mod
+    B, T, H, dkv = 3, 3, 4, 128
+    d = I.delta_inputs(kind, B, T, H, dkv, dkv, dtype="bf16", seed=31, state0="randn")
+    act = torch.bfloat16
+    n_slots = B * (T + 1)
+    chain = torch.zeros(n_slots, H, dkv, dkv, device="cuda")
+    slot_of = lambda t: np.arange(B, dtype=np.int32) * (T + 1) + t  # sequence b, step t
+    chain[torch.from_numpy(slot_of(0)).long().cuda()] = _dev(d.state0)
+    inplace = torch.zeros(B, H, dkv, dkv, device="cuda")
+    inplace[:] = _dev(d.state0)
+    for t in range(T):
+        q, k, v = (_dev(x[:, t], act) for x in (d.q, d.k, d.v))
+        beta, lg = _dev(d.beta[:, t]), _dev(d.log_gate[:, t])
+        src_before = chain[torch.from_numpy(slot_of(t)).long().cuda()].clone()
+        o1 = torch.empty(B, H, dkv, device="cuda", dtype=act)
+        hmd.delta_rule_decode_to(kind, q, k, v, beta, lg, chain, o1,
+                                 _dev(slot_of(t), torch.int32), _dev(slot_of(t + 1), torch.int32))
+        o2 = torch.empty_like(o1)
+        hmd.delta_rule_decode(kind, q, k, v, beta, lg, inplace, o2)
+        torch.cuda.synchronize()
+        assert hmd.hmd_device_errors(clear=True) == 0
+        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+        assert torch.equal(chain[torch.from_numpy(slot_of(t + 1)).long().cuda()], inplace)
+        assert torch.equal(chain[torch.from_numpy(slot_of(t)).long().cuda()], src_before)
+        _, st_ref = O.delta_recurrent(kind, d.q[:, :t + 1], d.k[:, :t + 1], d.v[:, :t + 1],
+                                      d.beta[:, :t + 1], d.log_gate[:, :t + 1], d.state0)
+        got = chain[torch.from_numpy(slot_of(t + 1)).long().cuda()].cpu().numpy()
+        assert O.rel_err(got, st_ref) < TOL["bf16"]
+
+
+def test_out_of_place_bad_destination_sets_device_error():
+    d = I.delta_inputs(I.GDN, 2, 1, 2, 64, 64, dtype="bf16", seed=32)
+    state = torch.zeros(4, 2, 64, 64, device="cuda")
+    before = state.clone()
+    o = torch.empty(2, 2, 64, device="cuda", dtype=torch.bfloat16)
+    hmd.delta_rule_decode_to(I.GDN, _dev(d.q[:, 0], torch.bfloat16), _dev(d.k[:, 0], torch.bfloat16),
+                             _dev(d.v[:, 0], torch.bfloat16), _dev(d.beta[:, 0]),
+                             _dev(d.log_gate[:, 0]), state, o, _dev(np.array([0, 1], np.int32), torch.int32),
+                             _dev(np.array([2, 4], np.int32), torch.int32))
+    torch.cuda.synchronize()
+    assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_SLOT
+    # sequence 0 (valid destination) was written to slot 2; sequence 1 skipped entirely
+    assert torch.equal(state[[0, 1, 3]], before[[0, 1, 3]])
