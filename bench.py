@@ -496,7 +496,7 @@ def run_kernel_workload(args):
                 f"paged bf16 KV (64-token pages, random permutation); value = tokens checked/s")
         roof = {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1), "peak": hbm,
                 "unit": "GB/s", "frac": round(byts / sec / 1e9 / hbm, 4),
-                "traffic": None, "algorithmic_bytes": byts}
+                "traffic": traffic_for(w), "algorithmic_bytes": byts}
         extra["verify"] = {"us_per_pass_by_n_q": {str(n): round(t * 1e6, 2) for n, t in per_nq.items()},
                            "cost_vs_one_token": round(per_nq[nq_max] / per_nq[1], 4)}
         launches = 2
