@@ -678,6 +678,59 @@ def run_spec(args):
             "gpu_launches": (la["draft"] + la["verify"]) * args.steps}
 
 
+def run_mixed(args):
+    """Mixed placements in one batch on the 48-layer mixer-only stack: B=64, context 32768,
+    H=32, Hkv=8, d=128; 32 sequences follow the 12 FA / 12 SWA / 12 KDA / 12 GDN placement and
+    32 the all-GDN placement, in one mixed step per token (each layer runs each of its mixers
+    over its group of sequences). The single-placement steps of the same stack at the same B
+    are timed alongside. Each step is one CUDA-graph replay."""
+    import torch
+
+    import hybrid_mixer_decoding_b200 as hmd
+    from hybrid_mixer_decoding_b200.stack import MixerStack, StackShape, layer_bytes
+
+    pk, _ = peaks()
+    hbm = float(pk["hbm_gbs"])
+    shape = StackShape(B=64, H=32, Hkv=8, d=128, ctx=32768, window=4096)
+    pls = {"hybrid": stack_placement(), "all_gdn": np.full(48, I.GDN, np.int8)}
+    st = MixerStack(pls, shape, fill_kv=False)
+    sp = np.array([0, 1] * 32, np.int32)  # interleaved: every other sequence on each preset
+    plan = st.batch_plan(sp)
+    graphs = {"mixed": st.capture(lambda: st.step_batch(plan)),
+              "hybrid": st.capture("hybrid"), "all_gdn": st.capture("all_gdn")}
+    sec = {}
+    for name, g in graphs.items():
+        sec[name] = _events_time(g.replay, args.steps, args.warmup)
+    assert hmd.hmd_device_errors(clear=True) == 0
+    half = StackShape(B=32, H=32, Hkv=8, d=128, ctx=32768, window=4096)
+    byts = sum(layer_bytes(int(k), half) for k in pls["hybrid"]) + \
+        sum(layer_bytes(int(k), half) for k in pls["all_gdn"])
+    launches = sum((2 if plan.group(l, k).size and k in (I.FA, I.SWA) else
+                    1 if plan.group(l, k).size else 0)
+                   for l in range(48) for k in (I.FA, I.SWA, I.KDA, I.GDN))
+    aliased = st.aliased
+    plan.free()
+    st.free()
+    t = sec["mixed"]
+    return {"metric": METRIC, "value": round(shape.B / t, 2), "unit": "tok/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init caches, no weights)",
+            "config": {"workload": ("mixed_stack: one batch of 64 sequences at ctx 32768 on the "
+                                    "48-layer mixer-only stack, 32 on the 12 FA/12 SWA/12 KDA/"
+                                    "12 GDN placement and 32 on all-GDN, one mixed step per token"),
+                       "kv_aliased": aliased,
+                       "inputs": "KV and states larger than L2"},
+            "roofline": {"bound": "hbm", "achieved": round(byts / t / 1e9, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(byts / t / 1e9 / hbm, 4), "traffic": None,
+                         "algorithmic_bytes": byts, "scope": "whole mixed step"},
+            "mixed": {"mixed_ms": round(t * 1e3, 4),
+                      "hybrid_B64_ms": round(sec["hybrid"] * 1e3, 4),
+                      "all_gdn_B64_ms": round(sec["all_gdn"] * 1e3, 4),
+                      "half_of_each_ms": round((sec["hybrid"] + sec["all_gdn"]) / 2 * 1e3, 4)},
+            "gpu_launches": launches * args.steps}
+
+
 SWEEP_CTX = (4096, 16384, 65536, 131072)
 
 
@@ -761,7 +814,7 @@ def main():
                     choices=["stack48", "attn_fa", "attn_swa", "prefill_fa", "prefill_swa",
                              "decode_kda", "decode_gdn",
                              "prefill_kda", "prefill_gdn", "verify_fa", "verify_swa",
-                             "spec_stack", "sweep"])
+                             "spec_stack", "mixed_stack", "sweep"])
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
@@ -775,6 +828,8 @@ def main():
         out = run_sweep(args)
     elif args.workload == "spec_stack":
         out = run_spec(args)
+    elif args.workload == "mixed_stack":
+        out = run_mixed(args)
     else:
         out = run_kernel_workload(args)
     if rank == 0 and out is not None:

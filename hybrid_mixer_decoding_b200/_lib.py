@@ -34,6 +34,13 @@ class DecodeIO(ctypes.Structure):
 
 _SIGS = {
     "delta_rule_decode": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _c_float, _vp]),
+    "hmd_group_sequences": (_c_int, [_c_int, _c_int, _vp, _c_int, _vp, _vp, _vp]),
+    "batch_plan_create": (_c_int, [_c_int, _c_int, _vp, _c_int, _vp, _vp, ctypes.POINTER(_vp)]),
+    "batch_plan_free": (_c_int, [_vp, _vp]),
+    "batch_plan_group": (_c_int, [_vp, _c_int, _c_int, ctypes.POINTER(_c_int),
+                                  ctypes.POINTER(ctypes.POINTER(ctypes.c_int32))]),
+    "batch_plan_workspace_size": (_sz, [_vp] + [_c_int] * 6),
+    "mixer_decode_step_batch": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "delta_rule_decode_to": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _vp, _c_float,
                                                                 _vp]),
     "delta_rule_prefill_chunked": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
@@ -331,6 +338,72 @@ def mixer_decode_step(placement, layer, io: DecodeIO, state_cache=None, kv_cache
                                  kv_cache.handle if kv_cache else None, ws, ws_bytes,
                                  _stream(stream))
     _check("mixer_decode_step", st)
+
+
+def group_sequences(placements, seq_placement):
+    """hmd_group_sequences (host only): placements int8 [n_placements][n_layers], seq_placement
+    int32 [B] -> (rows int32 [n_layers][B], offsets int32 [n_layers][5])."""
+    import numpy as np
+    pl = np.ascontiguousarray(placements, dtype=np.int8)
+    sp = np.ascontiguousarray(seq_placement, dtype=np.int32)
+    n_p, n_l = pl.shape
+    B = sp.shape[0]
+    rows = np.zeros((n_l, B), np.int32)
+    offs = np.zeros((n_l, 5), np.int32)
+    _check("hmd_group_sequences", lib().hmd_group_sequences(
+        n_l, n_p, pl.ctypes.data, B, sp.ctypes.data, rows.ctypes.data, offs.ctypes.data))
+    return rows, offs
+
+
+class BatchPlan:
+    """batch_plan_create / _group / _workspace_size / _free: the per-layer grouping of a
+    mixed batch's sequences by mixer kind, with the rows on the device."""
+
+    def __init__(self, placements, seq_placement, stream=None):
+        import numpy as np
+        pl = np.ascontiguousarray(placements, dtype=np.int8)
+        sp = np.ascontiguousarray(seq_placement, dtype=np.int32)
+        self.n_layers, self.B = pl.shape[1], sp.shape[0]
+        h = _vp()
+        _check("batch_plan_create", lib().batch_plan_create(self.n_layers, pl.shape[0],
+                                                            pl.ctypes.data, self.B,
+                                                            sp.ctypes.data, _stream(stream),
+                                                            ctypes.byref(h)))
+        self.handle = h.value
+
+    def group(self, layer, kind):
+        import numpy as np
+        n = _c_int()
+        ptr = ctypes.POINTER(ctypes.c_int32)()
+        _check("batch_plan_group", lib().batch_plan_group(self.handle, layer, kind,
+                                                          ctypes.byref(n), ctypes.byref(ptr)))
+        return np.ctypeslib.as_array(ptr, shape=(n.value,)).copy() if n.value else \
+            np.zeros(0, np.int32)
+
+    def workspace_size(self, window, Hq, Hkv, d, page_tokens, max_seq_len) -> int:
+        return int(lib().batch_plan_workspace_size(self.handle, window, Hq, Hkv, d, page_tokens,
+                                                   max_seq_len))
+
+    def free(self, stream=None):
+        if self.handle:
+            _check("batch_plan_free", lib().batch_plan_free(self.handle, _stream(stream)))
+            self.handle = None
+
+
+def mixer_decode_step_batch(plan: BatchPlan, layer, ios, state_cache=None, kv_cache=None,
+                            workspace=None, stream=None) -> None:
+    """One decode token for layer `layer` of a mixed batch: ios maps each kind present at the
+    layer to its DecodeIO (full-batch tensors)."""
+    arr = (ctypes.POINTER(DecodeIO) * 4)()
+    for kind, io in ios.items():
+        arr[kind] = ctypes.pointer(io)
+    ws = _p(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().mixer_decode_step_batch(plan.handle, layer, ctypes.cast(arr, _vp),
+                                       state_cache.handle if state_cache else None,
+                                       kv_cache.handle if kv_cache else None, ws, ws_bytes,
+                                       _stream(stream))
+    _check("mixer_decode_step_batch", st)
 
 
 def hmd_device_errors(clear=True, stream=None) -> int:

@@ -55,6 +55,7 @@ struct SplitParams {
     __nv_bfloat16 *k_pool, *v_pool;
     const int32_t *page_table;
     const int32_t *seq_lens;
+    const int32_t *rows;  // launch row r runs batch row rows[r] (NULL: r itself)
     float *ws_ml;   // [B*nq*Hq][n_splits][2]: running max (log2 domain), sum of exponentials
     float *ws_acc;  // [B*nq*Hq][n_splits][D]
     int B, Hq, Hkv, group, nq, n_pages, max_pages, window, swa, ring_pages;
@@ -80,7 +81,7 @@ constexpr int smem_bytes() {
 
 // Work item i of the split-K plan: sequence b, kv-head g, key range `split` of that sequence.
 struct Item {
-    int b, g, split, L, lo, last_page, t_begin, n_tiles;
+    int r, b, g, split, L, lo, last_page, t_begin, n_tiles;  // r: launch row, b: batch row
     bool bad_len;
 };
 
@@ -88,7 +89,8 @@ __device__ __forceinline__ Item item_info(const SplitParams &p, int i) {
     Item it;
     it.split = i % p.n_splits;
     it.g = (i / p.n_splits) % p.Hkv;
-    it.b = i / (p.n_splits * p.Hkv);
+    it.r = i / (p.n_splits * p.Hkv);
+    it.b = p.rows ? p.rows[it.r] : it.r;
     it.L = p.seq_lens[it.b];
     it.bad_len = it.L < p.nq || it.L > p.max_seq_len;
     // the earliest key any row reads: that of the first new token, at position L - nq
@@ -390,7 +392,7 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             }
         }
         const int ti = r / G;  // new token ti, query head g * G + (r - ti * G)
-        const size_t row = (((size_t)it.b * p.nq + ti) * p.Hq + it.g * G + (r - ti * G)) * p.n_splits + it.split;
+        const size_t row = (((size_t)it.r * p.nq + ti) * p.Hq + it.g * G + (r - ti * G)) * p.n_splits + it.split;
         p.ws_acc[row * D + dim] = acc;
         if (dim == 0) {
             p.ws_ml[row * 2] = M;
@@ -401,11 +403,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
 template <int D>
 __global__ void __launch_bounds__(D) attn_combine_kernel(const float *ws_ml, const float *ws_acc,
-                                                         int n_splits, __nv_bfloat16 *o) {
-    const size_t bh = blockIdx.x;
+                                                         int n_splits, __nv_bfloat16 *o,
+                                                         const int32_t *rows, int per_row) {
+    const size_t bh = blockIdx.x;  // query row of the launch: (launch row, token, head)
     const int dim = threadIdx.x;
     griddep_launch_dependents();
     griddep_wait();  // the partials are the split kernel's output
+    const size_t ob = rows ? (size_t)rows[bh / per_row] * per_row + bh % per_row : bh;
     const float *ml = ws_ml + bh * n_splits * 2;
     float M = -INFINITY;
     for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[2 * s]);
@@ -417,7 +421,7 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const float *ws_ml, con
             den += f * ml[2 * s + 1];
         }
     }
-    o[bh * D + dim] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+    o[ob * D + dim] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
 }
 
 // ---- host side --------------------------------------------------------------------------
@@ -479,7 +483,9 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     p.v_pool = static_cast<__nv_bfloat16 *>(a.v_pool);
     p.page_table = a.page_table;
     p.seq_lens = a.seq_lens;
-    const size_t rows = (size_t)a.B * a.nq * a.Hq * plan.n_splits;
+    p.rows = a.rows;
+    const int n_run = a.rows ? a.n_rows : a.B;  // batch rows this launch runs
+    const size_t rows = (size_t)n_run * a.nq * a.Hq * plan.n_splits;
     p.ws_ml = static_cast<float *>(a.workspace);
     p.ws_acc = p.ws_ml + ((rows * 2 + 3) & ~static_cast<size_t>(3));
     p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.group = group; p.nq = a.nq;
@@ -492,9 +498,9 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     cudaError_t e = launch_pdl(attn_split_kernel<D>, dim3((unsigned)plan.n_ctas), dim3(kThreads),
                                smem, s, tmk, tmv, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(a.B * a.nq * a.Hq)), dim3(D), 0, s,
+    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(n_run * a.nq * a.Hq)), dim3(D), 0, s,
                       (const float *)p.ws_ml, (const float *)p.ws_acc, plan.n_splits,
-                      static_cast<__nv_bfloat16 *>(a.o));
+                      static_cast<__nv_bfloat16 *>(a.o), a.rows, a.nq * a.Hq);
 }
 
 // SMs of the current device (148 when no device can be queried).
@@ -553,8 +559,8 @@ AttnPlan attn_decode_plan(bool swa, int window, int B, int Hq, int Hkv, int d, i
 }
 
 cudaError_t launch_attn_decode(const AttnDecodeArgs &a, cudaStream_t s) {
-    const AttnPlan plan = attn_decode_plan(a.swa, a.window, a.B, a.Hq, a.Hkv, a.d, a.page_tokens,
-                                           a.max_seq_len, a.nq);
+    const AttnPlan plan = attn_decode_plan(a.swa, a.window, a.rows ? a.n_rows : a.B, a.Hq, a.Hkv,
+                                           a.d, a.page_tokens, a.max_seq_len, a.nq);
     if (a.d == 128) return launch_d<128>(a, plan, s);
     if (a.d == 64) return launch_d<64>(a, plan, s);
     return cudaErrorInvalidValue;

@@ -55,8 +55,8 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     __shared__ int s_ok;
     const int slice = blockIdx.x % n_slices;
     const int bh = blockIdx.x / n_slices;
-    const int b = bh / a.H;
-    const int h = bh - b * a.H;
+    const int ri = bh / a.H;  // row of the launch: sequence ri, or rows[ri] for a sub-batch
+    const int h = bh - ri * a.H;
     const int tid = threadIdx.x;
     const int ct = tid % kColThreads;
     const int rt = tid / kColThreads;
@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     if (tid == 0) prefetch_tmap(&tm);
     griddep_launch_dependents();
     griddep_wait();  // q, k, v, gates and the state may come from the previous kernel
+    const int b = a.rows ? a.rows[ri] : ri;
     if (tid == 0) {
         const int slot = a.slots ? a.slots[b] : b;
         const int dst = a.dst_slots ? a.dst_slots[b] : slot;
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
 template <int DK>
 cudaError_t launch_dk(const DeltaDecodeArgs &a, cudaStream_t s) {
     const int n_slices = (a.dv + kSliceCols - 1) / kSliceCols;
-    const long long grid = (long long)a.B * a.H * n_slices;
+    const long long grid = (long long)(a.rows ? a.n_rows : a.B) * a.H * n_slices;
     if (grid <= 0) return cudaSuccess;
     // the state cache as a 2-D tensor [n_slots*H*DK rows][dv] fp32, read in 32-column boxes
     CUtensorMap tm;

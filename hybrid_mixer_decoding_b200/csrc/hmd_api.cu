@@ -23,6 +23,13 @@ struct hmd_state_cache {
     size_t layer_elems;
 };
 
+struct hmd_batch_plan {
+    int n_layers, B;
+    int32_t *rows_dev;             // [n_layers][B]: per layer, the rows of each kind in turn
+    std::vector<int32_t> rows;     // host copy
+    std::vector<int32_t> offsets;  // [n_layers][5]: kind k's rows are [offsets[k], offsets[k+1])
+};
+
 struct hmd_kv_cache {
     int n_layers, n_pools, n_pages, Hkv, d, page_tokens;
     std::vector<int32_t> layer_pool;
@@ -95,21 +102,38 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
 
 // ---- delta-rule mixers -------------------------------------------------------------------
 
-hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk, int dv,
-                                  hmd_dtype_t dtype, const void *q, const void *k, const void *v,
-                                  const float *beta, const float *log_gate, float *state,
-                                  int n_slots, const int32_t *slots, const int32_t *dst_slots,
-                                  void *o, float scale, hmd_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// delta_rule_decode_to over the batch rows `rows` (device, n_rows; NULL: every row of B).
+hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
+                       const void *q, const void *k, const void *v, const float *beta,
+                       const float *log_gate, float *state, int n_slots, const int32_t *slots,
+                       const int32_t *dst_slots, void *o, float scale, const int32_t *rows,
+                       int n_rows, hmd_stream_t stream) {
     const hmd_status_t st = check_delta_decode(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate,
                                                state, n_slots, o);
     if (st != HMD_OK) return fail(st);
-    if (B == 0) return HMD_OK;
+    if (B == 0 || (rows && n_rows == 0)) return HMD_OK;
     if (!slots && n_slots < B) return fail(HMD_ERR_SHAPE);
     hmd::DeltaDecodeArgs a{};
     a.kind = kind; a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.bf16 = dtype == HMD_BF16;
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
     a.n_slots = n_slots; a.slots = slots; a.dst_slots = dst_slots; a.o = o; a.scale = scale;
+    a.rows = rows; a.n_rows = n_rows;
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk, int dv,
+                                  hmd_dtype_t dtype, const void *q, const void *k, const void *v,
+                                  const float *beta, const float *log_gate, float *state,
+                                  int n_slots, const int32_t *slots, const int32_t *dst_slots,
+                                  void *o, float scale, hmd_stream_t stream) {
+    return delta_run(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate, state, n_slots, slots,
+                     dst_slots, o, scale, nullptr, 0, stream);
 }
 
 hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
@@ -288,12 +312,16 @@ size_t attn_decode_workspace_size(hmd_kind_t kind, int window, int B, int Hq, in
     return attn_verify_workspace_size(kind, window, 1, B, Hq, Hkv, d, page_tokens, max_seq_len);
 }
 
-hmd_status_t attn_verify(hmd_kind_t kind, int window, int ring_pages, int n_q, int B, int Hq,
-                         int Hkv, int d, int page_tokens, const void *q, const void *new_k,
-                         const void *new_v, void *k_pool, void *v_pool, int n_pages,
-                         const int32_t *page_table, int max_pages, const int32_t *seq_lens,
-                         int max_seq_len, void *o, void *workspace, size_t ws_bytes,
-                         hmd_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// attn_verify over the batch rows `rows` (device, n_rows of them; NULL: every row of B).
+hmd_status_t attn_run(hmd_kind_t kind, int window, int ring_pages, int n_q, int B, int Hq,
+                      int Hkv, int d, int page_tokens, const void *q, const void *new_k,
+                      const void *new_v, void *k_pool, void *v_pool, int n_pages,
+                      const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                      int max_seq_len, void *o, void *workspace, size_t ws_bytes,
+                      const int32_t *rows, int n_rows, hmd_stream_t stream) {
     if (kind != HMD_FA && kind != HMD_SWA) return fail(HMD_ERR_ARG);
     if (kind == HMD_SWA && window < 1) return fail(HMD_ERR_ARG);
     if (B < 0 || n_q < 1 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
@@ -318,17 +346,32 @@ hmd_status_t attn_verify(hmd_kind_t kind, int window, int ring_pages, int n_q, i
     if (!aligned16(q) || !aligned16(new_k) || !aligned16(new_v) || !aligned16(k_pool) ||
         !aligned16(v_pool) || !aligned16(workspace))
         return fail(HMD_ERR_ARG);
-    const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, B, Hq, Hkv, d,
-                                                   page_tokens, max_seq_len, n_q);
+    const hmd::AttnPlan pl = hmd::attn_decode_plan(kind == HMD_SWA, window, rows ? n_rows : B, Hq,
+                                                   Hkv, d, page_tokens, max_seq_len, n_q);
     if (ws_bytes < pl.ws_bytes) return fail(HMD_ERR_SHAPE);
     hmd::AttnDecodeArgs a{};
     a.swa = kind == HMD_SWA; a.window = window; a.ring_pages = ring_pages; a.nq = n_q;
+    a.rows = rows; a.n_rows = n_rows;
     a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
     a.page_tokens = page_tokens; a.q = q; a.new_k = new_k; a.new_v = new_v;
     a.k_pool = k_pool; a.v_pool = v_pool; a.n_pages = n_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seq_lens = seq_lens; a.max_seq_len = max_seq_len; a.o = o;
     a.workspace = workspace; a.ws_bytes = ws_bytes;
     return from_cuda(hmd::launch_attn_decode(a, as_stream(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+hmd_status_t attn_verify(hmd_kind_t kind, int window, int ring_pages, int n_q, int B, int Hq,
+                         int Hkv, int d, int page_tokens, const void *q, const void *new_k,
+                         const void *new_v, void *k_pool, void *v_pool, int n_pages,
+                         const int32_t *page_table, int max_pages, const int32_t *seq_lens,
+                         int max_seq_len, void *o, void *workspace, size_t ws_bytes,
+                         hmd_stream_t stream) {
+    return attn_run(kind, window, ring_pages, n_q, B, Hq, Hkv, d, page_tokens, q, new_k, new_v,
+                    k_pool, v_pool, n_pages, page_table, max_pages, seq_lens, max_seq_len, o,
+                    workspace, ws_bytes, nullptr, 0, stream);
 }
 
 hmd_status_t attn_decode(hmd_kind_t kind, int window, int B, int Hq, int Hkv, int d,
@@ -498,6 +541,141 @@ hmd_status_t mixer_decode_step(const int8_t *placement, int n_layers, int layer,
         default:
             return fail(HMD_ERR_ARG);
     }
+}
+
+// ---- mixed placements in one batch -------------------------------------------------------
+
+hmd_status_t hmd_group_sequences(int n_layers, int n_placements, const int8_t *placements, int B,
+                                 const int32_t *seq_placement, int32_t *rows, int32_t *offsets) {
+    if (!placements || !seq_placement || !rows || !offsets || n_layers < 1 || n_placements < 1 ||
+        B < 1)
+        return fail(HMD_ERR_ARG);
+    for (int p = 0; p < n_placements * n_layers; ++p)
+        if (placements[p] < HMD_FA || placements[p] > HMD_GDN) return fail(HMD_ERR_ARG);
+    for (int b = 0; b < B; ++b)
+        if (seq_placement[b] < 0 || seq_placement[b] >= n_placements) return fail(HMD_ERR_ARG);
+    for (int l = 0; l < n_layers; ++l) {
+        int32_t *r = rows + (size_t)l * B;
+        int32_t *off = offsets + (size_t)l * 5;
+        int n = 0;
+        for (int kind = HMD_FA; kind <= HMD_GDN; ++kind) {
+            off[kind] = n;
+            for (int b = 0; b < B; ++b)
+                if (placements[(size_t)seq_placement[b] * n_layers + l] == kind) r[n++] = b;
+        }
+        off[4] = n;
+    }
+    return HMD_OK;
+}
+
+hmd_status_t batch_plan_create(int n_layers, int n_placements, const int8_t *placements, int B,
+                               const int32_t *seq_placement, hmd_stream_t stream,
+                               hmd_batch_plan_t **out) {
+    if (!out) return fail(HMD_ERR_ARG);
+    *out = nullptr;
+    std::vector<int32_t> rows((size_t)n_layers * (B > 0 ? B : 0)), offs((size_t)n_layers * 5);
+    const hmd_status_t st = hmd_group_sequences(n_layers, n_placements, placements, B,
+                                                seq_placement, rows.data(), offs.data());
+    if (st != HMD_OK) return st;
+    void *dev = nullptr;
+    if (cudaMallocAsync(&dev, rows.size() * sizeof(int32_t), as_stream(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HMD_ERR_OOM);
+    }
+    // pageable source: the call returns once the host buffer has been staged
+    if (cudaMemcpyAsync(dev, rows.data(), rows.size() * sizeof(int32_t), cudaMemcpyHostToDevice,
+                        as_stream(stream)) != cudaSuccess) {
+        cudaFreeAsync(dev, as_stream(stream));
+        return fail(HMD_ERR_CUDA);
+    }
+    auto *pl = new (std::nothrow) hmd_batch_plan;
+    if (!pl) {
+        cudaFreeAsync(dev, as_stream(stream));
+        return fail(HMD_ERR_OOM);
+    }
+    pl->n_layers = n_layers;
+    pl->B = B;
+    pl->rows_dev = static_cast<int32_t *>(dev);
+    pl->rows = std::move(rows);
+    pl->offsets = std::move(offs);
+    *out = pl;
+    return HMD_OK;
+}
+
+hmd_status_t batch_plan_free(hmd_batch_plan_t *plan, hmd_stream_t stream) {
+    if (!plan) return HMD_OK;
+    const cudaError_t e = cudaFreeAsync(plan->rows_dev, as_stream(stream));
+    delete plan;
+    return e == cudaSuccess ? HMD_OK : fail(HMD_ERR_CUDA);
+}
+
+hmd_status_t batch_plan_group(const hmd_batch_plan_t *plan, int layer, hmd_kind_t kind,
+                              int *count, const int32_t **rows_host) {
+    if (!plan || !count || layer < 0 || layer >= plan->n_layers || kind < HMD_FA ||
+        kind > HMD_GDN)
+        return fail(HMD_ERR_ARG);
+    const int32_t *off = plan->offsets.data() + (size_t)layer * 5;
+    *count = off[kind + 1] - off[kind];
+    if (rows_host) *rows_host = plan->rows.data() + (size_t)layer * plan->B + off[kind];
+    return HMD_OK;
+}
+
+size_t batch_plan_workspace_size(const hmd_batch_plan_t *plan, int window, int Hq, int Hkv, int d,
+                                 int page_tokens, int max_seq_len) {
+    size_t best = 16;
+    if (!plan) return best;
+    for (int l = 0; l < plan->n_layers; ++l) {
+        const int32_t *off = plan->offsets.data() + (size_t)l * 5;
+        for (int kind = HMD_FA; kind <= HMD_SWA; ++kind) {
+            const int n = off[kind + 1] - off[kind];
+            if (n > 0)
+                best = std::max(best, attn_verify_workspace_size(static_cast<hmd_kind_t>(kind),
+                                                                 window, 1, n, Hq, Hkv, d,
+                                                                 page_tokens, max_seq_len));
+        }
+    }
+    return best;
+}
+
+hmd_status_t mixer_decode_step_batch(const hmd_batch_plan_t *plan, int layer,
+                                     const hmd_decode_io_t *const *io, hmd_state_cache_t *sc,
+                                     hmd_kv_cache_t *kc, void *workspace, size_t ws_bytes,
+                                     hmd_stream_t stream) {
+    if (!plan || !io || layer < 0 || layer >= plan->n_layers) return fail(HMD_ERR_ARG);
+    const int32_t *off = plan->offsets.data() + (size_t)layer * 5;
+    const int32_t *rows = plan->rows_dev + (size_t)layer * plan->B;
+    for (int kind = HMD_FA; kind <= HMD_GDN; ++kind) {
+        const int n = off[kind + 1] - off[kind];
+        if (n == 0) continue;
+        const hmd_decode_io_t *x = io[kind];
+        if (!x) return fail(HMD_ERR_ARG);
+        if (x->B != plan->B) return fail(HMD_ERR_SHAPE);
+        hmd_status_t st;
+        if (kind == HMD_GDN || kind == HMD_KDA) {
+            if (!sc || layer >= sc->n_layers) return fail(HMD_ERR_ARG);
+            if (x->H != sc->H || x->d != sc->dk || x->d != sc->dv) return fail(HMD_ERR_SHAPE);
+            if (!x->slots && x->B > sc->slots) return fail(HMD_ERR_SHAPE);
+            float *state = sc->base + sc->layer_elems * layer;
+            const float *lg = kind == HMD_GDN ? x->log_gate_scalar : x->log_gate_channel;
+            st = delta_run(static_cast<hmd_kind_t>(kind), x->B, x->H, x->d, x->d, x->dtype, x->q,
+                           x->k, x->v, x->beta, lg, state, sc->slots, x->slots, nullptr, x->o,
+                           x->scale, rows + off[kind], n, stream);
+        } else {
+            if (!kc || layer >= kc->n_layers || kc->layer_pool[layer] < 0) return fail(HMD_ERR_ARG);
+            if (x->dtype != HMD_BF16) return fail(HMD_ERR_DTYPE);
+            if (x->Hkv != kc->Hkv || x->d != kc->d) return fail(HMD_ERR_SHAPE);
+            const int p = kc->layer_pool[layer];
+            const int ring = kind == HMD_SWA && x->window >= 1
+                                 ? (x->window + kc->page_tokens - 1) / kc->page_tokens
+                                 : 0;
+            st = attn_run(static_cast<hmd_kind_t>(kind), x->window, ring, 1, x->B, x->H, x->Hkv,
+                          x->d, kc->page_tokens, x->q, x->k, x->v, kc->k_pools[p], kc->v_pools[p],
+                          kc->n_pages, x->page_table, x->max_pages, x->seq_lens, x->max_seq_len,
+                          x->o, workspace, ws_bytes, rows + off[kind], n, stream);
+        }
+        if (st != HMD_OK) return st;
+    }
+    return HMD_OK;
 }
 
 }  // extern "C"

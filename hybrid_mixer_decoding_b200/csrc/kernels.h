@@ -50,6 +50,8 @@ struct DeltaDecodeArgs {
     const int32_t *dst_slots;  // where the updated state goes (NULL: back to slots, in place)
     void *o;
     float scale;
+    const int32_t *rows = nullptr;  // batch rows to run (device, n_rows of them); NULL: all B
+    int n_rows = 0;
 };
 cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s);
 bool delta_decode_supported(int dk, int dv);
@@ -60,6 +62,8 @@ struct AttnDecodeArgs {
     int window;
     int ring_pages;  // SWA ring size in pages (>= ceil((window + nq - 1) / page_tokens))
     int nq = 1;      // new tokens per sequence (1: decode step; more: verification pass)
+    const int32_t *rows = nullptr;  // batch rows to run (device, n_rows of them); NULL: all B
+    int n_rows = 0;
     int B, Hq, Hkv, d, page_tokens;
     const void *q, *new_k, *new_v;
     void *k_pool, *v_pool;

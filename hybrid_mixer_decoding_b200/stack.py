@@ -54,6 +54,7 @@ class MixerStack:
         that many independent sets of per-layer input/output buffers (same initial values), so
         a caller can copy the next step's inputs into one set while a step runs on another."""
         self.placements = {k: np.asarray(v, dtype=np.int8) for k, v in placements.items()}
+        self.names = list(self.placements)
         self.n_layers = len(next(iter(self.placements.values())))
         assert all(len(p) == self.n_layers for p in self.placements.values())
         self.shape = s = shape
@@ -213,19 +214,39 @@ class MixerStack:
             if ev:
                 ev[1].record()
 
-    def capture(self, name: str, warmup: int = 2) -> "torch.cuda.CUDAGraph":
-        """Capture one step of placement `name` into a CUDA graph (the library's calls allocate
-        nothing and never synchronise, so the whole 48-layer step is one graph launch)."""
+    def batch_plan(self, seq_placement) -> "L.BatchPlan":
+        """A mixed-batch plan: sequence b follows placement names[seq_placement[b]] (names in
+        the order of self.names). Grows the attention workspace to what the plan needs."""
+        pl = np.stack([self.placements[n] for n in self.names])
+        plan = L.BatchPlan(pl, seq_placement)
+        s = self.shape
+        need = plan.workspace_size(s.window, s.H, s.Hkv, s.d, PAGE, s.ctx)
+        if need > self.ws.numel():
+            self.ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        return plan
+
+    def step_batch(self, plan: "L.BatchPlan", io_set: int = 0) -> None:
+        """One decode token for every sequence of a mixed batch: layer by layer, each mixer
+        runs over the sequences whose placement picks it there (mixer_decode_step_batch)."""
+        ios = self.io_sets[io_set]
+        for l in range(self.n_layers):
+            L.mixer_decode_step_batch(plan, l, ios[l], self.state, self.kv_for(l), self.ws)
+
+    def capture(self, name, warmup: int = 2) -> "torch.cuda.CUDAGraph":
+        """Capture one step into a CUDA graph (the library's calls allocate nothing and never
+        synchronise, so the whole 48-layer step is one graph launch). name: a placement name,
+        or a callable that runs one step."""
+        fn = name if callable(name) else (lambda: self.step(name))
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for _ in range(warmup):
-                self.step(name)
+                fn()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            self.step(name)
+            fn()
         torch.cuda.synchronize()
         return g
 

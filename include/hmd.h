@@ -302,6 +302,53 @@ HMD_API hmd_status_t mixer_decode_step(const int8_t *placement, int n_layers, in
                                hmd_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* Mixed placements in one batch. Placements switch between requests ("Super Apriel: One       */
+/* Checkpoint, Many Speeds", abstract; gist.science summary, section 2d); here each sequence  */
+/* of a batch may follow its own placement. A batch plan groups, for every layer, the          */
+/* sequences by the mixer their placement picks there; one step of a layer then runs each     */
+/* mixer once over its group through a device list of batch rows (no inputs are gathered or  */
+/* copied: every kernel reads and writes row b of the full-batch tensors directly).            */
+/* ------------------------------------------------------------------------------------------ */
+typedef struct hmd_batch_plan hmd_batch_plan_t;
+
+/* The grouping itself (host only, no device work): placements is a host int8 array
+ * [n_placements][n_layers] of kinds, seq_placement [B] names each sequence's placement.
+ * Writes rows [n_layers][B] (per layer: the FA rows, then SWA, KDA, GDN, each in increasing b)
+ * and offsets [n_layers][5] (kind k's rows are rows[l][offsets[l][k] .. offsets[l][k+1])).
+ * HMD_ERR_ARG for a bad kind, placement index or null pointer.                               */
+HMD_API hmd_status_t hmd_group_sequences(int n_layers, int n_placements, const int8_t *placements,
+                                         int B, const int32_t *seq_placement, int32_t *rows,
+                                         int32_t *offsets);
+
+/* Build a plan (the grouping above, with the rows uploaded to the device on `stream`; the
+ * plan owns that memory until batch_plan_free). Build it outside any CUDA-graph capture; the
+ * steps that use it can be captured.                                                          */
+HMD_API hmd_status_t batch_plan_create(int n_layers, int n_placements, const int8_t *placements,
+                                       int B, const int32_t *seq_placement, hmd_stream_t stream,
+                                       hmd_batch_plan_t **out);
+HMD_API hmd_status_t batch_plan_free(hmd_batch_plan_t *plan, hmd_stream_t stream);
+/* Size of kind's group at a layer, and (optional) its rows on the host. */
+HMD_API hmd_status_t batch_plan_group(const hmd_batch_plan_t *plan, int layer, hmd_kind_t kind,
+                                      int *count, const int32_t **rows_host);
+/* Attention workspace for every step of this plan: the largest attn_decode_workspace_size over
+ * the plan's FA and SWA groups (the figure depends on the group size). */
+HMD_API size_t batch_plan_workspace_size(const hmd_batch_plan_t *plan, int window, int Hq,
+                                         int Hkv, int d, int page_tokens, int max_seq_len);
+
+/* One decode token for layer `layer` of a mixed batch: for each kind with a non-empty group,
+ * runs that mixer over the group's rows, with io[kind] (an array of 4 pointers indexed by
+ * hmd_kind_t; entries of absent kinds may be NULL) describing the full-batch tensors of that
+ * mixer (io[kind]->B must equal the plan's B). FA and SWA groups of a layer share its
+ * registered pool (SWA on the ring of ceil(window / page_tokens) pages). The groups run in
+ * turn on `stream`, sharing `workspace` (batch_plan_workspace_size bytes). Each sequence's
+ * results are those of mixer_decode_step under its own placement.                              */
+HMD_API hmd_status_t mixer_decode_step_batch(const hmd_batch_plan_t *plan, int layer,
+                                             const hmd_decode_io_t *const *io,
+                                             hmd_state_cache_t *state_cache,
+                                             hmd_kv_cache_t *kv_cache, void *workspace,
+                                             size_t ws_bytes, hmd_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Diagnostics.                                                                               */
 /* ------------------------------------------------------------------------------------------ */
 HMD_API const char *hmd_status_string(hmd_status_t status);
