@@ -503,6 +503,49 @@ int oracle_attn_verify(int kind, int window, int ring_pages, int n_q, int B, int
     return bad ? -1 : 0;
 }
 
+/* The input activations of the GDN / KDA mixers, from the projections' raw outputs (the
+ * pages name the mixers but not their parameterisation; this is the standard one of the
+ * published GDN and KDA layers):
+ *   q = q_raw / sqrt(sum(q_raw^2) + eps), k likewise (L2 over d_k, per token and head);
+ *   beta = 1 / (1 + exp(-beta_logit));
+ *   log_gate = -exp(A_log[h]) * softplus(gate_logit + dt_bias),  softplus(x) = log(1 + exp(x)),
+ *   with dt_bias [H] and gate_logit [N][H] for GDN, dt_bias [H][dk] and gate_logit [N][H][dk]
+ *   for KDA. N counts the token rows (B*T, or B for one decode step).
+ *   q_raw, k_raw [N][H][dk] in, q, k out; beta_logit [N][H] in, beta out; log_gate out.
+ * Returns 0, or -1 on bad arguments.                                                          */
+int oracle_delta_activations(int kind, int N, int H, int dk, double eps, const double *q_raw,
+                             const double *k_raw, const double *beta_logit,
+                             const double *gate_logit, const double *A_log, const double *dt_bias,
+                             double *q, double *k, double *beta, double *log_gate) {
+    if ((kind != OR_GDN && kind != OR_KDA) || N < 0 || H < 1 || dk < 1 || !(eps >= 0.0))
+        return -1;
+    for (long row = 0; row < (long)N * H; ++row) {
+        const int h = (int)(row % H);
+        double sq = 0.0, sk = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            sq += q_raw[row * dk + i] * q_raw[row * dk + i];
+            sk += k_raw[row * dk + i] * k_raw[row * dk + i];
+        }
+        const double nq = sqrt(sq + eps), nk = sqrt(sk + eps);
+        for (int i = 0; i < dk; ++i) {
+            q[row * dk + i] = q_raw[row * dk + i] / nq;
+            k[row * dk + i] = k_raw[row * dk + i] / nk;
+        }
+        beta[row] = 1.0 / (1.0 + exp(-beta_logit[row]));
+        const double decay_rate = exp(A_log[h]);
+        if (kind == OR_GDN) {
+            const double x = gate_logit[row] + dt_bias[h];
+            log_gate[row] = -decay_rate * log1p(exp(x));
+        } else {
+            for (int i = 0; i < dk; ++i) {
+                const double x = gate_logit[row * dk + i] + dt_bias[(size_t)h * dk + i];
+                log_gate[row * dk + i] = -decay_rate * log1p(exp(x));
+            }
+        }
+    }
+    return 0;
+}
+
 /* The oracle's thread count after set-up (for reporting). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -55,10 +55,11 @@ def _load():
         lib.oracle_kv_slot_ring.argtypes = [c_int, c_int, c_int, I32, c_int, c_int, I32, I32]
         lib.oracle_attn_verify.argtypes = ([c_int] * 10 + [D, D, D, U16, U16, I32, c_int, I32, D,
                                                            c_int])
+        lib.oracle_delta_activations.argtypes = [c_int] * 4 + [c_double] + [D] * 10
         lib.oracle_max_threads.argtypes = []
         for f in ("oracle_delta_recurrent", "oracle_delta_chunked", "oracle_kv_slot",
                   "oracle_attn_decode", "oracle_attn_prefill", "oracle_kv_slot_ring",
-                  "oracle_attn_verify", "oracle_max_threads"):
+                  "oracle_attn_verify", "oracle_delta_activations", "oracle_max_threads"):
             getattr(lib, f).restype = c_int
         _lib = lib
     return _lib
@@ -209,6 +210,27 @@ def attn_verify(kind, window, ring_pages, q_bits, new_k_bits, new_v_bits, k_pool
     if rc:
         raise ValueError("oracle_attn_verify failed (bad arguments or page id)")
     return o
+
+
+def delta_activations(kind, q_raw, k_raw, beta_logit, gate_logit, A_log, dt_bias, eps=1e-6):
+    """Input activations of GDN/KDA from raw projections (see oracle.c): q_raw, k_raw
+    [..., H, dk]; beta_logit [..., H]; gate_logit [..., H] (GDN) or [..., H, dk] (KDA);
+    A_log [H]; dt_bias [H] or [H, dk]. Returns (q, k, beta, log_gate) in float64, same shapes."""
+    qr, kr = _d(q_raw), _d(k_raw)
+    bl, gl, al, db = _d(beta_logit), _d(gate_logit), _d(A_log), _d(dt_bias)
+    H, dk = qr.shape[-2], qr.shape[-1]
+    N = qr.size // (H * dk)
+    q, k = np.zeros_like(qr), np.zeros_like(kr)
+    beta, lg = np.zeros_like(bl), np.zeros_like(gl)
+    rc = _load().oracle_delta_activations(kind, N, H, dk, float(eps), _p(qr, ctypes.c_double),
+                                          _p(kr, ctypes.c_double), _p(bl, ctypes.c_double),
+                                          _p(gl, ctypes.c_double), _p(al, ctypes.c_double),
+                                          _p(db, ctypes.c_double), _p(q, ctypes.c_double),
+                                          _p(k, ctypes.c_double), _p(beta, ctypes.c_double),
+                                          _p(lg, ctypes.c_double))
+    if rc:
+        raise ValueError("oracle_delta_activations: bad arguments")
+    return q, k, beta, lg
 
 
 def rel_err(x, ref) -> float:

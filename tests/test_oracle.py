@@ -542,3 +542,59 @@ def test_ring_slot_formula_cases(oracle_mod):
     for w in (1, 4, 5, 9):
         for p in range(40):
             assert O.kv_slot_ring(I.SWA, -(-w // 4), 4, row, p) == O.kv_slot(I.SWA, w, 4, row, p)
+
+
+# --------------------------------------------------------------------------------------------
+# input activations of the delta-rule mixers (raw projections -> q, k, beta, log-gates)
+# --------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_activations_closed_forms(oracle_mod, kind):
+    O = oracle_mod
+    rng = np.random.default_rng(80)
+    N, H, dk = 5, 3, 8
+    qr, kr = rng.standard_normal((N, H, dk)) * 3, rng.standard_normal((N, H, dk)) * 0.1
+    gshape = (N, H) if kind == I.GDN else (N, H, dk)
+    bshape = (H,) if kind == I.GDN else (H, dk)
+    q, k, beta, lg = O.delta_activations(kind, qr, kr, np.zeros((N, H)), np.zeros(gshape),
+                                         np.zeros(H), np.zeros(bshape), eps=0.0)
+    # eps = 0: unit L2 norm, direction kept
+    np.testing.assert_allclose(np.linalg.norm(q, axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(np.linalg.norm(k, axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(q * np.linalg.norm(qr, axis=-1, keepdims=True), qr, rtol=1e-13)
+    # sigmoid(0) = 1/2; A_log = 0, logit + bias = 0: log gate = -log 2
+    np.testing.assert_array_equal(beta, 0.5)
+    np.testing.assert_allclose(lg, -math.log(2.0), rtol=1e-15)
+    # a large logit: softplus(x) -> x, so log gate -> -exp(A_log) * (x + b)
+    A = np.log(np.arange(1, H + 1, dtype=np.float64))
+    big = np.full(gshape, 40.0)
+    bias = np.full(bshape, 2.0)
+    _, _, _, lg2 = O.delta_activations(kind, qr, kr, np.zeros((N, H)), big, A, bias)
+    expect = -np.exp(A)[:, None] * 42.0 if kind == I.KDA else -np.exp(A)[None, :] * 42.0
+    np.testing.assert_allclose(lg2, np.broadcast_to(expect, gshape), rtol=1e-14)
+    # eps > 0 shrinks the norm: |q| = sqrt(s / (s + eps))
+    q3, _, b3, _ = O.delta_activations(kind, qr, kr, np.full((N, H), 2.0), np.zeros(gshape),
+                                       np.zeros(H), np.zeros(bshape), eps=0.5)
+    s2 = (qr ** 2).sum(-1)
+    np.testing.assert_allclose(np.linalg.norm(q3, axis=-1), np.sqrt(s2 / (s2 + 0.5)), rtol=1e-13)
+    np.testing.assert_allclose(b3, 1.0 / (1.0 + math.exp(-2.0)), rtol=1e-15)
+
+
+def test_activations_gate_is_per_head_and_per_channel(oracle_mod):
+    """GDN: one gate per (token, head) with the head's A_log and dt_bias; KDA: one per channel
+    with the channel's dt_bias: permuting heads / channels of every input permutes the gate."""
+    O = oracle_mod
+    rng = np.random.default_rng(81)
+    N, H, dk = 4, 3, 6
+    qr, kr = rng.standard_normal((N, H, dk)), rng.standard_normal((N, H, dk))
+    bl = rng.standard_normal((N, H))
+    A = rng.standard_normal(H) * 0.3
+    for kind, gl, db in ((I.GDN, rng.standard_normal((N, H)), rng.standard_normal(H)),
+                         (I.KDA, rng.standard_normal((N, H, dk)), rng.standard_normal((H, dk)))):
+        _, _, _, lg = O.delta_activations(kind, qr, kr, bl, gl, A, db)
+        perm = np.array([2, 0, 1])
+        _, _, _, lgp = O.delta_activations(kind, qr[:, perm], kr[:, perm], bl[:, perm],
+                                           gl[:, perm], A[perm], db[perm])
+        np.testing.assert_allclose(lgp, lg[:, perm], rtol=1e-15)
+        # softplus > 0 and exp(A_log) > 0: every log gate is negative
+        assert (lg < 0).all()

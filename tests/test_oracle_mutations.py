@@ -48,6 +48,14 @@ MUTANTS = [
                                   "ring_idx = pos;")]),
     ("verify_first_new_key_from_pool", [("if (j >= first_new) {", "if (j > first_new) {")]),
     ("verify_rows_shifted", [("const int P_pos = first_new + i;", "const int P_pos = first_new + i - (i > 0);")]),
+    ("act_norm_without_sqrt", [("const double nq = sqrt(sq + eps), nk = sqrt(sk + eps);",
+                                "const double nq = sq + eps, nk = sqrt(sk + eps);")]),
+    ("act_sigmoid_sign", [("beta[row] = 1.0 / (1.0 + exp(-beta_logit[row]));",
+                           "beta[row] = 1.0 / (1.0 + exp(beta_logit[row]));")]),
+    ("act_gate_bias_dropped", [("const double x = gate_logit[row * dk + i] + dt_bias[(size_t)h * dk + i];",
+                                "const double x = gate_logit[row * dk + i];")]),
+    ("act_gate_rate_not_exponentiated", [("const double decay_rate = exp(A_log[h]);",
+                                          "const double decay_rate = A_log[h];")]),
 ]
 
 
