@@ -23,6 +23,11 @@ _lib = None
 _c_int, _c_float, _vp, _sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
 
+class DeltaAct(ctypes.Structure):
+    """hmd_delta_act_t: fused input activations of the delta-rule mixers."""
+    _fields_ = [("A_log", _vp), ("dt_bias", _vp), ("l2_eps", _c_float)]
+
+
 class DecodeIO(ctypes.Structure):
     """hmd_decode_io_t."""
     _fields_ = [("B", _c_int), ("H", _c_int), ("Hkv", _c_int), ("d", _c_int), ("dtype", _c_int),
@@ -41,6 +46,10 @@ _SIGS = {
                                   ctypes.POINTER(ctypes.POINTER(ctypes.c_int32))]),
     "batch_plan_workspace_size": (_sz, [_vp] + [_c_int] * 6),
     "mixer_decode_step_batch": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "delta_rule_decode_act": (_c_int, [_c_int] * 6 + [_vp] * 7 + [_c_int, _vp, _vp, _vp,
+                                                                 _c_float, _vp]),
+    "delta_rule_prefill_chunked_act": (_c_int, [_c_int] * 7 + [_vp] * 7 + [_c_int, _vp, _vp,
+                                                                          _c_int, _c_float, _vp]),
     "delta_rule_decode_to": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _vp, _c_float,
                                                                 _vp]),
     "delta_rule_prefill_chunked": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
@@ -152,6 +161,39 @@ def delta_rule_decode_to(kind, q, k, v, beta, log_gate, state, o, slots, dst_slo
                                     _p(beta), _p(log_gate), _p(state), state.shape[0], _p(slots),
                                     _p(dst_slots), _p(o), float(scale), _stream(stream))
     _check("delta_rule_decode_to", st)
+
+
+def delta_rule_decode_act(kind, q_raw, k_raw, v, beta_logit, gate_logit, A_log, dt_bias, state,
+                          o, slots=None, dst_slots=None, scale=1.0, eps=1e-6,
+                          stream=None) -> None:
+    """delta_rule_decode_to on raw projections, the input activations fused in (see
+    include/hmd.h): A_log [H]; dt_bias [H] (GDN) or [H, dk] (KDA), fp32 on the device."""
+    _contig(q_raw, k_raw, v, beta_logit, gate_logit, A_log, dt_bias, state, o, slots, dst_slots)
+    B, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    act = DeltaAct(A_log.data_ptr(), dt_bias.data_ptr(), float(eps))
+    st = lib().delta_rule_decode_act(kind, B, H, dk, dv, _dtype_code(q_raw), _p(q_raw), _p(k_raw),
+                                     _p(v), _p(beta_logit), _p(gate_logit), ctypes.byref(act),
+                                     _p(state), state.shape[0], _p(slots), _p(dst_slots), _p(o),
+                                     float(scale), _stream(stream))
+    _check("delta_rule_decode_act", st)
+
+
+def delta_rule_prefill_chunked_act(kind, q_raw, k_raw, v, beta_logit, gate_logit, A_log, dt_bias,
+                                   state, o, slots=None, chunk=64, scale=1.0, eps=1e-6,
+                                   stream=None) -> None:
+    """delta_rule_prefill_chunked on raw projections, the input activations fused into the
+    chunk-parallel pass (bf16, dk = dv = 128, chunk 64; see include/hmd.h)."""
+    _contig(q_raw, k_raw, v, beta_logit, gate_logit, A_log, dt_bias, state, o, slots)
+    B, T, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    act = DeltaAct(A_log.data_ptr(), dt_bias.data_ptr(), float(eps))
+    st = lib().delta_rule_prefill_chunked_act(kind, B, T, H, dk, dv, _dtype_code(q_raw),
+                                              _p(q_raw), _p(k_raw), _p(v), _p(beta_logit),
+                                              _p(gate_logit), ctypes.byref(act), _p(state),
+                                              state.shape[0], _p(slots), _p(o), int(chunk),
+                                              float(scale), _stream(stream))
+    _check("delta_rule_prefill_chunked_act", st)
 
 
 def delta_rule_prefill_chunked(kind, q, k, v, beta, log_gate, state, o, slots=None, chunk=64,

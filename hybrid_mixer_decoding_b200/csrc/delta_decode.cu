@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     __shared__ __align__(128) float S[DK][kSliceCols];
     __shared__ float sk[DK], sq[DK], sa[DK];
     __shared__ float red[kWarps][kColThreads][9];
+    __shared__ float nrm[kWarps][2];
     __shared__ __align__(8) uint64_t bar;
     __shared__ int s_ok;
     const int slice = blockIdx.x % n_slices;
@@ -83,22 +84,59 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
         }
     }
     const size_t tok = (size_t)b * a.H + h;
+    const bool fused = a.act.A_log != nullptr;  // raw projections: activate them here
+    const float rate = fused ? expf(a.act.A_log[h]) : 0.f;
     if (a.kind == HMD_GDN) {
-        const float g = expf(a.log_gate[tok]);
+        float lg = a.log_gate[tok];
+        if (fused) lg = -rate * hmd_softplus(lg + a.act.dt_bias[h]);
+        const float g = expf(lg);
         for (int i = tid; i < DK; i += kThreads) sa[i] = g;
     } else {
-        for (int i = tid; i < DK; i += kThreads) sa[i] = expf(a.log_gate[tok * DK + i]);
+        for (int i = tid; i < DK; i += kThreads) {
+            float lg = a.log_gate[tok * DK + i];
+            if (fused) lg = -rate * hmd_softplus(lg + a.act.dt_bias[(size_t)h * DK + i]);
+            sa[i] = expf(lg);
+        }
     }
+    float ssk = 0.f, ssq = 0.f;
     for (int i = tid; i < DK; i += kThreads) {
-        sk[i] = act<BF16>(a.k, tok * DK + i);
-        sq[i] = act<BF16>(a.q, tok * DK + i);
+        const float kv = act<BF16>(a.k, tok * DK + i), qv = act<BF16>(a.q, tok * DK + i);
+        sk[i] = kv;
+        sq[i] = qv;
+        ssk += kv * kv;
+        ssq += qv * qv;
     }
     float vv[4] = {0.f, 0.f, 0.f, 0.f};
     if (active) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) vv[c] = act<BF16>(a.v, tok * a.dv + col + c);
     }
-    const float beta = a.beta[tok];
+    float beta = a.beta[tok];
+    if (fused) {
+        beta = 1.f / (1.f + expf(-beta));
+        // L2 norms of k and q over d_k: warp sums, then the kWarps partials
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            ssk += __shfl_xor_sync(0xffffffffu, ssk, off);
+            ssq += __shfl_xor_sync(0xffffffffu, ssq, off);
+        }
+        if ((tid & 31) == 0) {
+            nrm[tid >> 5][0] = ssk;
+            nrm[tid >> 5][1] = ssq;
+        }
+        __syncthreads();
+        float tk = 0.f, tq = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            tk += nrm[w][0];
+            tq += nrm[w][1];
+        }
+        const float fk = 1.f / sqrtf(tk + a.act.eps), fq = 1.f / sqrtf(tq + a.act.eps);
+        for (int i = tid; i < DK; i += kThreads) {
+            sk[i] *= fk;
+            sq[i] *= fq;
+        }
+    }
     __syncthreads();
     if (!s_ok) return;
     if (!mbar_wait_bounded(smem_u32(&bar), 0)) {

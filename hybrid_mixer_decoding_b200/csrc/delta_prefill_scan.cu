@@ -256,11 +256,16 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             for (int j = 0; j < 4; ++j) tma_load_4d(sb + A_G + j * 8192, &tmg, bar_in, j * 32, h, t0, b);
         }
     }
+    const bool fused = a.act.A_log != nullptr;  // raw projections: activate them here
+    const float rate = fused ? expf(a.act.A_log[h]) : 0.f;
     if (tid < kC) {
         const size_t tok = ((size_t)b * T + t0 + tid) * a.H + h;
-        sbeta[tid] = tid < n ? a.beta[tok] : 0.f;
+        float bt = tid < n ? a.beta[tok] : 0.f;
+        if (fused && tid < n) bt = 1.f / (1.f + expf(-bt));
+        sbeta[tid] = bt;
         if constexpr (!KDA) {
             float x = tid < n ? a.log_gate[tok] : 0.f;
+            if (fused && tid < n) x = -rate * hmd_softplus(x + a.act.dt_bias[h]);
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, off);
@@ -280,10 +285,13 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     if constexpr (KDA) {
         const int i = tid & (kD - 1), qr = tid >> 7;
         float *gcol = Gs + gidx(0, i);
+        const float bias = fused ? a.act.dt_bias[(size_t)h * kD + i] : 0.f;
         float run = 0.f;
 #pragma unroll
         for (int r = RPQ * qr; r < RPQ * qr + RPQ; ++r) {
-            run += gcol[r * 32];
+            float x = gcol[r * 32];
+            if (fused) x = r < n ? -rate * hmd_softplus(x + bias) : 0.f;
+            run += x;
             gcol[r * 32] = run;
         }
         qoff[qr * kD + i] = run;
@@ -330,13 +338,30 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             }
             const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w};
             const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+            float fq = 1.f, fk = 1.f;  // L2 normalisation of the row (fused activations)
+            if (fused) {
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    sq += bf16_lo(qw[e]) * bf16_lo(qw[e]) + bf16_hi(qw[e]) * bf16_hi(qw[e]);
+                    sk += bf16_lo(kw[e]) * bf16_lo(kw[e]) + bf16_hi(kw[e]) * bf16_hi(kw[e]);
+                }
+                // the row's 16 chunks of 8 channels sit in 16 consecutive lanes
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                }
+                fq = 1.f / sqrtf(sq + a.act.eps);
+                fk = 1.f / sqrtf(sk + a.act.eps);
+            }
             uint32_t kt[4], qt[4], kh[4], kcw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float ea = __expf(G[2 * e]), eb = __expf(G[2 * e + 1]);
                 const float ia = __expf(-G[2 * e]), ib = __expf(-G[2 * e + 1]);
-                const float ka = bf16_lo(kw[e]), kb = bf16_hi(kw[e]);
-                const float qa = bf16_lo(qw[e]), qb = bf16_hi(qw[e]);
+                const float ka = fk * bf16_lo(kw[e]), kb = fk * bf16_hi(kw[e]);
+                const float qa = fq * bf16_lo(qw[e]), qb = fq * bf16_hi(qw[e]);
                 kt[e] = pack_bf16x2(ka * ea, kb * eb);
                 qt[e] = pack_bf16x2(qa * ea, qb * eb);
                 kh[e] = pack_bf16x2(ka * ia, kb * ib);
@@ -736,7 +761,7 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
     PrefillScanArgs p;
     p.q = a.q; p.k = a.k; p.v = a.v; p.beta = a.beta; p.log_gate = a.log_gate;
     p.state = a.state; p.slots = a.slots; p.n_slots = a.n_slots; p.o = a.o;
-    p.B = a.B; p.T = a.T; p.H = a.H; p.scale = a.scale; p.ws = ws;
+    p.B = a.B; p.T = a.T; p.H = a.H; p.scale = a.scale; p.ws = ws; p.act = a.act;
     for (int cb = 0; cb < n_chunks; cb += seg) {
         p.chunk_begin = cb;
         p.n_seg = std::min(seg, n_chunks - cb);

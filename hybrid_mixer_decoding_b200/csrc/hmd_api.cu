@@ -110,7 +110,7 @@ hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_
                        const void *q, const void *k, const void *v, const float *beta,
                        const float *log_gate, float *state, int n_slots, const int32_t *slots,
                        const int32_t *dst_slots, void *o, float scale, const int32_t *rows,
-                       int n_rows, hmd_stream_t stream) {
+                       int n_rows, hmd_stream_t stream, const hmd_delta_act_t *act = nullptr) {
     const hmd_status_t st = check_delta_decode(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate,
                                                state, n_slots, o);
     if (st != HMD_OK) return fail(st);
@@ -121,6 +121,10 @@ hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_
     a.q = q; a.k = k; a.v = v; a.beta = beta; a.log_gate = log_gate; a.state = state;
     a.n_slots = n_slots; a.slots = slots; a.dst_slots = dst_slots; a.o = o; a.scale = scale;
     a.rows = rows; a.n_rows = n_rows;
+    if (act) {
+        if (!act->A_log || !act->dt_bias || !(act->l2_eps >= 0.f)) return fail(HMD_ERR_ARG);
+        a.act.A_log = act->A_log; a.act.dt_bias = act->dt_bias; a.act.eps = act->l2_eps;
+    }
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
 }
 }  // namespace
@@ -134,6 +138,18 @@ hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk, int dv,
                                   void *o, float scale, hmd_stream_t stream) {
     return delta_run(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate, state, n_slots, slots,
                      dst_slots, o, scale, nullptr, 0, stream);
+}
+
+hmd_status_t delta_rule_decode_act(hmd_kind_t kind, int B, int H, int dk, int dv,
+                                   hmd_dtype_t dtype, const void *q_raw, const void *k_raw,
+                                   const void *v, const float *beta_logit,
+                                   const float *gate_logit, const hmd_delta_act_t *act,
+                                   float *state, int n_slots, const int32_t *slots,
+                                   const int32_t *dst_slots, void *o, float scale,
+                                   hmd_stream_t stream) {
+    if (!act) return fail(HMD_ERR_ARG);
+    return delta_run(kind, B, H, dk, dv, dtype, q_raw, k_raw, v, beta_logit, gate_logit, state,
+                     n_slots, slots, dst_slots, o, scale, nullptr, 0, stream, act);
 }
 
 hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,
@@ -242,17 +258,29 @@ hmd_status_t delta_rule_prefill_chunked_ws(hmd_kind_t kind, int B, int T, int H,
     return from_cuda(hmd::launch_delta_prefill_scan(a, workspace, ws_bytes, as_stream(stream)));
 }
 
-hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
-                                        hmd_dtype_t dtype, const void *q, const void *k,
-                                        const void *v, const float *beta, const float *log_gate,
-                                        float *state, int n_slots, const int32_t *slots, void *o,
-                                        int chunk, float scale, hmd_stream_t stream) {
+}  // extern "C"
+
+namespace {
+hmd_status_t prefill_pooled(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                            hmd_dtype_t dtype, const void *q, const void *k, const void *v,
+                            const float *beta, const float *log_gate, float *state, int n_slots,
+                            const int32_t *slots, void *o, int chunk, float scale,
+                            const hmd_delta_act_t *act, hmd_stream_t stream) {
     const hmd_status_t st = check_prefill(kind, B, T, H, dk, dv, dtype, q, k, v, beta, log_gate,
                                           state, n_slots, slots, o, chunk);
     if (st != HMD_OK) return fail(st);
+    if (act) {
+        if (!act->A_log || !act->dt_bias || !(act->l2_eps >= 0.f)) return fail(HMD_ERR_ARG);
+        // the fused activations live in the tensor-core path's chunk-parallel pass
+        if (!hmd::delta_prefill_scan_supported(dk, dv, dtype == HMD_BF16, chunk))
+            return fail(HMD_ERR_UNSUPPORTED);
+    }
     if (B == 0 || T == 0) return HMD_OK;
-    const hmd::DeltaPrefillArgs a = prefill_args(kind, B, T, H, dk, dv, dtype, q, k, v, beta,
-                                                 log_gate, state, n_slots, slots, o, chunk, scale);
+    hmd::DeltaPrefillArgs a = prefill_args(kind, B, T, H, dk, dv, dtype, q, k, v, beta,
+                                           log_gate, state, n_slots, slots, o, chunk, scale);
+    if (act) {
+        a.act.A_log = act->A_log; a.act.dt_bias = act->dt_bias; a.act.eps = act->l2_eps;
+    }
     if (!hmd::delta_prefill_scan_supported(dk, dv, dtype == HMD_BF16, chunk))
         return from_cuda(hmd::launch_delta_prefill(a, as_stream(stream)));
     const size_t full = delta_rule_prefill_workspace_size(kind, B, T, H, dk, dv, dtype, chunk);
@@ -269,6 +297,30 @@ hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, in
     const cudaError_t f = cudaFreeAsync(ws, s);
     if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(f);
+}
+}  // namespace
+
+extern "C" {
+
+hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                        hmd_dtype_t dtype, const void *q, const void *k,
+                                        const void *v, const float *beta, const float *log_gate,
+                                        float *state, int n_slots, const int32_t *slots, void *o,
+                                        int chunk, float scale, hmd_stream_t stream) {
+    return prefill_pooled(kind, B, T, H, dk, dv, dtype, q, k, v, beta, log_gate, state, n_slots,
+                          slots, o, chunk, scale, nullptr, stream);
+}
+
+hmd_status_t delta_rule_prefill_chunked_act(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
+                                            hmd_dtype_t dtype, const void *q_raw,
+                                            const void *k_raw, const void *v,
+                                            const float *beta_logit, const float *gate_logit,
+                                            const hmd_delta_act_t *act, float *state,
+                                            int n_slots, const int32_t *slots, void *o, int chunk,
+                                            float scale, hmd_stream_t stream) {
+    if (!act) return fail(HMD_ERR_ARG);
+    return prefill_pooled(kind, B, T, H, dk, dv, dtype, q_raw, k_raw, v, beta_logit, gate_logit,
+                          state, n_slots, slots, o, chunk, scale, act, stream);
 }
 
 // ---- attention mixers --------------------------------------------------------------------

@@ -38,6 +38,26 @@ bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int hea
 bool make_tmap_bthd(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int B,
                     int T, int H, int d, int box_d, bool sw128);
 
+// Input activations of the delta-rule mixers, fused into their kernels when A_log is set: the
+// kernel then reads raw q, k (L2-normalised over d_k with eps), beta logits (sigmoid) and gate
+// logits (log-gate = -exp(A_log[h]) * softplus(logit + dt_bias), dt_bias [H] for GDN, [H][dk]
+// for KDA). A_log == nullptr: the inputs are already q, k, beta and log-gates.
+struct DeltaAct {
+    const float *A_log = nullptr;
+    const float *dt_bias = nullptr;
+    float eps = 0.f;
+};
+
+// softplus(x) = log(1 + e^x), from the definition: above 15 it is x + log(1 + e^-x) ~ x + e^-x;
+// below, with e = e^x, the series e - e^2/2 + e^3/3 - e^4/4 while e < 1/64 (next term e^5/5,
+// a relative 3e-8), else log(1 + e), where 1 + e keeps e to a relative 4e-6.
+__device__ __forceinline__ float hmd_softplus(float x) {
+    if (x > 15.f) return x + __expf(-x);
+    const float e = __expf(x);
+    if (e < 0.015625f) return e * (1.f - e * (0.5f - e * (1.f / 3.f - 0.25f * e)));
+    return __logf(1.f + e);
+}
+
 struct DeltaDecodeArgs {
     int kind;  // 2 = KDA (per-channel gate), 3 = GDN (scalar gate)
     int B, H, dk, dv;
@@ -52,6 +72,7 @@ struct DeltaDecodeArgs {
     float scale;
     const int32_t *rows = nullptr;  // batch rows to run (device, n_rows of them); NULL: all B
     int n_rows = 0;
+    DeltaAct act;
 };
 cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s);
 bool delta_decode_supported(int dk, int dv);
@@ -100,6 +121,7 @@ struct DeltaPrefillArgs {
     void *o;
     int chunk;
     float scale;
+    DeltaAct act;  // fused input activations (tensor-core path only)
 };
 cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s);
 bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk);
@@ -138,6 +160,7 @@ struct PrefillScanArgs {
     void *ws;         // records [B*H][n_seg][record bytes]
     int chunk_begin;  // first chunk of this segment
     int n_seg;        // chunks in this segment
+    DeltaAct act;     // fused input activations
 };
 bool delta_prefill_scan_supported(int dk, int dv, bool bf16, int chunk);
 size_t delta_prefill_scan_record_bytes();

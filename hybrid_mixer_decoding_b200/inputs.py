@@ -109,6 +109,45 @@ def delta_inputs(kind: int, B: int, T: int, H: int, dk: int, dv: int, dtype: str
 
 
 @dataclass
+class DeltaRawInputs:
+    """Raw projection outputs for the fused-activation entry points of GDN/KDA.
+
+    q_raw, k_raw [B,T,H,dk] ~ 2 N(0,1) (norms far from 1); v [B,T,H,dv] ~ N(0,1);
+    beta_logit [B,T,H] ~ N(0,1); gate_logit [B,T,H] (GDN) or [B,T,H,dk] (KDA) ~ N(0,1);
+    A_log [H] = log U(0.5, 2); dt_bias [H] (GDN) or [H,dk] (KDA) ~ U(-5, -3), so that the
+    per-token log-gates land near -0.02 as in the configured workloads; state0 [B,H,dk,dv].
+    bf16 values are bf16-representable fp32 (the raw q, k, v only).
+    """
+    kind: int
+    dtype: str
+    q_raw: np.ndarray
+    k_raw: np.ndarray
+    v: np.ndarray
+    beta_logit: np.ndarray
+    gate_logit: np.ndarray
+    A_log: np.ndarray
+    dt_bias: np.ndarray
+    state0: np.ndarray
+
+
+def delta_raw_inputs(kind: int, B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
+                     seed: int = 0) -> DeltaRawInputs:
+    assert kind in (KDA, GDN) and dtype in ("bf16", "f32")
+    g = rng(seed)
+    q = 2.0 * g.standard_normal((B, T, H, dk), dtype=np.float32)
+    k = 2.0 * g.standard_normal((B, T, H, dk), dtype=np.float32)
+    v = g.standard_normal((B, T, H, dv), dtype=np.float32)
+    bl = g.standard_normal((B, T, H), dtype=np.float32)
+    gl = g.standard_normal((B, T, H) if kind == GDN else (B, T, H, dk), dtype=np.float32)
+    A_log = np.log(g.uniform(0.5, 2.0, size=H)).astype(np.float32)
+    dt_bias = g.uniform(-5.0, -3.0, size=(H,) if kind == GDN else (H, dk)).astype(np.float32)
+    s0 = (g.standard_normal((B, H, dk, dv), dtype=np.float32) / np.float32(math.sqrt(dk)))
+    if dtype == "bf16":
+        q, k, v = bf16_round(q), bf16_round(k), bf16_round(v)
+    return DeltaRawInputs(kind, dtype, q, k, v, bl, gl, A_log, dt_bias, s0)
+
+
+@dataclass
 class AttnInputs:
     """Inputs of one FA or SWA decode step over a paged bf16 KV cache.
 

@@ -98,6 +98,30 @@ HMD_API hmd_status_t delta_rule_decode_to(hmd_kind_t kind, int B, int H, int dk,
                                           const int32_t *slots, const int32_t *dst_slots,
                                           void *o, float scale, hmd_stream_t stream);
 
+/* Input activations fused into the delta-rule kernels. The pages name GDN and KDA but not
+ * how their inputs are formed; this follows the published layers: from the projections' raw
+ * outputs, q and k are L2-normalised over d_k (x / sqrt(sum x^2 + l2_eps)), beta = sigmoid of
+ * its logit, and the log-gate = -exp(A_log[h]) * softplus(gate_logit + dt_bias) with
+ * softplus(x) = log(1 + e^x). A_log [H] fp32 (device); dt_bias [H] (GDN) or [H][dk] (KDA)
+ * fp32 (device).                                                                              */
+typedef struct {
+    const float *A_log;
+    const float *dt_bias;
+    float l2_eps;
+} hmd_delta_act_t;
+
+/* delta_rule_decode_to on raw projections: q_raw, k_raw as q, k; beta_logit as beta;
+ * gate_logit as log_gate (same shapes); activations as above, computed in fp32 inside the
+ * kernel. HMD_ERR_ARG for a null act, A_log or dt_bias, or a negative l2_eps.                 */
+HMD_API hmd_status_t delta_rule_decode_act(hmd_kind_t kind, int B, int H, int dk, int dv,
+                                           hmd_dtype_t dtype, const void *q_raw,
+                                           const void *k_raw, const void *v,
+                                           const float *beta_logit, const float *gate_logit,
+                                           const hmd_delta_act_t *act, float *state,
+                                           int n_slots, const int32_t *slots,
+                                           const int32_t *dst_slots, void *o, float scale,
+                                           hmd_stream_t stream);
+
 /* Chunked (WY / UT-transform) prefill over T tokens per sequence for one layer: the same
  * recurrence as delta_rule_decode applied to tokens 0..T-1 in order, computed chunk by chunk.
  *   q, k [B][T][H][dk]; v, o [B][T][H][dv] (dtype); beta [B][T][H] fp32;
@@ -125,6 +149,18 @@ HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, i
  * needs no scratch (the CUDA-core path) or the sizes are empty or invalid.                    */
 HMD_API size_t delta_rule_prefill_workspace_size(hmd_kind_t kind, int B, int T, int H, int dk,
                                                  int dv, hmd_dtype_t dtype, int chunk);
+
+/* delta_rule_prefill_chunked on raw projections (activations as for delta_rule_decode_act,
+ * fused into the chunk-parallel pass). Supported on the tensor-core path only: bf16 with
+ * dk = dv = 128 and chunk 64 (HMD_ERR_UNSUPPORTED otherwise).                                */
+HMD_API hmd_status_t delta_rule_prefill_chunked_act(hmd_kind_t kind, int B, int T, int H, int dk,
+                                                    int dv, hmd_dtype_t dtype, const void *q_raw,
+                                                    const void *k_raw, const void *v,
+                                                    const float *beta_logit,
+                                                    const float *gate_logit,
+                                                    const hmd_delta_act_t *act, float *state,
+                                                    int n_slots, const int32_t *slots, void *o,
+                                                    int chunk, float scale, hmd_stream_t stream);
 
 /* delta_rule_prefill_chunked with caller-owned scratch: `workspace` (device, 16-byte aligned)
  * of ws_bytes. Any size from one chunk's records for all B*H heads up works; with less than

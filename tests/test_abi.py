@@ -194,3 +194,23 @@ def test_attn_prefill_validation():
     assert _attn_prefill(kind=hmd.SWA, window=200, max_pages=3) == SHAPE  # ring of 4 pages
     assert _attn_prefill(ptr=None) == ARG
     assert _attn_prefill(T=0) == 0 and _attn_prefill(B=0) == 0
+
+
+def test_fused_activation_validation():
+    L = hmd.lib()
+    from hybrid_mixer_decoding_b200._lib import DeltaAct
+    good = DeltaAct(FAKE, FAKE, 1e-6)
+    dec = lambda act, B=2, dtype=hmd.BF16: L.delta_rule_decode_act(  # noqa: E731
+        hmd.GDN, B, 2, 64, 64, dtype, FAKE, FAKE, FAKE, FAKE, FAKE, act, FAKE, 4, None, None,
+        FAKE, 1.0, None)
+    assert dec(None) == ARG
+    assert dec(ctypes.byref(DeltaAct(None, FAKE, 1e-6))) == ARG
+    assert dec(ctypes.byref(DeltaAct(FAKE, None, 1e-6))) == ARG
+    assert dec(ctypes.byref(DeltaAct(FAKE, FAKE, -1.0))) == ARG
+    assert dec(ctypes.byref(good), B=0) == 0
+    pre = lambda act, dtype=hmd.BF16, dk=128: L.delta_rule_prefill_chunked_act(  # noqa: E731
+        hmd.KDA, 1, 64, 1, dk, dk, dtype, FAKE, FAKE, FAKE, FAKE, FAKE, act, FAKE, 1, None, FAKE,
+        64, 1.0, None)
+    assert pre(None) == ARG
+    assert pre(ctypes.byref(good), dtype=hmd.F32) == UNSUP   # fused only on the tensor-core path
+    assert pre(ctypes.byref(good), dk=64) == UNSUP
