@@ -17,11 +17,12 @@
 // memory in the 128-byte swizzled layout the tensor cores read; the CTA forms the gate factors,
 // then [Kt; Qt] Kh^T as ONE M = 128 tcgen05.mma product into TMEM (rows 0-63 give A, rows 64-127
 // give P), the blocked fp32 UT solve on the CUDA cores, and W^T, Ut^T as two M = 128 products
-// that read Kt and V MN-major. It writes one record per chunk: Qt, -W, Kc, P, Ut (bf16, in the
-// 128-byte XOR-swizzled tile layout pass B reads with ldmatrix) and e^{G_C} (fp32).
+// that read Kt and V MN-major. It writes one record per chunk: Qt, Kc, P, and -W^T, Ut^T (rows of
+// d_k / d_v, as the TMEM read-back delivers them), all bf16 in the 128-byte XOR-swizzled tile
+// layout pass B reads with ldmatrix, and e^{G_C} (fp32).
 // Pass B (prefill_scan_kernel, mma.sync m16n8k16): one CTA per (sequence, head, half of d_v)
-// walks the chunks in order. Each chunk's record arrives by one bulk copy into a 2-stage shared-memory ring while
-// the chunk before it computes; the state half lives in registers as MMA accumulator fragments.
+// walks the chunks in order. Each chunk's whole record arrives by one bulk copy into a 2-stage
+// shared-memory ring while the chunk before it computes; the state half lives in registers as MMA accumulator fragments.
 // Per chunk it does only the state-dependent products (U, O, state update): 7.3 MFLOP of the
 // chunk's 11.5 per head, split over two CTAs.
 #include <cuda_runtime.h>
@@ -46,12 +47,12 @@ constexpr int kDV = kD / kSplitV;      // 64 columns of d_v per pass-B CTA
 
 // ---- the per-chunk record (bytes) ----------------------------------------------------------
 constexpr uint32_t REC_QT = 0;         // Qt  bf16 [64][128], swizzled halves
-constexpr uint32_t REC_NW = 16384;     // -W  bf16 [64][128]
+constexpr uint32_t REC_NW = 16384;     // -W^T bf16 [128 d_k][64 tokens] (tile of 128 rows)
 constexpr uint32_t REC_KC = 32768;     // Kc  bf16 [64][128]
 constexpr uint32_t REC_P = 49152;      // P   bf16 [64][64]
 constexpr uint32_t REC_GAM = 57344;    // e^{G_C} fp32 [128]
-constexpr uint32_t REC_HEAD = 57856;   // bytes above, moved by one bulk copy
-constexpr uint32_t REC_UT = 57856;     // Ut  bf16 [64][128], swizzled halves
+constexpr uint32_t REC_HEAD = 57856;   // bytes above
+constexpr uint32_t REC_UT = 57856;     // Ut^T bf16 [128 d_v][64 tokens] (tile of 128 rows)
 constexpr uint32_t REC_BYTES = REC_UT + kC * kD * 2;  // 74240
 static_assert(REC_HEAD % 16 == 0 && REC_BYTES % 16 == 0, "bulk copies need 16-byte sizes");
 
@@ -62,17 +63,17 @@ constexpr uint32_t A_KQ = 0;           // [Kt; Qt], the K-major A operand of one
                                        //   (record layout) in the Kt rows; Kt is also read
                                        //   MN-major (halves 16 KiB apart)
 constexpr uint32_t A_KH = 32768;       // k, then Kh [64][128] (K-major B operand); then P, e^{G_C}
-constexpr uint32_t A_V = 49152;        // v [64][128] (MN-major A operand)
+constexpr uint32_t A_V = 49152;        // v [64][128] (MN-major A operand); at the end -W^T
 constexpr uint32_t A_G = 65536;        // KDA log-gates -> in-chunk prefix, fp32 [4][64][32]
 constexpr uint32_t A_AS = 65536;       // after the gate pass: A fp32 [64][68], then T bf16
 constexpr uint32_t A_XS = 82944;       // X fp32 [64][68]
 constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
-constexpr uint32_t A_UT = 65536;       // at the end: Ut bf16 (record layout, 16 KiB)
+constexpr uint32_t A_UT = 65536;       // at the end: Ut^T bf16 (record layout, 16 KiB)
 constexpr uint32_t A_SMALL = 104192;
 constexpr uint32_t S_BETA = 0, S_QOFF = 256, S_LGP = 1280, S_WSUM = 1536, S_EGC = 1552,
                    S_BAR = 2064, S_TMEM = 2080, S_SIZE = 2112;
 constexpr uint32_t A_SMEM = A_SMALL + S_SIZE + 1024;
-constexpr uint32_t A_T = A_AS;
+constexpr uint32_t A_T = A_KQ + 8192;  // T bf16 [64][64]: the Qt rows of the first half
 constexpr int AS_LD = 68;
 constexpr int YS_LD = 20;
 constexpr uint32_t kPrepTmemCols = 128;
@@ -84,7 +85,7 @@ static_assert(S_QOFF + (kPrepThreads / kD) * kD * 4 <= S_LGP, "gate part sums fi
 static_assert(S_BAR % 8 == 0 && S_TMEM + 4 <= S_SIZE, "small area");
 
 // ---- pass B shared memory ----------------------------------------------------------------
-constexpr uint32_t B_STAGE = 58368;        // one record head, padded to 1 KiB
+constexpr uint32_t B_STAGE = 74752;        // one whole record (one bulk copy), padded to 1 KiB
 constexpr uint32_t B_M = 2 * B_STAGE;      // M bf16 [128][64], two buffers (chunk parity)
 constexpr uint32_t B_U = B_M + 2 * 16384;  // U bf16 [64][64], two buffers
 constexpr uint32_t B_BAR = B_U + 2 * 8192;
@@ -116,7 +117,8 @@ constexpr int pow2_floor(int x) { return x >= 2 ? 2 * pow2_floor(x / 2) : 1; }
 // 4-column group) is shared by as many threads as the block has to spare (a power of two);
 // they split the sums and combine them by shuffles.
 template <int L>
-__device__ __forceinline__ void solve_level(const float *As, float *Xs, float *Ys, int tid) {
+__device__ __forceinline__ void solve_level(const float *As, float *Xs, float *Ys, int tid,
+                                            uint8_t *Tt, const float *sbeta) {
     constexpr int NB = 4 - L;                                  // blocks on this diagonal
     constexpr int TPI = pow2_floor(kPrepThreads / (NB * 64));  // threads per (block, row, group)
     constexpr int KPT = 16 * L / TPI;  // terms of Y per thread
@@ -161,9 +163,15 @@ __device__ __forceinline__ void solve_level(const float *As, float *Xs, float *Y
             acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
             acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
         }
-        if (part == 0)
+        if (part == 0) {
             *reinterpret_cast<float4 *>(Xs + (i * 16 + r) * AS_LD + j * 16 + cg * 4) =
                 make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            // the same four entries of T = X Diag(beta), bf16 (8 bytes of one 16-byte chunk)
+            const int s0 = j * 16 + cg * 4;
+            *reinterpret_cast<uint2 *>(Tt + toff(i * 16 + r, s0, 64)) =
+                make_uint2(pack_bf16x2(-acc.x * sbeta[s0], -acc.y * sbeta[s0 + 1]),
+                           pack_bf16x2(-acc.z * sbeta[s0 + 2], -acc.w * sbeta[s0 + 3]));
+        }
     }
     __syncthreads();
 }
@@ -439,10 +447,16 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         bulk_commit_group();
     }
 
-    // ---- X = (I + A)^-1 (16x16 blocks, fp32), T = X Diag(beta) ----------------------------
+    // ---- X = (I + A)^-1 (16x16 blocks, fp32) and, as its blocks appear, T = X Diag(beta)
+    //      (bf16 [r][s], the K-major B operand below) in the Qt slot, free once Qt's bulk store
+    //      has read it ------------------------------------------------------------------------
+    if (tid == 0) bulk_wait_group_read<1>();  // the Qt group; the P group may still be reading
+    __syncthreads();
+    uint8_t *Tt = sm + A_T;
     if (tid < 64) {  // diagonal blocks by forward substitution, one column per thread
         const int bi = tid >> 4, c0 = tid & 15;
         const float *ab = As + bi * 16 * AS_LD + bi * 16;
+        const float bc = sbeta[bi * 16 + c0];
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
@@ -451,20 +465,23 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             for (int s2 = 0; s2 < r; ++s2) acc += ab[r * AS_LD + s2] * x[s2];
             x[r] = r < c0 ? 0.f : (r == c0 ? 1.f : -acc);
             Xs[(bi * 16 + r) * AS_LD + bi * 16 + c0] = x[r];
+            *reinterpret_cast<__nv_bfloat16 *>(Tt + toff(bi * 16 + r, bi * 16 + c0, 64)) =
+                __float2bfloat16_rn(x[r] * bc);
+        }
+    } else {  // the blocks above the diagonal of T are zero: 6 blocks x 16 rows x 32 bytes
+        for (int idx = tid - 64; idx < 6 * 16 * 2; idx += NT - 64) {
+            const int blk = idx >> 5, rr = (idx >> 1) & 15, hh = idx & 1;
+            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);           // block row
+            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);  // block column > bi
+            *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + rr, bj * 16 + hh * 8, 64)) =
+                make_uint4(0, 0, 0, 0);
         }
     }
     __syncthreads();
-    solve_level<1>(As, Xs, Ys, tid);
-    solve_level<2>(As, Xs, Ys, tid);
-    solve_level<3>(As, Xs, Ys, tid);
-    // T overwrites A (no longer read): [r][s] bf16, the K-major B operand below
-    for (int idx = tid; idx < 64 * 32; idx += NT) {
-        const int r = idx >> 5, s0 = (idx & 31) * 2;
-        const float v0 = s0 <= r ? Xs[r * AS_LD + s0] * sbeta[s0] : 0.f;
-        const float v1 = s0 + 1 <= r ? Xs[r * AS_LD + s0 + 1] * sbeta[s0 + 1] : 0.f;
-        st_bf16x2(sm + A_T, toff(r, s0, 64), v0, v1);
-    }
-    fence_proxy_async_smem();
+    solve_level<1>(As, Xs, Ys, tid, Tt, sbeta);
+    solve_level<2>(As, Xs, Ys, tid, Tt, sbeta);
+    solve_level<3>(As, Xs, Ys, tid, Tt, sbeta);
+    fence_proxy_async_smem();  // T is read by the tensor cores
     __syncthreads();
 
     // ---- W^T = Kt^T T^T and Ut^T = V^T T^T: M = 128 (d), N = 64 (r), K = 64 (s), with Kt and V
@@ -487,28 +504,26 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
     tc_fence_after();
     {
-        const int quad = warp & 3, dd = 32 * quad + lane;  // this thread's row of d_k or d_v
+        // thread row dd of d_k (warps 0-3: -W^T, into the free V slot) or of d_v (warps 4-7:
+        // Ut^T); 32 token columns per TMEM load, stored as four 16-byte chunks of the row
+        const int quad = warp & 3, dd = 32 * quad + lane;
+        const bool w_side = warp < 4;
+        const float sgn = w_side ? -1.f : 1.f;
+        uint8_t *dst = sm + (w_side ? A_V : A_UT);
         uint32_t d[32];
-        if (warp < 4) {  // -W [r][d_k] bf16 (record layout) into the Kt rows of both halves
-            uint8_t *wb = sm + A_KQ + (dd >> 6) * 16384;
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 64 + 32 * hr, d);
-                tmem_wait_ld();
+        for (int hr = 0; hr < 2; ++hr) {
+            tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (w_side ? 64 : 0) + 32 * hr, d);
+            tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    *reinterpret_cast<__nv_bfloat16 *>(wb + toff(32 * hr + j, dd & 63, 64)) =
-                        __float2bfloat16_rn(-__uint_as_float(d[j]));
-            }
-        } else {  // Ut [r][d_v] bf16 (record layout)
+            for (int u = 0; u < 4; ++u) {
+                uint32_t w[4];
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * hr, d);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + A_UT + toff(32 * hr + j, dd, 64)) =
-                        __float2bfloat16_rn(__uint_as_float(d[j]));
+                for (int e = 0; e < 4; ++e)
+                    w[e] = pack_bf16x2(sgn * __uint_as_float(d[8 * u + 2 * e]),
+                                       sgn * __uint_as_float(d[8 * u + 2 * e + 1]));
+                *reinterpret_cast<uint4 *>(dst + toff(dd, 32 * hr + 8 * u, 128)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
     }
@@ -516,8 +531,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        bulk_store(rec + REC_NW, sb + A_KQ, 8192);
-        bulk_store(rec + REC_NW + 8192, sb + A_KQ + 16384, 8192);
+        bulk_store(rec + REC_NW, sb + A_V, 16384);
         bulk_store(rec + REC_UT, sb + A_UT, 16384);
         bulk_commit_group();
         bulk_wait_group_read0();  // shared memory must outlive the copies' reads
@@ -567,8 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
     __syncthreads();
     auto issue = [&](int c) {  // thread 0: chunk c's record head -> stage c & 1
         const uint32_t bar = smem_u32(&bars[c & 1]);
-        mbar_arrive_expect_tx(bar, REC_HEAD);
-        bulk_load(sb + (c & 1) * B_STAGE, record(a, bh, c), REC_HEAD, bar);
+        mbar_arrive_expect_tx(bar, REC_BYTES);
+        bulk_load(sb + (c & 1) * B_STAGE, record(a, bh, c), REC_BYTES, bar);
     };
     if (tid == 0) issue(0);
 
@@ -585,17 +599,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
     // U / O role: chunk rows 16*rt + g (+8), slice columns 32*chh + 8*j + 2*t4 (+1)
     const int rt = warp & 3, chh = warp >> 2;
     const int ur0 = 16 * rt + g, ur1 = ur0 + 8;
-    uint32_t un[4][2];  // Ut of the next chunk (bf16 pairs), prefetched
-    auto load_ut = [&](int c) {
-        const uint8_t *ut = record(a, bh, c) + REC_UT;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
-            un[j][0] = __ldg(reinterpret_cast<const unsigned int *>(ut + toff(ur0, cc, 64)));
-            un[j][1] = __ldg(reinterpret_cast<const unsigned int *>(ut + toff(ur1, cc, 64)));
-        }
-    };
-    load_ut(0);
 
     int aborted_at = -1;
     for (int c = 0; c < a.n_seg; ++c) {
@@ -631,16 +634,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
         float u[4][4], o[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            u[j][0] = bf16_lo(un[j][0]); u[j][1] = bf16_hi(un[j][0]);
-            u[j][2] = bf16_lo(un[j][1]); u[j][3] = bf16_hi(un[j][1]);
+            // Ut[token][cc], Ut[token][cc + 1] from rows cc, cc + 1 of the stage's Ut^T tile
+            const int cc = col0 + 32 * chh + 8 * j + 2 * t4;
+            const uint8_t *ut = sm + p * B_STAGE + REC_UT;
+            u[j][0] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ut + toff(cc, ur0, 128)));
+            u[j][1] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ut + toff(cc + 1, ur0, 128)));
+            u[j][2] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ut + toff(cc, ur1, 128)));
+            u[j][3] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ut + toff(cc + 1, ur1, 128)));
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[j][e] = 0.f;
         }
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
             uint32_t aw[4], aq[4];
-            ldmatrix_x4(stg + REC_NW + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), aw[0], aw[1],
-                        aw[2], aw[3]);
+            ldmatrix_x4_trans(stg + REC_NW + toff(kk * 16 + l7 + lb4 * 8, 16 * rt + lb3 * 8, 128),
+                              aw[0], aw[1], aw[2], aw[3]);
             ldmatrix_x4(stg + REC_QT + toff(16 * rt + l7 + lb3 * 8, kk * 16 + lb4 * 8, 64), aq[0], aq[1],
                         aq[2], aq[3]);
 #pragma unroll
@@ -660,7 +668,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_scan_kernel(const Prefill
             st_bf16x2(sm + B_U + p * 8192, toff(ur0, cc, 64), u[j][0], u[j][1]);
             st_bf16x2(sm + B_U + p * 8192, toff(ur1, cc, 64), u[j][2], u[j][3]);
         }
-        if (c + 1 < a.n_seg) load_ut(c + 1);
         __syncthreads();
 
         // ---- phase 3: O += P U and store it; st += Kc^T U ------------------------------------
