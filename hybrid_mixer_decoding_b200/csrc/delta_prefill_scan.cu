@@ -291,15 +291,29 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     // ---- gate prefix G (log domain): KDA per channel in place within NQ row parts, plus the
     //      parts' exclusive prefix; GDN per token -------------------------------------------------
     if constexpr (KDA) {
+        if (fused) {  // log-gates from the staged logits, in place, 4 channels per item
+            const float *db = a.act.dt_bias + (size_t)h * kD;
+#pragma unroll
+            for (int j = 0; j < kC * kD / 4 / NT; ++j) {
+                const int e = 4 * (tid + j * NT);
+                const int r = (e & 2047) >> 5, ch = (e >> 11) * 32 + (e & 31);  // gidx inverse
+                float4 x = *reinterpret_cast<const float4 *>(Gs + e);
+                const float4 bb = make_float4(db[ch], db[ch + 1], db[ch + 2], db[ch + 3]);
+                const bool live = r < n;  // rows past the sequence read as zero and stay zero
+                x.x = live ? -rate * hmd_softplus(x.x + bb.x) : 0.f;
+                x.y = live ? -rate * hmd_softplus(x.y + bb.y) : 0.f;
+                x.z = live ? -rate * hmd_softplus(x.z + bb.z) : 0.f;
+                x.w = live ? -rate * hmd_softplus(x.w + bb.w) : 0.f;
+                *reinterpret_cast<float4 *>(Gs + e) = x;
+            }
+            __syncthreads();
+        }
         const int i = tid & (kD - 1), qr = tid >> 7;
         float *gcol = Gs + gidx(0, i);
-        const float bias = fused ? a.act.dt_bias[(size_t)h * kD + i] : 0.f;
         float run = 0.f;
 #pragma unroll
         for (int r = RPQ * qr; r < RPQ * qr + RPQ; ++r) {
-            float x = gcol[r * 32];
-            if (fused) x = r < n ? -rate * hmd_softplus(x + bias) : 0.f;
-            run += x;
+            run += gcol[r * 32];
             gcol[r * 32] = run;
         }
         qoff[qr * kD + i] = run;

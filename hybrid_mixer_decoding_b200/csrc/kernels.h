@@ -48,14 +48,15 @@ struct DeltaAct {
     float eps = 0.f;
 };
 
-// softplus(x) = log(1 + e^x), from the definition: above 15 it is x + log(1 + e^-x) ~ x + e^-x;
-// below, with e = e^x, the series e - e^2/2 + e^3/3 - e^4/4 while e < 1/64 (next term e^5/5,
-// a relative 3e-8), else log(1 + e), where 1 + e keeps e to a relative 4e-6.
+// softplus(x) = log(1 + e^x) = max(x, 0) + log(1 + y), y = e^-|x| in (0, 1]; log(1 + y) is the
+// series y - y^2/2 + y^3/3 - y^4/4 while y < 1/64 (next term y^5/5, a relative 3e-8), else
+// log(1 + y), where 1 + y keeps y to a relative 4e-6. Both are computed and one is selected,
+// so a warp never diverges on it.
 __device__ __forceinline__ float hmd_softplus(float x) {
-    if (x > 15.f) return x + __expf(-x);
-    const float e = __expf(x);
-    if (e < 0.015625f) return e * (1.f - e * (0.5f - e * (1.f / 3.f - 0.25f * e)));
-    return __logf(1.f + e);
+    const float y = __expf(-fabsf(x));
+    const float ser = y * (1.f - y * (0.5f - y * (1.f / 3.f - 0.25f * y)));
+    const float lg = __logf(1.f + y);
+    return fmaxf(x, 0.f) + (y < 0.015625f ? ser : lg);
 }
 
 struct DeltaDecodeArgs {
