@@ -649,8 +649,14 @@ def run_spec(args):
     lin = lambda kind: layer_bytes(kind, shape)  # noqa: E731
     draft_bytes = nq * sum(lin(int(x)) for x in sp.drafter)
     attn = lambda keys: B * (keys * Hkv * d * 4 + nq * (2 * H * d * 2 + 2 * Hkv * d * 2))  # noqa: E731
-    verify_bytes = sum(attn(ctx) if x == I.FA else attn(w + k) if x == I.SWA else nq * lin(int(x))
-                       for x in target)
+    # a GDN/KDA layer of the target reads its state once and stores it after each of the nq
+    # positions (delta_rule_decode_chain): state (1 + nq) times, activations nq times
+    state_b = B * H * d * d * 4
+
+    def chain_bytes(kind):
+        return (1 + nq) * state_b + nq * (lin(kind) - 2 * state_b)
+    verify_bytes = sum(attn(ctx) if x == I.FA else attn(w + k) if x == I.SWA else
+                       chain_bytes(int(x)) for x in target)
     round_s = spec_s / args.steps
     byts = draft_bytes + verify_bytes
     la = sp.launches()

@@ -9,6 +9,7 @@ from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DE
                    KDA, SWA, DecodeIO, HmdError, KVCache, StateCache, attn_decode,
                    attn_decode_static_ws, attn_prefill, attn_decode_workspace_size, attn_verify,
                    attn_verify_workspace_size, delta_rule_decode, delta_rule_decode_act,
+                   delta_rule_decode_chain,
                    delta_rule_decode_to, delta_rule_prefill_chunked_act,
                    delta_rule_prefill_chunked, delta_rule_prefill_chunked_ws,
                    delta_rule_prefill_workspace_size, hmd_device_errors, hmd_last_error,
@@ -18,6 +19,7 @@ __all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "D
            "GDN", "KDA", "SWA", "DecodeIO", "HmdError", "KVCache", "StateCache", "attn_decode",
            "attn_decode_static_ws", "attn_decode_workspace_size", "attn_prefill", "attn_verify",
            "attn_verify_workspace_size", "delta_rule_decode", "delta_rule_decode_act",
+           "delta_rule_decode_chain",
            "delta_rule_decode_to", "delta_rule_prefill_chunked_act",
            "delta_rule_prefill_chunked", "delta_rule_prefill_chunked_ws",
            "delta_rule_prefill_workspace_size", "hmd_device_errors", "hmd_last_error",

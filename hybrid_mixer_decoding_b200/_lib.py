@@ -50,6 +50,8 @@ _SIGS = {
                                                                  _c_float, _vp]),
     "delta_rule_prefill_chunked_act": (_c_int, [_c_int] * 7 + [_vp] * 7 + [_c_int, _vp, _vp,
                                                                           _c_int, _c_float, _vp]),
+    "delta_rule_decode_chain": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_vp, _c_int, _vp, _vp,
+                                                                  _c_float, _vp]),
     "delta_rule_decode_to": (_c_int, [_c_int] * 6 + [_vp] * 6 + [_c_int, _vp, _vp, _vp, _c_float,
                                                                 _vp]),
     "delta_rule_prefill_chunked": (_c_int, [_c_int] * 7 + [_vp] * 6 + [_c_int, _vp, _vp, _c_int,
@@ -194,6 +196,24 @@ def delta_rule_prefill_chunked_act(kind, q_raw, k_raw, v, beta_logit, gate_logit
                                               state.shape[0], _p(slots), _p(o), int(chunk),
                                               float(scale), _stream(stream))
     _check("delta_rule_prefill_chunked_act", st)
+
+
+def delta_rule_decode_chain(kind, q, k, v, beta, log_gate, state, o, chain, scale=1.0,
+                            act=None, stream=None) -> None:
+    """n_q decode tokens per sequence along a slot chain (see include/hmd.h): q, k
+    [B,n_q,H,dk]; v, o [B,n_q,H,dv]; beta [B,n_q,H]; log_gate [B,n_q,H] or [B,n_q,H,dk];
+    chain int32 [n_q+1, B]; act: None, or (A_log, dt_bias, eps) for raw projections."""
+    _contig(q, k, v, beta, log_gate, state, o, chain)
+    B, n_q, H, dk = q.shape
+    dv = v.shape[-1]
+    a = None
+    if act is not None:
+        a = ctypes.byref(DeltaAct(act[0].data_ptr(), act[1].data_ptr(), float(act[2])))
+    st = lib().delta_rule_decode_chain(kind, n_q, B, H, dk, dv, _dtype_code(q), _p(q), _p(k),
+                                       _p(v), _p(beta), _p(log_gate), a, _p(state),
+                                       state.shape[0], _p(chain), _p(o), float(scale),
+                                       _stream(stream))
+    _check("delta_rule_decode_chain", st)
 
 
 def delta_rule_prefill_chunked(kind, q, k, v, beta, log_gate, state, o, slots=None, chunk=64,

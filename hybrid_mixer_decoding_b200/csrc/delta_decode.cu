@@ -43,10 +43,13 @@ __device__ __forceinline__ float act(const void *p, size_t i) {
     }
 }
 
-template <int DK, bool BF16>
+// CHAIN: nq tokens per launch along a slot chain (a.nq, a.chain); otherwise one token with
+// a.nq == 1, compiled without the token loop.
+template <int DK, bool BF16, bool CHAIN>
 __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_constant__ CUtensorMap tm,
                                                                 const DeltaDecodeArgs a,
                                                                 int n_slices) {
+    const int nq = CHAIN ? a.nq : 1;
     constexpr int RPT = DK / kRowThreads;  // rows per thread
     __shared__ __align__(128) float S[DK][kSliceCols];
     __shared__ float sk[DK], sq[DK], sa[DK];
@@ -68,10 +71,18 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     griddep_launch_dependents();
     griddep_wait();  // q, k, v, gates and the state may come from the previous kernel
     const int b = a.rows ? a.rows[ri] : ri;
+    // the slot read before token 0, and the slot written after token t
+    const int src = CHAIN ? a.chain[b] : (a.slots ? a.slots[b] : b);
+    auto dst_of = [&](int t) {
+        return CHAIN ? a.chain[(size_t)(t + 1) * a.B + b] : (a.dst_slots ? a.dst_slots[b] : src);
+    };
     if (tid == 0) {
-        const int slot = a.slots ? a.slots[b] : b;
-        const int dst = a.dst_slots ? a.dst_slots[b] : slot;
-        const bool ok = slot >= 0 && slot < a.n_slots && dst >= 0 && dst < a.n_slots;
+        const int slot = src;
+        bool ok = slot >= 0 && slot < a.n_slots;
+        for (int t = 0; t < nq; ++t) {
+            const int dst = dst_of(t);
+            ok = ok && dst >= 0 && dst < a.n_slots;
+        }
         s_ok = ok;
         if (ok) {
             const uint32_t bb = smem_u32(&bar);
@@ -83,8 +94,9 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
             atomicOr(&g_err, HMD_DEVERR_SLOT);
         }
     }
-    const size_t tok = (size_t)b * a.H + h;
     const bool fused = a.act.A_log != nullptr;  // raw projections: activate them here
+    for (int t = 0; t < nq; ++t) {  // body not re-indented: one token per iteration
+    const size_t tok = ((size_t)b * nq + t) * a.H + h;
     const float rate = fused ? expf(a.act.A_log[h]) : 0.f;
     if (a.kind == HMD_GDN) {
         float lg = a.log_gate[tok];
@@ -131,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
             tk += nrm[w][0];
             tq += nrm[w][1];
         }
-        const float fk = 1.f / sqrtf(tk + a.act.eps), fq = 1.f / sqrtf(tq + a.act.eps);
+        const float fk = rsqrtf(tk + a.act.eps), fq = rsqrtf(tq + a.act.eps);
         for (int i = tid; i < DK; i += kThreads) {
             sk[i] *= fk;
             sq[i] *= fq;
@@ -139,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     }
     __syncthreads();
     if (!s_ok) return;
-    if (!mbar_wait_bounded(smem_u32(&bar), 0)) {
+    if (t == 0 && !mbar_wait_bounded(smem_u32(&bar), 0)) {
         if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
         return;  // nothing was written; the state slice is left as it was
     }
@@ -174,6 +186,7 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
         }
         red[warp][lane][8] = kq;
     }
+    if (t > 0 && tid == 0) bulk_wait_group_read0();  // token t-1's store has read S
     __syncthreads();
     float W[4] = {0.f, 0.f, 0.f, 0.f}, PQ[4] = {0.f, 0.f, 0.f, 0.f}, KQ = 0.f;
 #pragma unroll
@@ -217,12 +230,11 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        const int slot = a.slots ? a.slots[b] : b;
-        const int dst = a.dst_slots ? a.dst_slots[b] : slot;
-        tma_store_2d(&tm, smem_u32(&S[0][0]), slice * kSliceCols, (dst * a.H + h) * DK);
+        tma_store_2d(&tm, smem_u32(&S[0][0]), slice * kSliceCols, (dst_of(t) * a.H + h) * DK);
         bulk_commit_group();
-        bulk_wait_group_read0();
     }
+    }  // tokens
+    if (tid == 0) bulk_wait_group_read0();  // shared memory must outlive the last store's read
 }
 
 template <int DK>
@@ -235,11 +247,16 @@ cudaError_t launch_dk(const DeltaDecodeArgs &a, cudaStream_t s) {
     if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.state, a.dv,
                       (long long)a.n_slots * a.H * DK, kSliceCols, DK))
         return cudaErrorInvalidValue;
+    const bool chain = a.chain != nullptr;
     if (a.bf16)
-        return launch_pdl(delta_decode_kernel<DK, true>, dim3((unsigned)grid), dim3(kThreads), 0, s,
-                          tm, a, n_slices);
-    return launch_pdl(delta_decode_kernel<DK, false>, dim3((unsigned)grid), dim3(kThreads), 0, s, tm,
-                      a, n_slices);
+        return chain ? launch_pdl(delta_decode_kernel<DK, true, true>, dim3((unsigned)grid),
+                                  dim3(kThreads), 0, s, tm, a, n_slices)
+                     : launch_pdl(delta_decode_kernel<DK, true, false>, dim3((unsigned)grid),
+                                  dim3(kThreads), 0, s, tm, a, n_slices);
+    return chain ? launch_pdl(delta_decode_kernel<DK, false, true>, dim3((unsigned)grid),
+                              dim3(kThreads), 0, s, tm, a, n_slices)
+                 : launch_pdl(delta_decode_kernel<DK, false, false>, dim3((unsigned)grid),
+                              dim3(kThreads), 0, s, tm, a, n_slices);
 }
 
 }  // namespace

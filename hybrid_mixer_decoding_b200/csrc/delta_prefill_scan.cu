@@ -374,8 +374,8 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     sq += __shfl_xor_sync(0xffffffffu, sq, off);
                     sk += __shfl_xor_sync(0xffffffffu, sk, off);
                 }
-                fq = 1.f / sqrtf(sq + a.act.eps);
-                fk = 1.f / sqrtf(sk + a.act.eps);
+                fq = rsqrtf(sq + a.act.eps);
+                fk = rsqrtf(sk + a.act.eps);
             }
             uint32_t kt[4], qt[4], kh[4], kcw[4];
 #pragma unroll

@@ -110,7 +110,8 @@ hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_
                        const void *q, const void *k, const void *v, const float *beta,
                        const float *log_gate, float *state, int n_slots, const int32_t *slots,
                        const int32_t *dst_slots, void *o, float scale, const int32_t *rows,
-                       int n_rows, hmd_stream_t stream, const hmd_delta_act_t *act = nullptr) {
+                       int n_rows, hmd_stream_t stream, const hmd_delta_act_t *act = nullptr,
+                       int nq = 1, const int32_t *chain = nullptr) {
     const hmd_status_t st = check_delta_decode(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate,
                                                state, n_slots, o);
     if (st != HMD_OK) return fail(st);
@@ -125,6 +126,7 @@ hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_
         if (!act->A_log || !act->dt_bias || !(act->l2_eps >= 0.f)) return fail(HMD_ERR_ARG);
         a.act.A_log = act->A_log; a.act.dt_bias = act->dt_bias; a.act.eps = act->l2_eps;
     }
+    a.nq = nq; a.chain = chain;
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
 }
 }  // namespace
@@ -150,6 +152,18 @@ hmd_status_t delta_rule_decode_act(hmd_kind_t kind, int B, int H, int dk, int dv
     if (!act) return fail(HMD_ERR_ARG);
     return delta_run(kind, B, H, dk, dv, dtype, q_raw, k_raw, v, beta_logit, gate_logit, state,
                      n_slots, slots, dst_slots, o, scale, nullptr, 0, stream, act);
+}
+
+hmd_status_t delta_rule_decode_chain(hmd_kind_t kind, int n_q, int B, int H, int dk, int dv,
+                                     hmd_dtype_t dtype, const void *q, const void *k,
+                                     const void *v, const float *beta, const float *log_gate,
+                                     const hmd_delta_act_t *act, float *state, int n_slots,
+                                     const int32_t *chain, void *o, float scale,
+                                     hmd_stream_t stream) {
+    if (n_q < 1) return fail(HMD_ERR_SHAPE);
+    if (!chain && B > 0) return fail(HMD_ERR_ARG);
+    return delta_run(kind, B, H, dk, dv, dtype, q, k, v, beta, log_gate, state, n_slots, nullptr,
+                     nullptr, o, scale, nullptr, 0, stream, act, n_q, chain);
 }
 
 hmd_status_t delta_rule_decode(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_t dtype,

@@ -74,6 +74,10 @@ struct DeltaDecodeArgs {
     const int32_t *rows = nullptr;  // batch rows to run (device, n_rows of them); NULL: all B
     int n_rows = 0;
     DeltaAct act;
+    // nq tokens per sequence in one launch (inputs [B][nq][H][...]): the state is read once
+    // from chain[0][b] and the state after token t is stored to chain[t + 1][b] ([nq+1][B])
+    int nq = 1;
+    const int32_t *chain = nullptr;
 };
 cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s);
 bool delta_decode_supported(int dk, int dv);

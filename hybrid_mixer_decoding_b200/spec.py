@@ -11,8 +11,9 @@ with no projections, MLPs or sampler (so no tokens): per round, for every sequen
           x_0, d_1, ..., d_k; step t reads state slot s_t and writes s_{t+1}
           (delta_rule_decode_to), so every intermediate state is kept;
   verify: the target placement checks the k + 1 positions at once: its attention layers in one
-          attn_verify pass (n_q = k + 1 query rows per sequence), its GDN/KDA layers as k + 1
-          decode steps along the same slot chain;
+          attn_verify pass (n_q = k + 1 query rows per sequence), its GDN/KDA layers in one
+          delta_rule_decode_chain launch (the state read once, the state after each position
+          stored along the same slot chain);
   accept: j_b of the k drafts are kept (plus the target's own token): the drafter's and the
           target's recurrent state are then slot s_{j_b + 1}, chosen without copying, and the
           attention caches keep L_b + j_b + 1 positions (the rejected ones are overwritten
@@ -138,28 +139,34 @@ class SpecStack:
         # per-layer inputs (resident; each round reads the same values)
         nq = self.n_q
 
-        def lin_inputs(l, kind, tag):
+        def lin_inputs(l, kind, tag, seq_major):
+            """[nq][B][...] for the drafter's token-by-token steps; [B][nq][...] for the
+            target's chain launches (plus token 0 alone, for its plain decode step)."""
+            shp = (B, nq) if seq_major else (nq, B)
             t = {}
-            t["q"] = torch.randn(nq, B, H, d, generator=_gen(layer_seed(l, tag) + seed), device=dev).to(bf)
-            kk = torch.randn(nq, B, H, d, generator=_gen(layer_seed(l, tag + 1) + seed), device=dev)
+            t["q"] = torch.randn(*shp, H, d, generator=_gen(layer_seed(l, tag) + seed), device=dev).to(bf)
+            kk = torch.randn(*shp, H, d, generator=_gen(layer_seed(l, tag + 1) + seed), device=dev)
             t["k"] = torch.nn.functional.normalize(kk, dim=-1).to(bf)
-            t["v"] = torch.randn(nq, B, H, d, generator=_gen(layer_seed(l, tag + 2) + seed), device=dev).to(bf)
-            t["beta"] = torch.sigmoid(torch.randn(nq, B, H, generator=_gen(layer_seed(l, tag + 3) + seed),
+            t["v"] = torch.randn(*shp, H, d, generator=_gen(layer_seed(l, tag + 2) + seed), device=dev).to(bf)
+            t["beta"] = torch.sigmoid(torch.randn(*shp, H, generator=_gen(layer_seed(l, tag + 3) + seed),
                                                   device=dev))
             if kind == KDA:
-                t["lg"] = -0.05 * torch.rand(nq, B, H, d, generator=_gen(layer_seed(l, tag + 4) + seed),
+                t["lg"] = -0.05 * torch.rand(*shp, H, d, generator=_gen(layer_seed(l, tag + 4) + seed),
                                              device=dev)
             else:
-                t["lg"] = -0.1 * torch.rand(nq, B, H, generator=_gen(layer_seed(l, tag + 4) + seed),
+                t["lg"] = -0.1 * torch.rand(*shp, H, generator=_gen(layer_seed(l, tag + 4) + seed),
                                             device=dev)
-            t["o"] = torch.empty(nq, B, H, d, device=dev, dtype=bf)
+            t["o"] = torch.empty(*shp, H, d, device=dev, dtype=bf)
+            if seq_major:
+                for x in ("q", "k", "v", "beta", "lg", "o"):
+                    t[x + "1"] = t[x][:, 0].contiguous()
             return t
 
         self.t_in, self.d_in = [], []
         for l in range(nl):
             kind = int(self.target[l])
             if kind in (GDN, KDA):
-                self.t_in.append(lin_inputs(l, kind, 20))
+                self.t_in.append(lin_inputs(l, kind, 20, seq_major=True))
             else:
                 t = {"q": torch.randn(B, nq, H, d, generator=_gen(layer_seed(l, 0) + seed), device=dev).to(bf),
                      "nk": torch.randn(B, nq, Hkv, d, generator=_gen(layer_seed(l, 6) + seed), device=dev).to(bf),
@@ -169,7 +176,7 @@ class SpecStack:
                 t["q1"], t["nk1"], t["nv1"] = (t[x][:, :1].contiguous() for x in ("q", "nk", "nv"))
                 t["o1"] = torch.empty(B, 1, H, d, device=dev, dtype=bf)
                 self.t_in.append(t)
-            self.d_in.append(lin_inputs(l, int(self.drafter[l]), 40))
+            self.d_in.append(lin_inputs(l, int(self.drafter[l]), 40, seq_major=False))
 
         ws = max([L.attn_verify_workspace_size(FA, 0, nq, B, H, Hkv, d, PAGE, s.ctx),
                   L.attn_verify_workspace_size(SWA, s.window, nq, B, H, Hkv, d, PAGE, s.ctx)])
@@ -203,10 +210,10 @@ class SpecStack:
             kind, t_in = int(self.target[l]), self.t_in[l]
             if kind in (FA, SWA):
                 self._attn(l, kind, t_in["q"], t_in["nk"], t_in["nv"], t_in["o"], self.lens_v)
-            else:
+            else:  # k + 1 tokens in one launch: the state read once, each step stored
                 st = self.t_state.layer_view(self.t_lin.index(l))
-                for t in range(self.n_q):
-                    self._lin_step(kind, t_in, st, t, self.slot_buf[t], self.slot_buf[t + 1])
+                L.delta_rule_decode_chain(kind, t_in["q"], t_in["k"], t_in["v"], t_in["beta"],
+                                          t_in["lg"], st, t_in["o"], self.slot_buf)
 
     def plain_step(self):
         """One ordinary decode token of the target placement (its states updated in place)."""
@@ -216,7 +223,9 @@ class SpecStack:
                 self._attn(l, kind, t_in["q1"], t_in["nk1"], t_in["nv1"], t_in["o1"], self.lens_1)
             else:
                 st = self.t_state.layer_view(self.t_lin.index(l))
-                self._lin_step(kind, t_in, st, 0, self.slot_buf[0], self.slot_buf[0])
+                L.delta_rule_decode_to(kind, t_in["q1"], t_in["k1"], t_in["v1"], t_in["beta1"],
+                                       t_in["lg1"], st, t_in["o1"], self.slot_buf[0],
+                                       self.slot_buf[0])
 
     def set_round(self, sched: Schedule, r: int, slots_dev: torch.Tensor, lens_dev: torch.Tensor):
         """Stream-ordered device-to-device copies of round r's slot chain and lengths."""
@@ -240,7 +249,7 @@ class SpecStack:
         n_lin_t = len(self.t_lin)
         n_att = self.n_layers - n_lin_t
         return {"draft": self.n_q * self.n_layers,
-                "verify": 2 * n_att + self.n_q * n_lin_t,
+                "verify": 2 * n_att + n_lin_t,
                 "plain": 2 * n_att + n_lin_t}
 
     def free(self):

@@ -122,6 +122,23 @@ HMD_API hmd_status_t delta_rule_decode_act(hmd_kind_t kind, int B, int H, int dk
                                            const int32_t *dst_slots, void *o, float scale,
                                            hmd_stream_t stream);
 
+/* n_q decode tokens per sequence in one launch, along a slot chain: the state is read once
+ * from slot chain[0][b] and, after token t, stored to slot chain[t + 1][b] (the state read is
+ * never written back). Equal to n_q delta_rule_decode_to calls stepping chain[t] ->
+ * chain[t + 1], bit for bit, while reading the state once instead of n_q times: the form a
+ * speculative verifier's GDN/KDA layers take, since its k + 1 positions are all known.
+ *   q, k [B][n_q][H][dk]; v, o [B][n_q][H][dv]; beta [B][n_q][H]; log_gate [B][n_q][H] (GDN)
+ *   or [B][n_q][H][dk] (KDA); chain int32 [n_q + 1][B] on the device, slots in [0, n_slots)
+ *   (a bad slot skips that sequence and sets HMD_DEVERR_SLOT), no slot shared between
+ *   sequences; act: NULL for activated inputs, else raw projections as in delta_rule_decode_act.
+ */
+HMD_API hmd_status_t delta_rule_decode_chain(hmd_kind_t kind, int n_q, int B, int H, int dk,
+                                             int dv, hmd_dtype_t dtype, const void *q,
+                                             const void *k, const void *v, const float *beta,
+                                             const float *log_gate, const hmd_delta_act_t *act,
+                                             float *state, int n_slots, const int32_t *chain,
+                                             void *o, float scale, hmd_stream_t stream);
+
 /* Chunked (WY / UT-transform) prefill over T tokens per sequence for one layer: the same
  * recurrence as delta_rule_decode applied to tokens 0..T-1 in order, computed chunk by chunk.
  *   q, k [B][T][H][dk]; v, o [B][T][H][dv] (dtype); beta [B][T][H] fp32;

@@ -181,3 +181,44 @@ def test_out_of_place_bad_destination_sets_device_error():
     assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_SLOT
     # sequence 0 (valid destination) was written to slot 2; sequence 1 skipped entirely
     assert torch.equal(state[[0, 1, 3]], before[[0, 1, 3]])
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_chain_launch_equals_steps_and_oracle(oracle_mod, kind, dtype):
+    """delta_rule_decode_chain over 4 tokens: every chain slot and output is bit-identical to
+    4 delta_rule_decode_to steps along the same chain, the first slot is never written, and the
+    slots match the oracle's recurrence after 1..4 tokens."""
+    O = oracle_mod
+    B, nq, H, dk, dv = 3, 4, 4, 128, 64
+    d = I.delta_inputs(kind, B, nq, H, dk, dv, dtype=dtype, seed=50, state0="randn")
+    act = torch.bfloat16 if dtype == "bf16" else torch.float32
+    chain = (np.arange(B)[None, :] * (nq + 1) + np.arange(nq + 1)[:, None]).astype(np.int32)
+    n_slots = B * (nq + 1)
+    st1 = torch.zeros(n_slots, H, dk, dv, device="cuda")
+    st1[torch.from_numpy(chain[0]).long().cuda()] = _dev(d.state0)
+    st2 = st1.clone()
+    o1 = torch.empty(B, nq, H, dv, device="cuda", dtype=act)
+    hmd.delta_rule_decode_chain(kind, _dev(d.q, act), _dev(d.k, act), _dev(d.v, act),
+                                _dev(d.beta), _dev(d.log_gate), st1, o1,
+                                _dev(chain, torch.int32))
+    outs = []
+    for t in range(nq):
+        o2 = torch.empty(B, H, dv, device="cuda", dtype=act)
+        hmd.delta_rule_decode_to(kind, _dev(d.q[:, t], act), _dev(d.k[:, t], act),
+                                 _dev(d.v[:, t], act), _dev(d.beta[:, t]), _dev(d.log_gate[:, t]),
+                                 st2, o2, _dev(chain[t], torch.int32), _dev(chain[t + 1], torch.int32))
+        outs.append(o2)
+    torch.cuda.synchronize()
+    assert hmd.hmd_device_errors(clear=True) == 0
+    assert torch.equal(st1, st2)
+    assert torch.equal(o1.view(torch.int16) if act == torch.bfloat16 else o1,
+                       (torch.stack(outs, 1).view(torch.int16) if act == torch.bfloat16
+                        else torch.stack(outs, 1)))
+    np.testing.assert_array_equal(st1[torch.from_numpy(chain[0]).long().cuda()].cpu().numpy(),
+                                  d.state0)
+    for t in range(nq):
+        _, s_ref = O.delta_recurrent(kind, d.q[:, :t + 1], d.k[:, :t + 1], d.v[:, :t + 1],
+                                     d.beta[:, :t + 1], d.log_gate[:, :t + 1], d.state0)
+        got = st1[torch.from_numpy(chain[t + 1]).long().cuda()].cpu().numpy()
+        assert O.rel_err(got, s_ref) < TOL[dtype]

@@ -1,6 +1,7 @@
 """GPU check of one self-speculative round on a 4-layer stack (FA, SWA, KDA, GDN target; all-GDN
 drafter): the verify pass matches the fp64 oracle on the cache as it stood, and each slot of
-the recurrent-state chain holds exactly the state of that many in-place decode steps."""
+the recurrent-state chain (one delta_rule_decode_chain launch per GDN/KDA layer) holds exactly
+the state of that many in-place decode steps."""
 import numpy as np
 import pytest
 import torch
@@ -49,12 +50,12 @@ def test_one_round(oracle_mod):
         t = sp.t_in[l]
         st = st0[l][torch.from_numpy(chain[0]).long().cuda()].clone()  # [B, H, d, d]
         for step in range(k + 1):
-            o = torch.empty_like(t["o"][step])
-            hmd.delta_rule_decode(int(target[l]), t["q"][step], t["k"][step], t["v"][step],
-                                  t["beta"][step], t["lg"][step], st, o)
+            x = {n: t[n][:, step].contiguous() for n in ("q", "k", "v", "beta", "lg", "o")}
+            o = torch.empty_like(x["o"])
+            hmd.delta_rule_decode(int(target[l]), x["q"], x["k"], x["v"], x["beta"], x["lg"], st, o)
             got = sp.t_state.layer_view(sp.t_lin.index(l))[torch.from_numpy(chain[step + 1]).long().cuda()]
             assert torch.equal(got, st), (l, step)
-            assert torch.equal(o.view(torch.int16), t["o"][step].view(torch.int16))
+            assert torch.equal(o.view(torch.int16), x["o"].view(torch.int16))
     sp.free()
 
 
