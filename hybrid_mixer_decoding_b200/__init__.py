@@ -7,7 +7,8 @@ include/hmd.h); this package is its ctypes binding plus the seeded input generat
 """
 from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DEVERR_PAGE, DEVERR_SEQLEN, DEVERR_SLOT, DEVERR_TIMEOUT, F32, FA, GDN,
                    KDA, SWA, DecodeIO, HmdError, KVCache, StateCache, attn_decode,
-                   attn_decode_static_ws, attn_prefill, attn_decode_workspace_size, attn_verify,
+                   attn_decode_static_ws, attn_prefill, attn_prefill_ext, attn_decode_workspace_size,
+                   attn_verify,
                    attn_verify_workspace_size, delta_rule_decode, delta_rule_decode_act,
                    delta_rule_decode_chain,
                    delta_rule_decode_to, delta_rule_prefill_chunked_act,
@@ -17,7 +18,8 @@ from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DE
 
 __all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "DEVERR_PAGE", "DEVERR_SEQLEN", "DEVERR_SLOT", "DEVERR_TIMEOUT", "F32", "FA",
            "GDN", "KDA", "SWA", "DecodeIO", "HmdError", "KVCache", "StateCache", "attn_decode",
-           "attn_decode_static_ws", "attn_decode_workspace_size", "attn_prefill", "attn_verify",
+           "attn_decode_static_ws", "attn_decode_workspace_size", "attn_prefill", "attn_prefill_ext",
+           "attn_verify",
            "attn_verify_workspace_size", "delta_rule_decode", "delta_rule_decode_act",
            "delta_rule_decode_chain",
            "delta_rule_decode_to", "delta_rule_prefill_chunked_act",

@@ -66,6 +66,8 @@ _SIGS = {
     "attn_decode": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _c_int, _vp,
                                                       _vp, _sz, _vp]),
     "attn_prefill": (_c_int, [_c_int] * 8 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp, _vp]),
+    "attn_prefill_ext": (_c_int, [_c_int] * 8 + [_vp] * 4 + [_c_int, _vp, _vp, _c_int, _vp,
+                                                             _c_int, _vp, _vp]),
     "attn_decode_static_ws": (_c_int, [_c_int] * 7 + [_vp] * 5 + [_c_int, _vp, _c_int, _vp,
                                                                 _c_int, _vp, _vp]),
     "state_cache_alloc": (_c_int, [_c_int] * 5 + [_vp, ctypes.POINTER(_vp)]),
@@ -316,6 +318,19 @@ def attn_prefill(kind, window, q, k, v, k_pool, v_pool, page_table, o, stream=No
                             _p(k_pool), _p(v_pool), n_pages, _p(page_table), page_table.shape[1],
                             _p(o), _stream(stream))
     _check("attn_prefill", st)
+
+
+def attn_prefill_ext(kind, window, q, k, v, prefix_lens, max_prefix, k_pool, v_pool, page_table,
+                     o, stream=None) -> None:
+    """attn_prefill after a cached prefix of prefix_lens[b] positions (device int32 [B],
+    multiples of 64; see include/hmd.h)."""
+    _contig(q, k, v, prefix_lens, k_pool, v_pool, page_table, o)
+    B, T, Hq, d = q.shape
+    n_pages, Hkv, PT, _ = k_pool.shape
+    st = lib().attn_prefill_ext(kind, int(window), B, T, Hq, Hkv, d, PT, _p(q), _p(k), _p(v),
+                                _p(prefix_lens), int(max_prefix), _p(k_pool), _p(v_pool), n_pages,
+                                _p(page_table), page_table.shape[1], _p(o), _stream(stream))
+    _check("attn_prefill_ext", st)
 
 
 class StateCache:

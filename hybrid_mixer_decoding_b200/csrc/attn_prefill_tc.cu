@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <float.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kernels.h"
@@ -70,8 +71,10 @@ struct TcParams {
     const __nv_bfloat16 *q, *k, *v;
     __nv_bfloat16 *k_pool, *v_pool, *o;
     const int32_t *page_table;
+    const int32_t *prefix_lens;  // cached positions before the prompt, per sequence (or NULL)
     int B, T, Hq, Hkv, G, QT, n_qb;
     int window, swa, ring_pages, max_pages, n_pages;
+    int defer_write;  // the prompt's K/V go to the cache in a later kernel (SWA with a prefix)
     float scale_log2;
 };
 
@@ -102,9 +105,13 @@ __device__ __forceinline__ void softmax_barrier() {  // warps 0-7 only (named ba
     asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
+// PREFIX: sequences may start after cached positions (p.prefix_lens); false compiles the
+// empty-cache prefill with every prefix path removed.
+template <bool PREFIX>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                       const TcParams p) {
+                       const __grid_constant__ CUtensorMap tmpk,
+                       const __grid_constant__ CUtensorMap tmpv, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -133,6 +140,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
         restart[0] = restart[1] = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
+        if constexpr (PREFIX) {
+            prefetch_tmap(&tmpk);
+            prefetch_tmap(&tmpv);
+        }
     }
     if (warp == 8) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -141,14 +152,24 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     griddep_launch_dependents();
     griddep_wait();  // the prompt and the cache may come from the previous kernel
 
-    const int kb_lo = key_lo(p, t_first) / kPT, kb_hi = t_last / kPT;
+    // positions: token t of the prompt sits at L0 + t after a cached prefix of L0 positions
+    int L0 = 0;
+    if constexpr (PREFIX) {
+        L0 = p.prefix_lens[b];
+        if (L0 < 0 || (L0 % kPT) != 0) {  // not a whole number of pages: report, run without it
+            if (tid == 0) atomicOr(&g_err, HMD_DEVERR_SEQLEN);
+            L0 = 0;
+        }
+    }
+    const int kb_lo = key_lo(p, L0 + t_first) / kPT, kb_hi = (L0 + t_last) / kPT;
     const int n_tiles = kb_hi - kb_lo + 1;
 
     // ---- Q rows -> shared memory (half a row per softmax thread); fused cache write ----------
     const int row = tid & (kRows - 1), ch = (tid >> 7) & 1;
     const int t_row = t_first + row % p.QT;
     const bool row_ok = t_row <= t_last;
-    const int lo_row = key_lo(p, t_row);
+    const int pos_row = L0 + t_row;  // the row's position: its last key
+    const int lo_row = key_lo(p, pos_row);
     const int h_row = g * p.G + row / p.QT;
     if (tid < kSoftmax) {
         const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -161,13 +182,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
         const int ring = p.ring_pages * kPT;
         const int n_tok = t_last - t_first + 1;
         constexpr int CH = kD / 8;
-        for (int idx = tid; idx < n_tok * 2 * CH; idx += kSoftmax) {
+        for (int idx = tid; idx < ((PREFIX && p.defer_write) ? 0 : n_tok * 2 * CH); idx += kSoftmax) {
             const int tt = idx / (2 * CH), rem = idx - tt * 2 * CH;
             const bool is_v = rem >= CH;
             const int chk = is_v ? rem - CH : rem;
             const int t = t_first + tt;
             if (p.swa && t < p.T - ring) continue;  // overwritten later in the ring
-            const int li = p.swa ? t % ring : t;
+            const int li = p.swa ? (L0 + t) % ring : L0 + t;
             const int lp = li / kPT;
             const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
             if (pg < 0 || pg >= p.n_pages) {
@@ -192,9 +213,27 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             int tiles_issued = 0, s_issued = 0, pv_issued = 0;
             auto issue_tile = [&](int i) {
                 const int st = i % kStages;
-                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: 4 boxes of 8 KiB
                 const uint32_t kb = sb + OFF_KV + st * STAGE, vb = kb + 16384;
-                const int z = b * p.T + (kb_lo + i) * kPT;
+                const int key0 = (kb_lo + i) * kPT;  // first position of the tile
+                if (PREFIX && key0 < L0) {  // a page of the cached prefix
+                    const int lp = (kb_lo + i) % (p.swa ? p.ring_pages : 0x7fffffff);
+                    const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+                    if (pg < 0 || pg >= p.n_pages) {
+                        atomicOr(&g_err, HMD_DEVERR_PAGE);
+                        mbar_arrive_expect_tx(bar(B_FULL + st), 0);  // complete with no copy
+                        return;
+                    }
+                    mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);
+                    const int y = (pg * p.Hkv + g) * kPT;
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        tma_load_2d(kb + hf * 8192, &tmpk, bar(B_FULL + st), hf * 64, y);
+                        tma_load_2d(vb + hf * 8192, &tmpv, bar(B_FULL + st), hf * 64, y);
+                    }
+                    return;
+                }
+                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: 4 boxes of 8 KiB
+                const int z = b * p.T + (key0 - L0);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     tma_load_3d(kb + hf * 8192, &tmk, bar(B_FULL + st), hf * 64, g, z);
@@ -299,14 +338,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             // ---- mask (edge tiles only), partial maximum; a restart if it outgrows the base ----
             const int j0 = (kb_lo + i) * kPT + ch * 32;
             float mx = -INFINITY;
-            if (row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= t_row) {
+            if (row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= pos_row) {
 #pragma unroll
                 for (int j = 0; j < kPT / 2; ++j) mx = fmaxf(mx, s[j]);
             } else {
 #pragma unroll
                 for (int j = 0; j < kPT / 2; ++j) {
                     const int key = j0 + j;
-                    const bool valid = row_ok && key >= lo_row && key <= t_row;
+                    const bool valid = row_ok && key >= lo_row && key <= pos_row;
                     s[j] = valid ? s[j] : -INFINITY;
                     mx = fmaxf(mx, s[j]);
                 }
@@ -405,6 +444,42 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     }
 }
 
+// The SWA ring write of a prompt that followed a cached prefix, after the attention kernel has
+// read every prefix key: the last R*64 positions of the prompt (the ones the ring keeps), one
+// 16-byte chunk of K or V per thread.
+__global__ void __launch_bounds__(256) attn_prefill_ring_write_kernel(const TcParams p) {
+    griddep_launch_dependents();
+    griddep_wait();  // the attention kernel has read the ring
+    const int ring = p.ring_pages * kPT;
+    const int t_lo = p.T > ring ? p.T - ring : 0;
+    constexpr int CH = kD / 8;
+    const long long n = (long long)p.B * (p.T - t_lo) * p.Hkv * 2 * CH;
+    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int chk = (int)(idx % CH);
+        long long r = idx / CH;
+        const bool is_v = (r & 1) != 0;
+        r >>= 1;
+        const int g = (int)(r % p.Hkv);
+        r /= p.Hkv;
+        const int t = t_lo + (int)(r % (p.T - t_lo));
+        const int b = (int)(r / (p.T - t_lo));
+        int L0 = p.prefix_lens ? p.prefix_lens[b] : 0;
+        if (L0 < 0 || (L0 % kPT) != 0) L0 = 0;  // reported by the attention kernel
+        const int li = (L0 + t) % ring;
+        const int lp = li / kPT;
+        const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+        if (pg < 0 || pg >= p.n_pages) {
+            atomicOr(&g_err, HMD_DEVERR_PAGE);
+            continue;
+        }
+        const size_t srco = (((size_t)b * p.T + t) * p.Hkv + g) * kD + chk * 8;
+        const size_t dsto = (((size_t)pg * p.Hkv + g) * kPT + (li % kPT)) * kD + chk * 8;
+        *reinterpret_cast<uint4 *>((is_v ? p.v_pool : p.k_pool) + dsto) =
+            *reinterpret_cast<const uint4 *>((is_v ? p.v : p.k) + srco);
+    }
+}
+
 }  // namespace
 
 bool attn_prefill_tc_supported(int d, int page_tokens, int group) {
@@ -417,15 +492,27 @@ cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_prefill_tc_kernel,
+        attr_err = cudaFuncSetAttribute(attn_prefill_tc_kernel<false>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(attn_prefill_tc_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap tmk, tmv;
+    CUtensorMap tmk, tmv, tmpk, tmpv;
     const long long n_tok = (long long)a.B * a.T;
     if (!make_tmap_tokens_sw128(&tmk, const_cast<void *>(a.k), n_tok, a.Hkv, kD) ||
         !make_tmap_tokens_sw128(&tmv, const_cast<void *>(a.v), n_tok, a.Hkv, kD))
         return cudaErrorInvalidValue;
+    if (a.prefix_lens) {
+        if (!make_tmap_pool_sw128(&tmpk, a.k_pool, a.n_pages, a.Hkv, kD) ||
+            !make_tmap_pool_sw128(&tmpv, a.v_pool, a.n_pages, a.Hkv, kD))
+            return cudaErrorInvalidValue;
+    } else {
+        tmpk = tmk;  // not read
+        tmpv = tmv;
+    }
     TcParams p;
     p.q = static_cast<const __nv_bfloat16 *>(a.q);
     p.k = static_cast<const __nv_bfloat16 *>(a.k);
@@ -434,6 +521,10 @@ cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     p.v_pool = static_cast<__nv_bfloat16 *>(a.v_pool);
     p.o = static_cast<__nv_bfloat16 *>(a.o);
     p.page_table = a.page_table;
+    p.prefix_lens = a.prefix_lens;
+    // with a prefix, SWA prompt tokens would overwrite ring slots of prefix keys that other
+    // CTAs still read: their cache write moves to a kernel that runs after the attention
+    p.defer_write = (a.swa && a.prefix_lens) ? 1 : 0;
     p.B = a.B; p.T = a.T; p.Hq = a.Hq; p.Hkv = a.Hkv;
     p.G = a.Hq / a.Hkv;
     p.QT = kRows / p.G;
@@ -443,8 +534,16 @@ cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     p.max_pages = a.max_pages; p.n_pages = a.n_pages;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
     const long long grid = (long long)p.n_qb * a.B * a.Hkv;
-    return launch_pdl(attn_prefill_tc_kernel, dim3((unsigned)grid), dim3(kThreads), SMEM_BYTES, s,
-                      tmk, tmv, p);
+    cudaError_t e = a.prefix_lens
+        ? launch_pdl(attn_prefill_tc_kernel<true>, dim3((unsigned)grid), dim3(kThreads),
+                     SMEM_BYTES, s, tmk, tmv, tmpk, tmpv, p)
+        : launch_pdl(attn_prefill_tc_kernel<false>, dim3((unsigned)grid), dim3(kThreads),
+                     SMEM_BYTES, s, tmk, tmv, tmpk, tmpv, p);
+    if (e != cudaSuccess || !p.defer_write) return e;
+    const int ring = p.ring_pages * kPT;
+    const long long n = (long long)a.B * std::min(a.T, ring) * a.Hkv * 2 * (kD / 8);
+    const unsigned blocks = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 16);
+    return launch_pdl(attn_prefill_ring_write_kernel, dim3(blocks), dim3(256), 0, s, p);
 }
 
 uint32_t attn_prefill_tc_read_errors(bool clear) {

@@ -339,30 +339,46 @@ hmd_status_t delta_rule_prefill_chunked_act(hmd_kind_t kind, int B, int T, int H
 
 // ---- attention mixers --------------------------------------------------------------------
 
-hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv, int d,
-                          int page_tokens, const void *q, const void *k, const void *v,
-                          void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
-                          int max_pages, void *o, hmd_stream_t stream) {
+hmd_status_t attn_prefill_ext(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv, int d,
+                              int page_tokens, const void *q, const void *k, const void *v,
+                              const int32_t *prefix_lens, int max_prefix, void *k_pool,
+                              void *v_pool, int n_pages, const int32_t *page_table, int max_pages,
+                              void *o, hmd_stream_t stream) {
     if (kind != HMD_FA && kind != HMD_SWA) return fail(HMD_ERR_ARG);
     if (kind == HMD_SWA && window < 1) return fail(HMD_ERR_ARG);
     if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || d < 1 || page_tokens < 1 || n_pages < 1 ||
-        max_pages < 1)
+        max_pages < 1 || max_prefix < 0)
         return fail(HMD_ERR_SHAPE);
     if (Hq % Hkv) return fail(HMD_ERR_SHAPE);
+    if (prefix_lens && max_prefix % page_tokens) return fail(HMD_ERR_SHAPE);
     if (B == 0 || T == 0) return HMD_OK;
     if (!q || !k || !v || !k_pool || !v_pool || !page_table || !o) return fail(HMD_ERR_ARG);
     if (!hmd::attn_prefill_supported(d, page_tokens, Hq / Hkv)) return fail(HMD_ERR_UNSUPPORTED);
+    // a cached prefix is read by the tensor-core kernel only
+    if (prefix_lens && !hmd::attn_prefill_tc_supported(d, page_tokens, Hq / Hkv))
+        return fail(HMD_ERR_UNSUPPORTED);
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_pool) ||
         !aligned16(v_pool))
         return fail(HMD_ERR_ARG);
+    const long long span = (long long)(prefix_lens ? max_prefix : 0) + T;
     const long long need = kind == HMD_SWA ? (window + page_tokens - 1) / page_tokens
-                                           : ((long long)T + page_tokens - 1) / page_tokens;
+                                           : (span + page_tokens - 1) / page_tokens;
     if (max_pages < need) return fail(HMD_ERR_SHAPE);
+    if ((long long)n_pages * Hkv * page_tokens >= (1LL << 31)) return fail(HMD_ERR_UNSUPPORTED);
     hmd::AttnPrefillArgs a{};
     a.swa = kind == HMD_SWA; a.window = window; a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
     a.page_tokens = page_tokens; a.q = q; a.k = k; a.v = v; a.k_pool = k_pool; a.v_pool = v_pool;
     a.n_pages = n_pages; a.page_table = page_table; a.max_pages = max_pages; a.o = o;
+    a.prefix_lens = prefix_lens;
     return from_cuda(hmd::launch_attn_prefill(a, as_stream(stream)));
+}
+
+hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv, int d,
+                          int page_tokens, const void *q, const void *k, const void *v,
+                          void *k_pool, void *v_pool, int n_pages, const int32_t *page_table,
+                          int max_pages, void *o, hmd_stream_t stream) {
+    return attn_prefill_ext(kind, window, B, T, Hq, Hkv, d, page_tokens, q, k, v, nullptr, 0,
+                            k_pool, v_pool, n_pages, page_table, max_pages, o, stream);
 }
 
 size_t attn_verify_workspace_size(hmd_kind_t kind, int window, int n_q, int B, int Hq, int Hkv,

@@ -37,6 +37,7 @@ bool make_tmap_2d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base,
 bool make_tmap_tokens_sw128(CUtensorMap *m, void *base, long long n_tok, int heads, int d);
 bool make_tmap_bthd(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, int B,
                     int T, int H, int d, int box_d, bool sw128);
+bool make_tmap_pool_sw128(CUtensorMap *m, void *pool, int n_pages, int heads, int d);
 
 // Input activations of the delta-rule mixers, fused into their kernels when A_log is set: the
 // kernel then reads raw q, k (L2-normalised over d_k with eps), beta logits (sigmoid) and gate
@@ -142,6 +143,9 @@ struct AttnPrefillArgs {
     const int32_t *page_table;
     int max_pages;
     void *o;
+    // cached prefix per sequence (device [B], multiples of page_tokens; NULL: none): token t
+    // sits at position prefix_lens[b] + t and also attends the cached keys (tcgen05 path)
+    const int32_t *prefix_lens = nullptr;
 };
 bool attn_prefill_supported(int d, int page_tokens, int group);
 cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s);

@@ -80,4 +80,19 @@ bool make_tmap_bthd(CUtensorMap *m, CUtensorMapDataType dt, int esize, const voi
            CUDA_SUCCESS;
 }
 
+// A paged pool [n_pages][heads][64][d] bf16 viewed as [n_pages*heads*64 rows][d], read in boxes
+// of 64 rows x 64 dims with the 128-byte swizzle: one box is half of one page of one head.
+bool make_tmap_pool_sw128(CUtensorMap *m, void *pool, int n_pages, int heads, int d) {
+    EncodeTiledFn enc = encode();
+    if (!enc) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)n_pages * heads * 64};
+    const cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool, gdim, gstride, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 }  // namespace hmd

@@ -270,6 +270,25 @@ HMD_API hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int
                                   const int32_t *page_table, int max_pages, void *o,
                                   hmd_stream_t stream);
 
+/* attn_prefill after a cached prefix (chunked prefill): sequence b already holds positions
+ * 0..prefix_lens[b]-1 in the paged cache (as attn_prefill / attn_decode wrote them); prompt
+ * token t sits at position P = prefix_lens[b] + t and attends keys [lo, P], lo = 0 (FA) or
+ * max(0, P + 1 - window) (SWA), reading the prefix keys from the cache and the prompt's own from
+ * k, v. The prompt's K and V are then written at their slots (SWA: the positions the ring of
+ * ceil(window / page_tokens) pages keeps; that write runs after every prefix key has been read).
+ *   prefix_lens: device int32 [B], each a multiple of page_tokens and <= max_prefix (a host
+ *   bound, itself a multiple of page_tokens); NULL is attn_prefill. FA needs
+ *   max_pages >= ceil((max_prefix + T) / page_tokens).
+ * Supported with a prefix: d = 128 (the tensor-core kernel), else HMD_ERR_UNSUPPORTED. A prefix
+ * length that is not a whole number of pages sets HMD_DEVERR_SEQLEN (that sequence then runs as
+ * if it had none).                                                                            */
+HMD_API hmd_status_t attn_prefill_ext(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv,
+                                      int d, int page_tokens, const void *q, const void *k,
+                                      const void *v, const int32_t *prefix_lens, int max_prefix,
+                                      void *k_pool, void *v_pool, int n_pages,
+                                      const int32_t *page_table, int max_pages, void *o,
+                                      hmd_stream_t stream);
+
 /* attn_decode without a caller-provided workspace. The paper has no counterpart to this entry
  * point: it exists for callers that cannot allocate device memory, such as a plugin whose host
  * application owns all device memory through its own allocator, or a serving loop that forbids

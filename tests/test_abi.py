@@ -214,3 +214,17 @@ def test_fused_activation_validation():
     assert pre(None) == ARG
     assert pre(ctypes.byref(good), dtype=hmd.F32) == UNSUP   # fused only on the tensor-core path
     assert pre(ctypes.byref(good), dk=64) == UNSUP
+
+
+def test_prefill_with_prefix_validation():
+    L = hmd.lib()
+    ext = lambda d=128, max_prefix=128, max_pages=8, T=64, kind=hmd.FA, w=0, pre=FAKE: (  # noqa: E731
+        L.attn_prefill_ext(kind, w, 2, T, 8, 2, d, 64, FAKE, FAKE, FAKE, pre, max_prefix, FAKE,
+                           FAKE, 16, FAKE, max_pages, FAKE, None))
+    assert ext(d=64) == UNSUP                  # a prefix needs the tensor-core kernel (d = 128)
+    assert ext(d=64, pre=None) != UNSUP        # no prefix: the d = 64 kernel is fine
+    assert ext(max_prefix=100) == SHAPE        # not a whole number of pages
+    assert ext(max_prefix=512, max_pages=8) == SHAPE  # FA table < (512 + 64) / 64 = 9 pages
+    assert ext(max_prefix=448, max_pages=8) != SHAPE
+    assert ext(max_prefix=-64) == SHAPE
+    assert ext(T=0) == 0

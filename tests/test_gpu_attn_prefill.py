@@ -131,3 +131,92 @@ def test_full_size_sampled_rows(oracle_mod, kind, window):
     ek, ev = expected_pools(O, a)
     np.testing.assert_array_equal(_bits_host(kp), ek)
     np.testing.assert_array_equal(_bits_host(vp), ev)
+
+
+# ---- prefill after a cached prefix (chunked prefill) ----------------------------------------
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_prefill_ext(a: I.AttnVerifyInputs, T):
+    """attn_prefill_ext of the T tokens in a (q, new_k, new_v as the prompt) after prefixes of
+    seq_lens - T positions, on device copies of a's pools."""
+    kp, vp = _bits_dev(a.k_pool), _bits_dev(a.v_pool)
+    o = torch.empty(a.B, T, a.Hq, a.d, dtype=torch.bfloat16, device="cuda")
+    pre = (a.seq_lens - T).astype(np.int32)
+    hmd.attn_prefill_ext(a.kind, a.window, _bits_dev(a.q), _bits_dev(a.new_k), _bits_dev(a.new_v),
+                         torch.from_numpy(pre).cuda(), int(pre.max()), kp, vp,
+                         torch.from_numpy(a.page_table).cuda(), o)
+    torch.cuda.synchronize()
+    assert hmd.hmd_device_errors(clear=True) == 0
+    return o, kp, vp
+
+
+def expected_pools_after_prefix(O, a: I.AttnVerifyInputs, T):
+    """The pools after the prompt's K/V are written: FA every position L0 + t, SWA the positions
+    its ring keeps (the last R*64 of the prompt); other slots unchanged."""
+    ek, ev = a.k_pool.copy(), a.v_pool.copy()
+    R64 = a.ring_pages * a.page_tokens
+    for b in range(a.B):
+        L0 = int(a.seq_lens[b]) - T
+        for t in range(T):
+            if a.kind == I.SWA and t < T - R64:
+                continue
+            pg, off = O.kv_slot_ring(a.kind, a.ring_pages, a.page_tokens, a.page_table[b], L0 + t)
+            ek[pg, :, off], ev[pg, :, off] = a.new_k[b, t], a.new_v[b, t]
+    return ek, ev
+
+
+PREFIX_CASES = [  # kind, window, T, Hq, Hkv, prefix lengths (multiples of 64)
+    (I.FA, 0, 200, 8, 2, [0, 64, 640]),
+    (I.FA, 0, 1, 8, 2, [128, 0, 64]),
+    (I.FA, 0, 130, 8, 8, [64, 192]),      # G = 1
+    (I.FA, 0, 70, 16, 1, [256, 64]),      # G = 16
+    (I.SWA, 100, 150, 8, 2, [0, 64, 640]),  # ring of 2 pages, prompt longer than the ring
+    (I.SWA, 64, 40, 8, 2, [128, 64]),
+    (I.SWA, 300, 500, 32, 8, [320, 1024]),
+]
+
+
+@pytest.mark.parametrize("kind,window,T,Hq,Hkv,prefixes", PREFIX_CASES)
+def test_prefill_after_prefix_matches_oracle(oracle_mod, kind, window, T, Hq, Hkv, prefixes):
+    O = oracle_mod
+    pre = np.array(prefixes, np.int32)
+    lens = pre + T
+    ring = -(-window // 64) if kind == I.SWA else 0
+    a = I.verify_inputs(kind, len(pre), T, Hq, Hkv, 128, int(lens.max()), window=window,
+                        ring_pages=ring, seed=int(lens.sum()) + T, seq_lens=lens)
+    o, kp, vp = run_prefill_ext(a, T)
+    ref = O.attn_verify(kind, window, a.ring_pages, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool,
+                        a.page_table, a.seq_lens)
+    assert O.rel_err(o.float().cpu().numpy(), ref) < 2e-2
+    ek, ev = expected_pools_after_prefix(O, a, T)
+    np.testing.assert_array_equal(_bits(kp), ek)
+    np.testing.assert_array_equal(_bits(vp), ev)
+
+
+@pytest.mark.parametrize("kind,window", [(I.FA, 0), (I.SWA, 200)])
+def test_two_chunks_equal_one_prefill(oracle_mod, kind, window):
+    """A prompt prefilled as 256 tokens, then 190 more after that cached prefix, gives the second
+    chunk the rows of the oracle's prefill over all 446 tokens."""
+    O = oracle_mod
+    B, T1, T2, Hq, Hkv, d = 2, 256, 190, 8, 2, 128
+    full = I.attn_prefill_inputs(kind, B, T1 + T2, Hq, Hkv, d, window=window, seed=91)
+    head = I.AttnPrefillInputs(kind, window, B, T1, Hq, Hkv, d, 64, full.q[:, :T1],
+                               full.k[:, :T1], full.v[:, :T1], full.page_table, full.n_pages)
+    _, kp, vp = run_prefill(head)
+    o2 = torch.empty(B, T2, Hq, d, dtype=torch.bfloat16, device="cuda")
+    hmd.attn_prefill_ext(kind, window, _bits_dev(full.q[:, T1:]), _bits_dev(full.k[:, T1:]),
+                         _bits_dev(full.v[:, T1:]), torch.full((B,), T1, dtype=torch.int32,
+                                                               device="cuda"),
+                         T1, kp, vp, torch.from_numpy(full.page_table).cuda(), o2)
+    torch.cuda.synchronize()
+    assert hmd.hmd_device_errors(clear=True) == 0
+    ref = O.attn_prefill(kind, window, O.bf16_bits_to_f64(full.q), O.bf16_bits_to_f64(full.k),
+                         O.bf16_bits_to_f64(full.v))
+    assert O.rel_err(o2.float().cpu().numpy(), ref[:, T1:]) < 2e-2
+    # and the cache then holds what one prefill of all 446 tokens leaves
+    ek, ev = expected_pools(O, full)
+    np.testing.assert_array_equal(_bits_host(kp), ek)
+    np.testing.assert_array_equal(_bits_host(vp), ev)
