@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     }
 }
 
-// 2-D tiled TMA load of one box into shared memory, completing on `bar` (no multicast).
+// 2-D tiled TMA load of one box into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int x,
                                             int y) {
     asm volatile(
@@ -77,7 +77,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
-// 3-D tiled TMA load of one box into shared memory, completing on `bar` (no multicast).
+// 3-D tiled TMA load of one box into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint32_t bar, int x,
                                             int y, int z) {
     asm volatile(
@@ -223,7 +223,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
-// 4-D tiled TMA load (no multicast).
+// 4-D tiled TMA load of one box into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint32_t bar, int c0,
                                             int c1, int c2, int c3) {
     asm volatile(
