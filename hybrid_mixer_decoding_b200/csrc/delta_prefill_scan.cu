@@ -71,7 +71,7 @@ constexpr uint32_t A_YS = 100352;      // Y fp32 [3][16][20]
 constexpr uint32_t A_UT = 65536;       // at the end: Ut^T bf16 (record layout, 16 KiB)
 constexpr uint32_t A_SMALL = 104192;
 constexpr uint32_t S_BETA = 0, S_QOFF = 256, S_LGP = 1280, S_WSUM = 1536, S_EGC = 1552,
-                   S_BAR = 2064, S_TMEM = 2080, S_SIZE = 2112;
+                   S_BAR = 2064, S_TMEM = 2080, S_NRM = 2112, S_SIZE = 2624;
 constexpr uint32_t A_SMEM = A_SMALL + S_SIZE + 1024;
 constexpr uint32_t A_T = A_KQ + 8192;  // T bf16 [64][64]: the Qt rows of the first half
 constexpr int AS_LD = 68;
@@ -197,6 +197,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     float *lgp = reinterpret_cast<float *>(sm + A_SMALL + S_LGP);     // [64] GDN log-gate prefix
     float *wsum = reinterpret_cast<float *>(sm + A_SMALL + S_WSUM);   // [2]
     float *egc = reinterpret_cast<float *>(sm + A_SMALL + S_EGC);     // [128] e^{G_C}
+    float *nrm = reinterpret_cast<float *>(sm + A_SMALL + S_NRM);     // [2][64] 1/|q|, 1/|k|
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + A_SMALL + S_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + A_SMALL + S_TMEM);
 
@@ -290,6 +291,31 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
     // ---- gate prefix G (log domain): KDA per channel in place within NQ row parts, plus the
     //      parts' exclusive prefix; GDN per token -------------------------------------------------
+    if (fused) {  // 1/|q| and 1/|k| of each row: 4 threads per row, 32 channels each
+        static_assert(NT == 4 * kC, "four threads per row");
+        const int r = tid >> 2, qq = tid & 3;
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int c0 = qq * 32 + c4 * 8;
+            const uint4 qv = *reinterpret_cast<const uint4 *>(sm + A_KQ + toff(64 + r, c0, 128));
+            const uint4 kv = *reinterpret_cast<const uint4 *>(sm + A_KH + toff(r, c0, 64));
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sq += bf16_lo(qw[e]) * bf16_lo(qw[e]) + bf16_hi(qw[e]) * bf16_hi(qw[e]);
+                sk += bf16_lo(kw[e]) * bf16_lo(kw[e]) + bf16_hi(kw[e]) * bf16_hi(kw[e]);
+            }
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+        if (qq == 0) {
+            nrm[r] = rsqrtf(sq + a.act.eps);
+            nrm[kC + r] = rsqrtf(sk + a.act.eps);
+        }
+    }
     if constexpr (KDA) {
         if (fused) {  // log-gates from the staged logits, in place, 4 channels per item
             const float *db = a.act.dt_bias + (size_t)h * kD;
@@ -360,23 +386,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             }
             const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w};
             const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
-            float fq = 1.f, fk = 1.f;  // L2 normalisation of the row (fused activations)
-            if (fused) {
-                float sq = 0.f, sk = 0.f;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    sq += bf16_lo(qw[e]) * bf16_lo(qw[e]) + bf16_hi(qw[e]) * bf16_hi(qw[e]);
-                    sk += bf16_lo(kw[e]) * bf16_lo(kw[e]) + bf16_hi(kw[e]) * bf16_hi(kw[e]);
-                }
-                // the row's 16 chunks of 8 channels sit in 16 consecutive lanes
-#pragma unroll
-                for (int off = 1; off < 16; off <<= 1) {
-                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
-                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
-                }
-                fq = rsqrtf(sq + a.act.eps);
-                fk = rsqrtf(sk + a.act.eps);
-            }
+            const float fq = fused ? nrm[r] : 1.f, fk = fused ? nrm[kC + r] : 1.f;
             uint32_t kt[4], qt[4], kh[4], kcw[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
