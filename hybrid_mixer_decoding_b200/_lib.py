@@ -72,6 +72,7 @@ _SIGS = {
                                                                 _c_int, _vp, _vp]),
     "state_cache_alloc": (_c_int, [_c_int] * 5 + [_vp, ctypes.POINTER(_vp)]),
     "state_cache_free": (_c_int, [_vp, _vp]),
+    "state_cache_save": (_c_int, [_vp, _c_int, _vp, _c_int, _vp, _vp]),
     "state_cache_layer": (_c_int, [_vp, _c_int, ctypes.POINTER(_vp)]),
     "state_cache_reset": (_c_int, [_vp, _c_int, _vp, _c_int, _vp, _vp]),
     "kv_cache_alloc": (_c_int, [_c_int, _vp] + [_c_int] * 5 + [_vp, ctypes.POINTER(_vp)]),
@@ -359,6 +360,12 @@ class StateCache:
         _check("state_cache_reset", lib().state_cache_reset(self.handle, layer, ids,
                                                             len(slot_ids), _p(init),
                                                             _stream(stream)))
+
+    def save(self, layer, slot_ids, out, stream=None):
+        """state_cache_save: copy the listed slots of one layer into out [n,H,dk,dv] fp32."""
+        ids = (ctypes.c_int32 * len(slot_ids))(*[int(x) for x in slot_ids])
+        _check("state_cache_save", lib().state_cache_save(self.handle, layer, ids, len(slot_ids),
+                                                          _p(out), _stream(stream)))
 
     def free(self, stream=None):
         if self.handle:

@@ -529,6 +529,23 @@ hmd_status_t state_cache_reset(hmd_state_cache_t *c, int layer, const int32_t *s
     return HMD_OK;
 }
 
+hmd_status_t state_cache_save(hmd_state_cache_t *c, int layer, const int32_t *slot_ids, int n,
+                              float *out, hmd_stream_t stream) {
+    if (!c || (n > 0 && (!slot_ids || !out))) return fail(HMD_ERR_ARG);
+    if (layer < 0 || layer >= c->n_layers || n < 0) return fail(HMD_ERR_ARG);
+    for (int i = 0; i < n; ++i)
+        if (slot_ids[i] < 0 || slot_ids[i] >= c->slots) return fail(HMD_ERR_ARG);
+    const size_t per = (size_t)c->H * c->dk * c->dv;
+    const float *blk = c->base + c->layer_elems * layer;
+    cudaStream_t s = as_stream(stream);
+    for (int i = 0; i < n; ++i) {  // one device-to-device copy per slot
+        if (cudaMemcpyAsync(out + per * i, blk + per * slot_ids[i], per * sizeof(float),
+                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return fail(HMD_ERR_CUDA);
+    }
+    return HMD_OK;
+}
+
 hmd_status_t kv_cache_alloc(int n_layers, const int32_t *layer_pool, int n_pools, int n_pages,
                             int Hkv, int d, int page_tokens, hmd_stream_t stream,
                             hmd_kv_cache_t **out) {

@@ -327,6 +327,12 @@ HMD_API hmd_status_t state_cache_alloc(int n_layers, int slots, int H, int dk, i
 HMD_API hmd_status_t state_cache_free(hmd_state_cache_t *cache, hmd_stream_t stream);
 /* Device pointer of layer `layer`'s [slots][H][dk][dv] block.                                 */
 HMD_API hmd_status_t state_cache_layer(hmd_state_cache_t *cache, int layer, float **out);
+/* Copy n slots (host array `slot_ids`) of one layer out to `out` [n][H][dk][dv] fp32 (device),
+ * asynchronously on `stream`: a request's recurrent state set aside (preemption, or a
+ * checkpoint of a long prompt), to come back with state_cache_reset(..., init = out).
+ * HMD_ERR_ARG for a bad layer, slot or null pointer.                                          */
+HMD_API hmd_status_t state_cache_save(hmd_state_cache_t *cache, int layer, const int32_t *slot_ids,
+                                      int n, float *out, hmd_stream_t stream);
 /* Reset n slots (host array `slot_ids`) of one layer to zero, or to init [n][H][dk][dv] fp32
  * (device) when init is not NULL.                                                            */
 HMD_API hmd_status_t state_cache_reset(hmd_state_cache_t *cache, int layer, const int32_t *slot_ids,

@@ -228,3 +228,9 @@ def test_prefill_with_prefix_validation():
     assert ext(max_prefix=448, max_pages=8) != SHAPE
     assert ext(max_prefix=-64) == SHAPE
     assert ext(T=0) == 0
+
+
+def test_state_cache_save_validation():
+    L = hmd.lib()
+    ids = (ctypes.c_int32 * 1)(0)
+    assert L.state_cache_save(None, 0, ids, 1, FAKE, None) == ARG

@@ -222,3 +222,23 @@ def test_chain_launch_equals_steps_and_oracle(oracle_mod, kind, dtype):
                                      d.beta[:, :t + 1], d.log_gate[:, :t + 1], d.state0)
         got = st1[torch.from_numpy(chain[t + 1]).long().cuda()].cpu().numpy()
         assert O.rel_err(got, s_ref) < TOL[dtype]
+
+
+def test_state_cache_save_and_restore_round_trip():
+    """state_cache_save copies slots out bit for bit; state_cache_reset(init=...) puts them back
+    (a preempted request's recurrent state set aside and restored)."""
+    sc = hmd.StateCache(2, 5, 3, 64, 32)
+    view = sc.layer_view(1)
+    view.normal_()
+    orig = view.clone()
+    out = torch.empty(2, 3, 64, 32, device="cuda")
+    sc.save(1, [3, 0], out)
+    torch.cuda.synchronize()
+    assert torch.equal(out[0], orig[3]) and torch.equal(out[1], orig[0])
+    sc.reset(1, [3, 0])
+    torch.cuda.synchronize()
+    assert not view[3].any() and not view[0].any()
+    sc.reset(1, [3, 0], init=out)
+    torch.cuda.synchronize()
+    assert torch.equal(view, orig)
+    sc.free()
