@@ -234,3 +234,37 @@ def test_state_cache_save_validation():
     L = hmd.lib()
     ids = (ctypes.c_int32 * 1)(0)
     assert L.state_cache_save(None, 0, ids, 1, FAKE, None) == ARG
+
+
+def test_header_is_c99_and_links_from_c(tmp_path):
+    """include/hmd.h compiles as strict C99, and a C program links against libhmd.so and calls
+    it (host-side calls only: version string, status strings, argument validation)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_hmd.c"
+    src.write_text(r"""
+#include "hmd.h"
+#include <stdio.h>
+#include <string.h>
+int main(void) {
+    if (strncmp(hmd_version(), "hmd", 3) != 0) return 1;
+    if (strcmp(hmd_status_string(HMD_OK), "ok") != 0) return 2;
+    /* a bad kind is rejected on the host, before any device work */
+    if (delta_rule_decode((hmd_kind_t)7, 1, 1, 64, 64, HMD_BF16, 0, 0, 0, 0, 0, 0, 1, 0, 0, 1.f,
+                          0) != HMD_ERR_ARG) return 3;
+    if (hmd_last_error() != HMD_ERR_ARG) return 4;
+    printf("ok\n");
+    return 0;
+}
+""")
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "use_hmd"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lhmd",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == "ok"
