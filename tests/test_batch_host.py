@@ -54,3 +54,28 @@ def test_grouping_rejects_bad_arguments():
     assert call(pl, np.array([-1, 0], np.int32)) == ARG
     assert call(pl, sp, B=0) == ARG
     assert L.mixer_decode_step_batch(None, 0, None, None, None, None, 0, None) == ARG
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.data())
+def test_grouping_properties(data):
+    """For any placements and assignment: each layer's rows are a permutation of the batch,
+    grouped by kind in FA, SWA, KDA, GDN order, increasing within a group, and each row sits
+    in the group of the kind its placement picks at that layer."""
+    n_p = data.draw(st.integers(1, 5))
+    n_l = data.draw(st.integers(1, 12))
+    B = data.draw(st.integers(1, 40))
+    pl = np.array(data.draw(st.lists(st.lists(st.integers(0, 3), min_size=n_l, max_size=n_l),
+                                     min_size=n_p, max_size=n_p)), np.int8)
+    sp = np.array(data.draw(st.lists(st.integers(0, n_p - 1), min_size=B, max_size=B)), np.int32)
+    rows, offs = hmd.group_sequences(pl, sp)
+    for l in range(n_l):
+        assert sorted(rows[l]) == list(range(B))
+        assert list(offs[l]) == sorted(offs[l]) and offs[l, 0] == 0 and offs[l, 4] == B
+        for k in range(4):
+            grp = rows[l, offs[l, k]:offs[l, k + 1]]
+            assert list(grp) == sorted(grp)
+            assert all(pl[sp[b], l] == k for b in grp)

@@ -42,3 +42,23 @@ def test_schedule_keeps_the_accepted_slot_and_length():
             assert (sch.slots[r + 1][0] == nxt).all()
         L = L + j + 1
     assert sch.slots.min() >= 0 and sch.slots.max() < B * (k + 2)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 20), k=st.integers(1, 6), rounds=st.integers(1, 15),
+       alpha=st.floats(0.0, 1.0), seed=st.integers(0, 1000))
+def test_schedule_properties(B, k, rounds, alpha, seed):
+    sch = make_schedule(B, k, rounds, 100, alpha, seed=seed)
+    assert ((sch.accepted >= 0) & (sch.accepted <= k)).all()
+    assert sch.slots.min() >= 0 and sch.slots.max() < B * (k + 2)
+    for r in range(rounds):
+        for b in range(B):  # a sequence's chain never leaves its own k + 2 slots
+            assert set(sch.slots[r, :, b]) == set(range(b * (k + 2), (b + 1) * (k + 2)))
+    # lengths grow by exactly the tokens each round produced
+    grow = (sch.accepted + 1).cumsum(axis=0)
+    assert (sch.lens[1:] - sch.lens[:-1] == sch.accepted[:-1] + 1).all()
+    if rounds > 1:
+        assert (sch.lens[-1] - sch.lens[0] == grow[-2]).all()
