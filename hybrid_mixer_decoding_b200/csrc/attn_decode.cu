@@ -463,12 +463,9 @@ template <int D>
 cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t s) {
     const int group = a.Hq / a.Hkv;
     constexpr int smem = smem_bytes<D>();
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_split_kernel<D>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        smem_bytes<D>());
+    const cudaError_t attr_err = once_per_device([] {
+        return cudaFuncSetAttribute(attn_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    smem_bytes<D>());
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap tmk, tmv;
@@ -505,19 +502,14 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
 
 // SMs of the current device (148 when no device can be queried).
 int device_sms() {
-    static int n = 0;
-    static std::once_flag once;
-    std::call_once(once, [] {
+    return once_per_device([] {
         int dev = 0, v = 0;
         if (cudaGetDevice(&dev) == cudaSuccess &&
             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-            n = v;
-        else {
-            cudaGetLastError();
-            n = 148;
-        }
+            return v;
+        cudaGetLastError();
+        return 148;
     });
-    return n;
 }
 
 }  // namespace

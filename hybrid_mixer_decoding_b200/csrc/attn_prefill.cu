@@ -334,11 +334,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_consta
 template <int D>
 cudaError_t launch_d(const AttnPrefillArgs &a, cudaStream_t s) {
     constexpr int smem = smem_bytes<D>();
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_prefill_kernel<D>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const cudaError_t attr_err = once_per_device([] {
+        return cudaFuncSetAttribute(attn_prefill_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap tmk, tmv;

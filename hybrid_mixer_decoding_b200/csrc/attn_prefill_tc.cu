@@ -489,15 +489,14 @@ bool attn_prefill_tc_supported(int d, int page_tokens, int group) {
 
 cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(attn_prefill_tc_kernel<false>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(attn_prefill_tc_kernel<true>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)SMEM_BYTES);
+    const cudaError_t attr_err = once_per_device([] {
+        cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(attn_prefill_tc_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        return e;
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap tmk, tmv, tmpk, tmpv;

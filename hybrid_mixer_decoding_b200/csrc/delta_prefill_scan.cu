@@ -759,7 +759,7 @@ size_t delta_prefill_scan_record_bytes() { return REC_BYTES; }
 
 cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_t ws_bytes,
                                       cudaStream_t s) {
-    static cudaError_t attr = [] {
+    const cudaError_t attr = once_per_device([] {
         cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel<true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A_SMEM);
         if (e == cudaSuccess)
@@ -769,7 +769,7 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
             e = cudaFuncSetAttribute(prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)B_SMEM);
         return e;
-    }();
+    });
     if (attr != cudaSuccess) return attr;
     const long long bhs = (long long)a.B * a.H;
     const int n_chunks = (a.T + kC - 1) / kC;

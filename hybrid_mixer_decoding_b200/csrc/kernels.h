@@ -6,9 +6,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
 
 namespace hmd {
+
+// Runs f() once for each device it is called on (the current device) and returns that first
+// result on every later call there. Kernel attributes (the dynamic shared-memory limit) and
+// device properties belong to one device, so a process that drives several GPUs sets and reads
+// them per device.
+constexpr int kMaxDevices = 64;
+template <typename F>
+auto once_per_device(F f) -> decltype(f()) {
+    static std::once_flag flags[kMaxDevices];
+    static decltype(f()) results[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        dev = 0;
+    }
+    std::call_once(flags[dev], [&] { results[dev] = f(); });
+    return results[dev];
+}
 
 // Launches `kernel` on stream s with programmatic stream serialisation: it may be scheduled
 // while the previous kernel in the stream drains, and waits for it (griddep_wait) before its
