@@ -364,11 +364,16 @@ def cpu_baseline(shape, pl, budget_s=15.0, n_seq=2):
                 break
         per_kind[kind] = float(np.median(ts))
     step_s = sum(per_kind[int(k)] for k in pl)  # one token for n_seq sequences, 48 layers
+    # the same sample on one host thread (each kind timed once), for the per-core figure
+    one = {kind: _oracle_layer_time(O, kind, _oracle_layer_inputs(kind, shape, 1, seed=kind), 1)
+           for kind in (I.FA, I.SWA, I.KDA, I.GDN)}
+    one_s = sum(one[int(k)] for k in pl)
     return {"value": round(n_seq / step_s, 4), "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "one_thread_tok_s": round(1.0 / one_s, 4),
             "sample": f"fp64 C oracle, {n_seq} sequences at the stack's per-layer shapes "
                       f"(H=32, Hkv=8, d=128, ctx 32768, w=4096); each mixer kind timed on one "
                       f"layer, summed over the placement's 48 layers; tokens/s = "
-                      f"{n_seq} / summed time",
+                      f"{n_seq} / summed time; one_thread_tok_s: one sequence on one thread",
             "per_layer_s": {I.KIND_NAMES[k]: round(v, 5) for k, v in per_kind.items()}}
 
 
