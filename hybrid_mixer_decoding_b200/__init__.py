@@ -5,7 +5,7 @@ The compute lives in libhmd.so (hand-written sm_100a CUDA kernels behind the C A
 include/hmd.h); this package is its ctypes binding plus the seeded input generator and the
 48-layer mixer-only stack driver.
 """
-from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DEVERR_PAGE, DEVERR_SEQLEN, DEVERR_SLOT, DEVERR_TIMEOUT, F32, FA, GDN,
+from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DEVERR_GATE, DEVERR_PAGE, DEVERR_SEQLEN, DEVERR_SLOT, DEVERR_TIMEOUT, F32, FA, GDN,
                    KDA, SWA, DecodeIO, HmdError, KVCache, StateCache, attn_decode,
                    attn_decode_static_ws, attn_prefill, attn_prefill_ext, attn_decode_workspace_size,
                    attn_verify,
@@ -16,7 +16,7 @@ from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DE
                    delta_rule_prefill_workspace_size, hmd_device_errors, hmd_last_error,
                    hmd_status_string, hmd_version, lib, mixer_decode_step)
 
-__all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "DEVERR_PAGE", "DEVERR_SEQLEN", "DEVERR_SLOT", "DEVERR_TIMEOUT", "F32", "FA",
+__all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "DEVERR_GATE", "DEVERR_PAGE", "DEVERR_SEQLEN", "DEVERR_SLOT", "DEVERR_TIMEOUT", "F32", "FA",
            "GDN", "KDA", "SWA", "DecodeIO", "HmdError", "KVCache", "StateCache", "attn_decode",
            "attn_decode_static_ws", "attn_decode_workspace_size", "attn_prefill", "attn_prefill_ext",
            "attn_verify",

@@ -15,7 +15,7 @@ F32, BF16 = 0, 1
 STATUS = {0: "HMD_OK", 1: "HMD_ERR_ARG", 2: "HMD_ERR_SHAPE", 3: "HMD_ERR_DTYPE",
           4: "HMD_ERR_OOM", 5: "HMD_ERR_CUDA", 6: "HMD_ERR_UNSUPPORTED",
           7: "HMD_ERR_DEVICE_CHECK"}
-DEVERR_TIMEOUT, DEVERR_PAGE, DEVERR_SLOT, DEVERR_SEQLEN = 0x1, 0x2, 0x4, 0x8
+DEVERR_TIMEOUT, DEVERR_PAGE, DEVERR_SLOT, DEVERR_SEQLEN, DEVERR_GATE = 0x1, 0x2, 0x4, 0x8, 0x10
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhmd.so")
 _lib = None

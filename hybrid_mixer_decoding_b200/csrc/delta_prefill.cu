@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
             }
             gl[i] = g;
             egl[i] = expf(g);
+            if (g < kPrefillGateFloor) atomicOr(&g_err, HMD_DEVERR_GATE);
         }
         for (int idx = tid; idx < kC * dvs; idx += kThreads) {
             const int r = idx / dvs, jj = idx % dvs;

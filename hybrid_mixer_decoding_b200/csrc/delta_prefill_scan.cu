@@ -353,11 +353,13 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                 acc += part;
             }
             egc[i] = __expf(acc);
+            if (acc < kPrefillGateFloor) atomicOr(&g_err, HMD_DEVERR_GATE);
         }
     } else {
         if (tid < kC) lgp[tid] += (warp == 1 ? wsum[0] : 0.f);
         __syncthreads();
         if (tid < kD) egc[tid] = __expf(lgp[kC - 1]);
+        if (tid == 0 && lgp[kC - 1] < kPrefillGateFloor) atomicOr(&g_err, HMD_DEVERR_GATE);
     }
     __syncthreads();
 

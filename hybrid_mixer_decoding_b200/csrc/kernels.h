@@ -11,6 +11,11 @@
 
 namespace hmd {
 
+// Lowest cumulative log-gate inside one chunk that the chunked prefill accepts. Its chunk form
+// factors e^{G_r - G_s} into k e^{G} and k e^{-G}, each of which must stay inside fp32's
+// normal range (|G| < 87); below this floor a chunk is reported with HMD_DEVERR_GATE.
+constexpr float kPrefillGateFloor = -80.f;
+
 // Runs f() once for each device it is called on (the current device) and returns that first
 // result on every later call there. Kernel attributes (the dynamic shared-memory limit) and
 // device properties belong to one device, so a process that drives several GPUs sets and reads

@@ -268,3 +268,12 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.strip() == "ok"
+
+
+def test_device_error_bits_match_the_header():
+    text = open(os.path.join(ROOT, "include", "hmd.h")).read()
+    bits = {m.group(1): int(m.group(2), 16)
+            for m in re.finditer(r"#define HMD_DEVERR_(\w+)\s+0x([0-9a-fA-F]+)u", text)}
+    assert bits == {"TIMEOUT": hmd.DEVERR_TIMEOUT, "PAGE": hmd.DEVERR_PAGE,
+                    "SLOT": hmd.DEVERR_SLOT, "SEQLEN": hmd.DEVERR_SEQLEN,
+                    "GATE": hmd.DEVERR_GATE}

@@ -153,6 +153,21 @@ def test_chunked_equals_recurrent(oracle_mod, kind, T, C):
     assert O.rel_err(s_c, s_r) < 1e-12
 
 
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_chunked_equals_recurrent_under_strong_decay(oracle_mod, kind):
+    # log-gates down to -20 per token: over a chunk of 64 the cumulative gate reaches about
+    # -640, so e^{G} and e^{-G} formed separately would underflow / overflow in fp64
+    # (e^{+-709} is the limit); the chunked form must still equal the recurrence
+    O = oracle_mod
+    d = I.delta_inputs(kind, 1, 150, 2, 16, 8, dtype="f32", seed=31, gate_lo=-20.0,
+                       state0="randn")
+    o_r, s_r = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    o_c, s_c = O.delta_chunked(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0, chunk=64)
+    assert np.isfinite(o_c).all() and np.isfinite(s_c).all()
+    assert O.rel_err(o_c, o_r) < 1e-12
+    assert O.rel_err(s_c, s_r) < 1e-12
+
+
 def test_oracle_thread_count_invariance(oracle_mod):
     O = oracle_mod
     d = I.delta_inputs(I.KDA, 2, 30, 4, 8, 8, dtype="f32", seed=8, state0="randn")
