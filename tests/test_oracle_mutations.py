@@ -32,6 +32,11 @@ MUTANTS = [
                                    "for (int s = 1; s < r; ++s) x -=")]),
     ("chunk_P_excludes_diagonal", [("(s <= r) ? p : 0.0", "(s < r) ? p : 0.0")]),
     ("chunk_state_decay_missing", [("double acc = exp(gC) * M[", "double acc = M[")]),
+    ("chunk_decay_split_into_factors", [
+        ("const double e = exp(G[(size_t)r * dk + i] - G[(size_t)s * dk + i]);",
+         "const double e = exp(G[(size_t)r * dk + i]) * exp(-G[(size_t)s * dk + i]);")]),
+    ("chunk_state_factor_split", [("* exp(gC - G[(size_t)s * dk + i]) *",
+                                   "* exp(gC) * exp(-G[(size_t)s * dk + i]) *")]),
     ("attn_scale_missing", [("s[j - lo] = acc * inv_sqrt_d;", "s[j - lo] = acc;")]),
     ("swa_window_off_by_one", [("? L - window : 0", "? L - window + 1 : 0")]),
     ("gqa_map_interleaved", [("g = h / group", "g = h % Hkv")]),
