@@ -15,6 +15,17 @@ Multi-GPU (torchrun): replicas only -- every rank runs its own copy of the workl
 caches (weak scaling, no collective on the data path); value = all ranks' tokens / the slowest
 rank's time.
 
+The headline is timed as K CUDA-graph replays of the 48-layer step with nothing else on the
+stream. At one GPU the line also carries, each measured after the headline:
+  per_mixer          each mixer's layer time inside the stack (a separate pass with events
+                     around every layer) and its fraction of the HBM roofline;
+  placement_switch   the first step after a placement switch against a steady step;
+  prefill, decode    tokens/s of each mixer at its own configuration (KDA/GDN prefill B=4,
+                     H=16, T=4096; FA/SWA prefill B=2, T=8192; KDA/GDN decode B=64, H=32;
+                     FA/SWA decode B=32, ctx 8192), each with its roofline and the fp64
+                     oracle's tokens/s on a bounded sample of the same work on the host's cores;
+  oracle_check       the fp32 GDN configuration (B=1, H=2, d=64, T=128) against the oracle.
+
 --impl reference times the fp64 CPU oracle (the only other implementation of the method) on a
 bounded sample of the same workload on this host's cores.
 """
@@ -183,7 +194,9 @@ def run_ours(args, rank, world, local_rank):
     cfg = WORKLOADS["stack48"]
     shape = StackShape(cfg["B"], cfg["H"], cfg["Hkv"], cfg["d"], cfg["ctx"], cfg["window"])
     pl = stack_placement()
-    st = MixerStack({"hybrid": pl}, shape, seed=0, io_sets=2)
+    # a second placement on the same caches (every layer as GDN), for the switch latency
+    st = MixerStack({"hybrid": pl, "all_gdn": np.full(len(pl), I.GDN, np.int8)}, shape, seed=0,
+                    io_sets=2)
 
     def barrier():
         if dist is not None:
@@ -193,29 +206,39 @@ def run_ours(args, rank, world, local_rank):
         st.step("hybrid")
     torch.cuda.synchronize()
     assert hmd.hmd_device_errors(clear=True) == 0
+    # one step = one CUDA-graph replay of the 48 mixer_decode_step calls (per io set)
+    graphs = [st.capture(lambda b_=b_: st.step("hybrid", io_set=b_), warmup=1) for b_ in range(2)]
+    for _ in range(args.warmup):
+        graphs[0].replay()
+    torch.cuda.synchronize()
 
-    # per-layer events for every layer (cheap: two event records per layer)
-    n_layers = st.n_layers
-    evs = [{l: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for l in range(n_layers)} for _ in range(args.steps)]
+    # ---- the timed region: K replays, nothing else on the stream ----------------------------
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
     clk.start()
     t0.record()
-    for k in range(args.steps):
-        st.step("hybrid", events=evs[k])
+    for _ in range(args.steps):
+        graphs[0].replay()
     t1.record()
     torch.cuda.synchronize()
     barrier()
     clocks = clk.stop()
+    assert hmd.hmd_device_errors(clear=True) == 0
     ms = max_over_ranks(t0.elapsed_time(t1), dist, "cuda")
     ms_per_step = ms / args.steps
     tokens = shape.B * args.steps * world
     value = job_throughput(shape.B * args.steps, world, ms)
 
-    # per-mixer achieved bandwidth from the per-layer events
+    # ---- per-mixer figures: a separate pass with events around every layer --------------------
+    n_layers = st.n_layers
+    n_pass = max(3, min(args.steps, 8))
+    evs = [{l: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for l in range(n_layers)} for _ in range(n_pass)]
+    for k in range(n_pass):
+        st.step("hybrid", events=evs[k])
+    torch.cuda.synchronize()
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     per_kind = {}
@@ -223,24 +246,31 @@ def run_ours(args, rank, world, local_rank):
         layers = [l for l in range(n_layers) if pl[l] == kind]
         if not layers:
             continue
-        durs = [evs[k][l][0].elapsed_time(evs[k][l][1]) for k in range(args.steps) for l in layers]
+        durs = [evs[k][l][0].elapsed_time(evs[k][l][1]) for k in range(n_pass) for l in layers]
         mean_ms = float(np.mean(durs))
         gbs = layer_bytes(kind, shape) / (mean_ms * 1e-3) / 1e9
         per_kind[I.KIND_NAMES[kind]] = {"layer_us": round(mean_ms * 1e3, 2),
                                         "achieved_gbs": round(gbs, 1),
                                         "frac": round(gbs / hbm, 4),
                                         "frac_nominal_8tbs": round(gbs / 8000.0, 4),
-                                        "bytes_per_layer": layer_bytes(kind, shape)}
+                                        "bytes_per_layer": layer_bytes(kind, shape),
+                                        "decode_tok_s_per_layer": round(shape.B / (mean_ms * 1e-3), 1)}
+    per_kind["measured"] = (f"separate pass after the timed region: {n_pass} eager steps with CUDA "
+                            f"events around each of the 48 layers on the launching stream")
     dom = per_kind["FA"]
     roofline = {"bound": "hbm", "achieved": dom["achieved_gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": dom["frac"], "traffic": traffic_for("attn_fa_stack48"),
                 "kernel": "attn_decode FA layer (attn_split_kernel<128> + attn_combine_kernel)",
-                "peak_source": pk_kind}
+                "peak_source": pk_kind,
+                "algorithmic_bytes_per_launch": dom["bytes_per_layer"],
+                "timing": "per-layer CUDA events of the per-mixer pass"}
+    switch = placement_switch(st, args.warmup)
     assert hmd.hmd_device_errors(clear=True) == 0
 
-    # end to end through the C ABI from pinned host buffers. Every step copies that step's
-    # inputs host->device and reads every layer's output device->host. A copy stream moves the
-    # next step's inputs into the other buffer set while the current step computes, and drains
+    # ---- end to end through the C ABI from pinned host buffers ----------------------------
+    # Every step copies that step's inputs host->device and reads every layer's output
+    # device->host. A copy stream moves the next step's inputs into the other buffer set while
+    # the current step computes (one graph replay of the 48 C-ABI calls on that set), and drains
     # the current step's outputs once it is done (events order every reuse of a buffer).
     host_in, dev_in, dev_out = [], [[], []], [[], []]
     for l in range(n_layers):
@@ -271,7 +301,7 @@ def run_ours(args, rank, world, local_rank):
         for k in range(n_steps):
             b_ = k % 2
             comp.wait_event(ev_in[b_])
-            st.step("hybrid", io_set=b_)
+            graphs[b_].replay()
             ev_done[b_].record(comp)
             with torch.cuda.stream(copy):
                 if k + 1 < n_steps:
@@ -294,9 +324,13 @@ def run_ours(args, rank, world, local_rank):
     e2e_run(args.steps, e0, e1)
     torch.cuda.synchronize()
     barrier()
+    assert hmd.hmd_device_errors(clear=True) == 0
     ems = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     e2e = {"value": round(tokens / (ems * 1e-3), 2), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h}
+           "d2h_bytes_per_step": d2h,
+           "how": "per step: pinned host inputs -> device, one graph replay of the 48 C-ABI "
+                  "calls, every layer's output -> pinned host; copies overlap the other buffer "
+                  "set's step"}
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "tok/s", "n_gpus": world,
@@ -308,20 +342,63 @@ def run_ours(args, rank, world, local_rank):
                                "Hkv=8, d=128, bf16 act/KV, fp32 state",
                    "global_batch": shape.B * world, "seq_len": shape.ctx,
                    "parallelism": f"replicas x{world}",
+                   "timed": "K CUDA-graph replays of the 48-layer step, no other work on the "
+                            "stream",
                    "l2": "working set per step ~122 GB >> L2 (126 MB); no flush",
                    "aliased_kv": st.aliased},
         "roofline": with_nominal(roofline),
         "per_mixer": per_kind,
+        "placement_switch": switch,
         "e2e": e2e,
         "gpu_launches": st.launches_per_step("hybrid") * args.steps,
         "clocks": clocks,
     }
+    del graphs
     st.free()
+    del st
+    torch.cuda.empty_cache()
     if rank == 0 and not args.skip_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(shape, pl, budget_s=args.cpu_budget)
     if dist is not None:
         dist.destroy_process_group()
     return out
+
+
+def placement_switch(st, warmup: int) -> dict:
+    """Latency of a placement switch on a registered stack: eager steps with CUDA events around
+    each whole step. Steady steps of each placement, then alternating steps (each one the first
+    after a switch). A switch passes another placement array; no cache is copied or reloaded,
+    so the first step after a switch should cost what a steady step of its placement costs."""
+    import torch
+
+    def timed_steps(names):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in names]
+        for (a, b), nm in zip(evs, names):
+            a.record()
+            st.step(nm)
+            b.record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    for nm in ("hybrid", "all_gdn"):
+        for _ in range(max(1, warmup // 2)):
+            st.step(nm)
+    n = 5
+    steady_h = timed_steps(["hybrid"] * n)[1:]
+    steady_g = timed_steps(["all_gdn"] * n)[1:]
+    alt = timed_steps(["hybrid", "all_gdn"] * n)
+    to_h = alt[0::2][1:]  # every hybrid step here directly follows an all-GDN step
+    to_g = alt[1::2]
+    sh, sg = float(np.median(steady_h)), float(np.median(steady_g))
+    fh, fg = float(np.median(to_h)), float(np.median(to_g))
+    return {"steady_step_ms": {"hybrid": round(sh, 4), "all_gdn": round(sg, 4)},
+            "first_step_after_switch_ms": {"to_hybrid": round(fh, 4), "to_all_gdn": round(fg, 4)},
+            "switch_cost_us": {"to_hybrid": round((fh - sh) * 1e3, 1),
+                               "to_all_gdn": round((fg - sg) * 1e3, 1)},
+            "how": "medians of eager steps timed with CUDA events; a switch passes another "
+                   "placement array to mixer_decode_step (the caches of both placements stay "
+                   "registered: nothing is copied or reloaded)"}
 
 
 # ------------------------------------------------------------------------------------------
@@ -434,7 +511,7 @@ def _events_time(fn, steps, warmup):
     return t0.elapsed_time(t1) / steps * 1e-3  # seconds per launch
 
 
-def run_kernel_workload(args):
+def measure_workload(w: str, steps: int, warmup: int) -> dict:
     """One mixer kernel at its configuration:
     attn_fa / attn_swa: B=32, Hq=32, Hkv=8, d=128, context 8192, SWA w=4096, paged bf16 KV
       (pages of 64, random page permutation), one new token per sequence;
@@ -452,7 +529,6 @@ def run_kernel_workload(args):
     bf = torch.bfloat16
     g = torch.Generator(device=dev)
     g.manual_seed(0)
-    w = args.workload
     extra = {}
     if w in ("attn_fa", "attn_swa"):
         kind = I.FA if w == "attn_fa" else I.SWA
@@ -472,7 +548,7 @@ def run_kernel_workload(args):
 
         def fn():
             hmd.attn_decode(kind, win, q, nk, nv, kp, vp, table, lens, L, o, ws)
-        sec = _events_time(fn, args.steps, args.warmup)
+        sec = _events_time(fn, steps, warmup)
         keys = L if kind == I.FA else win
         byts = B * (keys * Hkv * d * 4 + 2 * Hq * d * 2 + 2 * Hkv * d * 2)
         value, unit = B / sec, "tok/s"
@@ -503,7 +579,7 @@ def run_kernel_workload(args):
 
             def fn():
                 hmd.attn_verify(kind, win, ring, q, nk, nv, kp, vp, table, lens, L, o, ws)
-            per_nq[nq] = _events_time(fn, args.steps, args.warmup)
+            per_nq[nq] = _events_time(fn, steps, warmup)
         sec = per_nq[nq_max]
         keys = L if kind == I.FA else win + nq_max - 1
         byts = B * (keys * Hkv * d * 4 + nq_max * (2 * Hq * d * 2 + 2 * Hkv * d * 2))
@@ -532,7 +608,7 @@ def run_kernel_workload(args):
 
         def fn():
             hmd.attn_prefill(kind, win, q, k, v, kp, vp, table, o)
-        sec = _events_time(fn, args.steps, args.warmup)
+        sec = _events_time(fn, steps, warmup)
         keys = sum(min(t + 1, win) if kind == I.SWA else t + 1 for t in range(T))
         flops = 4 * d * Hq * B * keys  # S = q K^T and O = P V over the attended keys
         tf = float(pk["bf16_tflops"])
@@ -560,7 +636,7 @@ def run_kernel_workload(args):
         def fn():
             hmd.delta_rule_decode(kind, q, k, v, beta, lg, states[it[0] % 4], o)
             it[0] += 1
-        sec = _events_time(fn, args.steps, args.warmup)
+        sec = _events_time(fn, steps, warmup)
         byts = B * H * (2 * d * d * 4 + 4 * d * 2 + 4 + (4 * d if kind == I.KDA else 4))
         value, unit = B / sec, "tok/s"
         desc = f"{I.KIND_NAMES[kind]} decode step, B=64, H=32, d=128, bf16 act, fp32 state"
@@ -582,7 +658,7 @@ def run_kernel_workload(args):
 
         def fn():
             hmd.delta_rule_prefill_chunked(kind, q, k, v, beta, lg, st, o)
-        sec = _events_time(fn, args.steps, args.warmup)
+        sec = _events_time(fn, steps, warmup)
         per_tok = 768 + 256 + 4 + (512 if kind == I.KDA else 4)
         byts = B * T * H * per_tok + 2 * B * H * d * d * 4
         flops = B * T * H * (10 * 64 * d + 6 * d * d)
@@ -598,13 +674,174 @@ def run_kernel_workload(args):
     else:
         raise SystemExit(f"unknown workload {w}")
     assert hmd.hmd_device_errors(clear=True) == 0
-    out = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": 1,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 4),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic (seeded)", "config": {"workload": f"{w}: {desc}"},
-           "roofline": with_nominal(roof), "gpu_launches": launches * args.steps}
+    out = {"value": round(value, 2), "unit": unit, "ms_per_step": round(sec * 1e3, 4),
+           "workload": f"{w}: {desc}", "roofline": with_nominal(roof),
+           "launches_per_step": launches}
     out.update(extra)
     return out
+
+
+def run_kernel_workload(args):
+    """One mixer kernel at its configuration as the JSON line (see measure_workload)."""
+    m = measure_workload(args.workload, args.steps, args.warmup)
+    out = {"metric": METRIC, "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded)", "config": {"workload": m.pop("workload")},
+           "roofline": m.pop("roofline"),
+           "gpu_launches": m.pop("launches_per_step") * args.steps}
+    out.update(m)
+    if not args.skip_cpu_baseline and args.workload in ORACLE_SAMPLES:
+        out["cpu_baseline"] = workload_cpu_baseline(args.workload, args.cpu_budget / 4)
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# the oracle on a bounded sample of each per-mixer workload (reported baseline, not a target)
+# ------------------------------------------------------------------------------------------
+# workload -> (mixer, sample description); the sample's oracle time is scaled to the workload
+ORACLE_SAMPLES = {
+    "prefill_kda": (I.KDA, "sequence 0 of 4 (all 16 heads, T=4096, d=128), token by token"),
+    "prefill_gdn": (I.GDN, "sequence 0 of 4 (all 16 heads, T=4096, d=128), token by token"),
+    "prefill_fa": (I.FA, "the last 128 prompt tokens of sequence 0, kv-head group 0 (4 of 32 "
+                         "query heads) of B=2, T=8192; time scaled by the workload's attended "
+                         "query-key pairs over the sample's"),
+    "prefill_swa": (I.SWA, "the last 128 prompt tokens of sequence 0, kv-head group 0 (4 of 32 "
+                           "query heads) of B=2, T=8192, w=4096; time scaled by the workload's "
+                           "attended query-key pairs over the sample's"),
+    "decode_kda": (I.KDA, "2 of 64 sequences (all 32 heads, d=128), one token"),
+    "decode_gdn": (I.GDN, "2 of 64 sequences (all 32 heads, d=128), one token"),
+    "attn_fa": (I.FA, "2 of 32 sequences (32 query / 8 kv heads, ctx 8192), one token"),
+    "attn_swa": (I.SWA, "2 of 32 sequences (32 query / 8 kv heads, ctx 8192, w=4096), one token"),
+}
+
+
+def _repeat_time(fn, budget_s: float) -> float:
+    """Median seconds of fn() over repetitions until budget_s has passed (at least 2)."""
+    ts = []
+    t_start = time.perf_counter()
+    while len(ts) < 2 or (time.perf_counter() - t_start < budget_s and len(ts) < 50):
+        t0 = time.perf_counter()
+        fn()
+        ts.append(time.perf_counter() - t0)
+    return float(np.median(ts))
+
+
+def workload_cpu_baseline(w: str, budget_s: float = 2.0) -> dict:
+    """The fp64 oracle, as it stands, on the host's cores, on a bounded sample of workload w;
+    value in the workload's unit (tok/s)."""
+    from oracle import oracle as O
+    O.build()
+    cores = len(os.sched_getaffinity(0))
+    kind, sample = ORACLE_SAMPLES[w]
+    if w in ("prefill_kda", "prefill_gdn"):
+        T, H = 4096, 16
+        x = I.delta_inputs(kind, 1, T, H, 128, 128, dtype="bf16", seed=7)
+        sec = _repeat_time(lambda: O.delta_recurrent(kind, x.q, x.k, x.v, x.beta, x.log_gate,
+                                                     x.state0, n_threads=cores), budget_s)
+        value = T / sec  # the sample is one whole sequence of the workload
+    elif w in ("prefill_fa", "prefill_swa"):
+        T, n_q, win, Hq = 8192, 128, 4096, 4
+        window = win if kind == I.SWA else 0
+        x = I.verify_inputs(kind, 1, n_q, Hq, 1, 128, T, window=window, seed=7)
+        sec = _repeat_time(lambda: O.attn_verify(kind, window, x.ring_pages, x.q, x.new_k,
+                                                 x.new_v, x.k_pool, x.v_pool, x.page_table,
+                                                 x.seq_lens, n_threads=cores), budget_s)
+        keys = (lambda t: min(t + 1, win)) if kind == I.SWA else (lambda t: t + 1)
+        pairs_full = 2 * 32 * sum(keys(t) for t in range(T))   # B=2, Hq=32
+        pairs_sample = Hq * sum(keys(t) for t in range(T - n_q, T))
+        value = 2 * T / (sec * pairs_full / pairs_sample)
+    elif w in ("decode_kda", "decode_gdn"):
+        n = 2
+        x = I.delta_inputs(kind, n, 1, 32, 128, 128, dtype="bf16", seed=7, state0="randn")
+        sec = _repeat_time(lambda: O.delta_recurrent(kind, x.q, x.k, x.v, x.beta, x.log_gate,
+                                                     x.state0, n_threads=cores), budget_s)
+        value = n / sec
+    else:  # attn_fa, attn_swa (config 3)
+        n = 2
+        window = 4096 if kind == I.SWA else 0
+        x = I.attn_inputs(kind, n, 32, 8, 128, 8192, window=window, seed=7)
+        sec = _repeat_time(lambda: O.attn_decode(kind, window, x.q, x.new_k, x.new_v, x.k_pool,
+                                                 x.v_pool, x.page_table, x.seq_lens,
+                                                 n_threads=cores), budget_s)
+        value = n / sec
+    return {"value": round(value, 3), "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 C oracle on {cores} host threads: {sample}; median of repeats",
+            "sample_s": round(sec, 4)}
+
+
+def oracle_check_config1() -> dict:
+    """The single-layer GDN oracle check: B=1, H=2, d_k=d_v=64, T=128, fp32 (q, v ~ N(0,1),
+    k ~ N(0,1) L2-normalised, beta = sigmoid(N(0,1)), log g ~ U(-0.1, 0), S0 = 0, seed 0), run
+    on the GPU as 128 decode steps and as one chunked prefill (chunk 64), both against the fp64
+    recurrence at the fp32 tolerance 1e-4; the oracle's own time on the host is reported."""
+    import torch
+
+    import hybrid_mixer_decoding_b200 as hmd
+    from oracle import oracle as O
+    O.build()
+    x = I.delta_inputs(I.GDN, 1, 128, 2, 64, 64, dtype="f32", seed=0)
+    dev = "cuda"
+
+    def t(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    q, k, v, beta, lg = t(x.q), t(x.k), t(x.v), t(x.beta), t(x.log_gate)
+    # 128 decode steps
+    state = t(x.state0).clone()
+    o_dec = torch.empty(1, 128, 2, 64, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(128):
+        hmd.delta_rule_decode(I.GDN, q[:, i].contiguous(), k[:, i].contiguous(),
+                              v[:, i].contiguous(), beta[:, i].contiguous(),
+                              lg[:, i].contiguous(), state, o_dec[:, i])
+    e1.record()
+    torch.cuda.synchronize()
+    dec_ms = e0.elapsed_time(e1)
+    st_dec = state.cpu().numpy()
+    # one chunked prefill
+    state_p = t(x.state0).clone()
+    o_pre = torch.empty(1, 128, 2, 64, device=dev)
+    hmd.delta_rule_prefill_chunked(I.GDN, q, k, v, beta, lg, state_p, o_pre)
+    torch.cuda.synchronize()
+    assert hmd.hmd_device_errors(clear=True) == 0
+    cores = len(os.sched_getaffinity(0))
+    o_ref, s_ref = O.delta_recurrent(I.GDN, x.q, x.k, x.v, x.beta, x.log_gate, x.state0)
+    sec = _repeat_time(lambda: O.delta_recurrent(I.GDN, x.q, x.k, x.v, x.beta, x.log_gate,
+                                                 x.state0, n_threads=cores), 1.0)
+    errs = {"decode_o": O.rel_err(o_dec.cpu().numpy(), o_ref),
+            "decode_state": O.rel_err(st_dec, s_ref),
+            "prefill_o": O.rel_err(o_pre.cpu().numpy(), o_ref),
+            "prefill_state": O.rel_err(state_p.cpu().numpy(), s_ref)}
+    return {"config": "GDN B=1, H=2, d=64, T=128, fp32, S0=0, seed 0",
+            "rel_err": {k_: float(f"{v_:.3e}") for k_, v_ in errs.items()}, "tol": 1e-4,
+            "pass": all(v_ <= 1e-4 for v_ in errs.values()),
+            "gpu_decode_tok_s": round(128 / (dec_ms * 1e-3), 1),
+            "cpu_baseline": {"value": round(128 / sec, 1), "unit": "tok/s", "cores": cores,
+                             "kind": "oracle", "sample": "the whole config (128 tokens)"}}
+
+
+PREFILL_WORKLOADS = {"KDA": "prefill_kda", "GDN": "prefill_gdn", "FA": "prefill_fa",
+                     "SWA": "prefill_swa"}
+DECODE_WORKLOADS = {"KDA": "decode_kda", "GDN": "decode_gdn", "FA": "attn_fa", "SWA": "attn_swa"}
+
+
+def per_mixer_lines(args) -> dict:
+    """Prefill and decode tokens/s of each mixer at its configuration (bench steps/warmup),
+    each with its roofline and the oracle's throughput on a bounded sample of the same work."""
+    import torch
+    out = {}
+    for key, table in (("prefill", PREFILL_WORKLOADS), ("decode", DECODE_WORKLOADS)):
+        out[key] = {}
+        for mixer, w in table.items():
+            m = measure_workload(w, max(5, args.steps), args.warmup)
+            torch.cuda.empty_cache()
+            if not args.skip_cpu_baseline:
+                m["cpu_baseline"] = workload_cpu_baseline(w, budget_s=1.5)
+            out[key][mixer] = m
+    return out
+
+
 
 
 def run_spec(args):
@@ -833,6 +1070,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used for profiler runs)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="stack48: only the 48-layer line (no per-mixer prefill/decode lines)")
     ap.add_argument("--workload", default="stack48",
                     choices=["stack48", "attn_fa", "attn_swa", "prefill_fa", "prefill_swa",
                              "decode_kda", "decode_gdn",
@@ -847,6 +1086,10 @@ def main():
         out = run_reference(args, rank, world)
     elif args.workload == "stack48":
         out = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.headline_only:
+            # per-mixer prefill and decode lines and the fp32 oracle check, on this rank's GPU
+            out.update(per_mixer_lines(args))
+            out["oracle_check"] = oracle_check_config1()
     elif args.workload == "sweep":
         out = run_sweep(args)
     elif args.workload == "spec_stack":

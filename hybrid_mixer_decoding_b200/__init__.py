@@ -14,7 +14,8 @@ from ._lib import (BF16, BatchPlan, group_sequences, mixer_decode_step_batch, DE
                    delta_rule_decode_to, delta_rule_prefill_chunked_act,
                    delta_rule_prefill_chunked, delta_rule_prefill_chunked_ws,
                    delta_rule_prefill_workspace_size, hmd_device_errors, hmd_last_error,
-                   hmd_status_string, hmd_version, lib, mixer_decode_step)
+                   hmd_status_string, hmd_test_arm_copy_skip, hmd_version, lib,
+                   mixer_decode_step)
 
 __all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "DEVERR_GATE", "DEVERR_PAGE", "DEVERR_SEQLEN", "DEVERR_SLOT", "DEVERR_TIMEOUT", "F32", "FA",
            "GDN", "KDA", "SWA", "DecodeIO", "HmdError", "KVCache", "StateCache", "attn_decode",
@@ -25,4 +26,5 @@ __all__ = ["BF16", "BatchPlan", "group_sequences", "mixer_decode_step_batch", "D
            "delta_rule_decode_to", "delta_rule_prefill_chunked_act",
            "delta_rule_prefill_chunked", "delta_rule_prefill_chunked_ws",
            "delta_rule_prefill_workspace_size", "hmd_device_errors", "hmd_last_error",
-           "hmd_status_string", "hmd_version", "lib", "mixer_decode_step"]
+           "hmd_status_string", "hmd_test_arm_copy_skip", "hmd_version", "lib",
+           "mixer_decode_step"]

@@ -84,6 +84,7 @@ _SIGS = {
     "hmd_last_error": (_c_int, []),
     "hmd_device_errors": (_c_int, [_vp, ctypes.POINTER(ctypes.c_uint32), _c_int]),
     "hmd_version": (ctypes.c_char_p, []),
+    "hmd_test_arm_copy_skip": (_c_int, [_c_int, _c_int, ctypes.c_uint64]),
 }
 
 
@@ -507,3 +508,13 @@ def hmd_last_error() -> int:
 
 def hmd_version() -> str:
     return lib().hmd_version().decode()
+
+
+TEST_DELTA_DECODE, TEST_ATTN_SPLIT = 0, 1
+
+
+def hmd_test_arm_copy_skip(kernel: int, cta: int, wait_ns: int) -> None:
+    """Arm a one-shot missing copy in CTA `cta` of this thread's next launch of `kernel`
+    (TEST_DELTA_DECODE or TEST_ATTN_SPLIT), with every bounded wait of that launch limited to
+    wait_ns: the failure-detection tests' way to make a wait run out without an invalid access."""
+    _check("hmd_test_arm_copy_skip", lib().hmd_test_arm_copy_skip(kernel, cta, wait_ns))

@@ -61,6 +61,8 @@ struct SplitParams {
     int B, Hq, Hkv, group, nq, n_pages, max_pages, window, swa, ring_pages;
     int n_splits, pages_per_split, max_seq_len;
     float scale_log2;  // log2(e) / sqrt(d)
+    int skip_cta;      // fault injection (tests): this CTA arms its first tile with no copy
+    unsigned long long wait_ns;  // limit of every bounded wait
 };
 
 // Byte offset of the 16-byte chunk holding (row, dim..dim+7) in a page tile stored as D/64
@@ -193,10 +195,13 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 mbar_arrive_expect_tx(bar, 2 * TB);
                 const uint32_t kb = smem_base + s * 2 * TB, vb = kb + TB;
                 const int y = (pg * p.Hkv + it.g) * kPT;
+                // a test may arm the first tile's barrier with no copy
+                if (issued > 0 || (int)blockIdx.x != p.skip_cta) {
 #pragma unroll
-                for (int hf = 0; hf < D / 64; ++hf) {
-                    tma_load_2d(kb + hf * kPT * 128, &tmk, bar, hf * 64, y);
-                    tma_load_2d(vb + hf * kPT * 128, &tmv, bar, hf * 64, y);
+                    for (int hf = 0; hf < D / 64; ++hf) {
+                        tma_load_2d(kb + hf * kPT * 128, &tmk, bar, hf * 64, y);
+                        tma_load_2d(vb + hf * kPT * 128, &tmv, bar, hf * 64, y);
+                    }
                 }
             }
         }
@@ -228,15 +233,24 @@ attn_split_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
     for (int t = 0; t < it.n_tiles; ++t) {
         const int s = t % kStages;
-        const bool ok = mbar_wait_bounded(smem_u32(&full_bar[s]), (t / kStages) & 1);
+        const bool ok = mbar_wait_bounded(smem_u32(&full_bar[s]), (t / kStages) & 1, p.wait_ns);
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
                 // let the copies this CTA issued finish (bounded) before leaving
                 for (int u = t; u < issued; ++u)
-                    (void)mbar_wait_bounded(smem_u32(&full_bar[u % kStages]), (u / kStages) & 1);
+                    (void)mbar_wait_bounded(smem_u32(&full_bar[u % kStages]), (u / kStages) & 1,
+                                            p.wait_ns);
             }
-            return;  // no partials are written; the error word reports the step as failed
+            // mark this range's partials as missing (a negative sum of exponentials, which no
+            // completed range writes): the combine then leaves these rows' outputs untouched
+            for (int r = tid; r < p.nq * G; r += kThreads) {
+                const int ti = r / G;
+                const size_t row = (((size_t)it.r * p.nq + ti) * p.Hq + it.g * G + (r - ti * G)) *
+                                       p.n_splits + it.split;
+                p.ws_ml[row * 2 + 1] = -1.f;
+            }
+            return;  // the error word reports the step as failed
         }
         const int pg = stage_pg[s];
         const bool tile_ok = pg >= 0;
@@ -412,7 +426,12 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const float *ws_ml, con
     const size_t ob = rows ? (size_t)rows[bh / per_row] * per_row + bh % per_row : bh;
     const float *ml = ws_ml + bh * n_splits * 2;
     float M = -INFINITY;
-    for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[2 * s]);
+    bool missing = false;  // a key range whose CTA gave up (see the split kernel's abort path)
+    for (int s = 0; s < n_splits; ++s) {
+        M = fmaxf(M, ml[2 * s]);
+        missing |= ml[2 * s + 1] < 0.f;
+    }
+    if (missing) return;
     float num = 0.f, den = 0.f;
     if (M != -INFINITY) {
         for (int s = 0; s < n_splits; ++s) {
@@ -492,6 +511,8 @@ cudaError_t launch_d(const AttnDecodeArgs &a, const AttnPlan &plan, cudaStream_t
     p.n_splits = plan.n_splits; p.pages_per_split = plan.pages_per_split;
     p.max_seq_len = a.max_seq_len;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    p.skip_cta = a.skip.cta;
+    p.wait_ns = a.skip.wait_ns;
     cudaError_t e = launch_pdl(attn_split_kernel<D>, dim3((unsigned)plan.n_ctas), dim3(kThreads),
                                smem, s, tmk, tmv, p);
     if (e != cudaSuccess) return e;

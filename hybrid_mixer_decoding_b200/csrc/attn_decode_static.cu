@@ -20,11 +20,12 @@
 #include <mutex>
 
 #include "../../include/hmd.h"
+#include "kernels.h"
 
 namespace {
 
 constexpr size_t kStaticWsBytes = 16u << 20;  // 16 MiB
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = hmd::kMaxDevices;
 
 __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 
@@ -62,11 +63,12 @@ hmd_status_t attn_decode_static_ws(hmd_kind_t kind, int window, int B, int Hq, i
     if (B > 0 && Hq > 0 && Hkv > 0 && d > 0 && max_seq_len > 0) {
         const size_t need = attn_decode_workspace_size(kind, window, B, Hq, Hkv, d, page_tokens,
                                                        max_seq_len);
-        if (need > kStaticWsBytes) return HMD_ERR_UNSUPPORTED;  // too large for the fixed array
+        if (need > kStaticWsBytes)  // too large for the fixed array
+            return hmd::record_status(HMD_ERR_UNSUPPORTED);
     }
     void *ws = nullptr;
     const hmd_status_t st = static_ws_ptr(&ws);
-    if (st != HMD_OK) return st;
+    if (st != HMD_OK) return hmd::record_status(st);
     return attn_decode(kind, window, B, Hq, Hkv, d, page_tokens, q, new_k, new_v, k_pool, v_pool,
                        n_pages, page_table, max_pages, seq_lens, max_seq_len, o, ws,
                        kStaticWsBytes, stream);

@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
             mbar_init(bb, 1);
             fence_barrier_init();
             mbar_arrive_expect_tx(bb, DK * kSliceCols * 4);
-            tma_load_2d(smem_u32(&S[0][0]), &tm, bb, slice * kSliceCols, (slot * a.H + h) * DK);
+            if ((int)blockIdx.x != a.skip.cta)  // a test may arm this barrier with no copy
+                tma_load_2d(smem_u32(&S[0][0]), &tm, bb, slice * kSliceCols, (slot * a.H + h) * DK);
         } else {
             atomicOr(&g_err, HMD_DEVERR_SLOT);
         }
@@ -151,8 +152,13 @@ __global__ void __launch_bounds__(kThreads) delta_decode_kernel(const __grid_con
     }
     __syncthreads();
     if (!s_ok) return;
-    if (t == 0 && !mbar_wait_bounded(smem_u32(&bar), 0)) {
-        if (tid == 0) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+    // the CTA gives up together: one thread's timeout decides for all of them
+    if (t == 0 && __syncthreads_or(!mbar_wait_bounded(smem_u32(&bar), 0, a.skip.wait_ns))) {
+        if (tid == 0) {
+            atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+            // the copy may still land: let it finish (bounded) before the shared memory goes
+            (void)mbar_wait_bounded(smem_u32(&bar), 0, a.skip.wait_ns);
+        }
         return;  // nothing was written; the state slice is left as it was
     }
 

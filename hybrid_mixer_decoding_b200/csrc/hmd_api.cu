@@ -47,6 +47,9 @@ hmd_status_t fail(hmd_status_t s) {
 
 hmd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? HMD_OK : fail(HMD_ERR_CUDA); }
 
+// armed fault injections of this host thread (hmd_test_arm_copy_skip), one per test kernel
+thread_local hmd::CopySkip t_skip[2];
+
 cudaStream_t as_stream(hmd_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -67,7 +70,30 @@ hmd_status_t check_delta_decode(hmd_kind_t kind, int B, int H, int dk, int dv, h
 
 }  // namespace
 
+namespace hmd {
+hmd_status_t record_status(hmd_status_t s) { return s == HMD_OK ? s : fail(s); }
+
+CopySkip take_copy_skip(int kernel) {
+    const CopySkip c = t_skip[kernel];
+    t_skip[kernel] = CopySkip{};
+    return c;
+}
+}  // namespace hmd
+
 extern "C" {
+
+hmd_status_t hmd_test_arm_copy_skip(hmd_test_kernel_t kernel, int cta, uint64_t wait_ns) {
+    if ((kernel != HMD_TEST_DELTA_DECODE && kernel != HMD_TEST_ATTN_SPLIT) || cta < -1 ||
+        wait_ns < 1000 || wait_ns > 2000000000ull)
+        return fail(HMD_ERR_ARG);
+    if (cta == -1) {  // disarm
+        t_skip[kernel] = hmd::CopySkip{};
+        return HMD_OK;
+    }
+    t_skip[kernel].cta = cta;
+    t_skip[kernel].wait_ns = wait_ns;
+    return HMD_OK;
+}
 
 const char *hmd_version(void) { return "hmd 0.1 (sm_100a)"; }
 
@@ -127,6 +153,7 @@ hmd_status_t delta_run(hmd_kind_t kind, int B, int H, int dk, int dv, hmd_dtype_
         a.act.A_log = act->A_log; a.act.dt_bias = act->dt_bias; a.act.eps = act->l2_eps;
     }
     a.nq = nq; a.chain = chain;
+    a.skip = hmd::take_copy_skip(HMD_TEST_DELTA_DECODE);
     return from_cuda(hmd::launch_delta_decode(a, as_stream(stream)));
 }
 }  // namespace
@@ -439,6 +466,7 @@ hmd_status_t attn_run(hmd_kind_t kind, int window, int ring_pages, int n_q, int 
     a.k_pool = k_pool; a.v_pool = v_pool; a.n_pages = n_pages; a.page_table = page_table;
     a.max_pages = max_pages; a.seq_lens = seq_lens; a.max_seq_len = max_seq_len; a.o = o;
     a.workspace = workspace; a.ws_bytes = ws_bytes;
+    a.skip = hmd::take_copy_skip(HMD_TEST_ATTN_SPLIT);
     return from_cuda(hmd::launch_attn_decode(a, as_stream(stream)));
 }
 }  // namespace

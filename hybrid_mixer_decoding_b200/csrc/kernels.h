@@ -6,8 +6,11 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 #include <utility>
+
+#include "../../include/hmd.h"
 
 namespace hmd {
 
@@ -16,23 +19,50 @@ namespace hmd {
 // normal range (|G| < 87); below this floor a chunk is reported with HMD_DEVERR_GATE.
 constexpr float kPrefillGateFloor = -80.f;
 
-// Runs f() once for each device it is called on (the current device) and returns that first
-// result on every later call there. Kernel attributes (the dynamic shared-memory limit) and
-// device properties belong to one device, so a process that drives several GPUs sets and reads
-// them per device.
+// Runs f() for the current device until it succeeds once, then returns that result on every
+// later call there. Kernel attributes (the dynamic shared-memory limit) and device properties
+// belong to one device, so a process that drives several GPUs sets and reads them per device.
+// A CUDA error (for instance a transient failure to set an attribute) is returned to its caller
+// and not kept: f() runs again on the next call. When the current device cannot be determined,
+// f() runs uncached.
 constexpr int kMaxDevices = 64;
+template <typename R>
+inline bool once_cacheable(const R &) { return true; }
+inline bool once_cacheable(const cudaError_t &e) { return e == cudaSuccess; }
 template <typename F>
 auto once_per_device(F f) -> decltype(f()) {
-    static std::once_flag flags[kMaxDevices];
-    static decltype(f()) results[kMaxDevices];
-    int dev = 0;
+    using R = decltype(f());
+    static std::mutex mu;
+    static std::atomic<bool> done[kMaxDevices];
+    static R results[kMaxDevices];
+    int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
-        dev = 0;
+        return f();
     }
-    std::call_once(flags[dev], [&] { results[dev] = f(); });
+    if (done[dev].load(std::memory_order_acquire)) return results[dev];
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev].load(std::memory_order_relaxed)) {
+        const R r = f();
+        if (!once_cacheable(r)) return r;
+        results[dev] = r;
+        done[dev].store(true, std::memory_order_release);
+    }
     return results[dev];
 }
+
+// Records `s` as this host thread's last error (read by hmd_last_error) and returns it; for
+// entry points defined outside the API file.
+hmd_status_t record_status(hmd_status_t s);
+
+// One-shot fault injection for the failure-detection tests (hmd_test_arm_copy_skip): the next
+// launch of `kernel` on this host thread has CTA `cta` arm its first copy barrier without
+// issuing the copy, and every bounded wait in it gives up after wait_ns.
+struct CopySkip {
+    int cta = -1;                              // -1: nothing armed
+    unsigned long long wait_ns = 2000000000ull;  // the normal 2 s limit
+};
+CopySkip take_copy_skip(int kernel);
 
 // Launches `kernel` on stream s with programmatic stream serialisation: it may be scheduled
 // while the previous kernel in the stream drains, and waits for it (griddep_wait) before its
@@ -103,6 +133,7 @@ struct DeltaDecodeArgs {
     // from chain[0][b] and the state after token t is stored to chain[t + 1][b] ([nq+1][B])
     int nq = 1;
     const int32_t *chain = nullptr;
+    CopySkip skip;  // fault injection (tests only); inactive by default
 };
 cudaError_t launch_delta_decode(const DeltaDecodeArgs &a, cudaStream_t s);
 bool delta_decode_supported(int dk, int dv);
@@ -126,6 +157,7 @@ struct AttnDecodeArgs {
     void *o;
     void *workspace;
     size_t ws_bytes;
+    CopySkip skip;  // fault injection (tests only); inactive by default
 };
 struct AttnPlan {
     int n_splits;         // key ranges per (sequence, kv-head)

@@ -446,6 +446,23 @@ HMD_API hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int 
 /* Library version string. */
 HMD_API const char *hmd_version(void);
 
+/* ------------------------------------------------------------------------------------------ */
+/* Failure-detection testing hook. The paper has no counterpart: it exists so that the bounded */
+/* waits of the kernels (every wait on a copy barrier gives up instead of hanging, reports    */
+/* HMD_DEVERR_TIMEOUT and writes nothing) can be exercised without any invalid access.        */
+/* ------------------------------------------------------------------------------------------ */
+typedef enum { HMD_TEST_DELTA_DECODE = 0, HMD_TEST_ATTN_SPLIT = 1 } hmd_test_kernel_t;
+/* Arms a one-shot fault for the next launch of `kernel` made by this host thread (the delta-rule
+ * decode kernel of delta_rule_decode*, or the split kernel of attn_decode / attn_verify): CTA
+ * `cta` of that launch arms its first copy barrier for the copy's bytes but issues no copy, so
+ * its wait can never complete, and every bounded wait of the launch gives up after wait_ns
+ * nanoseconds (1e3 .. 2e9) instead of 2 s. That CTA then reports HMD_DEVERR_TIMEOUT and leaves
+ * its outputs untouched (delta decode: its state slice and its columns of o; attention: the
+ * query heads of its kv-head for that sequence, whose combine is skipped); every other CTA runs
+ * normally. A cta beyond the launch's grid arms nothing that fires; cta = -1 disarms.
+ * HMD_ERR_ARG for a bad kernel, cta < -1 or wait_ns out of range.                             */
+HMD_API hmd_status_t hmd_test_arm_copy_skip(hmd_test_kernel_t kernel, int cta, uint64_t wait_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -233,10 +233,36 @@ def delta_activations(kind, q_raw, k_raw, beta_logit, gate_logit, A_log, dt_bias
     return q, k, beta, lg
 
 
+# Every rel_err call is logged here with the elementwise figure beside the normwise one; the
+# test session prints the worst of each per test (tests/conftest.py).
+PARITY_LOG: list = []
+PARITY_LABEL = [""]  # the running test's id, set by the test session
+
+
+def elementwise_p99(x, ref) -> float:
+    """99th percentile over the elements of |x - ref| / max(|ref|, 1e-6 max|ref|): the
+    elementwise relative error, with an absolute floor so that entries near zero do not make it
+    undefined. Logged beside the normwise measure; the tolerances apply to the normwise one."""
+    x = np.asarray(x, dtype=np.float64).ravel()
+    ref = np.asarray(ref, dtype=np.float64).ravel()
+    if ref.size == 0:
+        return 0.0
+    floor = 1e-6 * float(np.max(np.abs(ref)))
+    den = np.maximum(np.abs(ref), floor)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        e = np.abs(x - ref) / den
+    e = np.where(den > 0, e, np.abs(x - ref))
+    return float(np.percentile(e, 99))
+
+
 def rel_err(x, ref) -> float:
-    """Normwise relative error max|x - ref| / max|ref| (the parity measure)."""
+    """Normwise relative error max|x - ref| / max|ref| (the parity measure). The elementwise
+    p99 (elementwise_p99) is logged beside it in PARITY_LOG."""
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     den = float(np.max(np.abs(ref))) if ref.size else 0.0
     num = float(np.max(np.abs(x - ref))) if ref.size else 0.0
-    return num / den if den > 0 else num
+    r = num / den if den > 0 else num
+    PARITY_LOG.append({"test": PARITY_LABEL[0], "shape": list(ref.shape), "normwise": r,
+                       "p99_elementwise": elementwise_p99(x, ref)})
+    return r

@@ -277,3 +277,20 @@ def test_device_error_bits_match_the_header():
     assert bits == {"TIMEOUT": hmd.DEVERR_TIMEOUT, "PAGE": hmd.DEVERR_PAGE,
                     "SLOT": hmd.DEVERR_SLOT, "SEQLEN": hmd.DEVERR_SEQLEN,
                     "GATE": hmd.DEVERR_GATE}
+
+
+def test_copy_skip_hook_validation():
+    """The failure-detection hook rejects bad arguments on the host; a valid arming launches
+    nothing by itself."""
+    L = hmd.lib()
+    hmd.hmd_last_error()
+    assert L.hmd_test_arm_copy_skip(7, 0, 10**6) == ARG          # no such kernel
+    assert L.hmd_test_arm_copy_skip(_lib.TEST_DELTA_DECODE, -2, 10**6) == ARG
+    assert L.hmd_test_arm_copy_skip(_lib.TEST_ATTN_SPLIT, 0, 10) == ARG        # below 1 us
+    assert L.hmd_test_arm_copy_skip(_lib.TEST_ATTN_SPLIT, 0, 3 * 10**9) == ARG  # above 2 s
+    assert hmd.hmd_last_error() == ARG
+    assert L.hmd_test_arm_copy_skip(_lib.TEST_DELTA_DECODE, 3, 10**6) == 0
+    # a call rejected on the host leaves the fault armed and launches nothing; cta = -1 disarms
+    # it, so no later test in this thread meets it
+    assert _decode(ptr=None) == ARG
+    assert L.hmd_test_arm_copy_skip(_lib.TEST_DELTA_DECODE, -1, 10**6) == 0

@@ -164,3 +164,18 @@ def test_gate_range_is_reported(oracle_mod, kind, dk, dtype):
     d = I.delta_inputs(kind, 1, 100, 2, dk, dk, dtype=dtype, seed=6, gate_lo=-4.0)
     run_prefill(d)
     assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_GATE
+
+
+@pytest.mark.parametrize("kind", [I.GDN, I.KDA])
+def test_long_prompt_does_not_drift(oracle_mod, kind):
+    """B=1, H=2, d=128, T=32768 (512 chunks): the scan rounds the state to bf16 as an MMA operand
+    in every chunk; the outputs of the last chunks and the final state must still match the
+    recurrence at the bf16 tolerance, so the rounding error does not grow with the chunk count."""
+    O = oracle_mod
+    d = I.delta_inputs(kind, 1, 32768, 2, 128, 128, dtype="bf16", seed=50, state0="randn")
+    o, st = run_prefill(d)
+    assert hmd.hmd_device_errors(clear=True) == 0
+    o_ref, st_ref = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
+    assert O.rel_err(o, o_ref) < 2e-2
+    assert O.rel_err(o[:, -4096:], o_ref[:, -4096:]) < 2e-2  # the last 64 chunks alone
+    assert O.rel_err(st, st_ref) < 2e-2
