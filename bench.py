@@ -171,6 +171,8 @@ def traffic_for(kernel_key: str):
     if not ent:
         return None
     src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src):
+        return None
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()[:16]
     if sha != ent.get("source_sha"):

@@ -4,18 +4,20 @@
 // Many Speeds", abstract; gist.science technical summary, section 2a); the recurrence is the
 // standard one (see delta_decode.cu). Over a chunk of C tokens starting from state M0, with
 // per-channel cumulative log-gates G[r][i] = sum_{s<=r} log a_{s,i}, it is exactly
-//   A[r][s] = beta_r (Kt_r . Kh_s)  (s < r)        Kt = k * exp(G),  Kh = k * exp(-G)
+//   A[r][s] = beta_r sum_i k_ri k_si e^(G_ri - G_si)  (s < r)
 //   T = (I + A)^{-1} Diag(beta)                    (unit lower-triangular solve)
-//   W = T Kt,  U = T V - W M0                      (U[r] is token r's delta-rule write)
-//   P[r][s] = Qt_r . Kh_s  (s <= r)                Qt = q * exp(G)
-//   O = Qt M0 + P U
-//   M_C = Diag(exp(G_C)) M0 + (Kh Diag(exp(G_C)))^T U,  G_C = G of the chunk's last token.
+//   U = T (V - Kt M0),  Kt = k * exp(G)            (U[r] is token r's delta-rule write)
+//   P[r][s] = sum_i q_ri k_si e^(G_ri - G_si)  (s <= r),  O = Qt M0 + P U,  Qt = q * exp(G)
+//   M_C = Diag(exp(G_C)) M0 + sum_s (k_s exp(G_C - G_s))^T U_s,  G_C = G of the chunk's last token.
+// The decays e^(G_r - G_s) are formed as e^G_r e^-G_s while every |G| of the chunk is at most
+// kPrefillFactorRange (both factors then stay inside fp32's range) and directly otherwise, so
+// any gate is accepted.
 //
 // bf16 inputs with d_k = d_v = 128 and C = 64 run on the tensor cores in two passes
-// (delta_prefill_scan.cu).
+// (delta_prefill_tc.cu).
 // This file holds the generic path: one CTA per (sequence, head, 32-column slice of d_v) runs
 // the chunks in order with the slice of the state resident in shared memory, all arithmetic in
-// fp32 on CUDA cores (so fp32 inputs keep fp32 accuracy). The k-side products (A, T, W, P) do
+// fp32 on CUDA cores (so fp32 inputs keep fp32 accuracy). The k-side products (A, T, P) do
 // not depend on d_v and are recomputed by every slice's CTA.
 #include "kernels.h"
 #include "ptx.cuh"
@@ -49,17 +51,17 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
                                                                    int n_slices, int dvs) {
     extern __shared__ float sm[];
     const int dk = a.dk, dv = a.dv;
-    float *Kt = sm;                         // [C][dk]
-    float *Kh = Kt + kC * dk;               // [C][dk]
-    float *Qt = Kh + kC * dk;               // [C][dk]
-    float *Wm = Qt + kC * dk;               // [C][dk]
-    float *Vs = Wm + kC * dk;               // [C][dvs]
+    float *Kr = sm;                         // [C][dk] k
+    float *Qr = Kr + kC * dk;               // [C][dk] q
+    float *Eg = Qr + kC * dk;               // [C][dk] e^G
+    float *Gx = Eg + kC * dk;               // [C][dk] e^-G (factored chunks) or G (direct ones)
+    float *Vs = Gx + kC * dk;               // [C][dvs]
     float *Us = Vs + kC * dvs;              // [C][dvs]
     float *Ms = Us + kC * dvs;              // [dk][dvs]
     float *Am = Ms + dk * dvs;              // [C][C]
     float *Tm = Am + kC * kC;               // [C][C]
     float *Pm = Tm + kC * kC;               // [C][C]
-    float *egl = Pm + kC * kC;              // [dk] exp(G_C)
+    float *egl = Pm + kC * kC;              // [dk] e^G_C
     float *gl = egl + dk;                   // [dk] G_C
     float *bt = gl + dk;                    // [C] beta
 
@@ -83,25 +85,31 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
     for (int t0 = 0; t0 < a.T; t0 += kC) {
         const int n = min(kC, a.T - t0);
         __syncthreads();  // previous chunk fully consumed
-        // gates, scaled q/k, v slice, beta
+        // gates: G per channel, and whether the factored form stays inside fp32's range
+        bool out_of_range = false;
         for (int i = tid; i < dk; i += kThreads) {
             float g = 0.f;
             for (int r = 0; r < kC; ++r) {
                 if (r < n) {
                     const size_t tok = ((size_t)b * a.T + t0 + r) * a.H + h;
                     g += a.kind == HMD_GDN ? a.log_gate[tok] : a.log_gate[tok * dk + i];
-                    const float e = expf(g), ie = expf(-g);
-                    const float kv = ld_act<BF16>(a.k, tok * dk + i);
-                    Kt[r * dk + i] = kv * e;
-                    Kh[r * dk + i] = kv * ie;
-                    Qt[r * dk + i] = ld_act<BF16>(a.q, tok * dk + i) * e;
-                } else {
-                    Kt[r * dk + i] = 0.f; Kh[r * dk + i] = 0.f; Qt[r * dk + i] = 0.f;
                 }
+                Gx[r * dk + i] = g;
+                out_of_range |= g < -kPrefillFactorRange || g > kPrefillFactorRange;
             }
             gl[i] = g;
             egl[i] = expf(g);
-            if (g < kPrefillGateFloor) atomicOr(&g_err, HMD_DEVERR_GATE);
+        }
+        const bool direct = __syncthreads_or(out_of_range);
+        // q, k, e^G and (factored chunks) e^-G, the v slice, beta
+        for (int idx = tid; idx < kC * dk; idx += kThreads) {
+            const int r = idx / dk, i = idx % dk;
+            const size_t tok = ((size_t)b * a.T + t0 + r) * a.H + h;
+            const float g = Gx[idx];
+            Kr[idx] = r < n ? ld_act<BF16>(a.k, tok * dk + i) : 0.f;
+            Qr[idx] = r < n ? ld_act<BF16>(a.q, tok * dk + i) : 0.f;
+            Eg[idx] = expf(g);
+            if (!direct) Gx[idx] = expf(-g);
         }
         for (int idx = tid; idx < kC * dvs; idx += kThreads) {
             const int r = idx / dvs, jj = idx % dvs;
@@ -111,15 +119,19 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
         for (int r = tid; r < kC; r += kThreads)
             bt[r] = r < n ? a.beta[((size_t)b * a.T + t0 + r) * a.H + h] : 0.f;
         __syncthreads();
-        // A (strictly lower, beta-scaled) and P (lower incl. diagonal)
+        // A (strictly lower, beta-scaled) and P (lower incl. diagonal):
+        // sum_i x_ri k_si e^(G_ri - G_si) with x = k (A) or q (P), the decay as e^G_r e^-G_s in a
+        // factored chunk, else formed directly
         for (int idx = tid; idx < kC * kC; idx += kThreads) {
             const int r = idx / kC, s = idx % kC;
             float av = 0.f, pv = 0.f;
             if (s <= r && r < n) {
                 for (int i = 0; i < dk; ++i) {
-                    const float kh = Kh[s * dk + i];
-                    av += Kt[r * dk + i] * kh;
-                    pv += Qt[r * dk + i] * kh;
+                    const float d = direct ? expf(Gx[r * dk + i] - Gx[s * dk + i])
+                                           : Eg[r * dk + i] * Gx[s * dk + i];
+                    const float ks = Kr[s * dk + i] * d;
+                    av += Kr[r * dk + i] * ks;
+                    pv += Qr[r * dk + i] * ks;
                 }
             }
             Am[idx] = s < r ? bt[r] * av : 0.f;
@@ -138,35 +150,29 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
             }
         }
         __syncthreads();
-        // W = T Kt ; U <- T V (first half of U = T V - W M0)
-        for (int idx = tid; idx < kC * dk; idx += kThreads) {
-            const int r = idx / dk, i = idx % dk;
-            float acc = 0.f;
-            for (int s = 0; s <= r; ++s) acc += Tm[r * kC + s] * Kt[s * dk + i];
-            Wm[idx] = acc;
-        }
+        // Z = V - Kt M0 (Kt = k e^G), into Us
         for (int idx = tid; idx < kC * dvs; idx += kThreads) {
             const int r = idx / dvs, jj = idx % dvs;
-            float acc = 0.f;
-            for (int s = 0; s <= r; ++s) acc += Tm[r * kC + s] * Vs[s * dvs + jj];
+            float acc = Vs[idx];
+            for (int i = 0; i < dk; ++i) acc -= Kr[r * dk + i] * Eg[r * dk + i] * Ms[i * dvs + jj];
             Us[idx] = acc;
         }
         __syncthreads();
-        // U = T V - W M0
+        // U = T Z (= T V - W M0 with W = T Kt), into Vs
         for (int idx = tid; idx < kC * dvs; idx += kThreads) {
             const int r = idx / dvs, jj = idx % dvs;
-            float acc = Us[idx];
-            for (int i = 0; i < dk; ++i) acc -= Wm[r * dk + i] * Ms[i * dvs + jj];
-            Us[idx] = acc;
+            float acc = 0.f;
+            for (int s = 0; s <= r; ++s) acc += Tm[r * kC + s] * Us[s * dvs + jj];
+            Vs[idx] = acc;
         }
         __syncthreads();
-        // O = Qt M0 + P U
+        // O = Qt M0 + P U (Qt = q e^G)
         for (int idx = tid; idx < kC * dvs; idx += kThreads) {
             const int r = idx / dvs, jj = idx % dvs;
             if (r >= n || jj >= ncols) continue;
             float acc = 0.f;
-            for (int i = 0; i < dk; ++i) acc += Qt[r * dk + i] * Ms[i * dvs + jj];
-            for (int s = 0; s <= r; ++s) acc += Pm[r * kC + s] * Us[s * dvs + jj];
+            for (int i = 0; i < dk; ++i) acc += Qr[r * dk + i] * Eg[r * dk + i] * Ms[i * dvs + jj];
+            for (int s = 0; s <= r; ++s) acc += Pm[r * kC + s] * Vs[s * dvs + jj];
             acc *= a.scale;
             const size_t oi = (((size_t)b * a.T + t0 + r) * a.H + h) * dv + j0 + jj;
             if constexpr (BF16) {
@@ -176,12 +182,15 @@ __global__ void __launch_bounds__(kThreads) prefill_generic_kernel(const DeltaPr
             }
         }
         __syncthreads();
-        // M_C = Diag(exp(G_C)) M0 + (Kh Diag(exp(G_C)))^T U
+        // M_C = Diag(e^G_C) M0 + sum_s (k_s e^(G_C - G_s))^T U_s
         for (int idx = tid; idx < dk * dvs; idx += kThreads) {
             const int i = idx / dvs, jj = idx % dvs;
             float acc = 0.f;
-            for (int s = 0; s < n; ++s) acc += Kh[s * dk + i] * Us[s * dvs + jj];
-            Ms[idx] = egl[i] * (Ms[idx] + acc);
+            for (int s = 0; s < n; ++s) {
+                const float d = direct ? expf(gl[i] - Gx[s * dk + i]) : egl[i] * Gx[s * dk + i];
+                acc += Kr[s * dk + i] * d * Vs[s * dvs + jj];
+            }
+            Ms[idx] = egl[i] * Ms[idx] + acc;
         }
     }
     __syncthreads();

@@ -14,10 +14,11 @@
 
 namespace hmd {
 
-// Lowest cumulative log-gate inside one chunk that the chunked prefill accepts. Its chunk form
-// factors e^{G_r - G_s} into k e^{G} and k e^{-G}, each of which must stay inside fp32's
-// normal range (|G| < 87); below this floor a chunk is reported with HMD_DEVERR_GATE.
-constexpr float kPrefillGateFloor = -80.f;
+// The chunked prefill factors each decay e^{G_r - G_s} into e^{G_r} and e^{-G_s} (so that the
+// chunk's products are plain matrix products) while every cumulative in-chunk log-gate |G| is at
+// most this bound: both factors then stay inside fp32's normal range (e^88 overflows). Chunks
+// beyond it form the decays directly.
+constexpr float kPrefillFactorRange = 80.f;
 
 // Runs f() for the current device until it succeeds once, then returns that result on every
 // later call there. Kernel attributes (the dynamic shared-memory limit) and device properties
@@ -226,6 +227,7 @@ struct PrefillScanArgs {
     int chunk_begin;  // first chunk of this segment
     int n_seg;        // chunks in this segment
     DeltaAct act;     // fused input activations
+    int prefetch_stride = 0;  // prep: CTA i prefetches the inputs of CTA i + stride into L2
 };
 bool delta_prefill_scan_supported(int dk, int dv, bool bf16, int chunk);
 size_t delta_prefill_scan_record_bytes();

@@ -57,8 +57,8 @@ typedef enum {
 #define HMD_DEVERR_PAGE      0x2u  /* a page-table entry was outside [0, n_pages) */
 #define HMD_DEVERR_SLOT      0x4u  /* a state-slot index was outside [0, n_slots) */
 #define HMD_DEVERR_SEQLEN    0x8u  /* a sequence length was < 1 or above the stated maximum */
-#define HMD_DEVERR_GATE      0x10u /* a chunked prefill's cumulative log-gate fell below -80
-                                      within one chunk (outside the range its factors cover) */
+#define HMD_DEVERR_GATE      0x10u /* reserved: no longer raised (the chunked prefill accepts
+                                      every gate range) */
 
 typedef void *hmd_stream_t;
 
@@ -157,11 +157,11 @@ HMD_API hmd_status_t delta_rule_decode_chain(hmd_kind_t kind, int n_q, int B, in
  * allocation from a pool the library keeps per device (up to 1 GiB stays cached between calls);
  * HMD_ERR_OOM if it cannot. Under stream capture, or to own the memory, call
  * delta_rule_prefill_chunked_ws instead.
- * Gate range: the chunk form splits each decay factor e^{G_r - G_s} (G the cumulative log-gate
- * inside a chunk) into k e^{G} and k e^{-G}, which stay in fp32's range only while every
- * channel's cumulative log-gate over a chunk stays >= -80 (an average log-gate >= -1.25 per
- * token). A chunk beyond that sets HMD_DEVERR_GATE and its results are not valid; the decode
- * entry points have no such limit.                                                            */
+ * Gate range: any log-gate <= 0 is accepted. The chunk form splits each decay e^{G_r - G_s}
+ * (G the cumulative log-gate inside a chunk) into e^{G_r} and e^{-G_s} while every |G| of the
+ * chunk is at most 80 (both factors then fit fp32), so that the chunk's products are plain
+ * matrix products; a chunk with stronger decay forms its decays directly, at a higher cost
+ * (KDA: on the CUDA cores; GDN's scalar decay needs no split).                                  */
 HMD_API hmd_status_t delta_rule_prefill_chunked(hmd_kind_t kind, int B, int T, int H, int dk, int dv,
                                         hmd_dtype_t dtype, const void *q, const void *k,
                                         const void *v, const float *beta, const float *log_gate,

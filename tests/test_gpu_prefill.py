@@ -144,26 +144,21 @@ def test_caller_workspace_segments_are_bit_exact(oracle_mod, kind):
 
 @pytest.mark.parametrize("kind", [I.GDN, I.KDA])
 @pytest.mark.parametrize("dk,dtype", [(128, "bf16"), (64, "f32")])
-def test_gate_range_is_reported(oracle_mod, kind, dk, dtype):
-    """The chunk form factors e^{G_r - G_s} into k e^{G} and k e^{-G}; a chunk whose cumulative
-    log-gate falls below -80 leaves fp32's range and must be reported (HMD_DEVERR_GATE), on the
-    tensor-core path (bf16, d = 128) and on the CUDA-core path alike. Gates just inside the
-    range are exact and report nothing."""
+@pytest.mark.parametrize("gate_lo", [-2.0, -4.0, -8.0])
+def test_strong_decay_matches_recurrence(oracle_mod, kind, dk, dtype, gate_lo):
+    """Per-token log-gates down to -8: a chunk's cumulative log-gate reaches about -256, far past
+    the range (|G| <= 80) in which the decays can be factored into e^G and e^-G. Those chunks form
+    their decays directly (the tensor-core path and the CUDA-core path alike) and must still match
+    the recurrence, with no device error reported. -2 stays inside the factored range."""
     O = oracle_mod
     hmd.hmd_device_errors(clear=True)
-    # per-token log-gates in [-2, 0]: a full chunk's cumulative gate between about -50 and -77
-    # (inside)
-    d = I.delta_inputs(kind, 1, 64, 2, dk, dk, dtype=dtype, seed=5, gate_lo=-2.0,
+    d = I.delta_inputs(kind, 2, 150, 2, dk, dk, dtype=dtype, seed=5, gate_lo=gate_lo,
                        state0="randn")
     o, st = run_prefill(d)
-    assert (hmd.hmd_device_errors(clear=True) & hmd.DEVERR_GATE) == 0
+    assert hmd.hmd_device_errors(clear=True) == 0
     o_ref, st_ref = O.delta_recurrent(kind, d.q, d.k, d.v, d.beta, d.log_gate, d.state0)
     assert O.rel_err(o, o_ref) < TOL[dtype]
     assert O.rel_err(st, st_ref) < TOL[dtype]
-    # per-token log-gates in [-4, 0]: about -128 over a chunk (outside)
-    d = I.delta_inputs(kind, 1, 100, 2, dk, dk, dtype=dtype, seed=6, gate_lo=-4.0)
-    run_prefill(d)
-    assert hmd.hmd_device_errors(clear=True) & hmd.DEVERR_GATE
 
 
 @pytest.mark.parametrize("kind", [I.GDN, I.KDA])
