@@ -29,8 +29,8 @@
 // Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks,
 // warp-specialised: a producer warp streams records into a 3-stage ring with bulk copies (enough
 // bytes in flight per SM to cover the copies' latency), one thread issues the tcgen05.mma
-// products, four warps hold the CTA's 64 fp32 state columns in registers (thread = row of d_k)
-// and two warps drain the outputs. Per chunk (N = the CTA's 64 columns):
+// products, eight warps hold the CTA's 64 fp32 state columns in registers (thread = row of d_k,
+// 32 columns) and two warps drain the outputs. Per chunk (N = the CTA's 64 columns):
 //   D_UO  = [-W; Qt] M                (M = 128, K = 128; lanes 0-63: -W M, 64-127: Qt M)
 //   U     = Ut + (-W M)               (threads, bf16 operand)
 //   D_UO += [- ; P] U,  D_S = Kc^T U  (lanes 64-127 of D_UO: O; D_S: the state increment)
@@ -737,11 +737,12 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 // ================================ pass B ==================================================
 // One CTA per (sequence, head, half of d_v): 64 state columns, the records streamed through a
 // 3-stage ring (each CTA reads the whole record but its own half of Ut).
-constexpr int kScanThreads = 256;  // 8 warps
+constexpr int kScanThreads = 384;  // 12 warps
 constexpr int kSplitV = 2;
 constexpr int kDV = kD / kSplitV;  // 64 state columns per CTA
 constexpr int kStages = 3;
-constexpr int kWarpProducer = 4, kWarpMma = 5;  // warps 0-3: state rows, 6-7: outputs
+constexpr int kStateWarps = 8;     // warp w: TMEM lanes 32 (w % 4) .., columns 32 (w / 4) ..
+constexpr int kWarpProducer = 8, kWarpMma = 9;  // 10-11: outputs
 constexpr uint32_t ST_WQ = 0, ST_KC = 32768, ST_P = 49152, ST_GAM = 57344, ST_UT = 57856,
                    ST_BYTES = 66560;  // one stage (1 KiB multiple)
 constexpr uint32_t ST_LOAD = ST_UT - ST_GAM + 57344 + kDV * kC * 2;  // bytes copied per stage
@@ -779,7 +780,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
     if (tid == 0) {
         for (int i = 0; i < N_BARS; ++i) {
             const bool by_threads = i == BAR_M || i == BAR_U || i == BAR_TEMPTY0 || i == BAR_TEMPTY0 + 1;
-            mbar_init(bar(i), i == BAR_M ? 4 : (by_threads ? 2 : 1));
+            mbar_init(bar(i), i == BAR_M ? kStateWarps : (i == BAR_U ? kStateWarps / 2 : (by_threads ? 2 : 1)));
         }
         fence_barrier_init();
         *s_abort = 0;
@@ -882,7 +883,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
             }
             umma_commit(bar(BAR_FINAL));  // every product issued has completed once this fires
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 10) {
         // ---- outputs: O rows from TMEM lanes 64-127 ----------------------------------------
         const int r = 32 * (warp & 3) - 64 + lane;  // token row 0..63
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
@@ -911,18 +912,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BAR_TEMPTY0 + u));
         }
-    } else if (warp < 4) {
-        // ---- state: thread = row i of d_k, this CTA's 64 columns --------------------------
-        // Per chunk c: warps 0-1 form U from D_UO; all four wait for D_S and update
+    } else if (warp < kStateWarps) {
+        // ---- state: thread = row i of d_k, 32 of this CTA's 64 columns --------------------
+        // Per chunk c: the warps over rows 0-63 form U from D_UO; all wait for D_S and update
         // M <- e^G_C(c) M + D_S, then write bf16(M) for chunk c + 1 right away (chunk c's first
         // product, the last reader of that tile, has completed by then).
-        const int i = 32 * warp + lane;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        float st[kDV];
+        const int quad = warp & 3, half = warp >> 2;
+        const int i = 32 * quad + lane, col0 = 32 * half;
+        const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+        float st[32];
         {
-            const float4 *src = reinterpret_cast<const float4 *>(Mg + (size_t)i * kD);
+            const float4 *src = reinterpret_cast<const float4 *>(Mg + (size_t)i * kD + col0);
 #pragma unroll
-            for (int q = 0; q < kDV / 4; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 const float4 v = src[q];
                 st[4 * q] = v.x; st[4 * q + 1] = v.y; st[4 * q + 2] = v.z; st[4 * q + 3] = v.w;
             }
@@ -936,8 +938,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
             if (!wait(BAR_FULL0 + s, (c / kStages) & 1)) return false;
             gam = reinterpret_cast<const float *>(sm + s * ST_BYTES + ST_GAM)[i];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                *reinterpret_cast<uint4 *>(mrow + ((q ^ (i & 7)) << 4)) =
+            for (int q = 0; q < 4; ++q) {
+                const int chunk = 4 * half + q;
+                *reinterpret_cast<uint4 *>(mrow + ((chunk ^ (i & 7)) << 4)) =
                     make_uint4(pack_bf16x2(st[8 * q], st[8 * q + 1]), pack_bf16x2(st[8 * q + 2], st[8 * q + 3]),
                                pack_bf16x2(st[8 * q + 4], st[8 * q + 5]), pack_bf16x2(st[8 * q + 6], st[8 * q + 7]));
             }
@@ -950,28 +953,30 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
         bool ok = nseg > 0 && publish_m(0);
         for (int c = 0; ok && c < nseg; ++c) {
             const int s = c % kStages, u = c & 1;
-            if (warp < 2) {
+            if (quad < 2) {
                 // U = Ut + (-W M) for token row i, bf16 into the U operand; Ut is read before the
                 // product lands
                 const uint8_t *utrow = sm + s * ST_BYTES + ST_UT + i * 128;
-                uint4 ut[8];
+                uint4 ut[4];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) ut[q] = *reinterpret_cast<const uint4 *>(utrow + ((q ^ (i & 7)) << 4));
+                for (int q = 0; q < 4; ++q)
+                    ut[q] = *reinterpret_cast<const uint4 *>(utrow + (((4 * half + q) ^ (i & 7)) << 4));
                 if (!wait(BAR_UO, c & 1)) break;
                 tc_fence_after();
-                uint32_t d[64];
-                tmem_ld64(tmem + lane_base + kDV * u, d);
+                uint32_t d[32];
+                tmem_ld32(tmem + lane_base + kDV * u + col0, d);
                 tmem_wait_ld();
                 uint8_t *urow = sm + SB_U + i * 128;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < 4; ++q) {
                     const uint32_t uw[4] = {ut[q].x, ut[q].y, ut[q].z, ut[q].w};
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         w[e] = pack_bf16x2(bf16_lo(uw[e]) + __uint_as_float(d[8 * q + 2 * e]),
                                            bf16_hi(uw[e]) + __uint_as_float(d[8 * q + 2 * e + 1]));
-                    *reinterpret_cast<uint4 *>(urow + ((q ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(urow + (((4 * half + q) ^ (i & 7)) << 4)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -982,19 +987,19 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
             if (!wait(BAR_S, c & 1)) break;
             tc_fence_after();
             {
-                uint32_t d[64];
-                tmem_ld64(tmem + lane_base + 2 * kDV, d);
+                uint32_t d[32];
+                tmem_ld32(tmem + lane_base + 2 * kDV + col0, d);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < kDV; ++e) st[e] = fmaf(gam, st[e], __uint_as_float(d[e]));
+                for (int e = 0; e < 32; ++e) st[e] = fmaf(gam, st[e], __uint_as_float(d[e]));
             }
             tc_fence_before();
             if (c + 1 < nseg && !publish_m(c + 1)) break;
         }
         if (!*s_abort) {
-            float4 *dst = reinterpret_cast<float4 *>(Mg + (size_t)i * kD);
+            float4 *dst = reinterpret_cast<float4 *>(Mg + (size_t)i * kD + col0);
 #pragma unroll
-            for (int q = 0; q < kDV / 4; ++q)
+            for (int q = 0; q < 8; ++q)
                 dst[q] = make_float4(st[4 * q], st[4 * q + 1], st[4 * q + 2], st[4 * q + 3]);
         }
     }
