@@ -20,8 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libhmd.so")
 SOURCES = ["hmd_api.cu", "delta_decode.cu", "attn_decode.cu", "delta_prefill.cu",
-           "attn_decode_static.cu", "delta_prefill_tc.cu", "attn_prefill.cu",
-           "attn_prefill_tc.cu",
+           "attn_decode_static.cu", "delta_prefill_tc.cu", "attn_prefill_tc.cu",
            "tmap.cu"]
 HEADERS = ["ptx.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

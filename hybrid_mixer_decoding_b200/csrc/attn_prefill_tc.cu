@@ -1,8 +1,9 @@
-// FA / SWA prefill on the 5th-generation tensor cores (tcgen05, TMEM), d = 128.
+// FA / SWA prefill on the 5th-generation tensor cores (tcgen05, TMEM), d = 64 or 128.
 //
-// Same operation, layouts and cache write as attn_prefill.cu (FA and SWA from the gist.science
-// technical summary of "Super Apriel: One Checkpoint, Many Speeds", sections 1 and 2a): token t
-// attends keys [lo_t, t], lo_t = 0 (FA) or max(0, t + 1 - w) (SWA).
+// FA and SWA from the gist.science technical summary of "Super Apriel: One Checkpoint, Many
+// Speeds", sections 1 and 2a: token t of a prompt attends keys [lo_t, t], lo_t = 0 (FA) or
+// max(0, t + 1 - w) (SWA), and the prompt's K and V are written to the paged cache at the slots
+// the decode step reads (SWA: the positions the ring of ceil(w / 64) pages keeps).
 //
 // One CTA per (sequence, kv-head, block of 128/G tokens), warp-specialised:
 //   warp 8 (one lane) issues the TMA copies of the K/V tiles (4-stage ring, 3-D boxes from the
@@ -38,23 +39,27 @@ namespace {
 
 __device__ unsigned int g_err;
 
-constexpr int kD = 128;
 constexpr int kPT = 64;          // keys per tile = tokens per page
 constexpr int kStages = 4;       // K/V tiles in flight
 constexpr int kSoftmax = 256;    // softmax threads (warps 0-7)
 constexpr int kThreads = kSoftmax + 32;  // + the TMA / MMA warp
 constexpr int kRows = 128;
-constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, PV at 128
+constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, PV at 128 (D columns)
 
-// shared memory (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;                  // Q [128 rows][128 dims]: 2 halves of 16 KiB
-constexpr uint32_t OFF_KV = 32768;             // stage s: K at +0, V at +16384 (2 halves each)
-constexpr uint32_t STAGE = 32768;
-constexpr uint32_t OFF_P = OFF_KV + kStages * STAGE;  // P [128 rows][64 keys] x 2 buffers
-constexpr uint32_t P_BYTES = 16384;
-constexpr uint32_t OFF_RED = OFF_P + 2 * P_BYTES;     // partial row maxima [2 tiles][2][128]
-constexpr uint32_t OFF_BAR = OFF_RED + 2048;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+// shared memory (bytes from a 1024-aligned base) for head size D (64 or 128): tiles are stored as
+// D / 64 blocks of [rows][128 B] with the 128-byte swizzle
+template <int D>
+struct Smem {
+    static constexpr uint32_t OFF_Q = 0;                  // Q [128 rows][D]: blocks of 16 KiB
+    static constexpr uint32_t OFF_KV = kRows * D * 2;     // stage s: K at +0, V at +STAGE / 2
+    static constexpr uint32_t STAGE = 2 * kPT * D * 2;
+    static constexpr uint32_t OFF_P = OFF_KV + kStages * STAGE;  // P [128 rows][64 keys] x 2
+    static constexpr uint32_t P_BYTES = 16384;
+    static constexpr uint32_t OFF_RED = OFF_P + 2 * P_BYTES;     // row maxima [2 tiles][2][128]
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2048;
+    static constexpr uint32_t BYTES = OFF_BAR + 128 + 1024;
+};
+static_assert(Smem<128>::BYTES <= 232448, "shared memory per CTA");
 // barrier indices
 constexpr int B_FULL = 0;    // [4] K/V tile landed (TMA)
 constexpr int B_SFULL = 4;   // [2] S_i computed (commit)
@@ -65,7 +70,22 @@ constexpr int N_BARS = 11;
 constexpr float kLazy = 8.f;  // log2 headroom before the exponent base moves
 
 constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);    // A = Q (K-major), B = K (K-major)
-constexpr uint32_t ID_PV = idesc_bf16(128, 128, 0, 1);  // A = P (K-major), B = V (MN-major)
+template <int D>
+constexpr uint32_t ID_PV = idesc_bf16(128, D, 0, 1);     // A = P (K-major), B = V (MN-major)
+
+// 2^x on the FMA pipe, for x <= 8: 2^x = 2^n 2^f with n = floor(x), f = x - n in [0, 1), and 2^f
+// by a cubic fitted to it on [0, 1) (least squares at Chebyshev nodes, reweighted towards the
+// minimax fit; largest relative error 7.5e-5, far below the bf16 rounding of P). x is clamped at
+// -126, where 2^x is below fp32's normal range and its share of a row sum that holds an entry
+// >= 1 is nil. Splitting the exponentials between this and ex2.approx keeps the softmax off a
+// single pipe.
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -126.f);
+    const float n = floorf(x);
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(0.07802451f, f, 0.22606717f), f, 0.69583356f), f, 0.99992520f);
+    return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
+}
 
 struct TcParams {
     const __nv_bfloat16 *q, *k, *v;
@@ -106,12 +126,16 @@ __device__ __forceinline__ void softmax_barrier() {  // warps 0-7 only (named ba
 }
 
 // PREFIX: sequences may start after cached positions (p.prefix_lens); false compiles the
-// empty-cache prefill with every prefix path removed.
-template <bool PREFIX>
+// empty-cache prefill with every prefix path removed. D: head size, 64 or 128.
+template <int D, bool PREFIX>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                        const __grid_constant__ CUtensorMap tmpk,
                        const __grid_constant__ CUtensorMap tmpv, const TcParams p) {
+    using L = Smem<D>;
+    constexpr uint32_t OFF_Q = L::OFF_Q, OFF_KV = L::OFF_KV, STAGE = L::STAGE, OFF_P = L::OFF_P,
+                       P_BYTES = L::P_BYTES, OFF_RED = L::OFF_RED, OFF_BAR = L::OFF_BAR;
+    constexpr int kD = D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -175,7 +199,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
         const uint4 *src = reinterpret_cast<const uint4 *>(
             p.q + (((size_t)b * p.T + (row_ok ? t_row : 0)) * p.Hq + h_row) * kD);
 #pragma unroll
-        for (int c = ch * 8; c < ch * 8 + 8; ++c) {
+        for (int c = ch * (kD / 16); c < (ch + 1) * (kD / 16); ++c) {
             const uint4 v = row_ok ? src[c] : make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(sm + OFF_Q + swz(row, c * 8, kRows)) = v;
         }
@@ -213,7 +237,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             int tiles_issued = 0, s_issued = 0, pv_issued = 0;
             auto issue_tile = [&](int i) {
                 const int st = i % kStages;
-                const uint32_t kb = sb + OFF_KV + st * STAGE, vb = kb + 16384;
+                const uint32_t kb = sb + OFF_KV + st * STAGE, vb = kb + STAGE / 2;
                 const int key0 = (kb_lo + i) * kPT;  // first position of the tile
                 if (PREFIX && key0 < L0) {  // a page of the cached prefix
                     const int lp = (kb_lo + i) % (p.swa ? p.ring_pages : 0x7fffffff);
@@ -226,16 +250,16 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);
                     const int y = (pg * p.Hkv + g) * kPT;
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
+                    for (int hf = 0; hf < kD / 64; ++hf) {
                         tma_load_2d(kb + hf * 8192, &tmpk, bar(B_FULL + st), hf * 64, y);
                         tma_load_2d(vb + hf * 8192, &tmpv, bar(B_FULL + st), hf * 64, y);
                     }
                     return;
                 }
-                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: 4 boxes of 8 KiB
+                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: boxes of 8 KiB
                 const int z = b * p.T + (key0 - L0);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < kD / 64; ++hf) {
                     tma_load_3d(kb + hf * 8192, &tmk, bar(B_FULL + st), hf * 64, g, z);
                     tma_load_3d(vb + hf * 8192, &tmv, bar(B_FULL + st), hf * 64, g, z);
                 }
@@ -252,12 +276,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             };
             auto issue_pv = [&](int i, bool fresh) {  // fresh: restart the TMEM sum
                 const uint32_t pbase = sb + OFF_P + (i & 1) * P_BYTES;
-                const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + 16384;
+                const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + STAGE / 2;
 #pragma unroll
                 for (int kk = 0; kk < kPT / 16; ++kk) {
                     const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
                     const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-                    umma_bf16(tmem + 128, ad, bd, ID_PV, (kk > 0 || !fresh) ? 1u : 0u);
+                    umma_bf16(tmem + 128, ad, bd, ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
                 }
                 umma_commit(bar(B_PVFULL));
             };
@@ -368,7 +392,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
 #pragma unroll
                         for (int c4 = 0; c4 < kD / 64; ++c4) {
                             uint32_t r[32];
-                            tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
+                            tmem_ld32(lane_base + 128 + ch * (kD / 2) + c4 * 32, r);
                             tmem_wait_ld();
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
@@ -390,7 +414,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     float e[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        e[u] = ex2_approx(fmaf(s[c * 8 + u], p.scale_log2, -mu));
+                        const float x = fmaf(s[c * 8 + u], p.scale_log2, -mu);
+                        e[u] = (u & 3) == 3 ? exp2_fma(x) : ex2_approx(x);
                         ls += e[u];
                     }
                     if (ok)
@@ -414,7 +439,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
 #pragma unroll
             for (int c4 = 0; c4 < kD / 64; ++c4) {
                 uint32_t r[32];
-                tmem_ld32(lane_base + 128 + ch * 64 + c4 * 32, r);
+                tmem_ld32(lane_base + 128 + ch * (kD / 2) + c4 * 32, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) o[c4 * 32 + j] += __uint_as_float(r[j]);
@@ -423,7 +448,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                 const float l = lb[row] + lb[kRows + row];
                 const float inv = l > 0.f ? 1.f / l : 0.f;
                 uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.o + (((size_t)b * p.T + t_row) * p.Hq + h_row) * kD + ch * 64);
+                    p.o + (((size_t)b * p.T + t_row) * p.Hq + h_row) * kD + ch * (kD / 2));
 #pragma unroll
                 for (int c = 0; c < kD / 16; ++c)
                     dst[c] = make_uint4(pack_bf16x2(o[c * 8] * inv, o[c * 8 + 1] * inv),
@@ -447,7 +472,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
 // The SWA ring write of a prompt that followed a cached prefix, after the attention kernel has
 // read every prefix key: the last R*64 positions of the prompt (the ones the ring keeps), one
 // 16-byte chunk of K or V per thread.
+template <int D>
 __global__ void __launch_bounds__(256) attn_prefill_ring_write_kernel(const TcParams p) {
+    constexpr int kD = D;
     griddep_launch_dependents();
     griddep_wait();  // the attention kernel has read the ring
     const int ring = p.ring_pages * kPT;
@@ -484,29 +511,31 @@ __global__ void __launch_bounds__(256) attn_prefill_ring_write_kernel(const TcPa
 
 bool attn_prefill_tc_supported(int d, int page_tokens, int group) {
     const bool g_ok = group == 1 || group == 2 || group == 4 || group == 8 || group == 16;
-    return d == kD && page_tokens == kPT && g_ok;
+    return (d == 64 || d == 128) && page_tokens == kPT && g_ok;
 }
 
-cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
-    if (a.B == 0 || a.T == 0) return cudaSuccess;
+namespace {
+template <int D>
+cudaError_t launch_tc(const AttnPrefillArgs &a, cudaStream_t s) {
+    constexpr uint32_t kSmem = Smem<D>::BYTES;
     const cudaError_t attr_err = once_per_device([] {
-        cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<false>,
+        cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
+                                             (int)Smem<D>::BYTES);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(attn_prefill_tc_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+            e = cudaFuncSetAttribute(attn_prefill_tc_kernel<D, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem<D>::BYTES);
         return e;
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap tmk, tmv, tmpk, tmpv;
     const long long n_tok = (long long)a.B * a.T;
-    if (!make_tmap_tokens_sw128(&tmk, const_cast<void *>(a.k), n_tok, a.Hkv, kD) ||
-        !make_tmap_tokens_sw128(&tmv, const_cast<void *>(a.v), n_tok, a.Hkv, kD))
+    if (!make_tmap_tokens_sw128(&tmk, const_cast<void *>(a.k), n_tok, a.Hkv, D) ||
+        !make_tmap_tokens_sw128(&tmv, const_cast<void *>(a.v), n_tok, a.Hkv, D))
         return cudaErrorInvalidValue;
     if (a.prefix_lens) {
-        if (!make_tmap_pool_sw128(&tmpk, a.k_pool, a.n_pages, a.Hkv, kD) ||
-            !make_tmap_pool_sw128(&tmpv, a.v_pool, a.n_pages, a.Hkv, kD))
+        if (!make_tmap_pool_sw128(&tmpk, a.k_pool, a.n_pages, a.Hkv, D) ||
+            !make_tmap_pool_sw128(&tmpv, a.v_pool, a.n_pages, a.Hkv, D))
             return cudaErrorInvalidValue;
     } else {
         tmpk = tmk;  // not read
@@ -531,18 +560,34 @@ cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     p.window = a.window; p.swa = a.swa ? 1 : 0;
     p.ring_pages = a.swa ? (a.window + kPT - 1) / kPT : 0;
     p.max_pages = a.max_pages; p.n_pages = a.n_pages;
-    p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     const long long grid = (long long)p.n_qb * a.B * a.Hkv;
     cudaError_t e = a.prefix_lens
-        ? launch_pdl(attn_prefill_tc_kernel<true>, dim3((unsigned)grid), dim3(kThreads),
-                     SMEM_BYTES, s, tmk, tmv, tmpk, tmpv, p)
-        : launch_pdl(attn_prefill_tc_kernel<false>, dim3((unsigned)grid), dim3(kThreads),
-                     SMEM_BYTES, s, tmk, tmv, tmpk, tmpv, p);
+        ? launch_pdl(attn_prefill_tc_kernel<D, true>, dim3((unsigned)grid), dim3(kThreads), kSmem,
+                     s, tmk, tmv, tmpk, tmpv, p)
+        : launch_pdl(attn_prefill_tc_kernel<D, false>, dim3((unsigned)grid), dim3(kThreads), kSmem,
+                     s, tmk, tmv, tmpk, tmpv, p);
     if (e != cudaSuccess || !p.defer_write) return e;
     const int ring = p.ring_pages * kPT;
-    const long long n = (long long)a.B * std::min(a.T, ring) * a.Hkv * 2 * (kD / 8);
+    const long long n = (long long)a.B * std::min(a.T, ring) * a.Hkv * 2 * (D / 8);
     const unsigned blocks = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 16);
-    return launch_pdl(attn_prefill_ring_write_kernel, dim3(blocks), dim3(256), 0, s, p);
+    return launch_pdl(attn_prefill_ring_write_kernel<D>, dim3(blocks), dim3(256), 0, s, p);
+}
+}  // namespace
+
+cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s) {
+    if (a.B == 0 || a.T == 0) return cudaSuccess;
+    if (a.d == 128) return launch_tc<128>(a, s);
+    if (a.d == 64) return launch_tc<64>(a, s);
+    return cudaErrorInvalidValue;
+}
+
+bool attn_prefill_supported(int d, int page_tokens, int group) {
+    return attn_prefill_tc_supported(d, page_tokens, group);
+}
+
+cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s) {
+    return launch_attn_prefill_tc(a, s);
 }
 
 uint32_t attn_prefill_tc_read_errors(bool clear) {

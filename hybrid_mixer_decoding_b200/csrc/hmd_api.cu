@@ -122,7 +122,7 @@ hmd_status_t hmd_device_errors(hmd_stream_t stream, uint32_t *bits, int clear) {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return fail(HMD_ERR_CUDA);
     *bits = hmd::delta_decode_read_errors(clear != 0) | hmd::attn_decode_read_errors(clear != 0) |
             hmd::delta_prefill_read_errors(clear != 0) | hmd::delta_prefill_scan_read_errors(clear != 0) |
-            hmd::attn_prefill_read_errors(clear != 0) | hmd::attn_prefill_tc_read_errors(clear != 0);
+            hmd::attn_prefill_tc_read_errors(clear != 0);
     return HMD_OK;
 }
 
@@ -381,17 +381,14 @@ hmd_status_t attn_prefill_ext(hmd_kind_t kind, int window, int B, int T, int Hq,
     if (B == 0 || T == 0) return HMD_OK;
     if (!q || !k || !v || !k_pool || !v_pool || !page_table || !o) return fail(HMD_ERR_ARG);
     if (!hmd::attn_prefill_supported(d, page_tokens, Hq / Hkv)) return fail(HMD_ERR_UNSUPPORTED);
-    // a cached prefix is read by the tensor-core kernel only
-    if (prefix_lens && !hmd::attn_prefill_tc_supported(d, page_tokens, Hq / Hkv))
-        return fail(HMD_ERR_UNSUPPORTED);
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_pool) ||
-        !aligned16(v_pool))
-        return fail(HMD_ERR_ARG);
     const long long span = (long long)(prefix_lens ? max_prefix : 0) + T;
     const long long need = kind == HMD_SWA ? (window + page_tokens - 1) / page_tokens
                                            : (span + page_tokens - 1) / page_tokens;
     if (max_pages < need) return fail(HMD_ERR_SHAPE);
     if ((long long)n_pages * Hkv * page_tokens >= (1LL << 31)) return fail(HMD_ERR_UNSUPPORTED);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_pool) ||
+        !aligned16(v_pool))
+        return fail(HMD_ERR_ARG);
     hmd::AttnPrefillArgs a{};
     a.swa = kind == HMD_SWA; a.window = window; a.B = B; a.T = T; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
     a.page_tokens = page_tokens; a.q = q; a.k = k; a.v = v; a.k_pool = k_pool; a.v_pool = v_pool;

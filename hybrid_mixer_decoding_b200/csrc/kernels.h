@@ -189,7 +189,7 @@ struct DeltaPrefillArgs {
 cudaError_t launch_delta_prefill(const DeltaPrefillArgs &a, cudaStream_t s);
 bool delta_prefill_supported(int dk, int dv, bool bf16, int chunk);
 uint32_t delta_prefill_read_errors(bool clear);
-// FA / SWA prefill from an empty cache (attn_prefill.cu)
+// FA / SWA prefill of a prompt into the paged cache (attn_prefill_tc.cu)
 struct AttnPrefillArgs {
     bool swa;
     int window;
@@ -206,8 +206,7 @@ struct AttnPrefillArgs {
 };
 bool attn_prefill_supported(int d, int page_tokens, int group);
 cudaError_t launch_attn_prefill(const AttnPrefillArgs &a, cudaStream_t s);
-uint32_t attn_prefill_read_errors(bool clear);
-// tcgen05 path (d = 128); launch_attn_prefill dispatches to it
+// the tcgen05 kernel (d = 64 or 128) behind launch_attn_prefill
 bool attn_prefill_tc_supported(int d, int page_tokens, int group);
 cudaError_t launch_attn_prefill_tc(const AttnPrefillArgs &a, cudaStream_t s);
 uint32_t attn_prefill_tc_read_errors(bool clear);

@@ -286,7 +286,7 @@ HMD_API hmd_status_t attn_prefill(hmd_kind_t kind, int window, int B, int T, int
  *   prefix_lens: device int32 [B], each a multiple of page_tokens and <= max_prefix (a host
  *   bound, itself a multiple of page_tokens); NULL is attn_prefill. FA needs
  *   max_pages >= ceil((max_prefix + T) / page_tokens).
- * Supported with a prefix: d = 128 (the tensor-core kernel), else HMD_ERR_UNSUPPORTED. A prefix
+ * Supported with a prefix: d in {64, 128}, as without one. A prefix
  * length that is not a whole number of pages sets HMD_DEVERR_SEQLEN (that sequence then runs as
  * if it had none).                                                                            */
 HMD_API hmd_status_t attn_prefill_ext(hmd_kind_t kind, int window, int B, int T, int Hq, int Hkv,

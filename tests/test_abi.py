@@ -120,18 +120,21 @@ def test_verify_validation():
     assert _verify(n_q=0) == SHAPE
     assert _verify(n_q=5) == UNSUP               # 5 tokens x GQA group 4 > 16 MMA rows
     assert _verify(n_q=4, Hq=16, Hkv=2) == UNSUP  # 4 x 8 > 16
-    assert _verify(n_q=16, Hq=8, Hkv=8) != UNSUP  # 16 x 1 rows fit
+    # a call that passes every check gets misaligned pointers (HMD_ERR_ARG, the last check
+    # before the launch), so that none of these calls can launch anything
+    MIS = FAKE + 2
+    assert _verify(n_q=16, Hq=8, Hkv=8, ptr=MIS) == ARG  # 16 x 1 rows fit
     # SWA ring must hold window + n_q - 1 = 103 positions: 2 pages of 64
     assert _verify(window=128, ring=2) == SHAPE  # 131 positions need 3 pages
-    assert _verify(window=128, ring=3, max_pages=3) != SHAPE
+    assert _verify(window=128, ring=3, max_pages=3, ptr=MIS) == ARG
     assert _verify(window=128, ring=3, max_pages=2, max_len=256) == SHAPE  # table < ring
-    assert _verify(window=128, ring=3, max_pages=2, max_len=100) != SHAPE  # short sequences
+    assert _verify(window=128, ring=3, max_pages=2, max_len=100, ptr=MIS) == ARG  # short sequences
     assert _verify(kind=hmd.FA, ring=0, max_pages=3) == SHAPE  # FA table < 256 tokens
     assert _verify(ws=16) == SHAPE
     assert _verify(ptr=None) == ARG
     assert _verify(B=0) == 0
     # one token on the default ring is the decode step's validation
-    assert _verify(window=4096, ring=64, n_q=1, max_pages=64, max_len=8192) != SHAPE
+    assert _verify(window=4096, ring=64, n_q=1, max_pages=64, max_len=8192, ptr=MIS) == ARG
     assert _verify(window=4096, ring=64, n_q=2, max_pages=64, max_len=8192) == SHAPE
 
 
@@ -217,15 +220,20 @@ def test_fused_activation_validation():
 
 
 def test_prefill_with_prefix_validation():
+    """Calls that pass every check get a misaligned output pointer, the last check before the
+    launch (HMD_ERR_ARG), so that none of them can launch anything."""
     L = hmd.lib()
-    ext = lambda d=128, max_prefix=128, max_pages=8, T=64, kind=hmd.FA, w=0, pre=FAKE: (  # noqa: E731
+    MIS = FAKE + 2
+    ext = lambda d=128, max_prefix=128, max_pages=8, T=64, kind=hmd.FA, w=0, pre=FAKE, o=MIS: (  # noqa: E731
         L.attn_prefill_ext(kind, w, 2, T, 8, 2, d, 64, FAKE, FAKE, FAKE, pre, max_prefix, FAKE,
-                           FAKE, 16, FAKE, max_pages, FAKE, None))
-    assert ext(d=64) == UNSUP                  # a prefix needs the tensor-core kernel (d = 128)
-    assert ext(d=64, pre=None) != UNSUP        # no prefix: the d = 64 kernel is fine
+                           FAKE, 16, FAKE, max_pages, o, None))
+    assert ext() == ARG                        # every shape check passes
+    assert ext(d=64) == ARG                    # d = 64 takes a cached prefix too
+    assert ext(d=64, pre=None) == ARG
+    assert ext(d=96) == UNSUP
     assert ext(max_prefix=100) == SHAPE        # not a whole number of pages
     assert ext(max_prefix=512, max_pages=8) == SHAPE  # FA table < (512 + 64) / 64 = 9 pages
-    assert ext(max_prefix=448, max_pages=8) != SHAPE
+    assert ext(max_prefix=448, max_pages=8) == ARG
     assert ext(max_prefix=-64) == SHAPE
     assert ext(T=0) == 0
 

@@ -49,6 +49,8 @@ def expected_pools(O, a: I.AttnPrefillInputs):
 
 CASES = [  # kind, window, B, T, Hq, Hkv, d
     (I.FA, 0, 2, 1, 8, 2, 128),
+    (I.FA, 0, 2, 1, 8, 2, 64),
+    (I.FA, 0, 1, 300, 16, 1, 64),     # G = 16 at d = 64
     (I.FA, 0, 2, 63, 8, 2, 128),
     (I.FA, 0, 2, 200, 8, 2, 128),
     (I.FA, 0, 1, 130, 8, 8, 128),     # G = 1: 128 tokens per block
@@ -168,24 +170,26 @@ def expected_pools_after_prefix(O, a: I.AttnVerifyInputs, T):
     return ek, ev
 
 
-PREFIX_CASES = [  # kind, window, T, Hq, Hkv, prefix lengths (multiples of 64)
-    (I.FA, 0, 200, 8, 2, [0, 64, 640]),
-    (I.FA, 0, 1, 8, 2, [128, 0, 64]),
-    (I.FA, 0, 130, 8, 8, [64, 192]),      # G = 1
-    (I.FA, 0, 70, 16, 1, [256, 64]),      # G = 16
-    (I.SWA, 100, 150, 8, 2, [0, 64, 640]),  # ring of 2 pages, prompt longer than the ring
-    (I.SWA, 64, 40, 8, 2, [128, 64]),
-    (I.SWA, 300, 500, 32, 8, [320, 1024]),
+PREFIX_CASES = [  # kind, window, T, Hq, Hkv, prefix lengths (multiples of 64), d
+    (I.FA, 0, 200, 8, 2, [0, 64, 640], 128),
+    (I.FA, 0, 1, 8, 2, [128, 0, 64], 128),
+    (I.FA, 0, 130, 8, 8, [64, 192], 128),      # G = 1
+    (I.FA, 0, 70, 16, 1, [256, 64], 128),      # G = 16
+    (I.SWA, 100, 150, 8, 2, [0, 64, 640], 128),  # ring of 2 pages, prompt longer than the ring
+    (I.SWA, 64, 40, 8, 2, [128, 64], 128),
+    (I.SWA, 300, 500, 32, 8, [320, 1024], 128),
+    (I.FA, 0, 200, 8, 2, [0, 64, 640], 64),
+    (I.SWA, 100, 150, 8, 4, [0, 128, 640], 64),
 ]
 
 
-@pytest.mark.parametrize("kind,window,T,Hq,Hkv,prefixes", PREFIX_CASES)
-def test_prefill_after_prefix_matches_oracle(oracle_mod, kind, window, T, Hq, Hkv, prefixes):
+@pytest.mark.parametrize("kind,window,T,Hq,Hkv,prefixes,d", PREFIX_CASES)
+def test_prefill_after_prefix_matches_oracle(oracle_mod, kind, window, T, Hq, Hkv, prefixes, d):
     O = oracle_mod
     pre = np.array(prefixes, np.int32)
     lens = pre + T
     ring = -(-window // 64) if kind == I.SWA else 0
-    a = I.verify_inputs(kind, len(pre), T, Hq, Hkv, 128, int(lens.max()), window=window,
+    a = I.verify_inputs(kind, len(pre), T, Hq, Hkv, d, int(lens.max()), window=window,
                         ring_pages=ring, seed=int(lens.sum()) + T, seq_lens=lens)
     o, kp, vp = run_prefill_ext(a, T)
     ref = O.attn_verify(kind, window, a.ring_pages, a.q, a.new_k, a.new_v, a.k_pool, a.v_pool,
