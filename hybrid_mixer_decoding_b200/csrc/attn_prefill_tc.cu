@@ -264,25 +264,26 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     tma_load_3d(vb + hf * 8192, &tmv, bar(B_FULL + st), hf * 64, g, z);
                 }
             };
+            // descriptors: the address field is the byte address / 16, so an offset is added as
+            // offset / 16 (every address here is below 256 KiB: no carry out of the field)
+            const uint64_t d_q = smem_desc_sw128(sb + OFF_Q, 16, 1024);
+            const uint64_t d_k = smem_desc_sw128(sb + OFF_KV, 16, 1024);
+            const uint64_t d_p = smem_desc_sw128(sb + OFF_P, 16, 1024);
+            const uint64_t d_v = smem_desc_sw128(sb + OFF_KV + STAGE / 2, 8192, 1024);
             auto issue_s = [&](int i) {
-                const uint32_t kbase = sb + OFF_KV + (i % kStages) * STAGE;
+                const uint64_t ko = ((i % kStages) * STAGE) >> 4;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(sb + OFF_Q + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    umma_bf16(tmem + (i & 1) * 64, ad, bd, ID_S, kk > 0);
-                }
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    umma_bf16(tmem + (i & 1) * 64, d_q + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                              d_k + ko + ((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), ID_S, kk > 0);
                 umma_commit(bar(B_SFULL + (i & 1)));
             };
             auto issue_pv = [&](int i, bool fresh) {  // fresh: restart the TMEM sum
-                const uint32_t pbase = sb + OFF_P + (i & 1) * P_BYTES;
-                const uint32_t vbase = sb + OFF_KV + (i % kStages) * STAGE + STAGE / 2;
+                const uint64_t po = ((i & 1) * P_BYTES) >> 4, vo = ((i % kStages) * STAGE) >> 4;
 #pragma unroll
-                for (int kk = 0; kk < kPT / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(pbase + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, 8192, 1024);
-                    umma_bf16(tmem + 128, ad, bd, ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kPT / 16; ++kk)
+                    umma_bf16(tmem + 128, d_p + po + ((kk * 32) >> 4), d_v + vo + ((kk * 2048) >> 4),
+                              ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
                 umma_commit(bar(B_PVFULL));
             };
             bool ok = true;
@@ -361,19 +362,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
             // ---- mask (edge tiles only), partial maximum; a restart if it outgrows the base ----
             const int j0 = (kb_lo + i) * kPT + ch * 32;
-            float mx = -INFINITY;
-            if (row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= pos_row) {
-#pragma unroll
-                for (int j = 0; j < kPT / 2; ++j) mx = fmaxf(mx, s[j]);
-            } else {
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // short chains
+            if (!(row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= pos_row)) {
 #pragma unroll
                 for (int j = 0; j < kPT / 2; ++j) {
                     const int key = j0 + j;
                     const bool valid = row_ok && key >= lo_row && key <= pos_row;
                     s[j] = valid ? s[j] : -INFINITY;
-                    mx = fmaxf(mx, s[j]);
                 }
             }
+#pragma unroll
+            for (int j = 0; j < kPT / 2; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
+            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;  // scores and maxima in the log2 domain from here on
             float *rb = red + (i & 1) * 2 * kRows;
             rb[ch * kRows + row] = mx;
@@ -407,7 +407,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             const float mu = (m_base == -INFINITY) ? 0.f : m_base;
             // ---- P_i half row -> shared memory (its buffer's last reader, PV_{i-2}, is done) ---
             {
-                float ls = 0.f;
+                float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short chains
                 uint8_t *prow = sm + OFF_P + (i & 1) * P_BYTES;
 #pragma unroll
                 for (int c = 0; c < kPT / 16; ++c) {
@@ -416,14 +416,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     for (int u = 0; u < 8; ++u) {
                         const float x = fmaf(s[c * 8 + u], p.scale_log2, -mu);
                         e[u] = (u & 3) == 3 ? exp2_fma(x) : ex2_approx(x);
-                        ls += e[u];
+                        ls4[u & 3] += e[u];
                     }
                     if (ok)
                         *reinterpret_cast<uint4 *>(prow + swz(row, ch * 32 + c * 8, kRows)) =
                             make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
                                        pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
                 }
-                l_run += ls;
+                l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
             }
             fence_proxy_async_smem();  // P is read by the tensor cores
             __syncwarp();
