@@ -367,40 +367,45 @@ def run_ours(args, rank, world, local_rank):
 
 
 def placement_switch(st, warmup: int) -> dict:
-    """Latency of a placement switch on a registered stack: eager steps with CUDA events around
-    each whole step. Steady steps of each placement, then alternating steps (each one the first
-    after a switch). A switch passes another placement array; no cache is copied or reloaded,
-    so the first step after a switch should cost what a steady step of its placement costs."""
+    """Latency of a placement switch on a registered stack. Each placement's step is one CUDA-graph
+    replay of its 48 mixer_decode_step calls (captured on the same caches), so the steps are
+    GPU-bound; steady replays of each placement are timed, then alternating replays (each one
+    the first step after a switch), all with CUDA events around every step. A switch passes
+    another placement array: no cache is copied or reloaded, so the first step after a switch
+    should cost what a steady step of its placement costs."""
     import torch
+
+    graphs = {nm: st.capture(nm, warmup=1) for nm in ("hybrid", "all_gdn")}
 
     def timed_steps(names):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in names]
         for (a, b), nm in zip(evs, names):
             a.record()
-            st.step(nm)
+            graphs[nm].replay()
             b.record()
         torch.cuda.synchronize()
         return [a.elapsed_time(b) for a, b in evs]
 
-    for nm in ("hybrid", "all_gdn"):
+    for nm in graphs:
         for _ in range(max(1, warmup // 2)):
-            st.step(nm)
-    n = 5
+            graphs[nm].replay()
+    n = 6
     steady_h = timed_steps(["hybrid"] * n)[1:]
     steady_g = timed_steps(["all_gdn"] * n)[1:]
     alt = timed_steps(["hybrid", "all_gdn"] * n)
     to_h = alt[0::2][1:]  # every hybrid step here directly follows an all-GDN step
     to_g = alt[1::2]
+    del graphs
     sh, sg = float(np.median(steady_h)), float(np.median(steady_g))
     fh, fg = float(np.median(to_h)), float(np.median(to_g))
     return {"steady_step_ms": {"hybrid": round(sh, 4), "all_gdn": round(sg, 4)},
             "first_step_after_switch_ms": {"to_hybrid": round(fh, 4), "to_all_gdn": round(fg, 4)},
             "switch_cost_us": {"to_hybrid": round((fh - sh) * 1e3, 1),
                                "to_all_gdn": round((fg - sg) * 1e3, 1)},
-            "how": "medians of eager steps timed with CUDA events; a switch passes another "
-                   "placement array to mixer_decode_step (the caches of both placements stay "
-                   "registered: nothing is copied or reloaded)"}
+            "how": "medians of CUDA-graph replays of each placement's step timed with CUDA "
+                   "events; a switch is a replay of the other placement's graph on the same "
+                   "registered caches (nothing is copied or reloaded)"}
 
 
 # ------------------------------------------------------------------------------------------

@@ -5,17 +5,20 @@
 // max(0, t + 1 - w) (SWA), and the prompt's K and V are written to the paged cache at the slots
 // the decode step reads (SWA: the positions the ring of ceil(w / 64) pages keeps).
 //
-// One CTA per (sequence, kv-head, block of 128/G tokens), warp-specialised:
-//   warp 8 (one lane) issues the TMA copies of the K/V tiles (4-stage ring, 3-D boxes from the
-//     prompt, 128-byte swizzle) and the tcgen05.mma products:
-//       S_i = Q K_i^T   M=128 N=64 K=128 (Q and K K-major) into TMEM buffer i & 1
-//       PV_i = P_i V_i  M=128 N=128 K=64 (P K-major, V MN-major) into TMEM
-//     in the order PV_{i-1}, S_{i+1}, so the tensor core works on them while the softmax warps
-//     process tile i;
+// One CTA per (sequence, kv-head, block of 128/G tokens), warp-specialised, key tiles of 128:
+//   warp 8 (one lane) issues the TMA copies of the K and V tiles (two rings of two stages each,
+//     3-D boxes of 64 tokens from the prompt or 2-D boxes of one page from the cache, 128-byte
+//     swizzle) and the tcgen05.mma products
+//       S_i = Q K_i^T   M=128 N=128 K=d (Q and K K-major) into TMEM buffer i & 1
+//       PV_i = P_i V_i  M=128 N=d K=128 (P K-major, V MN-major) into TMEM
+//     in the order PV_i, S_{i+2}, so the tensor core works on them while the softmax warps
+//     process tile i+1. A K stage is reloaded as soon as the S product that read it is done,
+//     a V stage once its PV product is;
 //   warps 0-7 run the softmax: query row r (head g*G + r / QT, token t_first + r % QT) is TMEM
-//     lane r; threads r and r + 128 split its columns (half of the scores, half of the output)
+//     lane r; threads r and r + 128 split its columns (64 of the 128 scores, half of the output)
 //     and exchange partial maxima through one 256-thread named barrier per tile. They read S
-//     with tcgen05.ld and write P (bf16) to shared memory in the swizzled K-major layout.
+//     with tcgen05.ld and write P (bf16) to shared memory in the swizzled K-major layout, once
+//     the previous tile's PV product has read it.
 // Lazy rescaling: PV accumulates in TMEM across tiles at a fixed exponent base per row, which
 // moves only when some row's maximum exceeds its base by more than 8 (P stays below 2^8). On
 // such a tile every row folds the TMEM accumulator into an fp32 register accumulator at the new
@@ -39,52 +42,96 @@ namespace {
 
 __device__ unsigned int g_err;
 
-constexpr int kPT = 64;          // keys per tile = tokens per page
-constexpr int kStages = 4;       // K/V tiles in flight
+constexpr int kPT = 64;          // tokens per page = keys per TMA box
+constexpr int kKT = 128;         // keys per tile
 constexpr int kSoftmax = 256;    // softmax threads (warps 0-7)
 constexpr int kThreads = kSoftmax + 32;  // + the TMA / MMA warp
 constexpr int kRows = 128;
-constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, PV at 128 (D columns)
+constexpr uint32_t kTmemCols = 512;  // S buffers at 0 and 128, PV at 256 (D columns)
+constexpr uint32_t kColPV = 256;
 
-// shared memory (bytes from a 1024-aligned base) for head size D (64 or 128): tiles are stored as
-// D / 64 blocks of [rows][128 B] with the 128-byte swizzle
+// shared memory (bytes from a 1024-aligned base) for head size D (64 or 128). Every operand tile
+// is stored as D / 64 (or, for P, 2) blocks of [128 rows][128 B] with the 128-byte swizzle; a
+// K or V tile's rows are its 128 keys, the two 64-key boxes at +0 and +8 KiB of each block.
 template <int D>
 struct Smem {
-    static constexpr uint32_t OFF_Q = 0;                  // Q [128 rows][D]: blocks of 16 KiB
-    static constexpr uint32_t OFF_KV = kRows * D * 2;     // stage s: K at +0, V at +STAGE / 2
-    static constexpr uint32_t STAGE = 2 * kPT * D * 2;
-    static constexpr uint32_t OFF_P = OFF_KV + kStages * STAGE;  // P [128 rows][64 keys] x 2
-    static constexpr uint32_t P_BYTES = 16384;
-    static constexpr uint32_t OFF_RED = OFF_P + 2 * P_BYTES;     // row maxima [2 tiles][2][128]
+    static constexpr uint32_t BLK = kRows * 128;               // one [128 rows][128 B] block
+    static constexpr uint32_t OFF_Q = 0;                       // Q: D / 64 blocks
+    static constexpr uint32_t TILE = (D / 64) * BLK;           // a K or V stage
+    static constexpr uint32_t OFF_K = OFF_Q + TILE;            // K stages 0, 1
+    static constexpr uint32_t OFF_V = OFF_K + 2 * TILE;        // V stages 0, 1
+    static constexpr uint32_t OFF_P = OFF_V + 2 * TILE;        // P [128 rows][128 keys]
+    static constexpr uint32_t P_BYTES = 2 * BLK;
+    static constexpr uint32_t OFF_RED = OFF_P + P_BYTES;       // row maxima [2 tiles][2][128]
     static constexpr uint32_t OFF_BAR = OFF_RED + 2048;
-    static constexpr uint32_t BYTES = OFF_BAR + 128 + 1024;
+    static constexpr uint32_t USED = OFF_BAR + 128 + 1024;
+    // at least 116 KiB, so that one CTA (and its 512 TMEM columns) holds an SM
+    static constexpr uint32_t BYTES = USED > 118784 ? USED : 118784;
 };
 static_assert(Smem<128>::BYTES <= 232448, "shared memory per CTA");
+static_assert(2 * Smem<64>::BYTES > 233472, "one CTA per SM");
 // barrier indices
-constexpr int B_FULL = 0;    // [4] K/V tile landed (TMA)
+constexpr int B_KFULL = 0;   // [2] K tile landed (TMA)
+constexpr int B_VFULL = 2;   // [2] V tile landed (TMA)
 constexpr int B_SFULL = 4;   // [2] S_i computed (commit)
 constexpr int B_SFREE = 6;   // [2] S_i read by the 8 softmax warps
-constexpr int B_PFULL = 8;   // [2] P_i written by the 8 softmax warps
-constexpr int B_PVFULL = 10; // PV_i computed (commit)
-constexpr int N_BARS = 11;
+constexpr int B_PFULL = 8;   // P_i written by the 8 softmax warps
+constexpr int B_PVFULL = 9;  // PV_i computed (commit)
+constexpr int N_BARS = 10;
 constexpr float kLazy = 8.f;  // log2 headroom before the exponent base moves
 
-constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);    // A = Q (K-major), B = K (K-major)
+constexpr uint32_t ID_S = idesc_bf16(128, kKT, 0, 0);   // A = Q (K-major), B = K (K-major)
 template <int D>
 constexpr uint32_t ID_PV = idesc_bf16(128, D, 0, 1);     // A = P (K-major), B = V (MN-major)
 
-// 2^x on the FMA pipe, for x <= 8: 2^x = 2^n 2^f with n = floor(x), f = x - n in [0, 1), and 2^f
-// by a cubic fitted to it on [0, 1) (least squares at Chebyshev nodes, reweighted towards the
-// minimax fit; largest relative error 7.5e-5, far below the bf16 rounding of P). x is clamped at
-// -126, where 2^x is below fp32's normal range and its share of a row sum that holds an entry
-// >= 1 is nil. Splitting the exponentials between this and ex2.approx keeps the softmax off a
-// single pipe.
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -126.f);
-    const float n = floorf(x);
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(0.07802451f, f, 0.22606717f), f, 0.69583356f), f, 0.99992520f);
-    return __int_as_float(__float_as_int(p) + (static_cast<int>(n) << 23));
+// ---- two fp32 lanes per instruction (sm_100 f32x2 arithmetic) ----------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe, for x <= 8: 2^x = 2^n 2^f with n = x rounded to the
+// nearest integer (adding 1.5 * 2^23 rounds it into the low mantissa bits) and f = x - n in
+// [-1/2, 1/2], 2^f by a cubic fitted to it on that interval (iteratively reweighted least
+// squares at Chebyshev nodes; largest relative error 7.5e-5, far below the bf16 rounding of P).
+// n is added to the exponent field straight from the rounded sum's bits (its low bits hold n,
+// the bits above them drop out of the shift). x is clamped at -125, where 2^x is below 1e-37
+// and its share of a row sum that holds an entry >= 1 is nil. Splitting the exponentials
+// between this and ex2.approx keeps the softmax off a single pipe.
+__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t x2) {
+    float a, b;
+    f2_split(x2, a, b);
+    x2 = f2(fmaxf(a, -125.f), fmaxf(b, -125.f));
+    const uint64_t j = f2_add(x2, f2(12582912.f, 12582912.f));
+    const uint64_t n = f2_add(j, f2(-12582912.f, -12582912.f));
+    const uint64_t f = f2_fma(n, f2(-1.f, -1.f), x2);
+    uint64_t p = f2_fma(f2(0.05517588f, 0.05517588f), f, f2(0.24261151f, 0.24261151f));
+    p = f2_fma(p, f, f2(0.6932602f, 0.6932602f));
+    p = f2_fma(p, f, f2(0.999928f, 0.999928f));
+    float p0, p1, j0, j1;
+    f2_split(p, p0, p1);
+    f2_split(j, j0, j1);
+    return f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23)),
+              __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23)));
 }
 
 struct TcParams {
@@ -133,8 +180,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                        const __grid_constant__ CUtensorMap tmpk,
                        const __grid_constant__ CUtensorMap tmpv, const TcParams p) {
     using L = Smem<D>;
-    constexpr uint32_t OFF_Q = L::OFF_Q, OFF_KV = L::OFF_KV, STAGE = L::STAGE, OFF_P = L::OFF_P,
-                       P_BYTES = L::P_BYTES, OFF_RED = L::OFF_RED, OFF_BAR = L::OFF_BAR;
+    constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, TILE = L::TILE,
+                       OFF_P = L::OFF_P, OFF_RED = L::OFF_RED, OFF_BAR = L::OFF_BAR, BLK = L::BLK;
     constexpr int kD = D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -144,7 +191,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * N_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 4);
-    volatile int *restart = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 8);  // [2]
+    // restart[i % 4]: tile i moved the exponent base (set by the softmax threads before the
+    // tile's named barrier, read by the issuing thread after P_i is full, cleared two tiles on)
+    volatile int *restart = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 8);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int bg = blockIdx.x % (p.B * p.Hkv);
@@ -155,13 +204,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
 
     if (tid == 0) {
         for (int i = 0; i < N_BARS; ++i) {
-            const bool by_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL ||
-                                  i == B_PFULL + 1;
+            const bool by_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL;
             mbar_init(bar(i), by_warps ? 8 : 1);
         }
         fence_barrier_init();
         *abort_flag = 0;
-        restart[0] = restart[1] = 0;
+        restart[0] = restart[1] = restart[2] = restart[3] = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
         if constexpr (PREFIX) {
@@ -170,6 +218,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
         }
     }
     if (warp == 8) {
+        __syncwarp();  // tcgen05.alloc is .sync.aligned: the whole warp, converged
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
@@ -185,7 +234,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             L0 = 0;
         }
     }
-    const int kb_lo = key_lo(p, L0 + t_first) / kPT, kb_hi = (L0 + t_last) / kPT;
+    const int kb_lo = key_lo(p, L0 + t_first) / kKT, kb_hi = (L0 + t_last) / kKT;
     const int n_tiles = kb_hi - kb_lo + 1;
 
     // ---- Q rows -> shared memory (half a row per softmax thread); fused cache write ----------
@@ -234,101 +283,127 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     if (warp == 8) {
         // ================= TMA and MMA issue (one lane) ================================
         if (lane == 0) {
-            int tiles_issued = 0, s_issued = 0, pv_issued = 0;
-            auto issue_tile = [&](int i) {
-                const int st = i % kStages;
-                const uint32_t kb = sb + OFF_KV + st * STAGE, vb = kb + STAGE / 2;
-                const int key0 = (kb_lo + i) * kPT;  // first position of the tile
-                if (PREFIX && key0 < L0) {  // a page of the cached prefix
-                    const int lp = (kb_lo + i) % (p.swa ? p.ring_pages : 0x7fffffff);
-                    const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
-                    if (pg < 0 || pg >= p.n_pages) {
-                        atomicOr(&g_err, HMD_DEVERR_PAGE);
-                        mbar_arrive_expect_tx(bar(B_FULL + st), 0);  // complete with no copy
-                        return;
-                    }
-                    mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);
-                    const int y = (pg * p.Hkv + g) * kPT;
+            int k_issued = 0, v_issued = 0, s_issued = 0, pv_issued = 0;
+            // K or V of tile i into stage i % 2: two boxes of 64 keys (a page of the cached
+            // prefix, or 64 prompt tokens; boxes past the prompt's end read zeros or another
+            // sequence's rows, masked by every row)
+            auto issue_kv = [&](int i, bool is_v) {
+                const int st = i & 1;
+                const uint32_t dst = sb + (is_v ? OFF_V : OFF_K) + st * TILE;
+                const uint32_t fb = bar((is_v ? B_VFULL : B_KFULL) + st);
+                const CUtensorMap *tm = is_v ? &tmv : &tmk;
+                int pg2[2] = {-1, -1};
+                uint32_t bytes = 0;
 #pragma unroll
-                    for (int hf = 0; hf < kD / 64; ++hf) {
-                        tma_load_2d(kb + hf * 8192, &tmpk, bar(B_FULL + st), hf * 64, y);
-                        tma_load_2d(vb + hf * 8192, &tmpv, bar(B_FULL + st), hf * 64, y);
+                for (int h = 0; h < 2; ++h) {
+                    const int key0 = (kb_lo + i) * kKT + h * kPT;  // first position of the box
+                    if (PREFIX && key0 < L0) {
+                        const int lp = (key0 / kPT) % (p.swa ? p.ring_pages : 0x7fffffff);
+                        const int pg = lp < p.max_pages ? p.page_table[(size_t)b * p.max_pages + lp] : -1;
+                        if (pg < 0 || pg >= p.n_pages) {
+                            atomicOr(&g_err, HMD_DEVERR_PAGE);
+                            continue;  // no copy: the call reports the error
+                        }
+                        pg2[h] = pg;
                     }
-                    return;
+                    bytes += (kD / 64) * 8192;
                 }
-                mbar_arrive_expect_tx(bar(B_FULL + st), STAGE);  // K and V: boxes of 8 KiB
-                const int z = b * p.T + (key0 - L0);
+                mbar_arrive_expect_tx(fb, bytes);
 #pragma unroll
-                for (int hf = 0; hf < kD / 64; ++hf) {
-                    tma_load_3d(kb + hf * 8192, &tmk, bar(B_FULL + st), hf * 64, g, z);
-                    tma_load_3d(vb + hf * 8192, &tmv, bar(B_FULL + st), hf * 64, g, z);
+                for (int h = 0; h < 2; ++h) {
+                    const int key0 = (kb_lo + i) * kKT + h * kPT;
+                    if (PREFIX && key0 < L0) {
+                        if (pg2[h] < 0) continue;
+                        const int y = (pg2[h] * p.Hkv + g) * kPT;
+#pragma unroll
+                        for (int hf = 0; hf < kD / 64; ++hf)
+                            tma_load_2d(dst + hf * BLK + h * 8192, is_v ? &tmpv : &tmpk, fb, hf * 64, y);
+                    } else {
+                        const int z = b * p.T + (key0 - L0);
+#pragma unroll
+                        for (int hf = 0; hf < kD / 64; ++hf)
+                            tma_load_3d(dst + hf * BLK + h * 8192, tm, fb, hf * 64, g, z);
+                    }
                 }
             };
             // descriptors: the address field is the byte address / 16, so an offset is added as
             // offset / 16 (every address here is below 256 KiB: no carry out of the field)
             const uint64_t d_q = smem_desc_sw128(sb + OFF_Q, 16, 1024);
-            const uint64_t d_k = smem_desc_sw128(sb + OFF_KV, 16, 1024);
+            const uint64_t d_k = smem_desc_sw128(sb + OFF_K, 16, 1024);
             const uint64_t d_p = smem_desc_sw128(sb + OFF_P, 16, 1024);
-            const uint64_t d_v = smem_desc_sw128(sb + OFF_KV + STAGE / 2, 8192, 1024);
+            const uint64_t d_v = smem_desc_sw128(sb + OFF_V, BLK, 1024);
             auto issue_s = [&](int i) {
-                const uint64_t ko = ((i % kStages) * STAGE) >> 4;
+                const uint64_t ko = ((i & 1) * TILE) >> 4;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    umma_bf16(tmem + (i & 1) * 64, d_q + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                              d_k + ko + ((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), ID_S, kk > 0);
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * BLK + (kk & 3) * 32;
+                    umma_bf16(tmem + (i & 1) * kKT, d_q + (off >> 4), d_k + ko + (off >> 4), ID_S, kk > 0);
+                }
                 umma_commit(bar(B_SFULL + (i & 1)));
             };
             auto issue_pv = [&](int i, bool fresh) {  // fresh: restart the TMEM sum
-                const uint64_t po = ((i & 1) * P_BYTES) >> 4, vo = ((i % kStages) * STAGE) >> 4;
+                const uint64_t vo = ((i & 1) * TILE) >> 4;
 #pragma unroll
-                for (int kk = 0; kk < kPT / 16; ++kk)
-                    umma_bf16(tmem + 128, d_p + po + ((kk * 32) >> 4), d_v + vo + ((kk * 2048) >> 4),
-                              ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    umma_bf16(tmem + kColPV, d_p + (((kk >> 2) * BLK + (kk & 3) * 32) >> 4),
+                              d_v + vo + ((kk * 2048) >> 4), ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
                 umma_commit(bar(B_PVFULL));
             };
             bool ok = true;
-            for (; tiles_issued < kStages && tiles_issued < n_tiles; ++tiles_issued) issue_tile(tiles_issued);
+            for (; k_issued < 2 && k_issued < n_tiles; ++k_issued) {
+                issue_kv(k_issued, false);
+                issue_kv(k_issued, true);
+                v_issued = k_issued + 1;
+            }
             for (; s_issued < 2 && s_issued < n_tiles && ok; ++s_issued) {
-                ok = wait_or_abort(bar(B_FULL + s_issued % kStages), (s_issued / kStages) & 1, abort_flag);
+                ok = wait_or_abort(bar(B_KFULL + s_issued), 0, abort_flag);
                 if (ok) {
                     tc_fence_after();
                     issue_s(s_issued);
                 }
             }
             for (int i = 0; i < n_tiles && ok; ++i) {
+                // K_{i+2} into the stage S_i read, as soon as S_i is done
+                if (i + 2 < n_tiles) {
+                    ok = wait_or_abort(bar(B_SFULL + (i & 1)), (i >> 1) & 1, abort_flag);
+                    if (!ok) break;
+                    issue_kv(i + 2, false);
+                    k_issued = i + 3;
+                }
                 // PV_i: P_i written (and, on a restart tile, the TMEM sum folded into registers)
-                ok = wait_or_abort(bar(B_PFULL + (i & 1)), (i >> 1) & 1, abort_flag);
+                ok = wait_or_abort(bar(B_PFULL), i & 1, abort_flag);
+                if (ok) ok = wait_or_abort(bar(B_VFULL + (i & 1)), (i >> 1) & 1, abort_flag);
                 if (!ok) break;
-                const bool fresh = restart[i & 1] != 0;
-                restart[i & 1] = 0;  // every softmax thread read it before arriving
+                const bool fresh = restart[i & 3] != 0;
                 tc_fence_after();
                 issue_pv(i, fresh || i == 0);
                 pv_issued = i + 1;
-                // S_{i+2} into the buffer S_i used: tile landed, S_i read
+                // S_{i+2} into the buffer S_i used: K landed, S_i read
                 if (i + 2 < n_tiles) {
-                    ok = wait_or_abort(bar(B_FULL + (i + 2) % kStages), ((i + 2) / kStages) & 1, abort_flag);
+                    ok = wait_or_abort(bar(B_KFULL + (i & 1)), ((i + 2) >> 1) & 1, abort_flag);
                     if (ok) ok = wait_or_abort(bar(B_SFREE + (i & 1)), (i >> 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
                     issue_s(i + 2);
                     s_issued = i + 3;
-                }
-                // tile i+kStages into the stage tile i used, once PV_i (hence S_i) is done
-                if (tiles_issued < n_tiles) {
+                    // V_{i+2} into the stage PV_i read, once PV_i is done
                     ok = wait_or_abort(bar(B_PVFULL), i & 1, abort_flag);
                     if (!ok) break;
-                    issue_tile(tiles_issued);
-                    ++tiles_issued;
+                    issue_kv(i + 2, true);
+                    v_issued = i + 3;
                 }
             }
             if (!ok) {
-                // let what this CTA started finish (bounded) before TMEM is freed
+                // let what this CTA started finish (bounded) before TMEM is freed: tcgen05
+                // products complete in issue order, so the last commit covers every product
                 atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
                 if (s_issued > 0)
                     (void)mbar_wait_bounded(bar(B_SFULL + ((s_issued - 1) & 1)), ((s_issued - 1) >> 1) & 1);
                 if (pv_issued > 0) (void)mbar_wait_bounded(bar(B_PVFULL), (pv_issued - 1) & 1);
-                for (int u = max(0, tiles_issued - kStages); u < tiles_issued; ++u)
-                    (void)mbar_wait_bounded(bar(B_FULL + u % kStages), (u / kStages) & 1);
+                for (int u = max(0, k_issued - 2); u < k_issued; ++u)
+                    (void)mbar_wait_bounded(bar(B_KFULL + (u & 1)), (u >> 1) & 1);
+                for (int u = max(0, v_issued - 2); u < v_issued; ++u)
+                    (void)mbar_wait_bounded(bar(B_VFULL + (u & 1)), (u >> 1) & 1);
             }
         }
     } else {
@@ -339,111 +414,138 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
 #pragma unroll
         for (int j = 0; j < kD / 2; ++j) o[j] = 0.f;
         float m_base = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
+        // folds the TMEM sum of this thread's output half into o at factor f (o = (o + acc) f)
+        auto fold_pv = [&](float f) {
+#pragma unroll
+            for (int c4 = 0; c4 < kD / 64; ++c4) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + kColPV + ch * (kD / 2) + c4 * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * f;
+            }
+        };
         // After an abort the loop keeps its shape (every wait then fails at once and the work
         // and arrivals are skipped), so every softmax thread meets the same barriers.
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
-            // ---- this thread's 32 scores of S_i; then hand the buffer back --------------------
+            // ---- this thread's 64 scores of S_i; then hand the buffer back --------------------
             if (ok) ok = wait_or_abort(bar(B_SFULL + (i & 1)), (i >> 1) & 1, abort_flag);
-            float s[kPT / 2];
+            ok = __all_sync(0xffffffffu, ok);  // the TMEM load below runs converged
+            float s[kKT / 2];
             if (ok) {
                 tc_fence_after();
-                uint32_t r[32];
-                tmem_ld32(lane_base + (i & 1) * 64 + ch * 32, r);
+                uint32_t r[64];
+                tmem_ld64(lane_base + (i & 1) * kKT + ch * 64, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(r[j]);
+                for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(r[j]);
                 tc_fence_before();
             } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) s[j] = 0.f;
+                for (int j = 0; j < 64; ++j) s[j] = 0.f;
             }
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
             // ---- mask (edge tiles only), partial maximum; a restart if it outgrows the base ----
-            const int j0 = (kb_lo + i) * kPT + ch * 32;
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // short chains
-            if (!(row_ok && j0 >= lo_row && j0 + kPT / 2 - 1 <= pos_row)) {
+            const int j0 = (kb_lo + i) * kKT + ch * 64;
+            if (!(row_ok && j0 >= lo_row && j0 + kKT / 2 - 1 <= pos_row)) {
 #pragma unroll
-                for (int j = 0; j < kPT / 2; ++j) {
+                for (int j = 0; j < kKT / 2; ++j) {
                     const int key = j0 + j;
                     const bool valid = row_ok && key >= lo_row && key <= pos_row;
                     s[j] = valid ? s[j] : -INFINITY;
                 }
             }
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // short chains
 #pragma unroll
-            for (int j = 0; j < kPT / 2; ++j) mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
+            for (int j = 0; j < kKT / 2; j += 8) {
+                mx4[0] = max3(mx4[0], s[j], s[j + 1]);
+                mx4[1] = max3(mx4[1], s[j + 2], s[j + 3]);
+                mx4[2] = max3(mx4[2], s[j + 4], s[j + 5]);
+                mx4[3] = max3(mx4[3], s[j + 6], s[j + 7]);
+            }
             float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;  // scores and maxima in the log2 domain from here on
             float *rb = red + (i & 1) * 2 * kRows;
             rb[ch * kRows + row] = mx;
-            if (mx > m_base + kLazy) restart[i & 1] = 1;
+            if (mx > m_base + kLazy) restart[i & 3] = 1;
             softmax_barrier();
-            const bool fold = restart[i & 1] != 0;
-            if (fold) {
+            if (tid == 0) restart[(i + 2) & 3] = 0;  // its last reader was done with it (see above)
+            bool pv_done = i == 0;  // PV_{i-1} has read P
+            if (restart[i & 3] != 0) {
                 // new base per row; the TMEM sum (PV up to i-1) joins the register sum there
                 const float m_new = fmaxf(m_base, fmaxf(rb[row], rb[kRows + row]));
                 const float mu = (m_new == -INFINITY) ? 0.f : m_new;
                 const float f = exp2f(m_base - mu);
                 if (i > 0) {
                     if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
                     if (ok) {
                         tc_fence_after();
-#pragma unroll
-                        for (int c4 = 0; c4 < kD / 64; ++c4) {
-                            uint32_t r[32];
-                            tmem_ld32(lane_base + 128 + ch * (kD / 2) + c4 * 32, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * f;
-                        }
+                        fold_pv(f);
                         tc_fence_before();
                     }
+                    pv_done = true;
                 }
                 l_run *= f;
                 m_base = m_new;
             }
             const float mu = (m_base == -INFINITY) ? 0.f : m_base;
-            // ---- P_i half row -> shared memory (its buffer's last reader, PV_{i-2}, is done) ---
+            // ---- exponentials, two lanes per instruction; the row sum in four partial chains ---
+            uint32_t pk[kKT / 4];
             {
-                float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: short chains
-                uint8_t *prow = sm + OFF_P + (i & 1) * P_BYTES;
+                const uint64_t sc2 = f2(p.scale_log2, p.scale_log2), nmu2 = f2(-mu, -mu);
+                uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < kPT / 16; ++c) {
-                    float e[8];
+                for (int c = 0; c < kKT / 16; ++c) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const float x = fmaf(s[c * 8 + u], p.scale_log2, -mu);
-                        e[u] = (u & 3) == 3 ? exp2_fma(x) : ex2_approx(x);
-                        ls4[u & 3] += e[u];
+                    for (int u = 0; u < 4; ++u) {
+                        const uint64_t x = f2_fma(f2(s[c * 8 + 2 * u], s[c * 8 + 2 * u + 1]), sc2, nmu2);
+                        uint64_t e;
+                        if (u == 3) {
+                            e = exp2_fma_x2(x);
+                        } else {
+                            float a0, a1;
+                            f2_split(x, a0, a1);
+                            e = f2(ex2_approx(a0), ex2_approx(a1));
+                        }
+                        acc[u & 1] = f2_add(acc[u & 1], e);
+                        float e0, e1;
+                        f2_split(e, e0, e1);
+                        pk[c * 4 + u] = pack_bf16x2(e0, e1);
                     }
-                    if (ok)
-                        *reinterpret_cast<uint4 *>(prow + swz(row, ch * 32 + c * 8, kRows)) =
-                            make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]),
-                                       pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
                 }
-                l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+                float a0, a1, b0, b1;
+                f2_split(acc[0], a0, a1);
+                f2_split(acc[1], b0, b1);
+                l_run += (a0 + a1) + (b0 + b1);
+            }
+            // ---- P_i half row -> shared memory, once PV_{i-1} has read the buffer ------------
+            if (!pv_done) {
+                if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (ok) {
+                uint8_t *prow = sm + OFF_P;
+#pragma unroll
+                for (int c = 0; c < kKT / 16; ++c)
+                    *reinterpret_cast<uint4 *>(prow + swz(row, ch * 64 + c * 8, kRows)) =
+                        make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
             }
             fence_proxy_async_smem();  // P is read by the tensor cores
             __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(B_PFULL + (i & 1)));
+            if (ok && lane == 0) mbar_arrive(bar(B_PFULL));
         }
         if (ok) ok = wait_or_abort(bar(B_PVFULL), (n_tiles - 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
         // the TMEM sum joins O (same base); the two halves' sums make the row's; normalise, store
         float *lb = red + (n_tiles & 1) * 2 * kRows;
         lb[ch * kRows + row] = l_run;
         softmax_barrier();
         if (ok) {
             tc_fence_after();
-#pragma unroll
-            for (int c4 = 0; c4 < kD / 64; ++c4) {
-                uint32_t r[32];
-                tmem_ld32(lane_base + 128 + ch * (kD / 2) + c4 * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) o[c4 * 32 + j] += __uint_as_float(r[j]);
-            }
+            fold_pv(1.f);
             if (row_ok) {
                 const float l = lb[row] + lb[kRows + row];
                 const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -808,7 +808,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
     const uint32_t tmem = *tmem_slot;
     float *Mg = a.state + ((size_t)slot * a.H + h) * kD * kD + sv * kDV;
 
-    // bounded wait that also gives up once another thread of the CTA has given up
+    // bounded wait that also gives up once another thread of the CTA has given up. A warp that
+    // goes on to a tcgen05 .sync.aligned instruction (a TMEM load) takes the decision as one
+    // (__all_sync), so the instruction always runs converged.
     auto wait = [&](int i, uint32_t parity) -> bool {
         const uint32_t bb = bar(i);
         if (mbar_try_wait(bb, parity)) return true;
@@ -889,7 +891,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         for (int c = 0; c < nseg; ++c) {
             const int u = c & 1;
-            if (!wait(BAR_OFULL0 + u, (c >> 1) & 1)) break;
+            if (!__all_sync(0xffffffffu, wait(BAR_OFULL0 + u, (c >> 1) & 1))) break;
             tc_fence_after();
             const int t0 = (a.chunk_begin + c) * kC;
             const int n = min(kC, T - t0);
@@ -935,7 +937,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
         float gam = 0.f;
         auto publish_m = [&](int c) -> bool {
             const int s = c % kStages;
-            if (!wait(BAR_FULL0 + s, (c / kStages) & 1)) return false;
+            if (!__all_sync(0xffffffffu, wait(BAR_FULL0 + s, (c / kStages) & 1))) return false;
             gam = reinterpret_cast<const float *>(sm + s * ST_BYTES + ST_GAM)[i];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -961,7 +963,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     ut[q] = *reinterpret_cast<const uint4 *>(utrow + (((4 * half + q) ^ (i & 7)) << 4));
-                if (!wait(BAR_UO, c & 1)) break;
+                if (!__all_sync(0xffffffffu, wait(BAR_UO, c & 1))) break;
                 tc_fence_after();
                 uint32_t d[32];
                 tmem_ld32(tmem + lane_base + kDV * u + col0, d);
@@ -984,7 +986,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) prefill_scan_kernel(const Pre
                 if (lane == 0) mbar_arrive(bar(BAR_U));
             }
             // M <- e^G_C M + Kc^T U
-            if (!wait(BAR_S, c & 1)) break;
+            if (!__all_sync(0xffffffffu, wait(BAR_S, c & 1))) break;
             tc_fence_after();
             {
                 uint32_t d[32];
