@@ -5,28 +5,28 @@
 // max(0, t + 1 - w) (SWA), and the prompt's K and V are written to the paged cache at the slots
 // the decode step reads (SWA: the positions the ring of ceil(w / 64) pages keeps).
 //
-// One CTA per (sequence, kv-head, block of 128/G tokens), warp-specialised, key tiles of 128:
-//   warp 8 (one lane) issues the TMA copies of the K and V tiles (two rings of two stages each,
-//     3-D boxes of 64 tokens from the prompt or 2-D boxes of one page from the cache, 128-byte
-//     swizzle) and the tcgen05.mma products
-//       S_i = Q K_i^T   M=128 N=128 K=d (Q and K K-major) into TMEM buffer i & 1
-//       PV_i = P_i V_i  M=128 N=d K=128 (P K-major, V MN-major) into TMEM
-//     in the order PV_i, S_{i+2}, so the tensor core works on them while the softmax warps
-//     process tile i+1. A K stage is reloaded as soon as the S product that read it is done,
-//     a V stage once its PV product is;
-//   warps 0-7 run the softmax: query row r (head g*G + r / QT, token t_first + r % QT) is TMEM
-//     lane r; threads r and r + 128 split its columns (64 of the 128 scores, half of the output)
-//     and exchange partial maxima through one 256-thread named barrier per tile. They read S
-//     with tcgen05.ld and write P (bf16) to shared memory in the swizzled K-major layout, once
-//     the previous tile's PV product has read it.
-// Lazy rescaling: PV accumulates in TMEM across tiles at a fixed exponent base per row, which
-// moves only when some row's maximum exceeds its base by more than 8 (P stays below 2^8). On
-// such a tile every row folds the TMEM accumulator into an fp32 register accumulator at the new
-// base and the tile's PV restarts the TMEM sum, so the threads never write TMEM.
-// The roles hand over through mbarriers only (S full / free, P full, PV full), so no CTA-wide
-// barrier sits in the tile loop. Accumulators are only read from TMEM (never written
-// by the threads). Every wait is bounded; a wait that gives up raises a shared abort flag that
-// ends every other wait of the CTA, and the error word reports the call as failed.
+// One CTA per (sequence, kv-head, block of 256/G tokens): two query tiles of 128 rows (row r of
+// tile j: head g*G + r / QT, token t_first + j*QT + r % QT, QT = 128/G) share every K/V tile.
+// Key tiles of 128. Warp-specialised, 320 threads:
+//   warp 9 (one lane) streams K and V tiles by TMA into two rings of two stages (3-D boxes of
+//     64 prompt tokens, or 2-D boxes of one cache page, 128-byte swizzle);
+//   warp 8 (one lane) issues the tcgen05.mma products, per key tile i and query tile j:
+//       S_j = Q_j K_i^T   M=128 N=128 K=d (both from shared memory, K-major) into TMEM S_j
+//       O_j += P_j V_i    M=128 N=d K=128 (P_j from TMEM, V MN-major from shared memory)
+//     in the order O_0(i), S_0(i+1), O_1(i), S_1(i+1): while one query tile's softmax runs, the
+//     tensor core works on the other's products;
+//   warps 4j .. 4j+3 are query tile j's softmax group: thread = query row = TMEM lane. A thread
+//     reads its row of S_j (tcgen05.ld), takes the maximum itself (no exchange), writes the
+//     row of P_j (bf16 pairs) into the TMEM columns of S_j it has read (tcgen05.st), and hands
+//     over through an mbarrier.
+// P_j (128 keys as bf16 pairs) lies in the first 64 columns of S_j: S_j(i+1) is issued after
+// O_j(i) by the same thread, and the tensor core runs one thread's products in order.
+// Lazy rescaling, per row: O_j accumulates at a fixed exponent base per row, which moves only
+// when the row's maximum exceeds it by more than 8 (P stays below 2^8); the thread then scales
+// its row of O_j in TMEM. S_j(i) is issued after O_j(i-1), so once S_j(i) is complete the
+// previous product into O_j is too, and the row can be rescaled before O_j(i) is issued.
+// Every wait is bounded; a wait that gives up raises a shared abort flag that ends every other
+// wait of the CTA, and the error word reports the call as failed.
 #include <cuda.h>
 #include <float.h>
 
@@ -44,27 +44,23 @@ __device__ unsigned int g_err;
 
 constexpr int kPT = 64;          // tokens per page = keys per TMA box
 constexpr int kKT = 128;         // keys per tile
-constexpr int kSoftmax = 256;    // softmax threads (warps 0-7)
-constexpr int kThreads = kSoftmax + 32;  // + the TMA / MMA warp
-constexpr int kRows = 128;
-constexpr uint32_t kTmemCols = 512;  // S buffers at 0 and 128, PV at 256 (D columns)
-constexpr uint32_t kColPV = 256;
+constexpr int kRows = 128;       // rows per query tile
+constexpr int kSoftmax = 256;    // softmax threads (warps 0-7: two groups of four)
+constexpr int kThreads = kSoftmax + 64;  // + the MMA warp (8) and the TMA warp (9)
+constexpr uint32_t kTmemCols = 512;  // query tile j: S_j (and P_j) at 256 j, O_j at 256 j + 128
 
 // shared memory (bytes from a 1024-aligned base) for head size D (64 or 128). Every operand tile
-// is stored as D / 64 (or, for P, 2) blocks of [128 rows][128 B] with the 128-byte swizzle; a
-// K or V tile's rows are its 128 keys, the two 64-key boxes at +0 and +8 KiB of each block.
+// is stored as D / 64 blocks of [128 rows][128 B] with the 128-byte swizzle; a K or V tile's
+// rows are its 128 keys, the two 64-key boxes at +0 and +8 KiB of each block.
 template <int D>
 struct Smem {
     static constexpr uint32_t BLK = kRows * 128;               // one [128 rows][128 B] block
-    static constexpr uint32_t OFF_Q = 0;                       // Q: D / 64 blocks
-    static constexpr uint32_t TILE = (D / 64) * BLK;           // a K or V stage
-    static constexpr uint32_t OFF_K = OFF_Q + TILE;            // K stages 0, 1
+    static constexpr uint32_t TILE = (D / 64) * BLK;           // a query tile, a K or a V stage
+    static constexpr uint32_t OFF_Q = 0;                       // Q_0, Q_1
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE;        // K stages 0, 1
     static constexpr uint32_t OFF_V = OFF_K + 2 * TILE;        // V stages 0, 1
-    static constexpr uint32_t OFF_P = OFF_V + 2 * TILE;        // P [128 rows][128 keys]
-    static constexpr uint32_t P_BYTES = 2 * BLK;
-    static constexpr uint32_t OFF_RED = OFF_P + P_BYTES;       // row maxima [2 tiles][2][128]
-    static constexpr uint32_t OFF_BAR = OFF_RED + 2048;
-    static constexpr uint32_t USED = OFF_BAR + 128 + 1024;
+    static constexpr uint32_t OFF_BAR = OFF_V + 2 * TILE;
+    static constexpr uint32_t USED = OFF_BAR + 256 + 1024;
     // at least 116 KiB, so that one CTA (and its 512 TMEM columns) holds an SM
     static constexpr uint32_t BYTES = USED > 118784 ? USED : 118784;
 };
@@ -73,16 +69,18 @@ static_assert(2 * Smem<64>::BYTES > 233472, "one CTA per SM");
 // barrier indices
 constexpr int B_KFULL = 0;   // [2] K tile landed (TMA)
 constexpr int B_VFULL = 2;   // [2] V tile landed (TMA)
-constexpr int B_SFULL = 4;   // [2] S_i computed (commit)
-constexpr int B_SFREE = 6;   // [2] S_i read by the 8 softmax warps
-constexpr int B_PFULL = 8;   // P_i written by the 8 softmax warps
-constexpr int B_PVFULL = 9;  // PV_i computed (commit)
-constexpr int N_BARS = 10;
-constexpr float kLazy = 8.f;  // log2 headroom before the exponent base moves
+constexpr int B_KFREE = 4;   // [2] both S products of the K tile done (commit)
+constexpr int B_VFREE = 6;   // [2] both PV products of the V tile done (commit)
+constexpr int B_SFULL = 8;   // [2] per query tile: S_j computed (commit)
+constexpr int B_PFULL = 10;  // [2] per query tile: P_j written (four warps)
+constexpr int B_ODONE = 12;  // [2] per query tile: the last PV product done (commit)
+constexpr int B_FINAL = 14;  // every product issued done (commit, teardown)
+constexpr int N_BARS = 15;
+constexpr float kLazy = 8.f;  // log2 headroom before a row's exponent base moves
 
 constexpr uint32_t ID_S = idesc_bf16(128, kKT, 0, 0);   // A = Q (K-major), B = K (K-major)
 template <int D>
-constexpr uint32_t ID_PV = idesc_bf16(128, D, 0, 1);     // A = P (K-major), B = V (MN-major)
+constexpr uint32_t ID_PV = idesc_bf16(128, D, 0, 1);     // A = P (TMEM), B = V (MN-major)
 
 // ---- two fp32 lanes per instruction (sm_100 f32x2 arithmetic) ----------------------------------
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
@@ -168,10 +166,6 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     }
 }
 
-__device__ __forceinline__ void softmax_barrier() {  // warps 0-7 only (named barrier 1)
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-}
-
 // PREFIX: sequences may start after cached positions (p.prefix_lens); false compiles the
 // empty-cache prefill with every prefix path removed. D: head size, 64 or 128.
 template <int D, bool PREFIX>
@@ -181,7 +175,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                        const __grid_constant__ CUtensorMap tmpv, const TcParams p) {
     using L = Smem<D>;
     constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, TILE = L::TILE,
-                       OFF_P = L::OFF_P, OFF_RED = L::OFF_RED, OFF_BAR = L::OFF_BAR, BLK = L::BLK;
+                       OFF_BAR = L::OFF_BAR, BLK = L::BLK;
     constexpr int kD = D;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -191,25 +185,18 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8 * N_BARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 4);
-    // restart[i % 4]: tile i moved the exponent base (set by the softmax threads before the
-    // tile's named barrier, read by the issuing thread after P_i is full, cleared two tiles on)
-    volatile int *restart = reinterpret_cast<volatile int *>(sm + OFF_BAR + 8 * N_BARS + 8);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int bg = blockIdx.x % (p.B * p.Hkv);
     const int qb = p.n_qb - 1 - (int)(blockIdx.x / (p.B * p.Hkv));  // longest blocks first
     const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-    const int t_first = qb * p.QT;
-    const int t_last = min(p.T, t_first + p.QT) - 1;
+    const int t_first = qb * 2 * p.QT;
+    const int t_last = min(p.T, t_first + 2 * p.QT) - 1;
 
     if (tid == 0) {
-        for (int i = 0; i < N_BARS; ++i) {
-            const bool by_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL;
-            mbar_init(bar(i), by_warps ? 8 : 1);
-        }
+        for (int i = 0; i < N_BARS; ++i) mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1) ? 4 : 1);
         fence_barrier_init();
         *abort_flag = 0;
-        restart[0] = restart[1] = restart[2] = restart[3] = 0;
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
         if constexpr (PREFIX) {
@@ -237,9 +224,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     const int kb_lo = key_lo(p, L0 + t_first) / kKT, kb_hi = (L0 + t_last) / kKT;
     const int n_tiles = kb_hi - kb_lo + 1;
 
-    // ---- Q rows -> shared memory (half a row per softmax thread); fused cache write ----------
-    const int row = tid & (kRows - 1), ch = (tid >> 7) & 1;
-    const int t_row = t_first + row % p.QT;
+    // ---- Q rows -> shared memory (one row per softmax thread); fused cache write -------------
+    const int qt = warp >> 2;  // the softmax thread's query tile
+    const int row = tid & (kRows - 1);
+    const int t_row = t_first + qt * p.QT + row % p.QT;
     const bool row_ok = t_row <= t_last;
     const int pos_row = L0 + t_row;  // the row's position: its last key
     const int lo_row = key_lo(p, pos_row);
@@ -248,9 +236,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
         const uint4 *src = reinterpret_cast<const uint4 *>(
             p.q + (((size_t)b * p.T + (row_ok ? t_row : 0)) * p.Hq + h_row) * kD);
 #pragma unroll
-        for (int c = ch * (kD / 16); c < (ch + 1) * (kD / 16); ++c) {
+        for (int c = 0; c < kD / 8; ++c) {
             const uint4 v = row_ok ? src[c] : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4 *>(sm + OFF_Q + swz(row, c * 8, kRows)) = v;
+            *reinterpret_cast<uint4 *>(sm + OFF_Q + qt * TILE + swz(row, c * 8, kRows)) = v;
         }
         const int ring = p.ring_pages * kPT;
         const int n_tok = t_last - t_first + 1;
@@ -280,10 +268,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ================= TMA and MMA issue (one lane) ================================
+    if (warp == 9) {
+        // ================= TMA producer (one lane) ======================================
         if (lane == 0) {
-            int k_issued = 0, v_issued = 0, s_issued = 0, pv_issued = 0;
+            int issued = 0;  // K/V tiles issued
             // K or V of tile i into stage i % 2: two boxes of 64 keys (a page of the cached
             // prefix, or 64 prompt tokens; boxes past the prompt's end read zeros or another
             // sequence's rows, masked by every row)
@@ -326,132 +314,117 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                     }
                 }
             };
+            bool ok = true;
+            for (int t = 0; t < n_tiles && ok; ++t) {
+                const int st = t & 1;
+                if (t >= 2) ok = wait_or_abort(bar(B_KFREE + st), ((t - 2) >> 1) & 1, abort_flag);
+                if (!ok) break;
+                issue_kv(t, false);
+                if (t >= 2) ok = wait_or_abort(bar(B_VFREE + st), ((t - 2) >> 1) & 1, abort_flag);
+                if (!ok) {
+                    issued = 2 * t + 1;
+                    break;
+                }
+                issue_kv(t, true);
+                issued = 2 * t + 2;
+            }
+            if (!ok) {
+                // the copies in flight land (bounded) before shared memory is released
+                atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+                for (int u = max(0, issued - 4); u < issued; ++u) {
+                    const int t = u >> 1;
+                    (void)mbar_wait_bounded(bar(((u & 1) ? B_VFULL : B_KFULL) + (t & 1)), (t >> 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 8) {
+        // ================= MMA issue (one lane) ========================================
+        if (lane == 0) {
             // descriptors: the address field is the byte address / 16, so an offset is added as
             // offset / 16 (every address here is below 256 KiB: no carry out of the field)
             const uint64_t d_q = smem_desc_sw128(sb + OFF_Q, 16, 1024);
             const uint64_t d_k = smem_desc_sw128(sb + OFF_K, 16, 1024);
-            const uint64_t d_p = smem_desc_sw128(sb + OFF_P, 16, 1024);
             const uint64_t d_v = smem_desc_sw128(sb + OFF_V, BLK, 1024);
-            auto issue_s = [&](int i) {
-                const uint64_t ko = ((i & 1) * TILE) >> 4;
+            auto issue_s = [&](int j, int i) {  // S_j = Q_j K_i^T
+                const uint64_t qo = (j * TILE) >> 4, ko = ((i & 1) * TILE) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * BLK + (kk & 3) * 32;
-                    umma_bf16(tmem + (i & 1) * kKT, d_q + (off >> 4), d_k + ko + (off >> 4), ID_S, kk > 0);
+                    umma_bf16(tmem + 256 * j, d_q + qo + (off >> 4), d_k + ko + (off >> 4), ID_S, kk > 0);
                 }
-                umma_commit(bar(B_SFULL + (i & 1)));
+                umma_commit(bar(B_SFULL + j));
             };
-            auto issue_pv = [&](int i, bool fresh) {  // fresh: restart the TMEM sum
+            auto issue_pv = [&](int j, int i) {  // O_j (+)= P_j V_i, P_j from TMEM
                 const uint64_t vo = ((i & 1) * TILE) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16(tmem + kColPV, d_p + (((kk >> 2) * BLK + (kk & 3) * 32) >> 4),
-                              d_v + vo + ((kk * 2048) >> 4), ID_PV<kD>, (kk > 0 || !fresh) ? 1u : 0u);
-                umma_commit(bar(B_PVFULL));
+                    umma_bf16_ts(tmem + 256 * j + 128, tmem + 256 * j + 8 * kk, d_v + vo + ((kk * 2048) >> 4),
+                                 ID_PV<kD>, (i > 0 || kk > 0) ? 1u : 0u);
             };
-            bool ok = true;
-            for (; k_issued < 2 && k_issued < n_tiles; ++k_issued) {
-                issue_kv(k_issued, false);
-                issue_kv(k_issued, true);
-                v_issued = k_issued + 1;
-            }
-            for (; s_issued < 2 && s_issued < n_tiles && ok; ++s_issued) {
-                ok = wait_or_abort(bar(B_KFULL + s_issued), 0, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    issue_s(s_issued);
-                }
+            bool ok = wait_or_abort(bar(B_KFULL), 0, abort_flag);
+            bool issued_any = false;
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_s(1, 0);
+                umma_commit(bar(B_KFREE));
+                issued_any = true;
             }
             for (int i = 0; i < n_tiles && ok; ++i) {
-                // K_{i+2} into the stage S_i read, as soon as S_i is done
-                if (i + 2 < n_tiles) {
-                    ok = wait_or_abort(bar(B_SFULL + (i & 1)), (i >> 1) & 1, abort_flag);
-                    if (!ok) break;
-                    issue_kv(i + 2, false);
-                    k_issued = i + 3;
-                }
-                // PV_i: P_i written (and, on a restart tile, the TMEM sum folded into registers)
-                ok = wait_or_abort(bar(B_PFULL), i & 1, abort_flag);
-                if (ok) ok = wait_or_abort(bar(B_VFULL + (i & 1)), (i >> 1) & 1, abort_flag);
-                if (!ok) break;
-                const bool fresh = restart[i & 3] != 0;
-                tc_fence_after();
-                issue_pv(i, fresh || i == 0);
-                pv_issued = i + 1;
-                // S_{i+2} into the buffer S_i used: K landed, S_i read
-                if (i + 2 < n_tiles) {
-                    ok = wait_or_abort(bar(B_KFULL + (i & 1)), ((i + 2) >> 1) & 1, abort_flag);
-                    if (ok) ok = wait_or_abort(bar(B_SFREE + (i & 1)), (i >> 1) & 1, abort_flag);
+#pragma unroll 1
+                for (int j = 0; j < 2 && ok; ++j) {
+                    ok = wait_or_abort(bar(B_PFULL + j), i & 1, abort_flag);
+                    if (ok && j == 0) ok = wait_or_abort(bar(B_VFULL + (i & 1)), (i >> 1) & 1, abort_flag);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(i + 2);
-                    s_issued = i + 3;
-                    // V_{i+2} into the stage PV_i read, once PV_i is done
-                    ok = wait_or_abort(bar(B_PVFULL), i & 1, abort_flag);
-                    if (!ok) break;
-                    issue_kv(i + 2, true);
-                    v_issued = i + 3;
+                    issue_pv(j, i);
+                    if (j == 1) umma_commit(bar(B_VFREE + (i & 1)));
+                    if (i == n_tiles - 1) umma_commit(bar(B_ODONE + j));
+                    if (i + 1 < n_tiles) {
+                        if (j == 0)
+                            ok = wait_or_abort(bar(B_KFULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(j, i + 1);
+                        if (j == 1) umma_commit(bar(B_KFREE + ((i + 1) & 1)));
+                    }
                 }
             }
-            if (!ok) {
-                // let what this CTA started finish (bounded) before TMEM is freed: tcgen05
-                // products complete in issue order, so the last commit covers every product
-                atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
-                if (s_issued > 0)
-                    (void)mbar_wait_bounded(bar(B_SFULL + ((s_issued - 1) & 1)), ((s_issued - 1) >> 1) & 1);
-                if (pv_issued > 0) (void)mbar_wait_bounded(bar(B_PVFULL), (pv_issued - 1) & 1);
-                for (int u = max(0, k_issued - 2); u < k_issued; ++u)
-                    (void)mbar_wait_bounded(bar(B_KFULL + (u & 1)), (u >> 1) & 1);
-                for (int u = max(0, v_issued - 2); u < v_issued; ++u)
-                    (void)mbar_wait_bounded(bar(B_VFULL + (u & 1)), (u >> 1) & 1);
+            if (!ok) atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
+            if (issued_any) {
+                // every product this thread issued is done before TMEM is freed (bounded)
+                umma_commit(bar(B_FINAL));
+                (void)mbar_wait_bounded(bar(B_FINAL), 0);
             }
         }
     } else {
-        // ================= softmax warps ==============================================
+        // ================= softmax: query tile qt, one thread per row ======================
         const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [2 tiles][2 halves][128]
-        float o[kD / 2];  // this thread's half of the row's output, at exponent base m_base
-#pragma unroll
-        for (int j = 0; j < kD / 2; ++j) o[j] = 0.f;
-        float m_base = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
-        // folds the TMEM sum of this thread's output half into o at factor f (o = (o + acc) f)
-        auto fold_pv = [&](float f) {
-#pragma unroll
-            for (int c4 = 0; c4 < kD / 64; ++c4) {
-                uint32_t r[32];
-                tmem_ld32(lane_base + kColPV + ch * (kD / 2) + c4 * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) o[c4 * 32 + j] = (o[c4 * 32 + j] + __uint_as_float(r[j])) * f;
-            }
-        };
-        // After an abort the loop keeps its shape (every wait then fails at once and the work
-        // and arrivals are skipped), so every softmax thread meets the same barriers.
+        const uint32_t s_col = lane_base + 256 * qt, o_col = s_col + 128;
+        float m_base = -INFINITY, l_run = 0.f;
         bool ok = true;
-        for (int i = 0; i < n_tiles; ++i) {
-            // ---- this thread's 64 scores of S_i; then hand the buffer back --------------------
-            if (ok) ok = wait_or_abort(bar(B_SFULL + (i & 1)), (i >> 1) & 1, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);  // the TMEM load below runs converged
-            float s[kKT / 2];
-            if (ok) {
-                tc_fence_after();
+        for (int i = 0; i < n_tiles && ok; ++i) {
+            ok = wait_or_abort(bar(B_SFULL + qt), i & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);  // the TMEM accesses below run converged
+            if (!ok) break;
+            tc_fence_after();
+            float s[kKT];
+            {
                 uint32_t r[64];
-                tmem_ld64(lane_base + (i & 1) * kKT + ch * 64, r);
+                tmem_ld64(s_col, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(r[j]);
-                tc_fence_before();
-            } else {
+                tmem_ld64(s_col + 64, r);
+                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; ++j) s[j] = 0.f;
+                for (int j = 0; j < 64; ++j) s[64 + j] = __uint_as_float(r[j]);
             }
-            __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(B_SFREE + (i & 1)));
-            // ---- mask (edge tiles only), partial maximum; a restart if it outgrows the base ----
-            const int j0 = (kb_lo + i) * kKT + ch * 64;
-            if (!(row_ok && j0 >= lo_row && j0 + kKT / 2 - 1 <= pos_row)) {
+            // ---- mask (edge tiles only), row maximum; the row's base moves if it outgrew it ----
+            const int j0 = (kb_lo + i) * kKT;
+            if (!(row_ok && j0 >= lo_row && j0 + kKT - 1 <= pos_row)) {
 #pragma unroll
-                for (int j = 0; j < kKT / 2; ++j) {
+                for (int j = 0; j < kKT; ++j) {
                     const int key = j0 + j;
                     const bool valid = row_ok && key >= lo_row && key <= pos_row;
                     s[j] = valid ? s[j] : -INFINITY;
@@ -459,51 +432,34 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
             }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // short chains
 #pragma unroll
-            for (int j = 0; j < kKT / 2; j += 8) {
+            for (int j = 0; j < kKT; j += 8) {
                 mx4[0] = max3(mx4[0], s[j], s[j + 1]);
                 mx4[1] = max3(mx4[1], s[j + 2], s[j + 3]);
                 mx4[2] = max3(mx4[2], s[j + 4], s[j + 5]);
                 mx4[3] = max3(mx4[3], s[j + 6], s[j + 7]);
             }
-            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-            mx *= p.scale_log2;  // scores and maxima in the log2 domain from here on
-            float *rb = red + (i & 1) * 2 * kRows;
-            rb[ch * kRows + row] = mx;
-            if (mx > m_base + kLazy) restart[i & 3] = 1;
-            softmax_barrier();
-            if (tid == 0) restart[(i + 2) & 3] = 0;  // its last reader was done with it (see above)
-            bool pv_done = i == 0;  // PV_{i-1} has read P
-            if (restart[i & 3] != 0) {
-                // new base per row; the TMEM sum (PV up to i-1) joins the register sum there
-                const float m_new = fmaxf(m_base, fmaxf(rb[row], rb[kRows + row]));
-                const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-                const float f = exp2f(m_base - mu);
-                if (i > 0) {
-                    if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (ok) {
-                        tc_fence_after();
-                        fold_pv(f);
-                        tc_fence_before();
-                    }
-                    pv_done = true;
-                }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.scale_log2;
+            const bool move = mx > m_base + kLazy;
+            float f = 1.f;  // factor of the row's earlier output and sum
+            if (move) {
+                f = exp2f(m_base - mx);  // 0 while the row had no key (m_base = -inf)
+                m_base = mx;
                 l_run *= f;
-                m_base = m_new;
             }
             const float mu = (m_base == -INFINITY) ? 0.f : m_base;
-            // ---- exponentials, two lanes per instruction; the row sum in four partial chains ---
-            uint32_t pk[kKT / 4];
+            __syncwarp();  // the row-dependent branches above rejoin before the TMEM stores
+            // ---- P row: exponentials two lanes per instruction, into TMEM over S's columns ----
             {
                 const uint64_t sc2 = f2(p.scale_log2, p.scale_log2), nmu2 = f2(-mu, -mu);
                 uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < kKT / 16; ++c) {
+                for (int c = 0; c < kKT / 32; ++c) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint64_t x = f2_fma(f2(s[c * 8 + 2 * u], s[c * 8 + 2 * u + 1]), sc2, nmu2);
+                    for (int u = 0; u < 16; ++u) {
+                        const uint64_t x = f2_fma(f2(s[c * 32 + 2 * u], s[c * 32 + 2 * u + 1]), sc2, nmu2);
                         uint64_t e;
-                        if (u == 3) {
+                        if ((u & 3) == 3) {
                             e = exp2_fma_x2(x);
                         } else {
                             float a0, a1;
@@ -513,50 +469,54 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_con
                         acc[u & 1] = f2_add(acc[u & 1], e);
                         float e0, e1;
                         f2_split(e, e0, e1);
-                        pk[c * 4 + u] = pack_bf16x2(e0, e1);
+                        pk[u] = pack_bf16x2(e0, e1);
                     }
+                    tmem_st16(s_col + 16 * c, pk);
                 }
                 float a0, a1, b0, b1;
                 f2_split(acc[0], a0, a1);
                 f2_split(acc[1], b0, b1);
                 l_run += (a0 + a1) + (b0 + b1);
             }
-            // ---- P_i half row -> shared memory, once PV_{i-1} has read the buffer ------------
-            if (!pv_done) {
-                if (ok) ok = wait_or_abort(bar(B_PVFULL), (i - 1) & 1, abort_flag);
-                ok = __all_sync(0xffffffffu, ok);
-            }
-            if (ok) {
-                uint8_t *prow = sm + OFF_P;
+            // ---- the row's earlier output to the new base (the product into it is done) -------
+            if (__any_sync(0xffffffffu, move) && i > 0) {
 #pragma unroll
-                for (int c = 0; c < kKT / 16; ++c)
-                    *reinterpret_cast<uint4 *>(prow + swz(row, ch * 64 + c * 8, kRows)) =
-                        make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(o_col + 32 * c, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * f);
+                    tmem_st32(o_col + 32 * c, r);
+                }
             }
-            fence_proxy_async_smem();  // P is read by the tensor cores
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(B_PFULL));
+            if (lane == 0) mbar_arrive(bar(B_PFULL + qt));
         }
-        if (ok) ok = wait_or_abort(bar(B_PVFULL), (n_tiles - 1) & 1, abort_flag);
+        if (ok) ok = wait_or_abort(bar(B_ODONE + qt), 0, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
-        // the TMEM sum joins O (same base); the two halves' sums make the row's; normalise, store
-        float *lb = red + (n_tiles & 1) * 2 * kRows;
-        lb[ch * kRows + row] = l_run;
-        softmax_barrier();
         if (ok) {
             tc_fence_after();
-            fold_pv(1.f);
-            if (row_ok) {
-                const float l = lb[row] + lb[kRows + row];
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.o + (((size_t)b * p.T + t_row) * p.Hq + h_row) * kD + ch * (kD / 2));
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (((size_t)b * p.T + t_row) * p.Hq + h_row) * kD);
 #pragma unroll
-                for (int c = 0; c < kD / 16; ++c)
-                    dst[c] = make_uint4(pack_bf16x2(o[c * 8] * inv, o[c * 8 + 1] * inv),
-                                        pack_bf16x2(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv),
-                                        pack_bf16x2(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv),
-                                        pack_bf16x2(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv));
+            for (int c = 0; c < kD / 32; ++c) {
+                __syncwarp();  // converged for the TMEM load after the row-dependent stores
+                uint32_t r[32];
+                tmem_ld32(o_col + 32 * c, r);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float *v = reinterpret_cast<const float *>(r + 8 * q4);
+                        dst[c * 4 + q4] = make_uint4(pack_bf16x2(v[0] * inv, v[1] * inv),
+                                                     pack_bf16x2(v[2] * inv, v[3] * inv),
+                                                     pack_bf16x2(v[4] * inv, v[5] * inv),
+                                                     pack_bf16x2(v[6] * inv, v[7] * inv));
+                    }
+                }
             }
         } else if (lane == 0) {
             atomicOr(&g_err, HMD_DEVERR_TIMEOUT);
@@ -658,7 +618,7 @@ cudaError_t launch_tc(const AttnPrefillArgs &a, cudaStream_t s) {
     p.B = a.B; p.T = a.T; p.Hq = a.Hq; p.Hkv = a.Hkv;
     p.G = a.Hq / a.Hkv;
     p.QT = kRows / p.G;
-    p.n_qb = (a.T + p.QT - 1) / p.QT;
+    p.n_qb = (a.T + 2 * p.QT - 1) / (2 * p.QT);
     p.window = a.window; p.swa = a.swa ? 1 : 0;
     p.ring_pages = a.swa ? (a.window + kPT - 1) / kPT : 0;
     p.max_pages = a.max_pages; p.n_pages = a.n_pages;
