@@ -17,8 +17,9 @@ rank's time.
 
 The headline is timed as K CUDA-graph replays of the 48-layer step with nothing else on the
 stream. At one GPU the line also carries, each measured after the headline:
-  per_mixer          each mixer's layer time inside the stack (a separate pass with events
-                     around every layer) and its fraction of the HBM roofline;
+  per_mixer          each mixer's layer time inside the stack (CUDA-graph replays of that
+                     kind's layers, and its marginal cost in the interleaved step) and its
+                     fraction of the HBM roofline;
   placement_switch   the first step after a placement switch against a steady step;
   prefill, decode    tokens/s of each mixer at its own configuration (KDA/GDN prefill B=4,
                      H=16, T=4096; FA/SWA prefill B=2, T=8192; KDA/GDN decode B=64, H=32;
@@ -233,14 +234,28 @@ def run_ours(args, rank, world, local_rank):
     tokens = shape.B * args.steps * world
     value = job_throughput(shape.B * args.steps, world, ms)
 
-    # ---- per-mixer figures: a separate pass with events around every layer --------------------
+    # ---- per-mixer figures: CUDA-graph replays, no events inside a replay --------------------
+    # (1) each kind's layers of the stack alone, back to back, as one graph: layer time = replay
+    #     time / layers; (2) the kind's marginal cost inside the interleaved step: the 48-layer
+    #     replay minus a replay of the same step without that kind's layers, per layer.
     n_layers = st.n_layers
-    n_pass = max(3, min(args.steps, 8))
-    evs = [{l: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for l in range(n_layers)} for _ in range(n_pass)]
-    for k in range(n_pass):
-        st.step("hybrid", events=evs[k])
-    torch.cuda.synchronize()
+    n_rep = max(5, min(args.steps, 20))
+
+    def graph_ms(layers):
+        g = st.capture(lambda: st.step("hybrid", layers=layers), warmup=1)
+        for _ in range(2):
+            g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(n_rep):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / n_rep
+
+    full_ms = graph_ms(list(range(n_layers)))
     pk, pk_kind = peaks()
     hbm = float(pk["hbm_gbs"])
     per_kind = {}
@@ -248,24 +263,31 @@ def run_ours(args, rank, world, local_rank):
         layers = [l for l in range(n_layers) if pl[l] == kind]
         if not layers:
             continue
-        durs = [evs[k][l][0].elapsed_time(evs[k][l][1]) for k in range(n_pass) for l in layers]
-        mean_ms = float(np.mean(durs))
+        mean_ms = graph_ms(layers) / len(layers)
+        rest = [l for l in range(n_layers) if pl[l] != kind]
+        marg_ms = (full_ms - graph_ms(rest)) / len(layers)
         gbs = layer_bytes(kind, shape) / (mean_ms * 1e-3) / 1e9
         per_kind[I.KIND_NAMES[kind]] = {"layer_us": round(mean_ms * 1e3, 2),
                                         "achieved_gbs": round(gbs, 1),
                                         "frac": round(gbs / hbm, 4),
                                         "frac_nominal_8tbs": round(gbs / 8000.0, 4),
+                                        "marginal_layer_us": round(marg_ms * 1e3, 2),
                                         "bytes_per_layer": layer_bytes(kind, shape),
                                         "decode_tok_s_per_layer": round(shape.B / (mean_ms * 1e-3), 1)}
-    per_kind["measured"] = (f"separate pass after the timed region: {n_pass} eager steps with CUDA "
-                            f"events around each of the 48 layers on the launching stream")
+    assert hmd.hmd_device_errors(clear=True) == 0
+    per_kind["measured"] = (f"separate pass after the timed region: layer_us = one CUDA-graph "
+                            f"replay of that kind's layers of the stack (same caches and inputs), "
+                            f"back to back, / layers, mean of {n_rep} replays timed "
+                            f"with CUDA events around the replays only; marginal_layer_us = (the "
+                            f"48-layer replay, {full_ms:.3f} ms, minus a replay of the step "
+                            f"without that kind's layers) / that kind's layers")
     dom = per_kind["FA"]
     roofline = {"bound": "hbm", "achieved": dom["achieved_gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": dom["frac"], "traffic": traffic_for("attn_fa_stack48"),
                 "kernel": "attn_decode FA layer (attn_split_kernel<128> + attn_combine_kernel)",
                 "peak_source": pk_kind,
                 "algorithmic_bytes_per_launch": dom["bytes_per_layer"],
-                "timing": "per-layer CUDA events of the per-mixer pass"}
+                "timing": "CUDA-graph replays of the stack's FA layers (events around replays only)"}
     switch = placement_switch(st, args.warmup)
     assert hmd.hmd_device_errors(clear=True) == 0
 

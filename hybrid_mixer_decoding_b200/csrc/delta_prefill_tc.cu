@@ -20,9 +20,9 @@
 //    range); beyond that, A and P are formed directly from the exponent differences on the CUDA
 //    cores, so no gate range is refused. GDN (scalar gate): [k; q] k^T on the tensor cores and
 //    the decay e^(G_r - G_s) <= 1 applied per entry, which holds for any gate.
-//  - T: the 16 x 16 diagonal blocks of (I + A)^-1 by forward substitution (fp32), then each
-//    block column of the off-diagonal blocks by one warp with tf32 mma.sync (no CTA barrier
-//    between levels): X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj.
+//  - T: the 16 x 16 diagonal blocks of (I + A)^-1 by row sweeps (fp32, one half-warp per
+//    block), then the blocks below the diagonal on tf32 mma.sync, merging 16 -> 32 -> 64
+//    (four dependent products): X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj.
 //  - [W | Ut] = T [Kt | V] as M = 128 tcgen05.mma (token rows in TMEM lanes 0-63).
 //  - One record per chunk: [-W; Qt], Kc, P, e^G_C, Ut (bf16 tiles in the operand layouts the
 //    scan's tensor cores read; e^G_C fp32).
@@ -103,13 +103,42 @@ constexpr uint32_t S_BETA = 0, S_NRM = 256, S_G = 768, S_BAR = 1024, S_TMEM = 10
 constexpr uint32_t PA_SMEM = PA_SMALL + S_SIZE + 1024;
 constexpr int AS_LD = 68;
 constexpr int YS_LD = 24;
-constexpr uint32_t PA_YS = PA_KH + 8192;  // three warps' 16 x 24 fp32 scratch (rows 64-127 of
-                                          // the T operand: lanes the W/Ut read-back ignores)
+constexpr uint32_t PA_YS = PA_KH + 8192;  // four 16 x 24 fp32 tiles of the solve (rows 64-127
+                                          // of the T operand: lanes the W/Ut read-back ignores)
 constexpr uint32_t kPrepTmemCols = 256;
 constexpr uint32_t ID_AP = idesc_bf16(128, 64, 0, 0);    // [Kt; Qt] Kh^T: both K-major
 constexpr uint32_t ID_WU = idesc_bf16(128, 128, 0, 1);   // [T; -] [Kt | V]: B MN-major
-static_assert(PA_YS + 3 * 16 * YS_LD * 4 <= PA_V, "warp scratch fits");
+static_assert(PA_YS + 4 * 16 * YS_LD * 4 <= PA_V, "warp scratch fits");
 static_assert(PA_XS + 64 * AS_LD * 4 <= PA_SMALL, "solve tiles fit");
+
+// acc += A B for 16 x 16 fp32 tiles in shared memory, on tf32 mma.sync m16n8k8 (g = lane / 4,
+// t4 = lane % 4; acc[nt] is the accumulator fragment of columns 8 nt .. 8 nt + 7)
+__device__ __forceinline__ void mma16_tf32(float (&acc)[2][4], const float *A, int lda,
+                                           const float *Bm, int ldb, int g, int t4) {
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const float *ar = A + g * lda + 8 * ks + t4;
+        const uint32_t af[4] = {to_tf32(ar[0]), to_tf32(ar[8 * lda]), to_tf32(ar[4]),
+                                to_tf32(ar[8 * lda + 4])};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float *br = Bm + (8 * ks + t4) * ldb + 8 * nt + g;
+            mma_tf32_1688(acc[nt], af, to_tf32(br[0]), to_tf32(br[4 * ldb]));
+        }
+    }
+}
+// C = sgn * acc (fragment layout as above)
+__device__ __forceinline__ void store16(float *C, int ldc, const float (&acc)[2][4], float sgn,
+                                        int g, int t4) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int cc = 8 * nt + 2 * t4;
+        C[g * ldc + cc] = sgn * acc[nt][0];
+        C[g * ldc + cc + 1] = sgn * acc[nt][1];
+        C[(g + 8) * ldc + cc] = sgn * acc[nt][2];
+        C[(g + 8) * ldc + cc + 1] = sgn * acc[nt][3];
+    }
+}
 
 template <bool KDA>
 __global__ void __launch_bounds__(kPrepThreads, 2)
@@ -592,21 +621,36 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
     // ---- T = (I + A)^-1 Diag(beta) ---------------------------------------------------------
     uint8_t *Tt = sm + PA_KH;  // bf16 [r][s], K-major, rows 0-63 of the W/Ut product's A operand
-    if (warp < 4 && lane < 16) {  // diagonal block `warp`, column `lane`: forward substitution
-        const int bi = warp, c0 = lane;
-        const float *ab = As + bi * 16 * AS_LD + bi * 16;
-        const float bc = sbeta[bi * 16 + c0];
-        float x[16];
+    if (warp < 2) {
+        // diagonal blocks by row sweeps: half-warp (warp w, half hh) takes block i = 2 w + hh,
+        // lane r its row r; after step s, row s is final and every row below it subtracts A_rs
+        // times row s (rows arrive by shuffles)
+        const int bi = 2 * warp + (lane >> 4), r = lane & 15;
+        const float *ap = As + (bi * 16 + r) * AS_LD + bi * 16;
+        float ar[16], x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums: a short dependence chain
-#pragma unroll
-            for (int s2 = 0; s2 < r; ++s2) acc[s2 & 3] += ab[r * AS_LD + s2] * x[s2];
-            x[r] = r < c0 ? 0.f : (r == c0 ? 1.f : -((acc[0] + acc[1]) + (acc[2] + acc[3])));
-            Xs[(bi * 16 + r) * AS_LD + bi * 16 + c0] = x[r];
-            *reinterpret_cast<__nv_bfloat16 *>(Tt + toff(bi * 16 + r, bi * 16 + c0, 64)) =
-                __float2bfloat16_rn(x[r] * bc);
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 v = *reinterpret_cast<const float4 *>(ap + 4 * q4);
+            ar[4 * q4] = v.x; ar[4 * q4 + 1] = v.y; ar[4 * q4 + 2] = v.z; ar[4 * q4 + 3] = v.w;
         }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) x[c] = c == r ? 1.f : 0.f;
+#pragma unroll
+        for (int s = 0; s < 15; ++s) {
+            const float f = r > s ? ar[s] : 0.f;
+#pragma unroll
+            for (int c = 0; c <= s; ++c) x[c] = fmaf(-f, __shfl_sync(0xffffffffu, x[c], s, 16), x[c]);
+        }
+        float *xr = Xs + (bi * 16 + r) * AS_LD + bi * 16;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<float4 *>(xr + 4 * q4) = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            w[e] = pack_bf16x2(x[2 * e] * sbeta[bi * 16 + 2 * e], x[2 * e + 1] * sbeta[bi * 16 + 2 * e + 1]);
+        *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16 + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
     } else if (warp >= 4) {  // blocks above the diagonal of T are zero: 6 blocks x 16 rows x 32 B
         for (int idx = tid - 128; idx < 6 * 16 * 2; idx += 128) {
             const int blk = idx >> 5, rr = (idx >> 1) & 15, hh = idx & 1;
@@ -617,58 +661,56 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         }
     }
     __syncthreads();
-    if (warp < 3) {  // block column j = warp: X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj, i = j+1..3
-        const int j = warp, g = lane >> 2, t4 = lane & 3;
-        float *Ys = reinterpret_cast<float *>(sm + PA_YS) + warp * 16 * YS_LD;
-        for (int i = j + 1; i < 4; ++i) {
-            float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            for (int k = j; k < i; ++k) {
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    const float *ar = As + (16 * i + g) * AS_LD + 16 * k + 8 * ks + t4;
-                    const uint32_t af[4] = {to_tf32(ar[0]), to_tf32(ar[8 * AS_LD]), to_tf32(ar[4]),
-                                            to_tf32(ar[8 * AS_LD + 4])};
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const float *xr = Xs + (16 * k + 8 * ks + t4) * AS_LD + 16 * j + 8 * nt + g;
-                        mma_tf32_1688(y[nt], af, to_tf32(xr[0]), to_tf32(xr[4 * AS_LD]));
-                    }
-                }
-            }
+    {
+        const int g8 = lane >> 2, t4 = lane & 3;
+        float *Ys = reinterpret_cast<float *>(sm + PA_YS);
+        auto store_t = [&](int bi, int bj, const float (&acc)[2][4], float sgn) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                Ys[g * YS_LD + 8 * nt + 2 * t4] = y[nt][0];
-                Ys[g * YS_LD + 8 * nt + 2 * t4 + 1] = y[nt][1];
-                Ys[(g + 8) * YS_LD + 8 * nt + 2 * t4] = y[nt][2];
-                Ys[(g + 8) * YS_LD + 8 * nt + 2 * t4 + 1] = y[nt][3];
+                const int cc = 16 * bj + 8 * nt + 2 * t4;
+                const float b0 = sgn * sbeta[cc], b1 = sgn * sbeta[cc + 1];
+                *reinterpret_cast<uint32_t *>(Tt + toff(16 * bi + g8, cc, 64)) =
+                    pack_bf16x2(acc[nt][0] * b0, acc[nt][1] * b1);
+                *reinterpret_cast<uint32_t *>(Tt + toff(16 * bi + g8 + 8, cc, 64)) =
+                    pack_bf16x2(acc[nt][2] * b0, acc[nt][3] * b1);
             }
+        };
+        // Below the diagonal, X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj, merging 16 -> 32 -> 64.
+        // The 32 x 32 halves: X_10 = -X_11 (A_10 X_00) (warp 0), X_32 = -X_33 (A_32 X_22) (warp 1)
+        if (warp < 2) {
+            const int i = warp == 0 ? 1 : 3, jj = i - 1;
+            float *Y = Ys + warp * 16 * YS_LD;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            mma16_tf32(acc, As + 16 * i * AS_LD + 16 * jj, AS_LD, Xs + 16 * jj * AS_LD + 16 * jj, AS_LD, g8, t4);
+            store16(Y, YS_LD, acc, 1.f, g8, t4);
             __syncwarp();
-            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const float *xr = Xs + (16 * i + g) * AS_LD + 16 * i + 8 * ks + t4;
-                const uint32_t af[4] = {to_tf32(xr[0]), to_tf32(xr[8 * AS_LD]), to_tf32(xr[4]),
-                                        to_tf32(xr[8 * AS_LD + 4])};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const float *yr = Ys + (8 * ks + t4) * YS_LD + 8 * nt + g;
-                    mma_tf32_1688(x[nt], af, to_tf32(yr[0]), to_tf32(yr[4 * YS_LD]));
-                }
+            float xa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            mma16_tf32(xa, Xs + 16 * i * AS_LD + 16 * i, AS_LD, Y, YS_LD, g8, t4);
+            store16(Xs + 16 * i * AS_LD + 16 * jj, AS_LD, xa, -1.f, g8, t4);
+            store_t(i, jj, xa, -1.f);
+        }
+        __syncthreads();
+        // the lower-left 32 x 32 quarter, X_BA = -X_B (A_BA X_A) with A = rows 0-31, B = rows
+        // 32-63; warp w takes block (i, j) = (2 + w / 2, w % 2): Y_ij = sum_k A_ik X_kj ...
+        if (warp < 4) {
+            const int i = 2 + (warp >> 1), jj = warp & 1;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            if (jj == 0) {
+                mma16_tf32(acc, As + 16 * i * AS_LD, AS_LD, Xs, AS_LD, g8, t4);
+                mma16_tf32(acc, As + 16 * i * AS_LD + 16, AS_LD, Xs + 16 * AS_LD, AS_LD, g8, t4);
+            } else {
+                mma16_tf32(acc, As + 16 * i * AS_LD + 16, AS_LD, Xs + 16 * AS_LD + 16, AS_LD, g8, t4);
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int cc = 16 * j + 8 * nt + 2 * t4;
-                const float b0 = sbeta[cc], b1 = sbeta[cc + 1];
-                Xs[(16 * i + g) * AS_LD + cc] = -x[nt][0];
-                Xs[(16 * i + g) * AS_LD + cc + 1] = -x[nt][1];
-                Xs[(16 * i + g + 8) * AS_LD + cc] = -x[nt][2];
-                Xs[(16 * i + g + 8) * AS_LD + cc + 1] = -x[nt][3];
-                *reinterpret_cast<uint32_t *>(Tt + toff(16 * i + g, cc, 64)) =
-                    pack_bf16x2(-x[nt][0] * b0, -x[nt][1] * b1);
-                *reinterpret_cast<uint32_t *>(Tt + toff(16 * i + g + 8, cc, 64)) =
-                    pack_bf16x2(-x[nt][2] * b0, -x[nt][3] * b1);
-            }
-            __syncwarp();
+            store16(Ys + warp * 16 * YS_LD, YS_LD, acc, 1.f, g8, t4);
+        }
+        __syncthreads();
+        // ... then X_2j = -X_22 Y_2j and X_3j = -(X_32 Y_2j + X_33 Y_3j)
+        if (warp < 4) {
+            const int i = 2 + (warp >> 1), jj = warp & 1;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            mma16_tf32(acc, Xs + 16 * i * AS_LD + 32, AS_LD, Ys + jj * 16 * YS_LD, YS_LD, g8, t4);
+            if (i == 3) mma16_tf32(acc, Xs + 48 * AS_LD + 48, AS_LD, Ys + (2 + jj) * 16 * YS_LD, YS_LD, g8, t4);
+            store_t(i, jj, acc, -1.f);
         }
     }
     fence_proxy_async_smem();  // T, Kt, Qt (GDN) are read by the tensor cores

@@ -196,14 +196,16 @@ class MixerStack:
     def pools_for(self, layer: int):
         return self.kv_for(layer).layer_pools(layer)
 
-    def step(self, name: str, events: dict | None = None, io_set: int = 0) -> None:
+    def step(self, name: str, events: dict | None = None, io_set: int = 0,
+             layers=None) -> None:
         """One decode token for every sequence through all layers under placement `name`,
         reading and writing the per-layer buffers of set `io_set`.
-        events: optional {layer: (start_event, end_event)} recorded around that layer."""
+        events: optional {layer: (start_event, end_event)} recorded around that layer.
+        layers: optional subset of the layer indices to run (in order); default all."""
         pl = self.placements[name]
         cpl = self.c_placements[name]
         ios = self.io_sets[io_set]
-        for l in range(self.n_layers):
+        for l in (range(self.n_layers) if layers is None else layers):
             kind = int(pl[l])
             ev = events.get(l) if events else None
             if ev:
