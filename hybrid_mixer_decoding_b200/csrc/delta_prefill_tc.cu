@@ -21,8 +21,9 @@
 //    cores, so no gate range is refused. GDN (scalar gate): [k; q] k^T on the tensor cores and
 //    the decay e^(G_r - G_s) <= 1 applied per entry, which holds for any gate.
 //  - T: the 16 x 16 diagonal blocks of (I + A)^-1 by row sweeps (fp32, one half-warp per
-//    block), then the blocks below the diagonal on tf32 mma.sync, merging 16 -> 32 -> 64
-//    (four dependent products): X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj.
+//    block, straight from the registers the A read-back left them in), then the blocks below
+//    the diagonal on tf32 mma.sync, merging 16 -> 32 -> 64 (four dependent products):
+//    X_ij = -X_ii sum_{k=j}^{i-1} A_ik X_kj.
 //  - [W | Ut] = T [Kt | V] as M = 128 tcgen05.mma (token rows in TMEM lanes 0-63).
 //  - One record per chunk: [-W; Qt], Kc, P, e^G_C, Ut (bf16 tiles in the operand layouts the
 //    scan's tensor cores read; e^G_C fp32).
@@ -137,6 +138,42 @@ __device__ __forceinline__ void store16(float *C, int ldc, const float (&acc)[2]
         C[g * ldc + cc + 1] = sgn * acc[nt][1];
         C[(g + 8) * ldc + cc] = sgn * acc[nt][2];
         C[(g + 8) * ldc + cc + 1] = sgn * acc[nt][3];
+    }
+}
+
+// The 16 x 16 diagonal block bi of X = (I + A)^-1 by a row sweep in fp32, run by one half-warp:
+// lane r (r = lane % 16) holds row r of the block, ar[s] = A_rs (s < r; the rest is ignored).
+// After step s row s is final and every row below it subtracts A_rs times row s, which arrives
+// by a shuffle. The row goes to Xs (fp32) and to T (bf16, times beta of its column).
+__device__ __forceinline__ void diag_sweep(const float (&ar)[16], int bi, int r, float *Xs,
+                                           uint8_t *Tt, const float *sbeta) {
+    float x[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) x[c] = c == r ? 1.f : 0.f;
+#pragma unroll
+    for (int s = 0; s < 15; ++s) {
+        const float f = r > s ? ar[s] : 0.f;
+#pragma unroll
+        for (int c = 0; c <= s; ++c) x[c] = fmaf(-f, __shfl_sync(0xffffffffu, x[c], s, 16), x[c]);
+    }
+    float *xr = Xs + (bi * 16 + r) * AS_LD + bi * 16;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<float4 *>(xr + 4 * q4) = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+    uint32_t w[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        w[e] = pack_bf16x2(x[2 * e] * sbeta[bi * 16 + 2 * e], x[2 * e + 1] * sbeta[bi * 16 + 2 * e + 1]);
+    *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16 + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+// T's blocks above the diagonal are zero: 6 blocks x 16 rows x 32 B, by 128 threads (t < 128)
+__device__ __forceinline__ void zero_upper_t(uint8_t *Tt, int t) {
+    for (int idx = t; idx < 6 * 16 * 2; idx += 128) {
+        const int blk = idx >> 5, rr = (idx >> 1) & 15, hh = idx & 1;
+        const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);              // block row
+        const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);  // block column > bi
+        *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + rr, bj * 16 + hh * 8, 64)) = make_uint4(0, 0, 0, 0);
     }
 }
 
@@ -565,15 +602,21 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (quad < 2) {  // A_rs = beta_r (.)_rs, s < r
             const float br = r < n ? sbeta[r] : 0.f;
             float *arow = As + r * AS_LD + s0;
+            float av[32];
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-                float v[4];
+            for (int ee = 0; ee < 32; ++ee) av[ee] = (s0 + ee < r) ? br * dec[ee] * __uint_as_float(d[ee]) : 0.f;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int ee = 4 * j4 + e;
-                    v[e] = (s0 + ee < r) ? br * dec[ee] * __uint_as_float(d[ee]) : 0.f;
-                }
-                *reinterpret_cast<float4 *>(arow + 4 * j4) = make_float4(v[0], v[1], v[2], v[3]);
+            for (int j4 = 0; j4 < 8; ++j4)
+                *reinterpret_cast<float4 *>(arow + 4 * j4) =
+                    make_float4(av[4 * j4], av[4 * j4 + 1], av[4 * j4 + 2], av[4 * j4 + 3]);
+            // warp 0 (rows 0-31, columns 0-31) holds diagonal blocks 0 and 1, warp 5 (rows 32-63,
+            // columns 32-63) blocks 2 and 3, one per half-warp: sweep them from these registers
+            if (warp == 0 || warp == 5) {
+                const int hh = lane >> 4;
+                float ar[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) ar[e] = hh ? av[16 + e] : av[e];
+                diag_sweep(ar, 2 * (warp == 5) + hh, lane & 15, Xs, sm + PA_KH, sbeta);
             }
         } else {  // P_rs, s <= r
 #pragma unroll
@@ -588,6 +631,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                 *reinterpret_cast<uint4 *>(rec + REC_P + toff(r, s0 + 8 * u, 64)) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
+            zero_upper_t(sm + PA_KH, (warp >> 2) * 64 + (quad - 2) * 32 + lane);
         }
         tc_fence_before();
         __syncthreads();
@@ -621,46 +665,24 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
     // ---- T = (I + A)^-1 Diag(beta) ---------------------------------------------------------
     uint8_t *Tt = sm + PA_KH;  // bf16 [r][s], K-major, rows 0-63 of the W/Ut product's A operand
-    if (warp < 2) {
-        // diagonal blocks by row sweeps: half-warp (warp w, half hh) takes block i = 2 w + hh,
-        // lane r its row r; after step s, row s is final and every row below it subtracts A_rs
-        // times row s (rows arrive by shuffles)
-        const int bi = 2 * warp + (lane >> 4), r = lane & 15;
-        const float *ap = As + (bi * 16 + r) * AS_LD + bi * 16;
-        float ar[16], x[16];
+    // the diagonal blocks: swept from the read-back registers above, or here after the
+    // CUDA-core A of a chunk beyond the factor range (then from As)
+    if (fallback) {
+        if (warp < 2) {
+            const int bi = 2 * warp + (lane >> 4), r = lane & 15;
+            const float *ap = As + (bi * 16 + r) * AS_LD + bi * 16;
+            float ar[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 v = *reinterpret_cast<const float4 *>(ap + 4 * q4);
-            ar[4 * q4] = v.x; ar[4 * q4 + 1] = v.y; ar[4 * q4 + 2] = v.z; ar[4 * q4 + 3] = v.w;
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 v = *reinterpret_cast<const float4 *>(ap + 4 * q4);
+                ar[4 * q4] = v.x; ar[4 * q4 + 1] = v.y; ar[4 * q4 + 2] = v.z; ar[4 * q4 + 3] = v.w;
+            }
+            diag_sweep(ar, bi, r, Xs, Tt, sbeta);
+        } else if (warp >= 4) {
+            zero_upper_t(Tt, tid - 128);
         }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) x[c] = c == r ? 1.f : 0.f;
-#pragma unroll
-        for (int s = 0; s < 15; ++s) {
-            const float f = r > s ? ar[s] : 0.f;
-#pragma unroll
-            for (int c = 0; c <= s; ++c) x[c] = fmaf(-f, __shfl_sync(0xffffffffu, x[c], s, 16), x[c]);
-        }
-        float *xr = Xs + (bi * 16 + r) * AS_LD + bi * 16;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<float4 *>(xr + 4 * q4) = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
-        uint32_t w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            w[e] = pack_bf16x2(x[2 * e] * sbeta[bi * 16 + 2 * e], x[2 * e + 1] * sbeta[bi * 16 + 2 * e + 1]);
-        *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + r, bi * 16 + 8, 64)) = make_uint4(w[4], w[5], w[6], w[7]);
-    } else if (warp >= 4) {  // blocks above the diagonal of T are zero: 6 blocks x 16 rows x 32 B
-        for (int idx = tid - 128; idx < 6 * 16 * 2; idx += 128) {
-            const int blk = idx >> 5, rr = (idx >> 1) & 15, hh = idx & 1;
-            const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);              // block row
-            const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);  // block column > bi
-            *reinterpret_cast<uint4 *>(Tt + toff(bi * 16 + rr, bj * 16 + hh * 8, 64)) =
-                make_uint4(0, 0, 0, 0);
-        }
+        __syncthreads();
     }
-    __syncthreads();
     {
         const int g8 = lane >> 2, t4 = lane & 3;
         float *Ys = reinterpret_cast<float *>(sm + PA_YS);
