@@ -25,7 +25,9 @@ stream. At one GPU the line also carries, each measured after the headline:
                      H=16, T=4096; FA/SWA prefill B=2, T=8192; KDA/GDN decode B=64, H=32;
                      FA/SWA decode B=32, ctx 8192), each with its roofline and the fp64
                      oracle's tokens/s on a bounded sample of the same work on the host's cores;
-  oracle_check       the fp32 GDN configuration (B=1, H=2, d=64, T=128) against the oracle.
+  oracle_check       the fp32 GDN configuration (B=1, H=2, d=64, T=128) against the oracle;
+  context_sweep      decode tok/s of all-FA and the hybrid placements at 8k and 128k context
+                     (B=16, 48 layers) and each one's speedup over all-FA.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of the method) on a
 bounded sample of the same workload on this host's cores.
@@ -1052,24 +1054,25 @@ def linear_cost_model(pls, res):
     return out
 
 
-def run_sweep(args):
-    """Context sweep: B=16, ctx in {4k, 16k, 64k, 128k}, 48-layer stack, placements all-FA,
-    24 FA + 24 GDN, 8 FA + 40 (20 KDA + 20 GDN), all-GDN, all-KDA; decode tok/s, speedup over
-    all-FA, and the linear per-layer cost model checked against the mixed placements.
+def run_sweep(args, ctxs=SWEEP_CTX, steps=None):
+    """Context sweep: B=16, ctx in {4k, 16k, 64k, 128k} (or `ctxs`), 48-layer stack, placements
+    all-FA, 24 FA + 24 GDN, 8 FA + 40 (20 KDA + 20 GDN), all-GDN, all-KDA; decode tok/s, speedup
+    over all-FA, and the linear per-layer cost model checked against the mixed placements.
     KV pools are zero-filled (timing only); FA layers share physical pools round-robin when the
     placement's KV exceeds device memory (each layer still streams its own full context)."""
     import torch
 
     from hybrid_mixer_decoding_b200.stack import MixerStack, StackShape, layer_bytes
     pls = sweep_placements()
+    steps = args.steps if steps is None else steps
     rows = []
-    for ctx in SWEEP_CTX:
+    for ctx in ctxs:
         shape = StackShape(16, 32, 8, 128, ctx, 4096)
         st = MixerStack(pls, shape, seed=0, fill_kv=False)
         res = {}
         graphs = {name: st.capture(name) for name in pls}
         for name in pls:
-            sec = _events_time(graphs[name].replay, args.steps, args.warmup)
+            sec = _events_time(graphs[name].replay, steps, args.warmup)
             byts = sum(layer_bytes(int(k), shape) for k in pls[name])
             res[name] = {"tok_s": round(16 / sec, 1), "ms_per_step": round(sec * 1e3, 3),
                          "achieved_gbs": round(byts / sec / 1e9, 1)}
@@ -1087,7 +1090,21 @@ def run_sweep(args):
     return {"metric": "decode tok/s per placement (BxCtx), context sweep", "workload":
             "sweep: 48-layer mixer-only stack, B=16, H=32, Hkv=8, d=128, SWA-free placements; "
             "each step one CUDA-graph replay of the 48 mixer_decode_step calls",
-            "steps": args.steps, "warmup": args.warmup, "rows": rows}
+            "steps": steps, "warmup": args.warmup, "rows": rows}
+
+
+def context_sweep_line(args) -> dict:
+    """The hybrid placements' decode speedup over all-FA at 8k and 128k context (B=16, 48 layers,
+    CUDA-graph replays), for the one-GPU bench line; the full sweep is --workload sweep."""
+    r = run_sweep(args, ctxs=(8192, 131072), steps=min(args.steps, 10))
+    return {"workload": r["workload"], "steps": r["steps"],
+            "rows": [{"ctx": row["ctx"], "aliased_fa_pools": row["aliased_fa_pools"],
+                      "tok_s": {n: v["tok_s"] for n, v in row["placements"].items()},
+                      "speedup_vs_all_fa": {n: v["speedup_vs_all_fa"] for n, v in row["placements"].items()},
+                      "predicted_by_bytes": {n: v["predicted_by_bytes"] for n, v in row["placements"].items()},
+                      "achieved_gbs": {n: v["achieved_gbs"] for n, v in row["placements"].items()},
+                      "linear_cost_model": row["linear_cost_model"]}
+                     for row in r["rows"]]}
 
 
 def main():
@@ -1119,6 +1136,7 @@ def main():
             # per-mixer prefill and decode lines and the fp32 oracle check, on this rank's GPU
             out.update(per_mixer_lines(args))
             out["oracle_check"] = oracle_check_config1()
+            out["context_sweep"] = context_sweep_line(args)
     elif args.workload == "sweep":
         out = run_sweep(args)
     elif args.workload == "spec_stack":
