@@ -130,3 +130,15 @@ def test_config3_full_size(oracle_mod, kind):
     w = 4096 if kind == I.SWA else 0
     a = I.attn_inputs(kind, 32, 32, 8, 128, 8192, window=w, seed=2)
     check(a, oracle_mod)
+
+
+@pytest.mark.parametrize("kind", [I.FA, I.SWA])
+def test_long_context_128k(oracle_mod, kind):
+    """The context sweep's longest context: B=2, Hq=32, Hkv=8, d=128, one sequence at 131072
+    tokens and one ragged at 100033 (the split plan's longest key ranges, and a last page that
+    holds only the new token), SWA window 4096, random page permutation: every output and the
+    append checked."""
+    w = 4096 if kind == I.SWA else 0
+    a = I.attn_inputs(kind, 2, 32, 8, 128, 131072, window=w, seed=5,
+                      seq_lens=np.array([131072, 100033], np.int32))
+    check(a, oracle_mod)
