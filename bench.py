@@ -27,7 +27,9 @@ stream. At one GPU the line also carries, each measured after the headline:
                      oracle's tokens/s on a bounded sample of the same work on the host's cores;
   oracle_check       the fp32 GDN configuration (B=1, H=2, d=64, T=128) against the oracle;
   context_sweep      decode tok/s of all-FA and the hybrid placements at 8k and 128k context
-                     (B=16, 48 layers) and each one's speedup over all-FA.
+                     (B=16, 48 layers) and each one's speedup over all-FA;
+  speculative,       self-speculative decoding (drafter all-GDN, k = 3) and one mixed batch of
+  mixed_batch        two placements on the stack, each with its roofline.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of the method) on a
 bounded sample of the same workload on this host's cores.
@@ -1093,6 +1095,27 @@ def run_sweep(args, ctxs=SWEEP_CTX, steps=None):
             "steps": steps, "warmup": args.warmup, "rows": rows}
 
 
+def next_row_lines(args) -> dict:
+    """Self-speculative decoding and a mixed-placement batch on the 48-layer stack (B=32 and
+    B=64 at ctx 32768), each with its roofline, for the one-GPU bench line; the full lines are
+    --workload spec_stack and mixed_stack. A failure is recorded in the line, not raised."""
+    import argparse as _ap
+
+    import torch
+    short = _ap.Namespace(**{**vars(args), "steps": min(args.steps, 10)})
+    keep = ("value", "unit", "ms_per_step", "roofline", "spec", "mixed", "config")
+    out = {}
+    for key, fn in (("speculative", run_spec), ("mixed_batch", run_mixed)):
+        try:
+            r = fn(short)
+            out[key] = {k: r[k] for k in keep if k in r}
+        except Exception as e:  # noqa: BLE001 - reported in the line
+            out[key] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 def context_sweep_line(args) -> dict:
     """The hybrid placements' decode speedup over all-FA at 8k and 128k context (B=16, 48 layers,
     CUDA-graph replays), for the one-GPU bench line; the full sweep is --workload sweep."""
@@ -1137,6 +1160,7 @@ def main():
             out.update(per_mixer_lines(args))
             out["oracle_check"] = oracle_check_config1()
             out["context_sweep"] = context_sweep_line(args)
+            out.update(next_row_lines(args))
     elif args.workload == "sweep":
         out = run_sweep(args)
     elif args.workload == "spec_stack":
