@@ -27,6 +27,8 @@
 //  - [W | Ut] = T [Kt | V] as M = 128 tcgen05.mma (token rows in TMEM lanes 0-63).
 //  - One record per chunk: [-W; Qt], Kc, P, e^G_C, Ut (bf16 tiles in the operand layouts the
 //    scan's tensor cores read; e^G_C fp32).
+//  - The fused input activations are a template parameter, so the plain kernel carries none of
+//    their code (a smaller kernel measured 2-3% faster).
 // Pass B (prefill_scan_kernel): one CTA per (sequence, head, half of d_v) walks the chunks,
 // warp-specialised: a producer warp streams records into a 3-stage ring with bulk copies (enough
 // bytes in flight per SM to cover the copies' latency), one thread issues the tcgen05.mma
@@ -177,7 +179,7 @@ __device__ __forceinline__ void zero_upper_t(uint8_t *Tt, int t) {
     }
 }
 
-template <bool KDA>
+template <bool KDA, bool FUSED>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmg,
@@ -203,7 +205,7 @@ prefill_prep_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     uint8_t *rec = record(a, bh, c);
     const uint32_t bar_in = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]),
                    bar_g = smem_u32(&bars[2]);
-    const bool fused = a.act.A_log != nullptr;  // raw projections: activate them here
+    constexpr bool fused = FUSED;  // raw projections (act.A_log set): activate them here
 
     if (tid == 0) {
         mbar_init(bar_in, 1);
@@ -1097,11 +1099,11 @@ size_t delta_prefill_scan_record_bytes() { return REC_BYTES; }
 cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_t ws_bytes,
                                       cudaStream_t s) {
     const cudaError_t attr = once_per_device([] {
-        cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(prefill_prep_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM);
+        cudaError_t e = cudaSuccess;
+        for (auto k : {prefill_prep_kernel<true, false>, prefill_prep_kernel<true, true>,
+                       prefill_prep_kernel<false, false>, prefill_prep_kernel<false, true>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PA_SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)SB_SMEM);
@@ -1142,7 +1144,9 @@ cudaError_t launch_delta_prefill_scan(const DeltaPrefillArgs &a, void *ws, size_
         p.chunk_begin = cb;
         p.n_seg = std::min(seg, n_chunks - cb);
         const unsigned grid_a = (unsigned)(bhs * p.n_seg);
-        cudaError_t e = launch_pdl(a.kind == HMD_KDA ? prefill_prep_kernel<true> : prefill_prep_kernel<false>,
+        const bool fused = a.act.A_log != nullptr;
+        cudaError_t e = launch_pdl(a.kind == HMD_KDA ? (fused ? prefill_prep_kernel<true, true> : prefill_prep_kernel<true, false>)
+                                                     : (fused ? prefill_prep_kernel<false, true> : prefill_prep_kernel<false, false>),
                                    dim3(grid_a), dim3(kPrepThreads), PA_SMEM, s, tmq, tmk, tmv, tmg, p);
         if (e != cudaSuccess) return e;
         e = launch_pdl(prefill_scan_kernel, dim3((unsigned)(bhs * kSplitV)), dim3(kScanThreads),
