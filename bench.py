@@ -715,20 +715,16 @@ def measure_workload(w: str, steps: int, warmup: int) -> dict:
 
 
 def run_kernel_workload(args):
-    """One mixer kernel at its configuration as the JSON line (see measure_workload), with the
-    SM clocks sampled while it runs."""
-    clk = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
-    clk.start()
-    try:
-        m = measure_workload(args.workload, args.steps, args.warmup)
-    finally:
-        clocks = clk.stop()
+    """One mixer kernel at its configuration as the JSON line (see measure_workload). Its timed
+    region lasts milliseconds, shorter than the clock sampler's period, so the line carries no
+    clock record; the default stack line does."""
+    m = measure_workload(args.workload, args.steps, args.warmup)
     out = {"metric": METRIC, "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": m.pop("ms_per_step"),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded)", "config": {"workload": m.pop("workload")},
            "roofline": m.pop("roofline"),
-           "gpu_launches": m.pop("launches_per_step") * args.steps, "clocks": clocks}
+           "gpu_launches": m.pop("launches_per_step") * args.steps}
     out.update(m)
     if not args.skip_cpu_baseline and args.workload in ORACLE_SAMPLES:
         out["cpu_baseline"] = workload_cpu_baseline(args.workload, args.cpu_budget / 4)
